@@ -1,0 +1,11 @@
+"""The oracle against the pages' printed values, library routines, brute force, closed
+forms and invariants (no GPU)."""
+import pytest
+
+import oracle
+import oracle_pins
+
+
+@pytest.mark.parametrize("pin", oracle_pins.ALL_PINS, ids=lambda f: f.__name__)
+def test_pin(pin):
+    pin(oracle)
