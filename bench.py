@@ -1,0 +1,430 @@
+"""Throughput of the binary convolution on B200: one JSON line per run.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload NAME|INDEX] [--no-e2e] [--no-cpu-baseline]
+
+A step is one forward of the layer (input transform + pack + A, beta, contraction and
+epilogue) over one batch of the workload: by default XNOR with beta scaling and input terms,
+batch 16, 56x56, 256 -> 256 channels, 3x3, ReLU.  ``value`` is nominal bit multiply-
+accumulates (every window tap, 1 op = 1 bit MAC) per second over all ranks, with inputs
+resident in HBM; four input/output buffer sets rotate so that one step's data is not in L2
+when it is next used (411 MB > the 126 MB L2).  ``e2e`` is the same metric through
+bconv_forward_host with page-locked host buffers (host-to-device copy, forward,
+device-to-host copy inside every step).  Multi-GPU runs (torchrun) are independent replicas
+with a batch each (weak scaling); their time is the maximum over ranks.
+
+``--impl reference`` times the oracle (the plain double-precision CPU loops) on the same
+workload, each step a bounded sample of output pixels, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from binarized_convolution_b200 import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "xnor_beta_n16_56x56_c256_k256_3x3"
+METRIC = "binary conv TOPS (1 op = 1 bit MAC) and images/s on 1 B200; % of roofline"
+UNIT = "TOPS"
+ROTATE = 4
+POPC_PER_CLK_PER_SM = 16  # 32-bit POPC lanes per clock per SM
+FP32_PER_CLK_PER_SM = 128  # FFMA lanes per clock per SM
+
+
+# ----------------------------------------------------------------------------------------
+# ranks
+# ----------------------------------------------------------------------------------------
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(
+        os.environ.get("LOCAL_RANK", "0"))
+
+
+def dist_init(backend: str):
+    import datetime
+
+    import torch.distributed as dist
+
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Maximum of a float over all ranks (identity for a single process)."""
+    import torch
+    import torch.distributed as dist
+
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+
+    if dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def replica_seed(base: int, rank: int) -> int:
+    """Each replica draws its own batch; rank 0 uses the workload's own seed."""
+    return base + 7919 * rank
+
+
+# ----------------------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; no setting is changed)
+# ----------------------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {"gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+               "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+
+    def start(self):
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self._h = h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 -- clocks are reported as unavailable
+            self._nvml = None
+            return self
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def _run(self):
+        p = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(p.nvmlDeviceGetClockInfo(self._h, p.NVML_CLOCK_SM))
+                self.reasons |= p.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:  # noqa: BLE001
+                pass
+            self._stop.wait(self.period)
+
+    def stop(self):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [k for k, v in self.REASONS.items() if self.reasons & v and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------------------
+# roofline bookkeeping
+# ----------------------------------------------------------------------------------------
+def kernel_source_digest(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, workload: str, sources) -> float | None:
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            table = json.load(f)
+    except (OSError, ValueError):
+        return None
+    rec = table.get(f"{kernel}:{workload}")
+    if not rec or rec.get("source_digest") != kernel_source_digest(sources):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+KERNEL_SOURCES = {
+    "popc_gemm": ["binarized_convolution_b200/csrc/popc_gemm.cu", "binarized_convolution_b200/csrc/common.cuh"],
+    "bw_conv": ["binarized_convolution_b200/csrc/bw_conv.cu", "binarized_convolution_b200/csrc/common.cuh"],
+}
+
+
+def contraction_kernel(w: synth.Workload) -> str:
+    return "bw_conv" if w.op == synth.BINARY_WEIGHTS else "popc_gemm"
+
+
+def derived_peak(w: synth.Workload, sms: int, sm_mhz: float) -> tuple[float, str, str]:
+    """(peak in TOPS, bound, how it was derived) for the contraction's instruction mix."""
+    if w.op == synth.BINARY_WEIGHTS:
+        p = sms * FP32_PER_CLK_PER_SM * sm_mhz * 1e6 / 1e12
+        return p, "alu", f"{sms} SMs x {FP32_PER_CLK_PER_SM} FP32 lanes/clk x {sm_mhz:.0f} MHz (1 op = 1 signed add)"
+    p = sms * POPC_PER_CLK_PER_SM * 32 * sm_mhz * 1e6 / 1e12
+    return p, "alu", f"{sms} SMs x {POPC_PER_CLK_PER_SM} POPC/clk x 32 bits x {sm_mhz:.0f} MHz"
+
+
+# ----------------------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample of output pixels
+# ----------------------------------------------------------------------------------------
+def oracle_sample_rate(w: synth.Workload, inp, target_s: float, rng_seed: int = 0):
+    """Times the oracle on output pixels of the workload; returns (TOPS, seconds, pixels, threads)."""
+    import oracle
+
+    otype = {synth.XNOR: oracle.ORACLE_XNOR, synth.AND: oracle.ORACLE_AND,
+             synth.BINARY_WEIGHTS: oracle.ORACLE_BINARY_WEIGHTS}[w.op]
+    rows_total = w.batch * w.out_h * w.out_w
+    ops_per_row = w.nominal_ops / rows_total
+    rng = np.random.default_rng(rng_seed)
+
+    def run(n):
+        rows = np.sort(rng.choice(rows_total, size=min(n, rows_total), replace=False)).astype(np.int64)
+        kw = dict(type=otype, scale=inp.scale, bias=inp.bias, in_scale=inp.in_scale, in_bias=inp.in_bias,
+                  use_beta=w.use_beta, relu=w.relu)
+        t0 = time.perf_counter()
+        if w.kind == "fc":
+            oracle.fc(inp.x, inp.wbits, rows=rows, **kw)
+        else:
+            oracle.conv(inp.x, inp.wbits, stride=(w.stride_y, w.stride_x), pixels=rows, **kw)
+        return time.perf_counter() - t0, len(rows)
+
+    threads = oracle.num_threads()
+    n = max(threads, 8)
+    dt, n = run(n)
+    while dt < 0.5 and n < rows_total:
+        n = min(rows_total, n * 4)
+        dt, n = run(n)
+    want = int(n * target_s / max(dt, 1e-6))
+    want = max(1, min(rows_total, want))
+    dt, n = run(want)
+    return n * ops_per_row / dt / 1e12, dt, n, threads
+
+
+# ----------------------------------------------------------------------------------------
+# native arm
+# ----------------------------------------------------------------------------------------
+def run_native(args, w: synth.Workload):
+    import torch
+
+    import binarized_convolution_b200 as bc
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init("nccl")
+
+    inp = synth.make_inputs(w, seed=replica_seed(w.seed, rank))
+    layer_kw = dict(op=w.op, scale=inp.scale, bias=inp.bias, in_scale=inp.in_scale, in_bias=inp.in_bias,
+                    use_beta=w.use_beta, relu=w.relu)
+    if w.kind == "fc":
+        layer = bc.BinaryFC(w.batch, w.in_h, w.in_w, w.in_channels, w.out_channels, wbits=inp.wbits, **layer_kw)
+        prof_begin, prof_end = bc.bfc_profile_begin, bc.bfc_profile_end
+    else:
+        layer = bc.BinaryConv2d(w.batch, w.in_h, w.in_w, w.in_channels, w.out_channels, (w.kernel_h, w.kernel_w),
+                                (w.stride_y, w.stride_x), wbits=inp.wbits, **layer_kw)
+        prof_begin, prof_end = bc.bconv_profile_begin, bc.bconv_profile_end
+    out_shape = layer.out_dims
+    xs = [torch.from_numpy(inp.x).to(device)]
+    for r in range(1, ROTATE):
+        xs.append(torch.from_numpy(synth.make_batch(w, seed=replica_seed(w.seed, rank) * 1000 + r)).to(device))
+    ys = [torch.empty(out_shape, dtype=torch.float32, device=device) for _ in range(ROTATE)]
+    stream = torch.cuda.current_stream(device)
+
+    for i in range(args.warmup):
+        layer.forward_into(xs[i % ROTATE], ys[i % ROTATE])
+    layer.sync_status(stream.cuda_stream)
+    torch.cuda.synchronize(device)
+
+    clocks = ClockSampler(local).start()
+    prof_begin(layer.handle, args.steps)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    ev0.record(stream)
+    for i in range(args.steps):
+        layer.forward_into(xs[i % ROTATE], ys[i % ROTATE])
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clock_info = clocks.stop()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    kern_ms, kern_n = prof_end(layer.handle)
+    layer.sync_status(stream.cuda_stream)
+    elapsed_ms = max_over_ranks(elapsed_ms, device)
+    kern_ms_max = max_over_ranks(kern_ms / max(kern_n, 1), device)
+
+    ops_step = w.nominal_ops
+    total_ops = ops_step * args.steps * world
+    value = total_ops / (elapsed_ms * 1e-3) / 1e12
+    images_s = w.batch * args.steps * world / (elapsed_ms * 1e-3)
+
+    # roofline of the contraction kernel: nominal ops of one launch / its mean event time
+    props = torch.cuda.get_device_properties(device)
+    sms = props.multi_processor_count
+    max_mhz = clock_info.get("sm_max_mhz") or 1965.0
+    peak, bound, how = derived_peak(w, sms, max_mhz)
+    achieved = ops_step / (kern_ms_max * 1e-3) / 1e12
+    kname = contraction_kernel(w)
+    traffic = measured_traffic(kname, w.name, KERNEL_SOURCES[kname])
+    roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+            "traffic": traffic, "kernel": kname, "kernel_ms": kern_ms_max, "peak_source": f"derived: {how}"}
+    sm_mhz = clock_info.get("sm_mhz")
+    if sm_mhz:
+        p_obs, _, _ = derived_peak(w, sms, sm_mhz)
+        roof["frac_at_observed_clock"] = achieved / p_obs
+    try:
+        probe = 0 if w.op != synth.BINARY_WEIGHTS else None
+        if probe is not None and rank == 0:
+            ops_s, mhz = bc.bconv_measure_peak(probe)
+            roof["probe_peak"] = ops_s / 1e12
+            roof["probe_sm_mhz"] = mhz
+    except Exception as e:  # noqa: BLE001
+        roof["probe_peak"] = f"unavailable: {e}"
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u32-bits/int32" if w.op != synth.BINARY_WEIGHTS else "f32",
+        "data": "synthetic (seeded N(0,1) inputs, Bernoulli weight bits)",
+        "config": {"workload": w.name, "batch_per_gpu": w.batch, "global_batch": w.batch * world,
+                   "in": [w.in_h, w.in_w, w.in_channels], "out_channels": w.out_channels,
+                   "kernel": [w.kernel_h, w.kernel_w], "stride": [w.stride_y, w.stride_x], "op": w.op,
+                   "beta": w.use_beta, "relu": w.relu, "input_terms": w.in_terms,
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"{ROTATE} rotating input/output sets, "
+                         f"{ROTATE * (inp.x.nbytes + int(np.prod(out_shape)) * 4) / 1e6:.0f} MB > 126 MB L2"},
+        "images_per_s": images_s,
+        "roofline": roof,
+        "clocks": clock_info,
+        "gpu_launches": layer.launches_per_forward() * args.steps,
+    }
+
+    # end to end through the C ABI with page-locked host buffers
+    if not args.no_e2e:
+        e2e_steps = max(3, min(args.steps, 20))
+        hin = torch.from_numpy(inp.x).pin_memory()
+        hout = torch.empty(out_shape, dtype=torch.float32).pin_memory()
+        fwd_host = bc.bfc_forward_host if w.kind == "fc" else bc.bconv_forward_host
+        for _ in range(2):
+            fwd_host(layer.handle, hin.data_ptr(), hout.data_ptr(), stream.cuda_stream)
+        barrier(device)
+        torch.cuda.synchronize(device)
+        t0 = time.perf_counter()
+        for _ in range(e2e_steps):
+            fwd_host(layer.handle, hin.data_ptr(), hout.data_ptr(), stream.cuda_stream)
+        t_e2e = time.perf_counter() - t0
+        t_e2e = max_over_ranks(t_e2e, device)
+        result["e2e"] = {"value": ops_step * e2e_steps * world / t_e2e / 1e12, "unit": UNIT,
+                         "h2d_bytes_per_step": int(hin.numel() * 4), "d2h_bytes_per_step": int(hout.numel() * 4),
+                         "steps": e2e_steps, "ms_per_step": t_e2e * 1e3 / e2e_steps,
+                         "api": "bfc_forward_host" if w.kind == "fc" else "bconv_forward_host"}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, dt, n, thr = oracle_sample_rate(w, inp, target_s=args.cpu_seconds)
+        result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": thr, "kind": "oracle",
+                                  "sample": f"{n} of {w.batch * w.out_h * w.out_w} output rows (all {w.out_channels} "
+                                            f"channels each), {dt:.1f} s"}
+    layer.close()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------------------
+# reference arm: the oracle, timed as it stands
+# ----------------------------------------------------------------------------------------
+def run_reference(args, w: synth.Workload):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    inp = synth.make_inputs(w)
+    total_steps = args.steps + args.warmup
+    per_step_s = min(10.0, args.reference_seconds / max(total_steps, 1))
+    rate, dt, n, thr = oracle_sample_rate(w, inp, target_s=per_step_s)  # calibrates the sample size
+    import oracle
+
+    otype = {synth.XNOR: oracle.ORACLE_XNOR, synth.AND: oracle.ORACLE_AND,
+             synth.BINARY_WEIGHTS: oracle.ORACLE_BINARY_WEIGHTS}[w.op]
+    rows_total = w.batch * w.out_h * w.out_w
+    ops_per_row = w.nominal_ops / rows_total
+    rng = np.random.default_rng(1)
+    kw = dict(type=otype, scale=inp.scale, bias=inp.bias, in_scale=inp.in_scale, in_bias=inp.in_bias,
+              use_beta=w.use_beta, relu=w.relu)
+
+    def step():
+        rows = np.sort(rng.choice(rows_total, size=n, replace=False)).astype(np.int64)
+        if w.kind == "fc":
+            oracle.fc(inp.x, inp.wbits, rows=rows, **kw)
+        else:
+            oracle.conv(inp.x, inp.wbits, stride=(w.stride_y, w.stride_x), pixels=rows, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    t = time.perf_counter() - t0
+    value = n * ops_per_row * args.steps / t / 1e12
+    result = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) inputs, Bernoulli weight bits)",
+        "config": {"workload": w.name, "batch_per_gpu": w.batch, "global_batch": w.batch * world,
+                   "parallelism": "rank 0 only (CPU oracle)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
+                         "sample": f"each step: {n} of {rows_total} output rows (all {w.out_channels} channels)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time of the cpu_baseline sample")
+    ap.add_argument("--reference-seconds", type=float, default=120.0, help="oracle time budget of --impl reference")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    key = int(args.workload) if args.workload.isdigit() else args.workload
+    w = synth.workload(key)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_native(args, w)
+
+
+if __name__ == "__main__":
+    main()

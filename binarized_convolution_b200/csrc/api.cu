@@ -1,0 +1,668 @@
+// C ABI of the binary convolution library: handles, validation, weight preparation and
+// the launch sequence of each forward.  The declarations and their contracts are in
+// include/bconv.h.
+//
+// A forward is, in stream order:
+//   XNOR / AND:       pack (x~, sign, bits [, A])  [-> beta]  -> POPC contraction + epilogue
+//   binaryWeights:    [pack (A only) -> beta ->]  FP32 contraction + epilogue (x~ fused)
+// Every buffer a forward touches besides the caller's input and output is allocated at
+// create time.
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "bconv.h"
+#include "common.cuh"
+
+namespace bconv {
+
+int current_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cache[dev] = sms;
+  return sms;
+}
+
+namespace {
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) {
+      ok = false;
+      return;
+    }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+// Device allocations owned by a handle, freed together.
+struct DevMem {
+  std::vector<void*> ptrs;
+  template <typename T>
+  cudaError_t alloc(T** p, size_t count) {
+    *p = nullptr;
+    if (count == 0) count = 1;
+    void* q = nullptr;
+    cudaError_t e = cudaMalloc(&q, count * sizeof(T));
+    if (e != cudaSuccess) return e;
+    ptrs.push_back(q);
+    *p = static_cast<T*>(q);
+    return cudaSuccess;
+  }
+  void release() {
+    for (void* p : ptrs) cudaFree(p);
+    ptrs.clear();
+  }
+};
+
+struct Profile {
+  std::vector<cudaEvent_t> start, stop;
+  int used = 0;
+  bool active = false;
+  void clear() {
+    for (auto e : start) cudaEventDestroy(e);
+    for (auto e : stop) cudaEventDestroy(e);
+    start.clear();
+    stop.clear();
+    used = 0;
+    active = false;
+  }
+};
+
+bconv_status_t from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return BCONV_OK;
+  if (e == cudaErrorMemoryAllocation) return BCONV_ERR_OOM;
+  if (e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver) return BCONV_ERR_NO_DEVICE;
+  return BCONV_ERR_CUDA;
+}
+
+// Everything both handle kinds share: parameters on the device, workspace, settings.
+struct Layer {
+  int device = 0;
+  int type = kXnor;
+  uint32_t flags = 0;
+  int relu = 0;
+  int algo = BCONV_ALGO_AUTO;
+  // geometry of the contraction
+  int N = 0, H = 0, W = 0, Ni = 0, No = 0, kh = 1, kw = 1, sy = 1, sx = 1, Ho = 1, Wo = 1;
+  bool fc = false;
+  int nw = 0, nw_pad = 0, no_pad = 0;
+  // binaryWeights contraction view: per-pixel channels (conv) or the whole flattened image
+  // as the channels of one pixel (FC), padded to whole pipeline steps
+  int bw_ni = 0, bw_ni_pad = 0;
+  float *bw_in_scale = nullptr, *bw_in_bias = nullptr;
+  // device parameters
+  float *scale = nullptr, *bias = nullptr, *in_scale = nullptr, *in_bias = nullptr;
+  uint32_t* wt = nullptr;  // POPC weights
+  int32_t* wpop = nullptr;
+  float* wf = nullptr;     // binaryWeights weights
+  // workspace
+  uint32_t* bits = nullptr;
+  float *A = nullptr, *beta = nullptr;
+  uint32_t* err = nullptr;
+  // host-buffer forward staging (allocated on first use)
+  float *stage_in = nullptr, *stage_out = nullptr;
+  DevMem mem;
+  Profile prof;
+
+  int64_t in_elems() const { return static_cast<int64_t>(N) * H * W * Ni; }
+  int64_t out_elems() const { return static_cast<int64_t>(N) * Ho * Wo * No; }
+  bool use_beta() const { return (flags & BCONV_FLAG_USE_BETA_SCALING) != 0; }
+};
+
+struct HandleBase {
+  uint32_t magic;
+  Layer L;
+};
+constexpr uint32_t kConvMagic = 0xBC0A7001u;
+constexpr uint32_t kFcMagic = 0xBC0A7002u;
+
+}  // namespace
+}  // namespace bconv
+
+struct bconv_handle_s : bconv::HandleBase {};
+struct bfc_handle_s : bconv::HandleBase {};
+
+namespace bconv {
+namespace {
+
+bool valid_type(int t) { return t == kBinaryWeights || t == kXnor || t == kAnd; }
+
+// Copy the parameter arrays (expanding defaults) and prepare the weights for the
+// contraction kernel of this layer type.
+bconv_status_t upload_params(Layer& L, const uint32_t* packed, const float* scale, const float* bias,
+                             const float* in_scale, const float* in_bias, float scale_value) {
+  const int taps = L.kh * L.kw;
+  std::vector<float> hs(L.No), hb(L.No, 0.f);
+  for (int c = 0; c < L.No; ++c) hs[c] = scale ? scale[c] : scale_value;
+  if (bias) memcpy(hb.data(), bias, sizeof(float) * L.No);
+  cudaError_t e = L.mem.alloc(&L.scale, L.No);
+  if (e == cudaSuccess) e = L.mem.alloc(&L.bias, L.No);
+  if (e == cudaSuccess) e = cudaMemcpy(L.scale, hs.data(), sizeof(float) * L.No, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(L.bias, hb.data(), sizeof(float) * L.No, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return from_cuda(e);
+  if (in_scale || in_bias) {  // both arrays exist on the device once either is given
+    std::vector<float> is(L.Ni, 1.f), ib(L.Ni, 0.f);
+    if (in_scale) memcpy(is.data(), in_scale, sizeof(float) * L.Ni);
+    if (in_bias) memcpy(ib.data(), in_bias, sizeof(float) * L.Ni);
+    e = L.mem.alloc(&L.in_scale, L.Ni);
+    if (e == cudaSuccess) e = L.mem.alloc(&L.in_bias, L.Ni);
+    if (e == cudaSuccess) e = cudaMemcpy(L.in_scale, is.data(), sizeof(float) * L.Ni, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(L.in_bias, ib.data(), sizeof(float) * L.Ni, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+
+  // Host weights: [No][taps][nw] LSB-first words.  Bits at or beyond Ni are cleared.
+  const int tail = L.Ni % kWordBits;
+  const uint32_t last_mask = tail ? ((1u << tail) - 1u) : 0xffffffffu;
+  auto wword = [&](int c, int t, int w) -> uint32_t {
+    uint32_t v = packed[(static_cast<int64_t>(c) * taps + t) * L.nw + w];
+    return w == L.nw - 1 ? (v & last_mask) : v;
+  };
+
+  if (L.type == kBinaryWeights) {
+    // [bw_ni_pad][no_pad] of +-1.0f, zero for padding rows and columns.  Row index
+    // t*ni_pad + f for a convolution; t*Ni + f (the flattened image) for the FC.
+    std::vector<float> hw(static_cast<size_t>(L.fc ? 1 : taps) * L.bw_ni_pad * L.no_pad, 0.f);
+    for (int c = 0; c < L.No; ++c)
+      for (int t = 0; t < taps; ++t)
+        for (int f = 0; f < L.Ni; ++f) {
+          const uint32_t bit = (wword(c, t, f / kWordBits) >> (f % kWordBits)) & 1u;
+          const int64_t row = L.fc ? static_cast<int64_t>(t) * L.Ni + f : static_cast<int64_t>(t) * L.bw_ni_pad + f;
+          hw[row * L.no_pad + c] = bit ? 1.f : -1.f;
+        }
+    e = L.mem.alloc(&L.wf, hw.size());
+    if (e == cudaSuccess) e = cudaMemcpy(L.wf, hw.data(), hw.size() * sizeof(float), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && L.fc && L.in_scale) {  // terms repeated over the flattened image
+      std::vector<float> is(static_cast<size_t>(L.bw_ni)), ib(static_cast<size_t>(L.bw_ni));
+      std::vector<float> s1(L.Ni, 1.f), b0(L.Ni, 0.f);
+      if (in_scale) memcpy(s1.data(), in_scale, sizeof(float) * L.Ni);
+      if (in_bias) memcpy(b0.data(), in_bias, sizeof(float) * L.Ni);
+      for (int64_t k = 0; k < L.bw_ni; ++k) {
+        is[k] = s1[k % L.Ni];
+        ib[k] = b0[k % L.Ni];
+      }
+      e = L.mem.alloc(&L.bw_in_scale, is.size());
+      if (e == cudaSuccess) e = L.mem.alloc(&L.bw_in_bias, ib.size());
+      if (e == cudaSuccess) e = cudaMemcpy(L.bw_in_scale, is.data(), is.size() * sizeof(float), cudaMemcpyHostToDevice);
+      if (e == cudaSuccess) e = cudaMemcpy(L.bw_in_bias, ib.data(), ib.size() * sizeof(float), cudaMemcpyHostToDevice);
+    } else {
+      L.bw_in_scale = L.in_scale;
+      L.bw_in_bias = L.in_bias;
+    }
+    return from_cuda(e);
+  }
+
+  // POPC weights: reduction-major [taps*nw_pad][no_pad], zero padding; per-tap popcounts.
+  const int64_t K = static_cast<int64_t>(taps) * L.nw_pad;
+  std::vector<uint32_t> hw(static_cast<size_t>(K) * L.no_pad, 0u);
+  std::vector<int32_t> hp(static_cast<size_t>(L.No) * taps, 0);
+  for (int c = 0; c < L.No; ++c)
+    for (int t = 0; t < taps; ++t) {
+      int32_t pc = 0;
+      for (int w = 0; w < L.nw; ++w) {
+        const uint32_t v = wword(c, t, w);
+        hw[(static_cast<int64_t>(t) * L.nw_pad + w) * L.no_pad + c] = v;
+        pc += __builtin_popcount(v);
+      }
+      hp[static_cast<size_t>(c) * taps + t] = pc;
+    }
+  e = L.mem.alloc(&L.wt, hw.size());
+  if (e == cudaSuccess) e = L.mem.alloc(&L.wpop, hp.size());
+  if (e == cudaSuccess) e = cudaMemcpy(L.wt, hw.data(), hw.size() * sizeof(uint32_t), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(L.wpop, hp.data(), hp.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+  return from_cuda(e);
+}
+
+bconv_status_t alloc_workspace(Layer& L) {
+  const int64_t npix = static_cast<int64_t>(L.N) * L.H * L.W;
+  cudaError_t e = L.mem.alloc(&L.err, 1);
+  if (e == cudaSuccess) e = cudaMemset(L.err, 0, sizeof(uint32_t));
+  if (e == cudaSuccess && L.type != kBinaryWeights) e = L.mem.alloc(&L.bits, npix * L.nw_pad);
+  if (e == cudaSuccess && L.use_beta()) e = L.mem.alloc(&L.A, npix);
+  if (e == cudaSuccess && L.use_beta()) e = L.mem.alloc(&L.beta, static_cast<int64_t>(L.N) * L.Ho * L.Wo);
+  return from_cuda(e);
+}
+
+bconv_status_t finish_create(Layer& L, const uint32_t* packed, const float* scale, const float* bias,
+                             const float* in_scale, const float* in_bias, float scale_value) {
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+    cudaGetLastError();
+    return BCONV_ERR_NO_DEVICE;
+  }
+  if (cudaGetDevice(&L.device) != cudaSuccess) return BCONV_ERR_CUDA;
+  L.nw = words_for(L.Ni);
+  L.nw_pad = round_up(L.nw, kWordPad);
+  L.bw_ni = L.fc ? L.H * L.W * L.Ni : L.Ni;
+  L.bw_ni_pad = round_up(L.bw_ni, kBwChanPad);
+  L.no_pad = round_up(L.No, kTileN);
+  bconv_status_t st = upload_params(L, packed, scale, bias, in_scale, in_bias, scale_value);
+  if (st == BCONV_OK) st = alloc_workspace(L);
+  if (st != BCONV_OK) L.mem.release();
+  return st;
+}
+
+// The launch sequence of one forward.
+bconv_status_t run_forward(Layer& L, const float* in, float* out, cudaStream_t s) {
+  const int64_t npix = static_cast<int64_t>(L.N) * L.H * L.W;
+  if (L.N == 0) return BCONV_OK;
+  cudaError_t e = cudaSuccess;
+  const bool beta = L.use_beta();
+
+  // 1. input transform + sign + pack (+ A)
+  if (L.type != kBinaryWeights || beta) {
+    PackArgs p{};
+    p.in = in;
+    p.npix = npix;
+    p.ni = L.Ni;
+    p.nw_pad = L.nw_pad;
+    p.in_scale = L.in_scale;
+    p.in_bias = L.in_bias;
+    p.bits = L.type != kBinaryWeights ? L.bits : nullptr;
+    p.A = beta ? L.A : nullptr;
+    e = launch_pack(p, s);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  // 2. beta
+  if (beta) {
+    BetaArgs b{L.A, L.beta, L.N, L.H, L.W, L.Ho, L.Wo, L.kh, L.kw, L.sy, L.sx};
+    e = L.fc ? launch_beta_image_mean(b, s) : launch_beta_conv(b, s);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  // 3. contraction + epilogue (timed when profiling)
+  const bool timed = L.prof.active && L.prof.used < static_cast<int>(L.prof.start.size());
+  if (timed) cudaEventRecord(L.prof.start[L.prof.used], s);
+  if (L.type == kBinaryWeights) {
+    BwArgs b{};
+    b.in = in;
+    b.in_scale = L.bw_in_scale;
+    b.in_bias = L.bw_in_bias;
+    b.wf = L.wf;
+    b.scale = L.scale;
+    b.bias = L.bias;
+    b.beta = beta ? L.beta : nullptr;
+    b.out = out;
+    b.ni = L.bw_ni; b.ni_pad = L.bw_ni_pad; b.no = L.No; b.no_pad = L.no_pad;
+    b.relu = L.relu;
+    b.vec_out = (L.No % 4 == 0) && (reinterpret_cast<uintptr_t>(out) & 15) == 0;
+    if (L.fc) {  // one "pixel" per image whose channels are the flattened image, one tap
+      b.N = L.N; b.H = 1; b.W = 1; b.Ho = 1; b.Wo = 1; b.kh = 1; b.kw = 1; b.sy = 1; b.sx = 1;
+    } else {
+      b.N = L.N; b.H = L.H; b.W = L.W; b.Ho = L.Ho; b.Wo = L.Wo;
+      b.kh = L.kh; b.kw = L.kw; b.sy = L.sy; b.sx = L.sx;
+    }
+    e = launch_bw_conv(b, s);
+  } else {
+    PopcArgs p{};
+    p.bits = L.bits;
+    p.wt = L.wt;
+    p.wpop = L.wpop;
+    p.scale = L.scale;
+    p.bias = L.bias;
+    p.beta = beta ? L.beta : nullptr;
+    p.out = out;
+    p.no = L.No;
+    p.no_pad = L.no_pad;
+    p.op = L.type;
+    p.relu = L.relu;
+    p.vec_out = (L.No % 4 == 0) && (reinterpret_cast<uintptr_t>(out) & 15) == 0;
+    if (L.fc) {  // one "pixel" per image holding all H*W*nw_pad words, one tap
+      p.N = L.N; p.H = 1; p.W = 1; p.Ho = 1; p.Wo = 1; p.kh = 1; p.kw = 1; p.sy = 1; p.sx = 1;
+      p.nw = L.H * L.W * L.nw_pad;
+      p.nbits = L.H * L.W * L.Ni;
+    } else {
+      p.N = L.N; p.H = L.H; p.W = L.W; p.Ho = L.Ho; p.Wo = L.Wo;
+      p.kh = L.kh; p.kw = L.kw; p.sy = L.sy; p.sx = L.sx;
+      p.nw = L.nw_pad;
+      p.nbits = L.Ni;
+    }
+    const int64_t m_tiles = ceil_div(static_cast<int64_t>(p.N) * p.Ho * p.Wo, 128);
+    const int ksteps = p.kh * p.kw * (p.nw / kWordPad);
+    p.split_k = popc_split_k_for(m_tiles, p.no_pad / kTileN, ksteps, current_sm_count());
+    e = launch_popc_gemm(p, s);
+  }
+  if (timed) cudaEventRecord(L.prof.stop[L.prof.used++], s);
+  return from_cuda(e);
+}
+
+bconv_status_t forward_host(Layer& L, const float* hin, float* hout, cudaStream_t s) {
+  if (!hin || !hout) return BCONV_ERR_INVALID_ARG;
+  cudaError_t e = cudaSuccess;
+  if (!L.stage_in) e = L.mem.alloc(&L.stage_in, L.in_elems());
+  if (e == cudaSuccess && !L.stage_out) e = L.mem.alloc(&L.stage_out, L.out_elems());
+  if (e != cudaSuccess) return from_cuda(e);
+  e = cudaMemcpyAsync(L.stage_in, hin, L.in_elems() * sizeof(float), cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return from_cuda(e);
+  bconv_status_t st = run_forward(L, L.stage_in, L.stage_out, s);
+  if (st != BCONV_OK) return st;
+  e = cudaMemcpyAsync(hout, L.stage_out, L.out_elems() * sizeof(float), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return from_cuda(e);
+}
+
+bconv_status_t sync_status(Layer& L, cudaStream_t s) {
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return from_cuda(e);
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, L.err, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return from_cuda(e);
+  if (word) {
+    cudaMemset(L.err, 0, sizeof(uint32_t));
+    if (word & kErrTimeout) return BCONV_ERR_TIMEOUT;
+    return BCONV_ERR_CUDA;
+  }
+  return BCONV_OK;
+}
+
+bconv_status_t set_algo(Layer& L, int algo) {
+  if (algo == BCONV_ALGO_AUTO) {
+    L.algo = algo;
+    return BCONV_OK;
+  }
+  if (algo == BCONV_ALGO_POPC && (L.type == kXnor || L.type == kAnd)) {
+    L.algo = algo;
+    return BCONV_OK;
+  }
+  if (algo == BCONV_ALGO_SIMT_F32 && L.type == kBinaryWeights) {
+    L.algo = algo;
+    return BCONV_OK;
+  }
+  if (algo < 0 || algo > BCONV_ALGO_SIMT_F32) return BCONV_ERR_INVALID_ARG;
+  return BCONV_ERR_UNSUPPORTED;
+}
+
+int launches_per_forward(const Layer& L) {
+  int n = 1;  // contraction
+  if (L.type != kBinaryWeights || L.use_beta()) n += 1;  // pack
+  if (L.use_beta()) n += 1;                              // beta
+  return n;
+}
+
+bconv_status_t profile_begin(Layer& L, int32_t n) {
+  if (n <= 0 || n > (1 << 20)) return BCONV_ERR_INVALID_ARG;
+  L.prof.clear();
+  for (int i = 0; i < n; ++i) {
+    cudaEvent_t a, b;
+    if (cudaEventCreate(&a) != cudaSuccess) return BCONV_ERR_CUDA;
+    if (cudaEventCreate(&b) != cudaSuccess) {
+      cudaEventDestroy(a);
+      return BCONV_ERR_CUDA;
+    }
+    L.prof.start.push_back(a);
+    L.prof.stop.push_back(b);
+  }
+  L.prof.active = true;
+  return BCONV_OK;
+}
+
+bconv_status_t profile_end(Layer& L, float* total_ms, int32_t* launches) {
+  float total = 0.f;
+  for (int i = 0; i < L.prof.used; ++i) {
+    if (cudaEventSynchronize(L.prof.stop[i]) != cudaSuccess) return BCONV_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, L.prof.start[i], L.prof.stop[i]) != cudaSuccess) return BCONV_ERR_CUDA;
+    total += ms;
+  }
+  if (total_ms) *total_ms = total;
+  if (launches) *launches = L.prof.used;
+  L.prof.clear();
+  return BCONV_OK;
+}
+
+void destroy(Layer& L) {
+  DeviceGuard g(L.device);
+  L.prof.clear();
+  L.mem.release();
+}
+
+template <typename H>
+H* checked(H* h, uint32_t magic) {
+  return (h && h->magic == magic) ? h : nullptr;
+}
+
+}  // namespace
+}  // namespace bconv
+
+using namespace bconv;
+
+extern "C" {
+
+bconv_status_t bconv_create(const bconv_desc_t* d, const uint32_t* packed_weights, const float* scale,
+                            const float* bias, const float* in_scale, const float* in_bias, bconv_type_t type,
+                            uint32_t flags, bconv_handle_t* out) {
+  if (!out) return BCONV_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!d || !packed_weights) return BCONV_ERR_INVALID_ARG;
+  if (!valid_type(type) || (flags & ~static_cast<uint32_t>(BCONV_FLAG_USE_BETA_SCALING))) return BCONV_ERR_INVALID_ARG;
+  if (d->neuron != BCONV_NEURON_NONE && d->neuron != BCONV_NEURON_RELU) return BCONV_ERR_INVALID_ARG;
+  if (d->batch < 0 || d->in_h <= 0 || d->in_w <= 0 || d->in_channels <= 0 || d->out_channels <= 0 ||
+      d->kernel_h <= 0 || d->kernel_w <= 0 || d->stride_y <= 0 || d->stride_x <= 0 || d->groups <= 0)
+    return BCONV_ERR_INVALID_ARG;
+  if (d->groups != 1) return BCONV_ERR_UNSUPPORTED;
+  if (d->kernel_h > d->in_h * 2 + 1 || d->kernel_w > d->in_w * 2 + 1 || d->kernel_h * d->kernel_w > 4096 ||
+      d->in_channels > (1 << 20) || d->out_channels > (1 << 20))
+    return BCONV_ERR_UNSUPPORTED;
+  bconv_handle_s* h = new (std::nothrow) bconv_handle_s();
+  if (!h) return BCONV_ERR_OOM;
+  h->magic = kConvMagic;
+  Layer& L = h->L;
+  L.type = type;
+  L.flags = flags;
+  L.relu = d->neuron == BCONV_NEURON_RELU;
+  L.N = d->batch; L.H = d->in_h; L.W = d->in_w; L.Ni = d->in_channels; L.No = d->out_channels;
+  L.kh = d->kernel_h; L.kw = d->kernel_w; L.sy = d->stride_y; L.sx = d->stride_x;
+  L.Ho = (L.H + L.sy - 1) / L.sy;
+  L.Wo = (L.W + L.sx - 1) / L.sx;
+  const bconv_status_t st = finish_create(L, packed_weights, scale, bias, in_scale, in_bias, d->scale_value);
+  if (st != BCONV_OK) {
+    h->magic = 0;
+    delete h;
+    return st;
+  }
+  *out = h;
+  return BCONV_OK;
+}
+
+bconv_status_t bconv_forward(bconv_handle_t h, const float* in, float* out, struct CUstream_st* stream) {
+  if (!checked(h, kConvMagic) || (h->L.N > 0 && (!in || !out))) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  if (!g.ok) return BCONV_ERR_CUDA;
+  return run_forward(h->L, in, out, stream);
+}
+
+bconv_status_t bconv_forward_host(bconv_handle_t h, const float* host_in, float* host_out,
+                                  struct CUstream_st* stream) {
+  if (!checked(h, kConvMagic)) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  if (!g.ok) return BCONV_ERR_CUDA;
+  return forward_host(h->L, host_in, host_out, stream);
+}
+
+bconv_status_t bconv_get_output_dims(bconv_handle_t h, int32_t* n, int32_t* ho, int32_t* wo, int32_t* c) {
+  if (!checked(h, kConvMagic)) return BCONV_ERR_INVALID_ARG;
+  if (n) *n = h->L.N;
+  if (ho) *ho = h->L.Ho;
+  if (wo) *wo = h->L.Wo;
+  if (c) *c = h->L.No;
+  return BCONV_OK;
+}
+
+int32_t bconv_input_feature_channels(bconv_handle_t h) { return checked(h, kConvMagic) ? h->L.Ni : -1; }
+int32_t bconv_output_feature_channels(bconv_handle_t h) { return checked(h, kConvMagic) ? h->L.No : -1; }
+
+bconv_status_t bconv_set_algo(bconv_handle_t h, bconv_algo_t algo) {
+  if (!checked(h, kConvMagic)) return BCONV_ERR_INVALID_ARG;
+  return set_algo(h->L, algo);
+}
+
+int32_t bconv_launches_per_forward(bconv_handle_t h) {
+  return checked(h, kConvMagic) ? launches_per_forward(h->L) : -1;
+}
+
+bconv_status_t bconv_sync_status(bconv_handle_t h, struct CUstream_st* stream) {
+  if (!checked(h, kConvMagic)) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  return sync_status(h->L, stream);
+}
+
+bconv_status_t bconv_profile_begin(bconv_handle_t h, int32_t max_launches) {
+  if (!checked(h, kConvMagic)) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  return profile_begin(h->L, max_launches);
+}
+
+bconv_status_t bconv_profile_end(bconv_handle_t h, float* total_ms, int32_t* launches) {
+  if (!checked(h, kConvMagic)) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  return profile_end(h->L, total_ms, launches);
+}
+
+bconv_status_t bconv_destroy(bconv_handle_t h) {
+  if (!h) return BCONV_OK;
+  if (!checked(h, kConvMagic)) return BCONV_ERR_INVALID_ARG;
+  destroy(h->L);
+  h->magic = 0;
+  delete h;
+  return BCONV_OK;
+}
+
+bconv_status_t bfc_create(const bfc_desc_t* d, const uint32_t* packed_weights, const float* scale,
+                          const float* bias, const float* in_scale, const float* in_bias, bconv_type_t type,
+                          uint32_t flags, bfc_handle_t* out) {
+  if (!out) return BCONV_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!d || !packed_weights) return BCONV_ERR_INVALID_ARG;
+  if (!valid_type(type) || (flags & ~static_cast<uint32_t>(BCONV_FLAG_USE_BETA_SCALING))) return BCONV_ERR_INVALID_ARG;
+  if (d->neuron != BCONV_NEURON_NONE && d->neuron != BCONV_NEURON_RELU) return BCONV_ERR_INVALID_ARG;
+  if (d->batch < 0 || d->in_h <= 0 || d->in_w <= 0 || d->in_channels <= 0 || d->out_channels <= 0 ||
+      d->groups <= 0)
+    return BCONV_ERR_INVALID_ARG;
+  if (d->stride_y != 1 || d->stride_x != 1) return BCONV_ERR_INVALID_ARG;
+  if (d->groups != 1) return BCONV_ERR_UNSUPPORTED;
+  const int64_t k_bits = static_cast<int64_t>(d->in_h) * d->in_w * d->in_channels;
+  if (k_bits > (1 << 26) || d->out_channels > (1 << 20)) return BCONV_ERR_UNSUPPORTED;
+  bfc_handle_s* h = new (std::nothrow) bfc_handle_s();
+  if (!h) return BCONV_ERR_OOM;
+  h->magic = kFcMagic;
+  Layer& L = h->L;
+  L.fc = true;
+  L.type = type;
+  L.flags = flags;
+  L.relu = d->neuron == BCONV_NEURON_RELU;
+  L.N = d->batch; L.H = d->in_h; L.W = d->in_w; L.Ni = d->in_channels; L.No = d->out_channels;
+  L.kh = d->in_h; L.kw = d->in_w; L.sy = 1; L.sx = 1;
+  L.Ho = 1;
+  L.Wo = 1;
+  const bconv_status_t st = finish_create(L, packed_weights, scale, bias, in_scale, in_bias, d->scale_value);
+  if (st != BCONV_OK) {
+    h->magic = 0;
+    delete h;
+    return st;
+  }
+  *out = h;
+  return BCONV_OK;
+}
+
+bconv_status_t bfc_forward(bfc_handle_t h, const float* in, float* out, struct CUstream_st* stream) {
+  if (!checked(h, kFcMagic) || (h->L.N > 0 && (!in || !out))) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  if (!g.ok) return BCONV_ERR_CUDA;
+  return run_forward(h->L, in, out, stream);
+}
+
+bconv_status_t bfc_forward_host(bfc_handle_t h, const float* host_in, float* host_out, struct CUstream_st* stream) {
+  if (!checked(h, kFcMagic)) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  if (!g.ok) return BCONV_ERR_CUDA;
+  return forward_host(h->L, host_in, host_out, stream);
+}
+
+int32_t bfc_input_feature_channels(bfc_handle_t h) { return checked(h, kFcMagic) ? h->L.Ni : -1; }
+int32_t bfc_output_feature_channels(bfc_handle_t h) { return checked(h, kFcMagic) ? h->L.No : -1; }
+
+bconv_status_t bfc_set_algo(bfc_handle_t h, bconv_algo_t algo) {
+  if (!checked(h, kFcMagic)) return BCONV_ERR_INVALID_ARG;
+  return set_algo(h->L, algo);
+}
+
+int32_t bfc_launches_per_forward(bfc_handle_t h) { return checked(h, kFcMagic) ? launches_per_forward(h->L) : -1; }
+
+bconv_status_t bfc_sync_status(bfc_handle_t h, struct CUstream_st* stream) {
+  if (!checked(h, kFcMagic)) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  return sync_status(h->L, stream);
+}
+
+bconv_status_t bfc_profile_begin(bfc_handle_t h, int32_t max_launches) {
+  if (!checked(h, kFcMagic)) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  return profile_begin(h->L, max_launches);
+}
+
+bconv_status_t bfc_profile_end(bfc_handle_t h, float* total_ms, int32_t* launches) {
+  if (!checked(h, kFcMagic)) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  return profile_end(h->L, total_ms, launches);
+}
+
+bconv_status_t bfc_destroy(bfc_handle_t h) {
+  if (!h) return BCONV_OK;
+  if (!checked(h, kFcMagic)) return BCONV_ERR_INVALID_ARG;
+  destroy(h->L);
+  h->magic = 0;
+  delete h;
+  return BCONV_OK;
+}
+
+const char* bconv_status_string(bconv_status_t s) {
+  switch (s) {
+    case BCONV_OK: return "ok";
+    case BCONV_ERR_INVALID_ARG: return "invalid argument";
+    case BCONV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case BCONV_ERR_CUDA: return "CUDA error";
+    case BCONV_ERR_OOM: return "out of device memory";
+    case BCONV_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    case BCONV_ERR_NO_DEVICE: return "no CUDA device";
+  }
+  return "unknown status";
+}
+
+bconv_status_t bconv_pack_bits(const uint8_t* bits, int64_t rows, int32_t nbits, uint32_t* out) {
+  if (!bits || !out || rows < 0 || nbits <= 0) return BCONV_ERR_INVALID_ARG;
+  const int nw = words_for(nbits);
+  for (int64_t r = 0; r < rows; ++r) {
+    const uint8_t* src = bits + r * nbits;
+    uint32_t* dst = out + r * nw;
+    for (int w = 0; w < nw; ++w) dst[w] = 0u;
+    for (int f = 0; f < nbits; ++f)
+      if (src[f]) dst[f / kWordBits] |= 1u << (f % kWordBits);
+  }
+  return BCONV_OK;
+}
+
+int32_t bconv_version(void) { return 100; }
+
+bconv_status_t bconv_measure_peak(int32_t kind, double* ops_per_s, double* sm_mhz) {
+  if (kind < 0 || kind > 2 || !ops_per_s) return BCONV_ERR_INVALID_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+    cudaGetLastError();
+    return BCONV_ERR_NO_DEVICE;
+  }
+  return from_cuda(probe_peak(kind, ops_per_s, sm_mhz));
+}
+
+}  // extern "C"

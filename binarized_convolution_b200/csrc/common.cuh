@@ -1,0 +1,104 @@
+// Internal declarations shared by the library's translation units (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace bconv {
+
+enum Op : int { kBinaryWeights = 0, kXnor = 1, kAnd = 2 };
+
+// Error word bits the kernels may set (read by *_sync_status).
+enum : uint32_t { kErrTimeout = 1u };
+
+constexpr int kWordBits = 32;
+// Words per pixel are padded to this many (32 bytes) so that a pixel's words start on a
+// 16-byte boundary and every pipeline stage of the POPC contraction reads whole chunks.
+constexpr int kWordPad = 8;
+
+inline int words_for(int bits) { return (bits + kWordBits - 1) / kWordBits; }
+inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Multiprocessor count of the current device (cached per device).
+int current_sm_count();
+
+// ------------------------------------------------------------------------------------
+// Input transform, sign and pack (one pass over the fp32 input).
+// ------------------------------------------------------------------------------------
+struct PackArgs {
+  const float* in;        // [npix][ni] fp32
+  int64_t npix;
+  int ni;
+  int nw_pad;             // words written per pixel (>= ceil(ni/32), multiple of kWordPad)
+  const float* in_scale;  // [ni] or nullptr
+  const float* in_bias;   // [ni] or nullptr
+  uint32_t* bits;         // [npix][nw_pad] or nullptr (A only)
+  float* A;               // [npix] or nullptr (no beta)
+};
+cudaError_t launch_pack(const PackArgs& a, cudaStream_t s);
+
+// ------------------------------------------------------------------------------------
+// Beta: box filter of A over the window (conv) or mean of A over the image (FC).
+// ------------------------------------------------------------------------------------
+struct BetaArgs {
+  const float* A;  // [N][H][W]
+  float* beta;     // [N][Ho][Wo] (conv) or [N] (FC)
+  int N, H, W, Ho, Wo, kh, kw, sy, sx;
+};
+cudaError_t launch_beta_conv(const BetaArgs& a, cudaStream_t s);
+cudaError_t launch_beta_image_mean(const BetaArgs& a, cudaStream_t s);
+
+// ------------------------------------------------------------------------------------
+// POPC implicit-GEMM contraction with the fused epilogue (XNOR / AND).
+// Geometry of the convolution as a GEMM: rows = output pixels, columns = output
+// channels, reduction = taps x words.  The FC case is a 1x1 "convolution" whose single
+// pixel per image holds all H*W*nw words.
+// ------------------------------------------------------------------------------------
+struct PopcArgs {
+  const uint32_t* bits;   // [N][H][W][nw] packed input bits
+  const uint32_t* wt;     // [kh*kw*nw][no_pad] packed weights, reduction-major
+  const int32_t* wpop;    // [no][kh*kw] weight popcount per tap (XNOR border correction)
+  const float* scale;     // [no]
+  const float* bias;      // [no]
+  const float* beta;      // [N*Ho*Wo] or nullptr
+  float* out;             // [N*Ho*Wo][no]
+  int N, H, W, Ho, Wo, kh, kw, sy, sx;
+  int nw;                 // words per pixel (multiple of kWordPad)
+  int nbits;              // real bits per tap (Ni, or H*W*Ni for the FC)
+  int no, no_pad;
+  int op;                 // kXnor or kAnd
+  int relu;
+  int split_k;            // 1, or CTAs of a cluster sharing one output tile
+  int vec_out;            // out is 16-byte aligned and no % 4 == 0: float4 stores
+};
+cudaError_t launch_popc_gemm(const PopcArgs& a, cudaStream_t s);
+int popc_split_k_for(int64_t m_tiles, int64_t n_tiles, int ksteps, int sm_count);
+
+// ------------------------------------------------------------------------------------
+// binaryWeights: FP32 signed-add contraction with the transform fused into the loads.
+// ------------------------------------------------------------------------------------
+struct BwArgs {
+  const float* in;        // [N][H][W][ni] raw input
+  const float* in_scale;  // [ni] or nullptr
+  const float* in_bias;   // [ni] or nullptr
+  const float* wf;        // [kh*kw*ni_pad][no_pad] weights as +-1.0f (0 in padding)
+  const float* scale;     // [no]
+  const float* bias;      // [no]
+  const float* beta;      // [N*Ho*Wo] or nullptr
+  float* out;             // [N*Ho*Wo][no]
+  int N, H, W, Ho, Wo, kh, kw, sy, sx;
+  int ni, ni_pad, no, no_pad;
+  int relu;
+  int vec_out;            // out is 16-byte aligned and no % 4 == 0: float4 stores
+};
+cudaError_t launch_bw_conv(const BwArgs& a, cudaStream_t s);
+constexpr int kBwChanPad = 32;  // channels per pipeline stage of the FP32 kernel
+constexpr int kTileN = 128;     // output channels per CTA tile (both contraction kernels)
+
+// ------------------------------------------------------------------------------------
+// Peak probes.
+// ------------------------------------------------------------------------------------
+cudaError_t probe_peak(int kind, double* ops_per_s, double* sm_mhz);
+
+}  // namespace bconv

@@ -1,0 +1,96 @@
+// Input transform + sign + bit-pack + channel mean |x~|, in one pass over the fp32 input.
+//
+// Follows the Apple page "MPSCNNBinaryConvolution", Overview: the input is pre-offset and
+// scaled by inputScaleTerms / inputBiasTerms before binarization and before the beta image
+// ("The scaling of input values happens before possible beta-image computation"), is
+// binarized by bin(x) = x < 0 ? -1 : 1 (bit 1 <-> +1), and A[i,x,y] = sum_c |in| / Nc feeds
+// beta.  x~ is one fused multiply-add, so its sign is the sign of the exact affine value.
+//
+// Layout: one warp per pixel.  Lane l takes channel 32*w + l of word w, so a warp load is
+// one coalesced 128-byte line and __ballot_sync assembles the word in channel order
+// (LSB = lowest channel).  Eight words are loaded before any is used so that each warp
+// keeps a kilobyte in flight; the kernel is bound by the fp32 read.
+#include "common.cuh"
+
+namespace bconv {
+namespace {
+
+constexpr int kPackThreads = 256;
+constexpr int kWordsInFlight = 8;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <bool kTerms, bool kBits, bool kA>
+__global__ void __launch_bounds__(kPackThreads) pack_kernel(PackArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kPackThreads) >> 5;
+  const int ni = a.ni;
+  const int nw = (ni + kWordBits - 1) / kWordBits;
+
+  for (int64_t p = warp; p < a.npix; p += nwarps) {
+    const float* row = a.in + p * ni;
+    uint32_t* brow = kBits ? a.bits + p * a.nw_pad : nullptr;
+    float asum = 0.f;
+    for (int w0 = 0; w0 < nw; w0 += kWordsInFlight) {
+      float x[kWordsInFlight];
+#pragma unroll
+      for (int j = 0; j < kWordsInFlight; ++j) {
+        const int f = (w0 + j) * kWordBits + lane;
+        x[j] = (f < ni) ? __ldcs(row + f) : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < kWordsInFlight; ++j) {
+        const int w = w0 + j;
+        if (w >= nw) break;  // warp-uniform
+        const int f = w * kWordBits + lane;
+        const bool valid = f < ni;
+        float xt = x[j];
+        if (kTerms && valid) xt = fmaf(xt, __ldg(a.in_scale + f), __ldg(a.in_bias + f));
+        if (kA) asum += valid ? fabsf(xt) : 0.f;
+        if (kBits) {
+          const uint32_t word = __ballot_sync(0xffffffffu, valid && !(xt < 0.f));
+          if (lane == 0) brow[w] = word;
+        }
+      }
+    }
+    if (kBits)
+      for (int w = nw + lane; w < a.nw_pad; w += 32) brow[w] = 0u;
+    if (kA) {
+      asum = warp_sum(asum);
+      if (lane == 0) a.A[p] = asum / static_cast<float>(ni);
+    }
+  }
+}
+
+template <bool kTerms>
+cudaError_t launch_pack_t(const PackArgs& a, cudaStream_t s) {
+  const int sms = current_sm_count();
+  const int64_t warps_per_block = kPackThreads / 32;
+  int64_t blocks = ceil_div(a.npix, warps_per_block);
+  const int64_t cap = static_cast<int64_t>(sms) * 8;  // 8 x 256 threads = 64 warps per SM
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  const dim3 grid(static_cast<unsigned>(blocks));
+  if (a.bits && a.A)
+    pack_kernel<kTerms, true, true><<<grid, kPackThreads, 0, s>>>(a);
+  else if (a.bits)
+    pack_kernel<kTerms, true, false><<<grid, kPackThreads, 0, s>>>(a);
+  else if (a.A)
+    pack_kernel<kTerms, false, true><<<grid, kPackThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const PackArgs& a, cudaStream_t s) {
+  if (a.npix == 0 || (!a.bits && !a.A)) return cudaSuccess;
+  if (a.in_scale) return launch_pack_t<true>(a, s);
+  return launch_pack_t<false>(a, s);
+}
+
+}  // namespace bconv

@@ -1,0 +1,227 @@
+/*
+ * bconv.h -- C ABI of the B200 binary convolution library (libbconv.so).
+ *
+ * The operation is the binary convolution of the Apple page "MPSCNNBinaryConvolution",
+ * Overview:
+ *
+ *     out[i,x,y,c] = act( (sum_{dx,dy,f} in[i,x+dx,y+dy,f] (op) B[c,dx,dy,f])
+ *                         * scale[c] * beta[i,x,y] + bias[c] )
+ *
+ * with three operators (the MPSCNNBinaryConvolutionType bullets): binaryWeights (input
+ * not binarized, weights [0,1] -> {-1,1}), XNOR (input binarized by bin(x) = x<0 ? -1 : 1,
+ * each 32-bit word contributes 32 - 2*popcount(x^y)) and AND (same binarization, each word
+ * contributes popcount(x&y)); optional input terms applied before binarization and before
+ * beta ("inputScaleTerms"/"inputBiasTerms"); and optional beta scaling (the beta and A
+ * formulas, enabled by the useBetaScaling flag).  The bfc_* entry points are the
+ * fully-connected special case of the page "MPSCNNFullyConnected" (kernel = source size,
+ * a 1x1xNo output).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are fp32, NHWC, contiguous.  in[n][y][x][f], out[n][oy][ox][c].
+ *   - Packed bits are LSB-first: channel f is bit (f % 32) of word (f / 32); each pixel
+ *     (or weight tap) holds ceil(Ni/32) words; bits at or beyond Ni are ignored.
+ *     Bit 1 means +1 (XNOR, binaryWeights) or 1 (AND).
+ *   - Pointers documented as "host" are read during the call only.  Pointers documented
+ *     as "device" must be device memory on the device the handle was created on, are
+ *     owned by the caller, and must stay valid until the work on `stream` completes.
+ *   - A stream argument is a cudaStream_t (NULL = the legacy default stream).
+ *   - Every call returns a status; nothing aborts the process.  Launch failures come back
+ *     from the call that launched; device-side failures (an error word the kernels set)
+ *     come back from *_sync_status.
+ *   - A handle's workspace is used by one stream at a time: forwards on one handle that
+ *     overlap on the GPU race.
+ */
+#ifndef BCONV_H_
+#define BCONV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* the type behind cudaStream_t */
+
+/* Status of a call. */
+typedef enum {
+  BCONV_OK = 0,
+  BCONV_ERR_INVALID_ARG = 1, /* NULL where a pointer is required, bad size, bad enum     */
+  BCONV_ERR_UNSUPPORTED = 2, /* a valid request this library does not do (groups > 1)  */
+  BCONV_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed            */
+  BCONV_ERR_OOM = 4,         /* device allocation failed                               */
+  BCONV_ERR_TIMEOUT = 5,     /* a kernel gave up a bounded wait and set the error word */
+  BCONV_ERR_NO_DEVICE = 6    /* no CUDA device is visible                              */
+} bconv_status_t;
+
+/* The convolution operator (MPSCNNBinaryConvolutionType). */
+typedef enum {
+  BCONV_TYPE_BINARY_WEIGHTS = 0,
+  BCONV_TYPE_XNOR = 1,
+  BCONV_TYPE_AND = 2
+} bconv_type_t;
+
+/* Flags (MPSCNNBinaryConvolutionFlags). */
+enum { BCONV_FLAG_NONE = 0u, BCONV_FLAG_USE_BETA_SCALING = 1u };
+
+/* The activation neuron applied last (the closing sentence of the Overview). */
+typedef enum { BCONV_NEURON_NONE = 0, BCONV_NEURON_RELU = 1 } bconv_neuron_t;
+
+/* Kernel family used for the contraction.  AUTO picks the fastest one this build has. */
+typedef enum {
+  BCONV_ALGO_AUTO = 0,
+  BCONV_ALGO_POPC = 1,     /* XNOR/AND: LOP3 XOR/AND + POPC into int32 registers     */
+  BCONV_ALGO_SIMT_F32 = 2  /* binaryWeights: FP32 signed-add contraction on the SIMT */
+} bconv_algo_t;
+
+/*
+ * Convolution descriptor.  Output extent: Ho = ceil(in_h/stride_y), Wo = ceil(in_w/stride_x);
+ * output (oy, ox) is centred on input (oy*stride_y, ox*stride_x) and its window covers rows
+ * dy in [-floor(kernel_h/2), floor((kernel_h-1)/2)] (columns likewise).  Taps outside the
+ * image contribute 0.  `groups` must be 1 (the Note on the MPSCNNBinaryConvolution page).
+ * `scale_value` is used for every output channel when no scale array is given (the
+ * init(device:convolutionData:scaleValue:type:flags:) form).
+ */
+typedef struct {
+  int32_t batch, in_h, in_w, in_channels, out_channels;
+  int32_t kernel_h, kernel_w, stride_y, stride_x, groups;
+  int32_t neuron; /* bconv_neuron_t */
+  float scale_value;
+} bconv_desc_t;
+
+typedef struct bconv_handle_s* bconv_handle_t;
+
+/*
+ * Create a convolution (MPSCNNBinaryConvolution initializer with outputBiasTerms,
+ * outputScaleTerms, inputBiasTerms, inputScaleTerms, type and flags).
+ *   desc            host; copied.
+ *   packed_weights  host uint32 [out_channels][kernel_h][kernel_w][ceil(in_channels/32)];
+ *                   required; copied to the device (bits beyond in_channels are cleared).
+ *   scale           host float [out_channels] or NULL (then desc->scale_value for all).
+ *   bias            host float [out_channels] or NULL (then 0).
+ *   in_scale        host float [in_channels] or NULL (then 1).
+ *   in_bias         host float [in_channels] or NULL (then 0).
+ *   flags           BCONV_FLAG_* bits; unknown bits are rejected.
+ *   out             host; receives the handle.
+ * Allocates on the current device every buffer the forward needs (weights, terms and
+ * workspace), so forwards never allocate.  Errors: INVALID_ARG, UNSUPPORTED (groups != 1),
+ * OOM, CUDA, NO_DEVICE; *out is left NULL on any error.
+ */
+bconv_status_t bconv_create(const bconv_desc_t* desc, const uint32_t* packed_weights, const float* scale,
+                            const float* bias, const float* in_scale, const float* in_bias, bconv_type_t type,
+                            uint32_t flags, bconv_handle_t* out);
+
+/*
+ * Run the layer: in (device fp32 [batch][in_h][in_w][in_channels]) -> out (device fp32
+ * [batch][Ho][Wo][out_channels]).  Asynchronous on `stream`; allocates nothing.
+ */
+bconv_status_t bconv_forward(bconv_handle_t h, const float* in, float* out, struct CUstream_st* stream);
+
+/*
+ * Same as bconv_forward with HOST buffers: copies host_in to the device, runs the layer
+ * and copies the result into host_out, all on `stream`, then waits for the stream.  Use
+ * page-locked host memory for full copy bandwidth.  The first call on a handle allocates
+ * the device staging buffers it needs and keeps them until bconv_destroy.
+ */
+bconv_status_t bconv_forward_host(bconv_handle_t h, const float* host_in, float* host_out,
+                                  struct CUstream_st* stream);
+
+/* Output dimensions (n, Ho, Wo, out_channels).  Any pointer may be NULL. */
+bconv_status_t bconv_get_output_dims(bconv_handle_t h, int32_t* n, int32_t* ho, int32_t* wo, int32_t* c);
+
+/* The inputFeatureChannels / outputFeatureChannels properties; -1 for a NULL handle. */
+int32_t bconv_input_feature_channels(bconv_handle_t h);
+int32_t bconv_output_feature_channels(bconv_handle_t h);
+
+/* Choose the kernel family (BCONV_ALGO_*).  UNSUPPORTED if the family does not do this type. */
+bconv_status_t bconv_set_algo(bconv_handle_t h, bconv_algo_t algo);
+
+/* Kernel launches one bconv_forward makes with the current settings. */
+int32_t bconv_launches_per_forward(bconv_handle_t h);
+
+/*
+ * Wait for `stream`, then read and clear the handle's device error word.  Returns OK,
+ * TIMEOUT (a kernel gave up a bounded wait), or CUDA (a pending CUDA error).
+ */
+bconv_status_t bconv_sync_status(bconv_handle_t h, struct CUstream_st* stream);
+
+/*
+ * Timing of the contraction kernel.  After bconv_profile_begin(h, n), each of the next n
+ * forwards records a CUDA event pair around its contraction kernel on its own stream;
+ * bconv_profile_end waits for the events and returns the summed milliseconds and the
+ * number of launches timed, then stops recording.
+ */
+bconv_status_t bconv_profile_begin(bconv_handle_t h, int32_t max_launches);
+bconv_status_t bconv_profile_end(bconv_handle_t h, float* total_ms, int32_t* launches);
+
+/* Free everything the handle owns (waits for the device first).  NULL is a no-op (OK). */
+bconv_status_t bconv_destroy(bconv_handle_t h);
+
+/* ------------------------------------------------------------------------------------
+ * Fully-connected special case (MPSCNNFullyConnected Overview and Note): the kernel is
+ * the whole source image, the output is 1x1xNo per image, and the result equals the
+ * flattened (y, x, f) input vector times an No x (H*W*Ni) weight matrix.  Stride and
+ * groups must be 1.  With beta, beta_n = sum over all pixels of A / (H*W).
+ * ------------------------------------------------------------------------------------ */
+typedef struct {
+  int32_t batch, in_h, in_w, in_channels, out_channels;
+  int32_t stride_y, stride_x, groups; /* each must be 1 */
+  int32_t neuron;                     /* bconv_neuron_t */
+  float scale_value;
+} bfc_desc_t;
+
+typedef struct bfc_handle_s* bfc_handle_t;
+
+/*
+ * packed_weights: host uint32 [out_channels][in_h][in_w][ceil(in_channels/32)].
+ * Other arguments and errors as for bconv_create; stride or groups != 1 -> INVALID_ARG
+ * and UNSUPPORTED respectively.
+ */
+bconv_status_t bfc_create(const bfc_desc_t* desc, const uint32_t* packed_weights, const float* scale,
+                          const float* bias, const float* in_scale, const float* in_bias, bconv_type_t type,
+                          uint32_t flags, bfc_handle_t* out);
+/* in: device fp32 [batch][in_h][in_w][in_channels]; out: device fp32 [batch][out_channels]. */
+bconv_status_t bfc_forward(bfc_handle_t h, const float* in, float* out, struct CUstream_st* stream);
+bconv_status_t bfc_forward_host(bfc_handle_t h, const float* host_in, float* host_out, struct CUstream_st* stream);
+int32_t bfc_input_feature_channels(bfc_handle_t h);
+int32_t bfc_output_feature_channels(bfc_handle_t h);
+bconv_status_t bfc_set_algo(bfc_handle_t h, bconv_algo_t algo);
+int32_t bfc_launches_per_forward(bfc_handle_t h);
+bconv_status_t bfc_sync_status(bfc_handle_t h, struct CUstream_st* stream);
+bconv_status_t bfc_profile_begin(bfc_handle_t h, int32_t max_launches);
+bconv_status_t bfc_profile_end(bfc_handle_t h, float* total_ms, int32_t* launches);
+bconv_status_t bfc_destroy(bfc_handle_t h);
+
+/* ------------------------------------------------------------------------------------
+ * Host helpers
+ * ------------------------------------------------------------------------------------ */
+
+/* A short English description of a status. */
+const char* bconv_status_string(bconv_status_t s);
+
+/*
+ * Pack 0/1 bytes into LSB-first words: bits (host uint8 [rows][nbits], each byte 0 or
+ * nonzero) -> out (host uint32 [rows][ceil(nbits/32)]); bit f of a row goes to bit
+ * (f % 32) of word (f / 32), unused high bits are 0.  For weights, rows = out_channels *
+ * kernel_h * kernel_w and nbits = in_channels.
+ */
+bconv_status_t bconv_pack_bits(const uint8_t* bits, int64_t rows, int32_t nbits, uint32_t* out);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t bconv_version(void);
+
+/*
+ * Measured peak of an instruction the contraction kernels are bound by, on the current
+ * device: kind 0 = POPC (32-bit population count, reported as bit-ops/s = 32 x
+ * instructions/s), 1 = LOP3 (32-bit logic op, instructions/s x 32), 2 = b1 tensor MMA
+ * mma.sync m16n8k256 .xor.popc (bit multiply-accumulates/s).  Runs a few short kernels
+ * (milliseconds) and waits for them.  *sm_mhz receives the SM clock the kernels saw,
+ * derived from clock64() over the event-timed interval (may be NULL).
+ */
+bconv_status_t bconv_measure_peak(int32_t kind, double* ops_per_s, double* sm_mhz);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BCONV_H_ */

@@ -22,3 +22,13 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+def pytest_sessionstart(session):
+    # Build the in-tree CUDA library and the oracle if their sources changed.
+    from binarized_convolution_b200 import build as _build
+
+    _build.build()
+    import oracle
+
+    oracle.build()

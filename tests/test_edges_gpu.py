@@ -1,0 +1,108 @@
+"""Edge cases of the CUDA library against the oracle on tiny inputs (runs on the B200 machine):
+channel counts around word boundaries, odd and even kernels, strides, non-square and tiny
+images, signed zeros, empty batches, ragged output channels and the FC with a partial last
+word."""
+import itertools
+
+import numpy as np
+import pytest
+
+from binarized_convolution_b200 import synth
+import binarized_convolution_b200 as bc
+import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(w, inp=None):
+    inp = inp if inp is not None else synth.make_inputs(w)
+    S_ref, beta_ref, y_ref = pu.run_oracle(w, inp)
+    y = pu.run_device(w, inp)
+    pu.assert_outputs_close(w, inp, y, S_ref, beta_ref, y_ref)
+    if w.op != synth.BINARY_WEIGHTS:
+        S_dev = pu.run_device(w, inp, sums=True)
+        S_sum, _, _ = pu.run_oracle(w, inp, sums=True)
+        pu.assert_sums_exact(S_dev, S_sum)
+
+
+SWEEP = []
+for i, (ni, k, s, op) in enumerate(itertools.product([1, 31, 32, 33, 100], [1, 2, 3, 5, 7], [1, 2],
+                                                     [synth.XNOR, synth.AND, synth.BINARY_WEIGHTS])):
+    if (i % 3) != 0 and k not in (2, 3):  # keep the sweep small: every even/3x3 kernel, a third of the rest
+        continue
+    SWEEP.append(synth.small_case(batch=1 + (i % 2), h=7 + (i % 3), w=9 - (i % 4), ni=ni, no=5 + (i % 7), k=k,
+                                  stride=s, op=op, use_beta=bool(i % 2), relu=bool((i // 2) % 2),
+                                  in_terms=bool((i // 3) % 2), seed=1000 + i))
+
+
+@pytest.mark.parametrize("w", SWEEP, ids=lambda w: w.name)
+def test_sweep(w, cuda_device):
+    _check(w)
+
+
+@pytest.mark.parametrize("op", [synth.XNOR, synth.AND, synth.BINARY_WEIGHTS])
+def test_kernel_larger_than_image(op, cuda_device):
+    _check(synth.small_case(batch=2, h=3, w=2, ni=40, no=3, k=7, kw=5, op=op, use_beta=True, in_terms=True, seed=7))
+
+
+@pytest.mark.parametrize("op", [synth.XNOR, synth.AND])
+def test_signed_zeros_binarize_to_plus_one(op, cuda_device):
+    w = synth.small_case(batch=1, h=6, w=5, ni=48, no=9, k=3, op=op, seed=8)
+    inp = synth.make_inputs(w)
+    inp.x[..., :8] = 0.0
+    inp.x[..., 8:16] = -0.0
+    _check(w, inp)
+    # the same layer with in_bias that maps some inputs exactly onto +-0
+    w2 = synth.small_case(batch=1, h=6, w=5, ni=48, no=9, k=3, op=op, in_terms=True, seed=9)
+    inp2 = synth.make_inputs(w2)
+    inp2.in_scale[:] = 1.0
+    inp2.in_bias[:4] = 0.5
+    inp2.x[..., :4] = -0.5
+    _check(w2, inp2)
+
+
+@pytest.mark.parametrize("op", [synth.XNOR, synth.AND, synth.BINARY_WEIGHTS])
+def test_fc_partial_last_word(op, cuda_device):
+    _check(synth.small_case(batch=5, h=3, w=5, ni=7, no=11, kind="fc", op=op, use_beta=True, in_terms=True, seed=10))
+    _check(synth.small_case(batch=3, h=1, w=1, ni=1, no=1, kind="fc", op=op, use_beta=True, seed=11))
+
+
+@pytest.mark.parametrize("op", [synth.XNOR, synth.AND, synth.BINARY_WEIGHTS])
+def test_ragged_channels_and_tiles(op, cuda_device):
+    # No = 1 and No = 129 (one past a 128-channel tile), M = 129 (one past a 128-pixel tile)
+    _check(synth.small_case(batch=1, h=3, w=43, ni=65, no=1, k=3, op=op, use_beta=True, seed=12))
+    _check(synth.small_case(batch=1, h=3, w=43, ni=65, no=129, k=3, op=op, relu=True, seed=13))
+
+
+def test_empty_batch(cuda_device):
+    import torch
+
+    for op in (synth.XNOR, synth.BINARY_WEIGHTS):
+        layer = bc.BinaryConv2d(0, 5, 5, 8, 4, 3, 1, wbits=np.ones((4, 3, 3, 8), np.uint8), op=op, use_beta=True)
+        y = layer(torch.empty((0, 5, 5, 8), device="cuda"))
+        layer.sync_status()
+        assert tuple(y.shape) == (0, 5, 5, 4)
+        layer.close()
+
+
+def test_forward_host_matches_device(cuda_device):
+    w = synth.small_case(batch=2, h=9, w=10, ni=96, no=40, k=3, op=synth.XNOR, use_beta=True, relu=True,
+                         in_terms=True, seed=14)
+    inp = synth.make_inputs(w)
+    y_dev = pu.run_device(w, inp)
+    layer = pu.make_layer(w, inp)
+    y_host = layer.forward_host(inp.x)
+    layer.close()
+    np.testing.assert_array_equal(y_host.reshape(y_dev.shape), y_dev)
+
+
+def test_properties_and_algo(cuda_device):
+    w = synth.small_case(batch=1, h=5, w=5, ni=70, no=6, k=3, op=synth.XNOR, seed=15)
+    inp = synth.make_inputs(w)
+    layer = pu.make_layer(w, inp)
+    assert layer.input_feature_channels == 70 and layer.output_feature_channels == 6
+    layer.set_algo(bc.ALGO_POPC)
+    with pytest.raises(bc.BconvError):
+        layer.set_algo(bc.ALGO_SIMT_F32)
+    assert layer.launches_per_forward() == 2
+    layer.close()
