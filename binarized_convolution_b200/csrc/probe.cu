@@ -35,7 +35,7 @@ __global__ void __launch_bounds__(kProbeThreads) popc_probe(int iters, uint32_t*
 #pragma unroll
   for (int j = 0; j < kChains; ++j) s += acc[j];
   out[tid] = s;
-  if (tid == 0) *cycles = t1 - t0;
+  if ((threadIdx.x & 31) == 0) atomicMax(reinterpret_cast<unsigned long long*>(cycles), static_cast<unsigned long long>(t1 - t0));
 }
 
 __global__ void __launch_bounds__(kProbeThreads) lop3_probe(int iters, uint32_t* out, long long* cycles) {
@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(kProbeThreads) lop3_probe(int iters, uint32_t*
 #pragma unroll
   for (int j = 0; j < kChains; ++j) s ^= x[j];
   out[tid] = s;
-  if (tid == 0) *cycles = t1 - t0;
+  if ((threadIdx.x & 31) == 0) atomicMax(reinterpret_cast<unsigned long long*>(cycles), static_cast<unsigned long long>(t1 - t0));
 }
 
 constexpr int kMmaChains = 4;
@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(kProbeThreads) b1mma_probe(int iters, uint32_t
 #pragma unroll
     for (int j = 0; j < 4; ++j) s += d[c][j];
   out[tid] = static_cast<uint32_t>(s);
-  if (tid == 0) *cycles = t1 - t0;
+  if ((threadIdx.x & 31) == 0) atomicMax(reinterpret_cast<unsigned long long*>(cycles), static_cast<unsigned long long>(t1 - t0));
 }
 
 }  // namespace
@@ -113,6 +113,7 @@ cudaError_t probe_peak(int kind, double* ops_per_s, double* sm_mhz) {
   float best_ms = 0.f;
   long long cycles = 0;
   for (int rep = 0; rep < 4 && err == cudaSuccess; ++rep) {
+    cudaMemset(cyc, 0, sizeof(long long));
     cudaEventRecord(e0, 0);
     if (kind == 0)
       popc_probe<<<blocks, kProbeThreads>>>(iters, out, cyc);
