@@ -29,6 +29,8 @@ from ._native import (  # noqa: F401
     bconv_destroy,
     bconv_forward,
     bconv_forward_host,
+    bconv_forward_noalloc,
+    NOALLOC_SCRATCH_BYTES,
     bconv_get_output_dims,
     bconv_input_feature_channels,
     bconv_launches_per_forward,

@@ -78,7 +78,9 @@ _SIGS = {
     "bconv_pack_bits": (_I32, [_P, ctypes.c_int64, _I32, _P]),
     "bconv_version": (_I32, []),
     "bconv_measure_peak": (_I32, [_I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
+    "bconv_forward_noalloc": (_I32, [ctypes.POINTER(bconv_desc_t), _I32, ctypes.c_uint32] + [_P] * 8),
 }
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def library_path() -> str:
@@ -281,3 +283,12 @@ def bconv_measure_peak(kind: int):
     ops, mhz = ctypes.c_double(), ctypes.c_double()
     _check(load_library().bconv_measure_peak(int(kind), ctypes.byref(ops), ctypes.byref(mhz)), "bconv_measure_peak")
     return ops.value, mhz.value
+
+
+def bconv_forward_noalloc(desc: bconv_desc_t, type: int, flags: int, weights_ptr: int, scale_ptr: int | None,
+                          bias_ptr: int | None, in_scale_ptr: int | None, in_bias_ptr: int | None, in_ptr: int,
+                          out_ptr: int, stream: int = 0):
+    """XNOR/AND forward that allocates nothing; every pointer is a device address (or None)."""
+    _check(load_library().bconv_forward_noalloc(ctypes.byref(desc), int(type), int(flags), weights_ptr, scale_ptr,
+                                                bias_ptr, in_scale_ptr, in_bias_ptr, in_ptr, out_ptr, stream),
+           "bconv_forward_noalloc")

@@ -220,6 +220,49 @@ int32_t bconv_version(void);
  */
 bconv_status_t bconv_measure_peak(int32_t kind, double* ops_per_s, double* sm_mhz);
 
+/* ------------------------------------------------------------------------------------
+ * Forward without any allocation.  (The pages have no counterpart to this entry point; it
+ * exists for callers of this library that cannot allocate device memory when they run a
+ * layer: code whose device memory is all owned by its own pool, real-time loops where an
+ * allocation may stall on a device-wide synchronisation, or work issued while a stream is
+ * being captured into a CUDA graph, where allocation calls are not permitted.  Such callers
+ * cannot use bconv_create, which allocates.)
+ * ------------------------------------------------------------------------------------ */
+
+/* Size of the one fixed scratch array this entry point works in (16 MiB).  Every device that
+ * loads the library holds it until the process exits. */
+#define BCONV_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * XNOR or AND convolution (the same result as bconv_create + bconv_forward with the same
+ * arguments), computed with no cudaMalloc, cudaFree or other allocating call.
+ *   desc            host; as for bconv_create (groups must be 1).
+ *   type            BCONV_TYPE_XNOR or BCONV_TYPE_AND (binaryWeights -> INVALID_ARG).
+ *   flags           BCONV_FLAG_* bits.
+ *   packed_weights  DEVICE uint32 [out_channels][kernel_h][kernel_w][ceil(in_channels/32)],
+ *                   LSB-first as for bconv_create; bits beyond in_channels are ignored.
+ *   scale, bias     DEVICE float [out_channels] or NULL (desc->scale_value / 0).
+ *   in_scale, in_bias DEVICE float [in_channels] or NULL (1 / 0).
+ *   in, out         DEVICE fp32 NHWC input and output, as for bconv_forward.
+ *   stream          the stream all work is queued on (asynchronous).
+ * Working buffers come from the library's fixed scratch array.  Their total is
+ *   P*W + T*W*C + No*T*4 [+ P*4 + N*Ho*Wo*4 with beta] [+ 4*No per missing scale/bias]
+ *   [+ 4*Ni if exactly one of in_scale/in_bias is given]
+ * bytes, each piece rounded up to 256, with P = batch*in_h*in_w, W = 4*round_up(ceil(Ni/32), 8),
+ * T = kernel_h*kernel_w, C = round_up(out_channels, 128); a call needing more than
+ * BCONV_NOALLOC_SCRATCH_BYTES returns BCONV_ERR_UNSUPPORTED before queuing any work.  Each call
+ * rewrites every part of the scratch it reads, so no state carries over from earlier calls,
+ * but all calls share the one array: calls whose GPU work can overlap (different streams or
+ * host threads without ordering between them) race and corrupt each other's results.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current) and caches it; make that first call before any stream capture begins.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA, NO_DEVICE.
+ */
+bconv_status_t bconv_forward_noalloc(const bconv_desc_t* desc, bconv_type_t type, uint32_t flags,
+                                     const uint32_t* packed_weights, const float* scale, const float* bias,
+                                     const float* in_scale, const float* in_bias, const float* in, float* out,
+                                     struct CUstream_st* stream);
+
 #ifdef __cplusplus
 }
 #endif
