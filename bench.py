@@ -171,15 +171,35 @@ def measured_traffic(kernel: str, workload: str, sources) -> float | None:
 KERNEL_SOURCES = {
     "popc_gemm": ["binarized_convolution_b200/csrc/popc_gemm.cu", "binarized_convolution_b200/csrc/common.cuh"],
     "bw_conv": ["binarized_convolution_b200/csrc/bw_conv.cu", "binarized_convolution_b200/csrc/common.cuh"],
+    "tc_conv": ["binarized_convolution_b200/csrc/tc_conv.cu", "binarized_convolution_b200/csrc/tc_conv.cuh"],
 }
+ALGO_KERNEL = {1: "popc_gemm", 2: "bw_conv", 3: "tc_conv"}
+BF16_FALLBACK_TFLOPS = 1590.0  # recipe fallback when MEASURED_PEAKS.json is absent
 
 
-def contraction_kernel(w: synth.Workload) -> str:
-    return "bw_conv" if w.op == synth.BINARY_WEIGHTS else "popc_gemm"
+def measured_peaks() -> dict:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return {}
 
 
-def derived_peak(w: synth.Workload, sms: int, sm_mhz: float) -> tuple[float, str, str]:
+def tensor_peak() -> tuple[float, str]:
+    """Dense int8 tensor-core multiply-accumulates per second, in T: the measured bf16 burst
+    TFLOP/s x 2 (the nominal int8/bf16 ratio, 4.5/2.25) / 2 (ops per MAC)."""
+    p = measured_peaks()
+    if "bf16_tflops" in p:
+        v = float(p["bf16_tflops"])
+        return v, f"of measured: bf16 burst {v:.1f} TFLOP/s x 2 (int8/bf16 nominal) / 2 ops per MAC"
+    return BF16_FALLBACK_TFLOPS, "of fallback: 1590 TFLOP/s bf16 x 2 / 2 ops per MAC"
+
+
+def derived_peak(w: synth.Workload, sms: int, sm_mhz: float, kernel: str = "") -> tuple[float, str, str]:
     """(peak in TOPS, bound, how it was derived) for the contraction's instruction mix."""
+    if kernel == "tc_conv":
+        v, how = tensor_peak()
+        return v, "tensor", how
     if w.op == synth.BINARY_WEIGHTS:
         p = sms * FP32_PER_CLK_PER_SM * sm_mhz * 1e6 / 1e12
         return p, "alu", f"{sms} SMs x {FP32_PER_CLK_PER_SM} FP32 lanes/clk x {sm_mhz:.0f} MHz (1 op = 1 signed add)"
@@ -246,6 +266,8 @@ def run_native(args, w: synth.Workload):
         layer = bc.BinaryConv2d(w.batch, w.in_h, w.in_w, w.in_channels, w.out_channels, (w.kernel_h, w.kernel_w),
                                 (w.stride_y, w.stride_x), wbits=inp.wbits, **layer_kw)
         prof_begin, prof_end = bc.bconv_profile_begin, bc.bconv_profile_end
+    if args.algo != "auto":
+        layer.set_algo({"popc": bc.ALGO_POPC, "tcgen05": bc.ALGO_TCGEN05, "simt_f32": bc.ALGO_SIMT_F32}[args.algo])
     out_shape = layer.out_dims
     xs = [torch.from_numpy(inp.x).to(device)]
     for r in range(1, ROTATE):
@@ -285,18 +307,19 @@ def run_native(args, w: synth.Workload):
     props = torch.cuda.get_device_properties(device)
     sms = props.multi_processor_count
     max_mhz = clock_info.get("sm_max_mhz") or 1965.0
-    peak, bound, how = derived_peak(w, sms, max_mhz)
+    kname = ALGO_KERNEL[layer.effective_algo()]
+    peak, bound, how = derived_peak(w, sms, max_mhz, kname)
     achieved = ops_step / (kern_ms_max * 1e-3) / 1e12
-    kname = contraction_kernel(w)
     traffic = measured_traffic(kname, w.name, KERNEL_SOURCES[kname])
     roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
-            "traffic": traffic, "kernel": kname, "kernel_ms": kern_ms_max, "peak_source": f"derived: {how}"}
+            "traffic": traffic, "kernel": kname, "kernel_ms": kern_ms_max,
+            "peak_source": how if bound == "tensor" else f"derived: {how}"}
     sm_mhz = clock_info.get("sm_mhz")
-    if sm_mhz:
-        p_obs, _, _ = derived_peak(w, sms, sm_mhz)
+    if sm_mhz and bound == "alu":
+        p_obs, _, _ = derived_peak(w, sms, sm_mhz, kname)
         roof["frac_at_observed_clock"] = achieved / p_obs
     try:
-        probe = 0 if w.op != synth.BINARY_WEIGHTS else None
+        probe = 0 if kname == "popc_gemm" else None
         if probe is not None and rank == 0:
             ops_s, mhz = bc.bconv_measure_peak(probe)
             roof["probe_peak"] = ops_s / 1e12
@@ -307,13 +330,13 @@ def run_native(args, w: synth.Workload):
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "u32-bits/int32" if w.op != synth.BINARY_WEIGHTS else "f32",
+        "dtype": {"popc_gemm": "u32 bits / int32", "tc_conv": "int8 codes / int32", "bw_conv": "f32"}[kname],
         "data": "synthetic (seeded N(0,1) inputs, Bernoulli weight bits)",
         "config": {"workload": w.name, "batch_per_gpu": w.batch, "global_batch": w.batch * world,
                    "in": [w.in_h, w.in_w, w.in_channels], "out_channels": w.out_channels,
                    "kernel": [w.kernel_h, w.kernel_w], "stride": [w.stride_y, w.stride_x], "op": w.op,
                    "beta": w.use_beta, "relu": w.relu, "input_terms": w.in_terms,
-                   "parallelism": f"replicas x{world}",
+                   "parallelism": f"replicas x{world}", "algo": kname,
                    "l2": f"{ROTATE} rotating input/output sets, "
                          f"{ROTATE * (inp.x.nbytes + int(np.prod(out_shape)) * 4) / 1e6:.0f} MB > 126 MB L2"},
         "images_per_s": images_s,
@@ -411,6 +434,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--algo", choices=["auto", "popc", "tcgen05", "simt_f32"], default="auto",
+                    help="kernel family of the contraction (auto = the library's choice)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time of the cpu_baseline sample")

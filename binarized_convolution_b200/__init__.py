@@ -16,6 +16,7 @@ from ._native import (  # noqa: F401
     ALGO_AUTO,
     ALGO_POPC,
     ALGO_SIMT_F32,
+    ALGO_TCGEN05,
     FLAG_NONE,
     FLAG_USE_BETA_SCALING,
     NEURON_NONE,
@@ -27,6 +28,7 @@ from ._native import (  # noqa: F401
     bconv_create,
     bconv_desc_t,
     bconv_destroy,
+    bconv_effective_algo,
     bconv_forward,
     bconv_forward_host,
     bconv_forward_noalloc,
@@ -46,6 +48,7 @@ from ._native import (  # noqa: F401
     bfc_create,
     bfc_desc_t,
     bfc_destroy,
+    bfc_effective_algo,
     bfc_forward,
     bfc_forward_host,
     bfc_input_feature_channels,

@@ -23,7 +23,7 @@ _HEADER = os.path.join(_ROOT, "include", "bconv.h")
 TYPE_BINARY_WEIGHTS, TYPE_XNOR, TYPE_AND = 0, 1, 2
 FLAG_NONE, FLAG_USE_BETA_SCALING = 0, 1
 NEURON_NONE, NEURON_RELU = 0, 1
-ALGO_AUTO, ALGO_POPC, ALGO_SIMT_F32 = 0, 1, 2
+ALGO_AUTO, ALGO_POPC, ALGO_SIMT_F32, ALGO_TCGEN05 = 0, 1, 2, 3
 
 _STATUS = {0: "BCONV_OK", 1: "BCONV_ERR_INVALID_ARG", 2: "BCONV_ERR_UNSUPPORTED", 3: "BCONV_ERR_CUDA",
            4: "BCONV_ERR_OOM", 5: "BCONV_ERR_TIMEOUT", 6: "BCONV_ERR_NO_DEVICE"}
@@ -59,6 +59,7 @@ _SIGS = {
     "bconv_output_feature_channels": (_I32, [_P]),
     "bconv_set_algo": (_I32, [_P, _I32]),
     "bconv_launches_per_forward": (_I32, [_P]),
+    "bconv_effective_algo": (_I32, [_P]),
     "bconv_sync_status": (_I32, [_P, _P]),
     "bconv_profile_begin": (_I32, [_P, _I32]),
     "bconv_profile_end": (_I32, [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_I32)]),
@@ -70,6 +71,7 @@ _SIGS = {
     "bfc_output_feature_channels": (_I32, [_P]),
     "bfc_set_algo": (_I32, [_P, _I32]),
     "bfc_launches_per_forward": (_I32, [_P]),
+    "bfc_effective_algo": (_I32, [_P]),
     "bfc_sync_status": (_I32, [_P, _P]),
     "bfc_profile_begin": (_I32, [_P, _I32]),
     "bfc_profile_end": (_I32, [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_I32)]),
@@ -217,6 +219,14 @@ def bconv_launches_per_forward(h) -> int:
 
 def bfc_launches_per_forward(h) -> int:
     return load_library().bfc_launches_per_forward(h)
+
+
+def bconv_effective_algo(h) -> int:
+    return load_library().bconv_effective_algo(h)
+
+
+def bfc_effective_algo(h) -> int:
+    return load_library().bfc_effective_algo(h)
 
 
 def bconv_sync_status(h, stream: int = 0):

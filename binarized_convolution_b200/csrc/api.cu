@@ -10,11 +10,16 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
 #include <new>
 #include <vector>
 
 #include "bconv.h"
 #include "common.cuh"
+#include "tc_conv.cuh"
 
 namespace bconv {
 
@@ -112,6 +117,15 @@ struct Layer {
   uint32_t* bits = nullptr;
   float *A = nullptr, *beta = nullptr;
   uint32_t* err = nullptr;
+  // tensor-core path: int8 codes [N][H][W][cip], int8 weights [no_tc][taps*cip], tensor maps
+  bool tc_ok = false;
+  int cip = 0;
+  int8_t* codes = nullptr;
+  int8_t* wq = nullptr;
+  float* ws = nullptr;  // FC split-K partial sums [N][No]
+  TcArgs tc{};
+  CUtensorMap tmA{}, tmB{}, tmWs{}, tmOut{};
+  const float* tm_out_ptr = nullptr;
   // host-buffer forward staging (allocated on first use)
   float *stage_in = nullptr, *stage_out = nullptr;
   DevMem mem;
@@ -139,6 +153,153 @@ namespace bconv {
 namespace {
 
 bool valid_type(int t) { return t == kBinaryWeights || t == kXnor || t == kAnd; }
+
+// cuTensorMapEncodeTiled from the driver, found through the runtime (the library does not
+// link the driver library, so it loads on machines without one).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 4-D tiled map, dims innermost first, 128-byte swizzle, out-of-range elements read as 0.
+bool encode_4d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, const uint64_t dims[4],
+               const uint64_t strides_bytes[3], const uint32_t box[4]) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, dt, 4, const_cast<void*>(base), reinterpret_cast<const cuuint64_t*>(dims),
+             reinterpret_cast<const cuuint64_t*>(strides_bytes), reinterpret_cast<const cuuint32_t*>(box), estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1, uint64_t stride1,
+               uint32_t b0, uint32_t b1) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {d0, d1};
+  const cuuint64_t strides[1] = {stride1};
+  const cuuint32_t box[2] = {b0, b1};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int next_pow2(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+// Output map over `out` ([N][Ho][Wo][No] fp32) with the tile's box.
+bool encode_out_map(Layer& L, CUtensorMap* m, const float* out) {
+  const uint64_t dims[4] = {static_cast<uint64_t>(L.No), static_cast<uint64_t>(L.Ho), static_cast<uint64_t>(L.Wo),
+                            static_cast<uint64_t>(L.N)};
+  uint64_t d[4] = {dims[0], dims[2], dims[1], dims[3]};  // {No, Wo, Ho, N}
+  const uint64_t row = static_cast<uint64_t>(L.No) * 4;
+  const uint64_t strides[3] = {row, row * L.Wo, row * L.Wo * L.Ho};
+  const uint32_t box[4] = {32, static_cast<uint32_t>(L.tc.Cw), static_cast<uint32_t>(L.tc.R),
+                           static_cast<uint32_t>(L.tc.Bn)};
+  return encode_4d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, out, d, strides, box);
+}
+
+// The tensor-core path covers XNOR/AND with stride 1 (or the FC) and No % 4 == 0 (16-byte
+// output rows for the TMA store).  Sets up its buffers, weights and maps.
+bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
+  if (L.type == kBinaryWeights || L.No % 4 != 0 || (!L.fc && (L.sy != 1 || L.sx != 1)) || L.N == 0) return BCONV_OK;
+  if (!tensor_map_encoder()) return BCONV_OK;
+  const int taps = L.kh * L.kw;
+  L.cip = round_up(L.Ni, 128);
+  TcArgs& t = L.tc;
+  t.BN = std::min(256, round_up(L.No, 32));
+  t.n_tiles = (L.No + t.BN - 1) / t.BN;
+  t.No = L.No;
+  t.N = L.N;
+  t.tmem_cols = static_cast<uint32_t>(std::max(32, next_pow2(2 * t.BN)));
+  t.relu = L.relu;
+  t.err = L.err;
+  t.scale = L.scale;
+  t.bias = L.bias;
+  if (L.fc) {
+    t.Ho = 1; t.Wo = 1; t.kh = 1; t.kw = 1;
+    t.kb_per_tap = L.H * L.W * L.cip / 128;
+    t.R = 1; t.Cw = 1; t.Bn = 128;
+    t.tiles_x = 1; t.tiles_y = 1;
+  } else {
+    t.Ho = L.Ho; t.Wo = L.Wo; t.kh = L.kh; t.kw = L.kw;
+    t.kb_per_tap = L.cip / 128;
+    t.Cw = std::min(128, next_pow2(L.Wo));
+    t.R = std::min(128 / t.Cw, next_pow2(L.Ho));
+    t.Bn = 128 / (t.Cw * t.R);
+    t.tiles_x = (L.Wo + t.Cw - 1) / t.Cw;
+    t.tiles_y = (L.Ho + t.R - 1) / t.R;
+  }
+  t.m_tiles = t.tiles_x * t.tiles_y * ((L.N + t.Bn - 1) / t.Bn);
+  const int kb_total = t.kh * t.kw * t.kb_per_tap;
+  t.k_splits = 1;
+  if (L.fc) {  // spread the reduction so that the tiles fill the GPU
+    const int sms = current_sm_count();
+    const int64_t tiles = static_cast<int64_t>(t.m_tiles) * t.n_tiles;
+    int64_t best = -1;
+    for (int s = 1; s <= 16 && kb_total / s >= 4; ++s) {
+      const int64_t cost = ceil_div(tiles * s, sms) * ceil_div(kb_total, s);
+      if (best < 0 || cost < best) {
+        best = cost;
+        t.k_splits = s;
+      }
+    }
+  }
+
+  // int8 weights [no_tc][taps*cip]: +-1 (XNOR) or 0/1 (AND) codes, 0 in every padding slot.
+  const int no_tc = t.n_tiles * t.BN;
+  const int64_t kt = static_cast<int64_t>(taps) * L.cip;
+  std::vector<int8_t> hq(static_cast<size_t>(no_tc) * kt, 0);
+  const int8_t one = 1, zero_code = (L.type == kXnor) ? -1 : 0;
+  for (int c = 0; c < L.No; ++c)
+    for (int tp = 0; tp < taps; ++tp)
+      for (int f = 0; f < L.Ni; ++f) {
+        const uint32_t word = packed[(static_cast<int64_t>(c) * taps + tp) * L.nw + f / kWordBits];
+        hq[static_cast<size_t>(c) * kt + static_cast<int64_t>(tp) * L.cip + f] =
+            ((word >> (f % kWordBits)) & 1u) ? one : zero_code;
+      }
+  const int64_t npix = static_cast<int64_t>(L.N) * L.H * L.W;
+  cudaError_t e = L.mem.alloc(&L.wq, hq.size());
+  if (e == cudaSuccess) e = cudaMemcpy(L.wq, hq.data(), hq.size(), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = L.mem.alloc(&L.codes, static_cast<size_t>(npix) * L.cip);
+  if (e == cudaSuccess && t.k_splits > 1) e = L.mem.alloc(&L.ws, static_cast<size_t>(L.N) * L.No);
+  if (e != cudaSuccess) return from_cuda(e);
+
+  bool ok = true;
+  if (L.fc) {
+    const uint64_t K = static_cast<uint64_t>(L.H) * L.W * L.cip;
+    const uint64_t dims[4] = {K, 1, 1, static_cast<uint64_t>(L.N)};
+    const uint64_t strides[3] = {K, K, K};
+    const uint32_t box[4] = {128, 1, 1, 128};
+    ok = encode_4d(&L.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.codes, dims, strides, box);
+  } else {
+    const uint64_t dims[4] = {static_cast<uint64_t>(L.cip), static_cast<uint64_t>(L.W), static_cast<uint64_t>(L.H),
+                              static_cast<uint64_t>(L.N)};
+    const uint64_t strides[3] = {static_cast<uint64_t>(L.cip), static_cast<uint64_t>(L.cip) * L.W,
+                                 static_cast<uint64_t>(L.cip) * L.W * L.H};
+    const uint32_t box[4] = {128, static_cast<uint32_t>(t.Cw), static_cast<uint32_t>(t.R), static_cast<uint32_t>(t.Bn)};
+    ok = encode_4d(&L.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.codes, dims, strides, box);
+  }
+  ok = ok && encode_2d(&L.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(kt),
+                       static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128, static_cast<uint32_t>(t.BN));
+  if (ok && t.k_splits > 1) ok = encode_out_map(L, &L.tmWs, L.ws);
+  if (!ok) return BCONV_OK;  // the POPC path stays available
+  L.tc_ok = true;
+  return BCONV_OK;
+}
 
 // Copy the parameter arrays (expanding defaults) and prepare the weights for the
 // contraction kernel of this layer type.
@@ -251,12 +412,61 @@ bconv_status_t finish_create(Layer& L, const uint32_t* packed, const float* scal
   L.no_pad = round_up(L.No, kTileN);
   bconv_status_t st = upload_params(L, packed, scale, bias, in_scale, in_bias, scale_value);
   if (st == BCONV_OK) st = alloc_workspace(L);
+  if (st == BCONV_OK) st = setup_tc(L, packed);
   if (st != BCONV_OK) L.mem.release();
   return st;
 }
 
+bool use_tc(const Layer& L) {
+  return L.tc_ok && (L.algo == BCONV_ALGO_AUTO || L.algo == BCONV_ALGO_TCGEN05);
+}
+
+// Tensor-core forward: int8 codes (+ A) -> [beta] -> tcgen05 contraction [-> finalize].
+bconv_status_t run_forward_tc(Layer& L, const float* in, float* out, cudaStream_t s) {
+  const bool beta = L.use_beta();
+  PackI8Args p{};
+  p.in = in;
+  p.npix = static_cast<int64_t>(L.N) * L.H * L.W;
+  p.ni = L.Ni;
+  p.cip = L.cip;
+  p.in_scale = L.in_scale;
+  p.in_bias = L.in_bias;
+  p.codes = L.codes;
+  p.A = beta ? L.A : nullptr;
+  p.op = L.type;
+  cudaError_t e = launch_pack_i8(p, s);
+  if (e != cudaSuccess) return from_cuda(e);
+  if (beta) {
+    BetaArgs b{L.A, L.beta, L.N, L.H, L.W, L.Ho, L.Wo, L.kh, L.kw, L.sy, L.sx};
+    e = L.fc ? launch_beta_image_mean(b, s) : launch_beta_conv(b, s);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  TcArgs t = L.tc;
+  t.beta = beta ? L.beta : nullptr;
+  const CUtensorMap* om = &L.tmWs;
+  if (t.k_splits > 1) {
+    e = cudaMemsetAsync(L.ws, 0, sizeof(float) * static_cast<size_t>(L.N) * L.No, s);
+    if (e != cudaSuccess) return from_cuda(e);
+  } else {
+    if (out != L.tm_out_ptr) {
+      if (!encode_out_map(L, &L.tmOut, out)) return BCONV_ERR_CUDA;
+      L.tm_out_ptr = out;
+    }
+    om = &L.tmOut;
+  }
+  const bool timed = L.prof.active && L.prof.used < static_cast<int>(L.prof.start.size());
+  if (timed) cudaEventRecord(L.prof.start[L.prof.used], s);
+  e = launch_tc_conv(&L.tmA, &L.tmB, om, t, s);
+  if (timed) cudaEventRecord(L.prof.stop[L.prof.used++], s);
+  if (e != cudaSuccess) return from_cuda(e);
+  if (t.k_splits > 1)
+    e = launch_tc_finalize(L.ws, out, L.scale, L.bias, t.beta, static_cast<int64_t>(L.N) * L.No, L.No, 1, L.relu, s);
+  return from_cuda(e);
+}
+
 // The launch sequence of one forward.
 bconv_status_t run_forward(Layer& L, const float* in, float* out, cudaStream_t s) {
+  if (L.N > 0 && use_tc(L)) return run_forward_tc(L, in, out, s);
   const int64_t npix = static_cast<int64_t>(L.N) * L.H * L.W;
   if (L.N == 0) return BCONV_OK;
   cudaError_t e = cudaSuccess;
@@ -380,15 +590,25 @@ bconv_status_t set_algo(Layer& L, int algo) {
     L.algo = algo;
     return BCONV_OK;
   }
-  if (algo < 0 || algo > BCONV_ALGO_SIMT_F32) return BCONV_ERR_INVALID_ARG;
+  if (algo == BCONV_ALGO_TCGEN05 && L.tc_ok) {
+    L.algo = algo;
+    return BCONV_OK;
+  }
+  if (algo < 0 || algo > BCONV_ALGO_TCGEN05) return BCONV_ERR_INVALID_ARG;
   return BCONV_ERR_UNSUPPORTED;
 }
 
 int launches_per_forward(const Layer& L) {
+  if (L.N > 0 && use_tc(L)) return 2 + (L.use_beta() ? 1 : 0) + (L.tc.k_splits > 1 ? 2 : 0);  // memset counted
   int n = 1;  // contraction
   if (L.type != kBinaryWeights || L.use_beta()) n += 1;  // pack
   if (L.use_beta()) n += 1;                              // beta
   return n;
+}
+
+int effective_algo(const Layer& L) {
+  if (use_tc(L)) return BCONV_ALGO_TCGEN05;
+  return L.type == kBinaryWeights ? BCONV_ALGO_SIMT_F32 : BCONV_ALGO_POPC;
 }
 
 bconv_status_t profile_begin(Layer& L, int32_t n) {
@@ -512,6 +732,8 @@ int32_t bconv_launches_per_forward(bconv_handle_t h) {
   return checked(h, kConvMagic) ? launches_per_forward(h->L) : -1;
 }
 
+int32_t bconv_effective_algo(bconv_handle_t h) { return checked(h, kConvMagic) ? effective_algo(h->L) : -1; }
+
 bconv_status_t bconv_sync_status(bconv_handle_t h, struct CUstream_st* stream) {
   if (!checked(h, kConvMagic)) return BCONV_ERR_INVALID_ARG;
   DeviceGuard g(h->L.device);
@@ -599,6 +821,8 @@ bconv_status_t bfc_set_algo(bfc_handle_t h, bconv_algo_t algo) {
 }
 
 int32_t bfc_launches_per_forward(bfc_handle_t h) { return checked(h, kFcMagic) ? launches_per_forward(h->L) : -1; }
+
+int32_t bfc_effective_algo(bfc_handle_t h) { return checked(h, kFcMagic) ? effective_algo(h->L) : -1; }
 
 bconv_status_t bfc_sync_status(bfc_handle_t h, struct CUstream_st* stream) {
   if (!checked(h, kFcMagic)) return BCONV_ERR_INVALID_ARG;

@@ -94,3 +94,93 @@ cudaError_t launch_pack(const PackArgs& a, cudaStream_t s) {
 }
 
 }  // namespace bconv
+
+// ------------------------------------------------------------------------------------
+// int8 operand codes for the tensor-core contraction, with the same transform and A.
+// A warp per pixel; with 4-aligned channels each lane turns one float4 into 4 codes (one
+// 32-bit store), so a warp writes 128 contiguous code bytes per step.
+// ------------------------------------------------------------------------------------
+#include "tc_conv.cuh"
+
+namespace bconv {
+namespace {
+
+template <bool kTerms, bool kA, int kOp, bool kVec>
+__global__ void __launch_bounds__(kPackThreads) pack_i8_kernel(PackI8Args a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kPackThreads) >> 5;
+  const int ni = a.ni;
+  constexpr uint32_t kPos = kOp == kXnor ? 0x01u : 0x01u;
+  constexpr uint32_t kNeg = kOp == kXnor ? 0xFFu : 0x00u;
+  for (int64_t p = warp; p < a.npix; p += nwarps) {
+    const float* row = a.in + p * ni;
+    int8_t* crow = a.codes + p * a.cip;
+    float asum = 0.f;
+    if constexpr (kVec) {
+      for (int f0 = 0; f0 < a.cip; f0 += 128) {
+        const int f = f0 + lane * 4;
+        uint32_t word = 0u;
+        if (f < ni) {
+          float4 v = __ldcs(reinterpret_cast<const float4*>(row + f));
+          if (kTerms) {
+            v.x = fmaf(v.x, __ldg(a.in_scale + f + 0), __ldg(a.in_bias + f + 0));
+            v.y = fmaf(v.y, __ldg(a.in_scale + f + 1), __ldg(a.in_bias + f + 1));
+            v.z = fmaf(v.z, __ldg(a.in_scale + f + 2), __ldg(a.in_bias + f + 2));
+            v.w = fmaf(v.w, __ldg(a.in_scale + f + 3), __ldg(a.in_bias + f + 3));
+          }
+          if (kA) asum += (fabsf(v.x) + fabsf(v.y)) + (fabsf(v.z) + fabsf(v.w));
+          word = ((v.x < 0.f) ? kNeg : kPos) | (((v.y < 0.f) ? kNeg : kPos) << 8) |
+                 (((v.z < 0.f) ? kNeg : kPos) << 16) | (((v.w < 0.f) ? kNeg : kPos) << 24);
+        }
+        *reinterpret_cast<uint32_t*>(crow + f) = word;
+      }
+    } else {
+      for (int f0 = 0; f0 < a.cip; f0 += 32) {
+        const int f = f0 + lane;
+        uint32_t code = 0u;
+        if (f < ni) {
+          float v = __ldcs(row + f);
+          if (kTerms) v = fmaf(v, __ldg(a.in_scale + f), __ldg(a.in_bias + f));
+          if (kA) asum += fabsf(v);
+          code = (v < 0.f) ? kNeg : kPos;
+        }
+        crow[f] = static_cast<int8_t>(code);
+      }
+    }
+    if (kA) {
+      asum = warp_sum(asum);
+      if (lane == 0) a.A[p] = asum / static_cast<float>(ni);
+    }
+  }
+}
+
+template <bool kTerms, bool kA, int kOp>
+cudaError_t launch_i8_t(const PackI8Args& a, bool vec, dim3 grid, cudaStream_t s) {
+  if (vec)
+    pack_i8_kernel<kTerms, kA, kOp, true><<<grid, kPackThreads, 0, s>>>(a);
+  else
+    pack_i8_kernel<kTerms, kA, kOp, false><<<grid, kPackThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <bool kTerms, bool kA>
+cudaError_t launch_i8_op(const PackI8Args& a, bool vec, dim3 grid, cudaStream_t s) {
+  return a.op == kXnor ? launch_i8_t<kTerms, kA, kXnor>(a, vec, grid, s) : launch_i8_t<kTerms, kA, kAnd>(a, vec, grid, s);
+}
+
+}  // namespace
+
+cudaError_t launch_pack_i8(const PackI8Args& a, cudaStream_t s) {
+  if (a.npix == 0) return cudaSuccess;
+  const int sms = current_sm_count();
+  int64_t blocks = ceil_div(a.npix, kPackThreads / 32);
+  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  if (blocks > cap) blocks = cap;
+  const dim3 grid(static_cast<unsigned>(blocks));
+  const bool vec = (a.ni % 4) == 0 && (reinterpret_cast<uintptr_t>(a.in) & 15) == 0;
+  if (a.in_scale) return a.A ? launch_i8_op<true, true>(a, vec, grid, s) : launch_i8_op<true, false>(a, vec, grid, s);
+  return a.A ? launch_i8_op<false, true>(a, vec, grid, s) : launch_i8_op<false, false>(a, vec, grid, s);
+}
+
+}  // namespace bconv

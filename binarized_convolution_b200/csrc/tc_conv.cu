@@ -1,0 +1,449 @@
+// Binary convolution on the 5th-generation tensor cores (tcgen05.mma kind::i8).
+//
+// What it computes (Apple page "MPSCNNBinaryConvolution", Overview, XNOR and AND bullets):
+// a product of two binarized values is +-1 (XNOR) or 0/1 (AND), so the window sum
+//   S = sum_{valid taps, f} a(x~[f]) * w[f]
+// is an exact integer dot product of int8 operands: XNOR codes a = bin(x~) in {-1,+1} and
+// w in {-1,+1}; AND codes a, w in {0,1}.  With int32 accumulation the result equals the
+// popcount form 32 - 2*popcount(x^y) (resp. popcount(x&y)) summed over the words, bit for
+// bit.  Out-of-image taps and padding channels are zero codes, which add exactly 0, so no
+// border correction is needed.  The epilogue is out = act(S * scale[c] * beta + bias[c]).
+// The fully-connected layer (page "MPSCNNFullyConnected") is the same contraction with one
+// tap spanning the flattened image.
+//
+// Structure: a persistent kernel, one CTA per SM, 6 warps.
+//   warp 0      TMA producer: per k-block, one 128-row x 128-byte activation tile (a box of
+//               Bn images x R rows x Cw columns of the int8 NHWC codes, shifted by the tap
+//               offset; out-of-image coordinates read zeros) and one BN x 128-byte weight
+//               tile, both 128-byte swizzled, into a 4-stage ring guarded by mbarriers.
+//   warp 1      allocates TMEM (two BN-column int32 accumulators) and, from one thread,
+//               issues tcgen05.mma M=128 x N=BN x K=32 per 32-byte step; tcgen05.commit frees
+//               each stage and publishes each finished accumulator.
+//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time (one TMEM lane = one output
+//               pixel), apply scale/beta/bias/neuron in fp32, stage through 128-byte
+//               swizzled shared memory, and TMA-store the box (clipped at the tensor edges).
+//               With a split reduction (the FC layer), the partial sums are instead added
+//               into an fp32 workspace by TMA reduce-add (integers below 2^24 add exactly) and
+//               a small kernel applies the epilogue.
+// Every mbarrier wait gives up after one second of %globaltimer, sets the error word and
+// makes all roles stop; TMEM is released on every exit path.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "tc_conv.cuh"
+
+namespace bconv {
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kABytes = 128 * 128;  // 128 rows x 128 bytes
+constexpr int kThreadsTc = 192;
+constexpr int kEpiThreads = 128;
+constexpr int kStageOutBytes = 128 * 128;  // 128 rows x 32 fp32
+constexpr uint64_t kTimeoutNs = 1000000000ull;
+
+struct __align__(8) Barriers {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t done;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; false after the time limit or, when
+// `follow_abort`, as soon as another role has given up (the caller then stops).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Barriers* B, uint32_t* err,
+                                          bool follow_abort = true) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try(bar, parity)) return true;
+    if (follow_abort && *reinterpret_cast<volatile uint32_t*>(&B->abort_flag)) return false;
+    if (globaltimer() - t0 > kTimeoutNs) {
+      atomicOr(err, kErrTimeout);
+      atomicExch(&B->abort_flag, 1u);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
+                                            int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
+                                                  int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void epi_barrier() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, M = 128, N and K=32 from the descriptors.
+__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 consecutive 32-bit columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tc_ld_32x32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, rows of 128 bytes with the 128-byte
+// swizzle, 8-row groups 1024 bytes apart (tile base 1024-byte aligned).
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
+  const uint32_t a = smem_u32(p);
+  uint64_t d = static_cast<uint64_t>((a & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1) << 16;          // leading byte offset (unused for this layout)
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;  // stride byte offset: 8 rows x 128 bytes
+  d |= static_cast<uint64_t>(1) << 46;          // descriptor version
+  d |= static_cast<uint64_t>(2) << 61;          // 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor: s32 accumulator, signed int8 A and B, both K-major, M=128, N=bn.
+__host__ __device__ constexpr uint32_t idesc_i8(int bn) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(bn >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+struct TileCoord {
+  int n0, oy0, ox0, ntile, split;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const TcArgs& a, int t) {
+  TileCoord c;
+  c.split = t % a.k_splits;
+  t /= a.k_splits;
+  c.ntile = t % a.n_tiles;
+  t /= a.n_tiles;
+  const int tx = t % a.tiles_x;
+  t /= a.tiles_x;
+  const int ty = t % a.tiles_y;
+  t /= a.tiles_y;
+  c.n0 = t * a.Bn;
+  c.oy0 = ty * a.R;
+  c.ox0 = tx * a.Cw;
+  return c;
+}
+
+template <bool kSplit>
+__global__ void __launch_bounds__(kThreadsTc, 1)
+    tc_conv_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmOut, const TcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte aligned base for the swizzled tiles
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int b_bytes = a.BN * 128;
+  const int stage_bytes = kABytes + b_bytes;
+  uint8_t* stage_out = smem + kStages * stage_bytes;  // 2 x 16 KB epilogue staging
+  Barriers* B = reinterpret_cast<Barriers*>(stage_out + 2 * kStageOutBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total_tiles = a.m_tiles * a.n_tiles * a.k_splits;
+  const int kb_total = a.kh * a.kw * a.kb_per_tap;
+  const int kb_per_split = (kb_total + a.k_splits - 1) / a.k_splits;
+  const uint32_t tmem_cols = a.tmem_cols;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&B->full[s], 1);
+      mbar_init(&B->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&B->tmem_full[b], 1);
+      mbar_init(&B->tmem_empty[b], kEpiThreads / 32);
+    }
+    mbar_init(&B->done, 1);
+    B->abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&B->tmem_base)),
+                 "r"(tmem_cols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = B->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = tile_coord(a, t);
+        const int kb0 = tc.split * kb_per_split;
+        const int kb1 = min(kb0 + kb_per_split, kb_total);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&B->empty[stage], phase ^ 1u, B, a.err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * stage_bytes;
+          uint8_t* sb = sa + kABytes;
+          mbar_expect_tx(&B->full[stage], static_cast<uint32_t>(stage_bytes));
+          const int tap = kb / a.kb_per_tap, cb = kb - tap * a.kb_per_tap;
+          const int ky = tap / a.kw, kx = tap - ky * a.kw;
+          tma_load_4d(sa, &tmA, &B->full[stage], cb * 128, tc.ox0 + kx - a.kw / 2, tc.oy0 + ky - a.kh / 2, tc.n0);
+          tma_load_2d(sb, &tmB, &B->full[stage], kb * 128, tc.ntile * a.BN);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      const uint32_t idesc = idesc_i8(a.BN);
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = tile_coord(a, t);
+        const int kb0 = tc.split * kb_per_split;
+        const int kb1 = min(kb0 + kb_per_split, kb_total);
+        if (!mbar_wait(&B->tmem_empty[acc], acc_phase ^ 1u, B, a.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&B->full[stage], phase, B, a.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint8_t* sa = smem + stage * stage_bytes;
+          const uint64_t da = smem_desc_sw128(sa), db = smem_desc_sw128(sa + kABytes);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)  // four K=32 steps across the 128-byte row
+            tc_mma_i8(d_tmem, da + 2u * j, db + 2u * j, idesc, (kb > kb0 || j > 0) ? 1u : 0u);
+          tc_commit(&B->empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&B->tmem_full[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      // all MMAs issued by this thread have completed once `done` fires (waited even after an
+      // abort, so that TMEM is never released under a running MMA)
+      tc_commit(&B->done);
+      mbar_wait(&B->done, 0, B, a.err, false);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    const int et = threadIdx.x - 64;  // 0..127 within the epilogue group
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int chunk_count = 0;
+    const int rc = a.R * a.Cw;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+      const TileCoord tc = tile_coord(a, t);
+      if (!mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err)) break;
+      tc_fence_after();
+      const int n = tc.n0 + row / rc, oy = tc.oy0 + (row / a.Cw) % a.R, ox = tc.ox0 + row % a.Cw;
+      const bool valid = n < a.N && oy < a.Ho && ox < a.Wo;
+      float beta = 1.f;
+      if (!kSplit && a.beta && valid) beta = __ldg(a.beta + (static_cast<int64_t>(n) * a.Ho + oy) * a.Wo + ox);
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
+      for (int ch = 0; ch < a.BN / 32; ++ch) {
+        uint32_t v[32];
+        tc_ld_32x32(tbase + static_cast<uint32_t>(ch * 32), v);
+        if (ch == a.BN / 32 - 1) {  // accumulator fully read: hand it back to the MMA warp
+          tc_fence_before();
+          if (lane == 0) mbar_arrive(&B->tmem_empty[acc]);
+        }
+        const int buf = chunk_count & 1;
+        ++chunk_count;
+        uint8_t* so = stage_out + buf * kStageOutBytes;
+        epi_barrier();  // the store that last read `so` has finished (waited below by et 0)
+        const int c0 = tc.ntile * a.BN + ch * 32;
+        float y[32];
+        if (kSplit) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) y[j] = static_cast<float>(static_cast<int32_t>(v[j]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int c = c0 + j;
+            const float sc = c < a.No ? __ldg(a.scale + c) : 0.f;
+            const float bi = c < a.No ? __ldg(a.bias + c) : 0.f;
+            const float s = static_cast<float>(static_cast<int32_t>(v[j]));
+            float r = a.beta ? fmaf(s * sc, beta, bi) : fmaf(s, sc, bi);
+            if (a.relu) r = fmaxf(r, 0.f);
+            y[j] = r;
+          }
+        }
+        // 128-byte swizzled row: 16-byte chunk k of row r lives at chunk k ^ (r % 8)
+        float4* orow = reinterpret_cast<float4*>(so + row * 128);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          orow[k ^ (row & 7)] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
+        fence_proxy_async();
+        epi_barrier();
+        if (et == 0) {
+          if (c0 < a.No) {  // a box past the last channel would write nothing; skip it
+            if (kSplit)
+              tma_reduce_add_4d(&tmOut, so, c0, tc.ox0, tc.oy0, tc.n0);
+            else
+              tma_store_4d(&tmOut, so, c0, tc.ox0, tc.oy0, tc.n0);
+          }
+          bulk_commit();  // one group per chunk (possibly empty) keeps the buffer accounting
+          bulk_wait_read_1();
+        }
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (et == 0) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(tmem_cols));
+  }
+}
+
+// y = act(S * scale[c] * beta[n] + bias[c]) over the fp32 partial-sum workspace [N][No].
+__global__ void tc_finalize_kernel(const float* __restrict__ ws, float* __restrict__ out, const float* __restrict__ scale,
+                                   const float* __restrict__ bias, const float* __restrict__ beta, int64_t total, int no,
+                                   int rows_per_beta, int relu) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= total) return;
+  const int c = static_cast<int>(i % no);
+  const float s = ws[i];
+  float r = beta ? fmaf(s * __ldg(scale + c), __ldg(beta + (i / no) / rows_per_beta), __ldg(bias + c))
+                 : fmaf(s, __ldg(scale + c), __ldg(bias + c));
+  if (relu) r = fmaxf(r, 0.f);
+  out[i] = r;
+}
+
+}  // namespace
+
+int tc_smem_bytes(int bn) { return kStages * (kABytes + bn * 128) + 2 * kStageOutBytes + 256 + 1024; }
+
+cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmOut, const TcArgs& a,
+                           cudaStream_t s) {
+  const int smem = tc_smem_bytes(a.BN);
+  const int total_tiles = a.m_tiles * a.n_tiles * a.k_splits;
+  if (total_tiles == 0) return cudaSuccess;
+  int grid = current_sm_count();
+  if (grid > total_tiles) grid = total_tiles;
+  cudaError_t e;
+  if (a.k_splits > 1) {
+    e = cudaFuncSetAttribute(tc_conv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    tc_conv_kernel<true><<<grid, kThreadsTc, smem, s>>>(*tmA, *tmB, *tmOut, a);
+  } else {
+    e = cudaFuncSetAttribute(tc_conv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    tc_conv_kernel<false><<<grid, kThreadsTc, smem, s>>>(*tmA, *tmB, *tmOut, a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc_finalize(const float* ws, float* out, const float* scale, const float* bias, const float* beta,
+                               int64_t total, int no, int rows_per_beta, int relu, cudaStream_t s) {
+  if (total == 0) return cudaSuccess;
+  tc_finalize_kernel<<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(ws, out, scale, bias, beta, total, no,
+                                                                                 rows_per_beta, relu);
+  return cudaGetLastError();
+}
+
+}  // namespace bconv

@@ -87,6 +87,9 @@ class BinaryConv2d(_Layer):
     def launches_per_forward(self) -> int:
         return nat.bconv_launches_per_forward(self.handle)
 
+    def effective_algo(self) -> int:
+        return nat.bconv_effective_algo(self.handle)
+
     def forward_into(self, x, out):
         import torch
 
@@ -147,6 +150,9 @@ class BinaryFC(_Layer):
 
     def launches_per_forward(self) -> int:
         return nat.bfc_launches_per_forward(self.handle)
+
+    def effective_algo(self) -> int:
+        return nat.bfc_effective_algo(self.handle)
 
     def forward_into(self, x, out):
         import torch

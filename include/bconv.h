@@ -71,7 +71,10 @@ typedef enum { BCONV_NEURON_NONE = 0, BCONV_NEURON_RELU = 1 } bconv_neuron_t;
 typedef enum {
   BCONV_ALGO_AUTO = 0,
   BCONV_ALGO_POPC = 1,     /* XNOR/AND: LOP3 XOR/AND + POPC into int32 registers     */
-  BCONV_ALGO_SIMT_F32 = 2  /* binaryWeights: FP32 signed-add contraction on the SIMT */
+  BCONV_ALGO_SIMT_F32 = 2, /* binaryWeights: FP32 signed-add contraction on the SIMT */
+  BCONV_ALGO_TCGEN05 = 3   /* XNOR/AND: +-1 / {0,1} int8 codes on the tcgen05 tensor
+                              cores, int32 accumulation in TMEM (stride 1 or the FC, and
+                              out_channels % 4 == 0); exact, like the POPC family */
 } bconv_algo_t;
 
 /*
@@ -139,6 +142,9 @@ bconv_status_t bconv_set_algo(bconv_handle_t h, bconv_algo_t algo);
 /* Kernel launches one bconv_forward makes with the current settings. */
 int32_t bconv_launches_per_forward(bconv_handle_t h);
 
+/* The kernel family (BCONV_ALGO_*, never AUTO) the next forward will use; -1 for a bad handle. */
+int32_t bconv_effective_algo(bconv_handle_t h);
+
 /*
  * Wait for `stream`, then read and clear the handle's device error word.  Returns OK,
  * TIMEOUT (a kernel gave up a bounded wait), or CUDA (a pending CUDA error).
@@ -187,6 +193,7 @@ int32_t bfc_input_feature_channels(bfc_handle_t h);
 int32_t bfc_output_feature_channels(bfc_handle_t h);
 bconv_status_t bfc_set_algo(bfc_handle_t h, bconv_algo_t algo);
 int32_t bfc_launches_per_forward(bfc_handle_t h);
+int32_t bfc_effective_algo(bfc_handle_t h);
 bconv_status_t bfc_sync_status(bfc_handle_t h, struct CUstream_st* stream);
 bconv_status_t bfc_profile_begin(bfc_handle_t h, int32_t max_launches);
 bconv_status_t bfc_profile_end(bfc_handle_t h, float* total_ms, int32_t* launches);

@@ -43,6 +43,18 @@ def make_layer(w: synth.Workload, inp: synth.Inputs, *, sums: bool = False):
                         (w.stride_y, w.stride_x), wbits=inp.wbits, **kw)
 
 
+def algo_for(w: synth.Workload, name: str):
+    """Library algorithm code for a test parameter: 'auto', or 'popc' (XNOR/AND only; None
+    for binaryWeights, which has one kernel family)."""
+    import binarized_convolution_b200 as bc
+
+    if name == "auto":
+        return bc.ALGO_AUTO
+    if w.op == synth.BINARY_WEIGHTS:
+        return None
+    return bc.ALGO_POPC
+
+
 def run_device(w: synth.Workload, inp: synth.Inputs, *, sums: bool = False, algo=None):
     """Output of the library, as float32 [rows, No] (rows = output pixels or images)."""
     import torch

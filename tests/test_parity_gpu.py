@@ -41,13 +41,17 @@ MEDIUM = [
 ]
 
 
+@pytest.mark.parametrize("algo", ["auto", "popc"])
 @pytest.mark.parametrize("w", MEDIUM, ids=lambda w: w.name)
-def test_medium_all_outputs(w, cuda_device):
+def test_medium_all_outputs(w, algo, cuda_device):
+    a = pu.algo_for(w, algo)
+    if a is None:
+        pytest.skip("binaryWeights has a single kernel family")
     inp = synth.make_inputs(w)
     S_ref, beta_ref, y_ref = pu.run_oracle(w, inp)
-    y = pu.run_device(w, inp)
+    y = pu.run_device(w, inp, algo=a)
     pu.assert_outputs_close(w, inp, y, S_ref, beta_ref, y_ref)
-    S_dev = pu.run_device(w, inp, sums=True)
+    S_dev = pu.run_device(w, inp, sums=True, algo=a)
     S_sum, _, _ = pu.run_oracle(w, inp, sums=True)
     if w.op == synth.BINARY_WEIGHTS:
         pu.assert_outputs_close(w, synth.Inputs(inp.x, inp.wbits, np.ones_like(inp.scale),
@@ -57,16 +61,20 @@ def test_medium_all_outputs(w, cuda_device):
         pu.assert_sums_exact(S_dev, S_sum)
 
 
+@pytest.mark.parametrize("algo", ["auto", "popc"])
 @pytest.mark.parametrize("idx", range(5), ids=lambda i: synth.WORKLOAD_ORDER[i])
-def test_workload_full_size(idx, cuda_device):
+def test_workload_full_size(idx, algo, cuda_device):
     w = synth.workload(idx)
+    a = pu.algo_for(w, algo)
+    if a is None:
+        pytest.skip("binaryWeights has a single kernel family")
     inp = synth.make_inputs(w)
     rows = pu.sample_rows(w, seed=idx)
-    y = pu.run_device(w, inp)
+    y = pu.run_device(w, inp, algo=a)
     S_ref, beta_ref, y_ref = pu.run_oracle(w, inp, rows=rows)
     pu.assert_outputs_close(w, inp, y[rows], S_ref, beta_ref, y_ref, rows=rows)
 
-    S_dev = pu.run_device(w, inp, sums=True)
+    S_dev = pu.run_device(w, inp, sums=True, algo=a)
     S_sum, _, _ = pu.run_oracle(w, inp, rows=rows, sums=True)
     if w.op == synth.BINARY_WEIGHTS:
         ones = synth.Inputs(inp.x, inp.wbits, np.ones_like(inp.scale), np.zeros_like(inp.bias), inp.in_scale,
