@@ -124,7 +124,7 @@ struct Layer {
   int8_t* wq = nullptr;
   float* ws = nullptr;  // FC split-K partial sums [N][No]
   TcArgs tc{};
-  CUtensorMap tmA{}, tmB{}, tmWs{}, tmOut{};
+  CUtensorMap tmA{}, tmB{}, tmBp{}, tmWs{}, tmOut{};
   const float* tm_out_ptr = nullptr;
   // host-buffer forward staging (allocated on first use)
   float *stage_in = nullptr, *stage_out = nullptr;
@@ -220,11 +220,14 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   const int taps = L.kh * L.kw;
   L.cip = round_up(L.Ni, 128);
   TcArgs& t = L.tc;
-  t.BN = std::min(256, round_up(L.No, 32));
+  // The FC keeps a batch of up to 256 images in one CTA tile (two 128-row sub-tiles sharing
+  // every weight stage), so its large weight matrix streams from memory once.
+  t.mt = (L.fc && L.N > 128) ? 2 : 1;
+  t.BN = std::min(t.mt == 2 ? 128 : 256, round_up(L.No, 32));
   t.n_tiles = (L.No + t.BN - 1) / t.BN;
   t.No = L.No;
   t.N = L.N;
-  t.tmem_cols = static_cast<uint32_t>(std::max(32, next_pow2(2 * t.BN)));
+  t.tmem_cols = static_cast<uint32_t>(std::max(32, next_pow2(2 * t.mt * t.BN)));
   t.relu = L.relu;
   t.err = L.err;
   t.scale = L.scale;
@@ -243,7 +246,7 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
     t.tiles_x = (L.Wo + t.Cw - 1) / t.Cw;
     t.tiles_y = (L.Ho + t.R - 1) / t.R;
   }
-  t.m_tiles = t.tiles_x * t.tiles_y * ((L.N + t.Bn - 1) / t.Bn);
+  t.m_tiles = t.tiles_x * t.tiles_y * ((L.N + t.Bn * t.mt - 1) / (t.Bn * t.mt));
   const int kb_total = t.kh * t.kw * t.kb_per_tap;
   t.k_splits = 1;
   if (L.fc) {  // spread the reduction so that the tiles fill the GPU
@@ -295,6 +298,10 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   }
   ok = ok && encode_2d(&L.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(kt),
                        static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128, static_cast<uint32_t>(t.BN));
+  tc_plan(t, current_sm_count());  // work list for this device: tail tiles cut along N
+  ok = ok && encode_2d(&L.tmBp, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(kt),
+                       static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128,
+                       static_cast<uint32_t>(t.BN / t.pieces));
   if (ok && t.k_splits > 1) ok = encode_out_map(L, &L.tmWs, L.ws);
   if (!ok) return BCONV_OK;  // the POPC path stays available
   L.tc_ok = true;
@@ -436,13 +443,16 @@ bconv_status_t run_forward_tc(Layer& L, const float* in, float* out, cudaStream_
   p.op = L.type;
   cudaError_t e = launch_pack_i8(p, s);
   if (e != cudaSuccess) return from_cuda(e);
-  if (beta) {
+  if (beta && L.fc) {  // the convolution forms beta from A inside its epilogue
     BetaArgs b{L.A, L.beta, L.N, L.H, L.W, L.Ho, L.Wo, L.kh, L.kw, L.sy, L.sx};
-    e = L.fc ? launch_beta_image_mean(b, s) : launch_beta_conv(b, s);
+    e = launch_beta_image_mean(b, s);
     if (e != cudaSuccess) return from_cuda(e);
   }
   TcArgs t = L.tc;
   t.beta = beta ? L.beta : nullptr;
+  t.A = (beta && !L.fc) ? L.A : nullptr;
+  t.H = L.H;
+  t.W = L.W;
   const CUtensorMap* om = &L.tmWs;
   if (t.k_splits > 1) {
     e = cudaMemsetAsync(L.ws, 0, sizeof(float) * static_cast<size_t>(L.N) * L.No, s);
@@ -456,7 +466,7 @@ bconv_status_t run_forward_tc(Layer& L, const float* in, float* out, cudaStream_
   }
   const bool timed = L.prof.active && L.prof.used < static_cast<int>(L.prof.start.size());
   if (timed) cudaEventRecord(L.prof.start[L.prof.used], s);
-  e = launch_tc_conv(&L.tmA, &L.tmB, om, t, s);
+  e = launch_tc_conv(&L.tmA, &L.tmB, &L.tmBp, om, t, s);
   if (timed) cudaEventRecord(L.prof.stop[L.prof.used++], s);
   if (e != cudaSuccess) return from_cuda(e);
   if (t.k_splits > 1)
@@ -572,7 +582,7 @@ bconv_status_t sync_status(Layer& L, cudaStream_t s) {
   if (word) {
     cudaMemset(L.err, 0, sizeof(uint32_t));
     if (word & kErrTimeout) return BCONV_ERR_TIMEOUT;
-    return BCONV_ERR_CUDA;
+    return BCONV_ERR_CUDA;  // kErrLayout: a kernel refused an unexpected shared-memory layout
   }
   return BCONV_OK;
 }
@@ -599,7 +609,8 @@ bconv_status_t set_algo(Layer& L, int algo) {
 }
 
 int launches_per_forward(const Layer& L) {
-  if (L.N > 0 && use_tc(L)) return 2 + (L.use_beta() ? 1 : 0) + (L.tc.k_splits > 1 ? 2 : 0);  // memset counted
+  if (L.N > 0 && use_tc(L))  // pack, contraction; the FC adds beta, memset and finalize
+    return 2 + ((L.fc && L.use_beta()) ? 1 : 0) + (L.tc.k_splits > 1 ? 2 : 0);
   int n = 1;  // contraction
   if (L.type != kBinaryWeights || L.use_beta()) n += 1;  // pack
   if (L.use_beta()) n += 1;                              // beta

@@ -9,7 +9,7 @@ namespace bconv {
 enum Op : int { kBinaryWeights = 0, kXnor = 1, kAnd = 2 };
 
 // Error word bits the kernels may set (read by *_sync_status).
-enum : uint32_t { kErrTimeout = 1u };
+enum : uint32_t { kErrTimeout = 1u, kErrLayout = 2u };
 
 constexpr int kWordBits = 32;
 // Words per pixel are padded to this many (32 bytes) so that a pixel's words start on a

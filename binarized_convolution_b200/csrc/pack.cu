@@ -105,48 +105,117 @@ cudaError_t launch_pack(const PackArgs& a, cudaStream_t s) {
 namespace bconv {
 namespace {
 
-template <bool kTerms, bool kA, int kOp, bool kVec>
-__global__ void __launch_bounds__(kPackThreads) pack_i8_kernel(PackI8Args a) {
+// Codes for 4 transformed values as one little-endian word.
+template <int kOp>
+__device__ __forceinline__ uint32_t codes4(const float4& v) {
+  constexpr uint32_t kPos = 0x01u;
+  constexpr uint32_t kNeg = kOp == kXnor ? 0xFFu : 0x00u;
+  return ((v.x < 0.f) ? kNeg : kPos) | (((v.y < 0.f) ? kNeg : kPos) << 8) | (((v.z < 0.f) ? kNeg : kPos) << 16) |
+         (((v.w < 0.f) ? kNeg : kPos) << 24);
+}
+
+template <bool kTerms>
+__device__ __forceinline__ float4 transform4(float4 v, const float* __restrict__ sc, const float* __restrict__ bi,
+                                             int f) {
+  if (kTerms) {
+    const float4 s = __ldg(reinterpret_cast<const float4*>(sc + f));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(bi + f));
+    v.x = fmaf(v.x, s.x, b.x);
+    v.y = fmaf(v.y, s.y, b.y);
+    v.z = fmaf(v.z, s.z, b.z);
+    v.w = fmaf(v.w, s.w, b.w);
+  }
+  return v;
+}
+
+// Vector path: kC chunks of 128 channels per pixel (a compile-time 1, 2 or 4), a group of
+// 8 / kC pixels per warp step with all 8 float4 loads per lane issued before any is used.
+// Lane l always handles channels chunk*128 + 4l .. 4l+3, so its input terms stay in registers.
+template <bool kTerms, bool kA, int kOp, int kC>
+__global__ void __launch_bounds__(kPackThreads, 3) pack_i8_vec_kernel(PackI8Args a) {
+  constexpr int kG = 8 / kC;  // pixels per warp step
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kPackThreads) >> 5;
   const int ni = a.ni;
-  constexpr uint32_t kPos = kOp == kXnor ? 0x01u : 0x01u;
+  const float* __restrict__ in = a.in;
+  int8_t* __restrict__ codes = a.codes;
+  float4 sc[kC], bi[kC];
+  bool live[kC];
+#pragma unroll
+  for (int c = 0; c < kC; ++c) {
+    const int f = c * 128 + lane * 4;
+    live[c] = f < ni;
+    sc[c] = make_float4(1.f, 1.f, 1.f, 1.f);
+    bi[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (kTerms && live[c]) {
+      sc[c] = __ldg(reinterpret_cast<const float4*>(a.in_scale + f));
+      bi[c] = __ldg(reinterpret_cast<const float4*>(a.in_bias + f));
+    }
+  }
+  for (int64_t p0 = warp * kG; p0 < a.npix; p0 += nwarps * kG) {
+    float4 v[kG][kC];
+#pragma unroll
+    for (int g = 0; g < kG; ++g)
+#pragma unroll
+      for (int c = 0; c < kC; ++c) {
+        const int64_t p = p0 + g;
+        v[g][c] = (p < a.npix && live[c])
+                      ? __ldcs(reinterpret_cast<const float4*>(in + p * ni + c * 128 + lane * 4))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+    for (int g = 0; g < kG; ++g) {
+      const int64_t p = p0 + g;
+      if (p >= a.npix) break;  // warp-uniform
+      float asum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kC; ++c) {
+        uint32_t word = 0u;
+        if (live[c]) {
+          float4 t = v[g][c];
+          if (kTerms) {
+            t.x = fmaf(t.x, sc[c].x, bi[c].x);
+            t.y = fmaf(t.y, sc[c].y, bi[c].y);
+            t.z = fmaf(t.z, sc[c].z, bi[c].z);
+            t.w = fmaf(t.w, sc[c].w, bi[c].w);
+          }
+          if (kA) asum += (fabsf(t.x) + fabsf(t.y)) + (fabsf(t.z) + fabsf(t.w));
+          word = codes4<kOp>(t);
+        }
+        *reinterpret_cast<uint32_t*>(codes + p * a.cip + c * 128 + lane * 4) = word;
+      }
+      if (kA) {
+        asum = warp_sum(asum);
+        if (lane == 0) a.A[p] = asum / static_cast<float>(ni);
+      }
+    }
+  }
+}
+
+// Any channel count: one byte per lane per step.
+template <bool kTerms, bool kA, int kOp>
+__global__ void __launch_bounds__(kPackThreads) pack_i8_scalar_kernel(PackI8Args a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kPackThreads) >> 5;
+  const int ni = a.ni;
+  constexpr uint32_t kPos = 0x01u;
   constexpr uint32_t kNeg = kOp == kXnor ? 0xFFu : 0x00u;
   for (int64_t p = warp; p < a.npix; p += nwarps) {
     const float* row = a.in + p * ni;
     int8_t* crow = a.codes + p * a.cip;
     float asum = 0.f;
-    if constexpr (kVec) {
-      for (int f0 = 0; f0 < a.cip; f0 += 128) {
-        const int f = f0 + lane * 4;
-        uint32_t word = 0u;
-        if (f < ni) {
-          float4 v = __ldcs(reinterpret_cast<const float4*>(row + f));
-          if (kTerms) {
-            v.x = fmaf(v.x, __ldg(a.in_scale + f + 0), __ldg(a.in_bias + f + 0));
-            v.y = fmaf(v.y, __ldg(a.in_scale + f + 1), __ldg(a.in_bias + f + 1));
-            v.z = fmaf(v.z, __ldg(a.in_scale + f + 2), __ldg(a.in_bias + f + 2));
-            v.w = fmaf(v.w, __ldg(a.in_scale + f + 3), __ldg(a.in_bias + f + 3));
-          }
-          if (kA) asum += (fabsf(v.x) + fabsf(v.y)) + (fabsf(v.z) + fabsf(v.w));
-          word = ((v.x < 0.f) ? kNeg : kPos) | (((v.y < 0.f) ? kNeg : kPos) << 8) |
-                 (((v.z < 0.f) ? kNeg : kPos) << 16) | (((v.w < 0.f) ? kNeg : kPos) << 24);
-        }
-        *reinterpret_cast<uint32_t*>(crow + f) = word;
+    for (int f0 = 0; f0 < a.cip; f0 += 32) {
+      const int f = f0 + lane;
+      uint32_t code = 0u;
+      if (f < ni) {
+        float v = __ldcs(row + f);
+        if (kTerms) v = fmaf(v, __ldg(a.in_scale + f), __ldg(a.in_bias + f));
+        if (kA) asum += fabsf(v);
+        code = (v < 0.f) ? kNeg : kPos;
       }
-    } else {
-      for (int f0 = 0; f0 < a.cip; f0 += 32) {
-        const int f = f0 + lane;
-        uint32_t code = 0u;
-        if (f < ni) {
-          float v = __ldcs(row + f);
-          if (kTerms) v = fmaf(v, __ldg(a.in_scale + f), __ldg(a.in_bias + f));
-          if (kA) asum += fabsf(v);
-          code = (v < 0.f) ? kNeg : kPos;
-        }
-        crow[f] = static_cast<int8_t>(code);
-      }
+      crow[f] = static_cast<int8_t>(code);
     }
     if (kA) {
       asum = warp_sum(asum);
@@ -156,17 +225,22 @@ __global__ void __launch_bounds__(kPackThreads) pack_i8_kernel(PackI8Args a) {
 }
 
 template <bool kTerms, bool kA, int kOp>
-cudaError_t launch_i8_t(const PackI8Args& a, bool vec, dim3 grid, cudaStream_t s) {
-  if (vec)
-    pack_i8_kernel<kTerms, kA, kOp, true><<<grid, kPackThreads, 0, s>>>(a);
+cudaError_t launch_i8_t(const PackI8Args& a, int chunks, dim3 grid, cudaStream_t s) {
+  if (chunks == 1)
+    pack_i8_vec_kernel<kTerms, kA, kOp, 1><<<grid, kPackThreads, 0, s>>>(a);
+  else if (chunks == 2)
+    pack_i8_vec_kernel<kTerms, kA, kOp, 2><<<grid, kPackThreads, 0, s>>>(a);
+  else if (chunks == 4)
+    pack_i8_vec_kernel<kTerms, kA, kOp, 4><<<grid, kPackThreads, 0, s>>>(a);
   else
-    pack_i8_kernel<kTerms, kA, kOp, false><<<grid, kPackThreads, 0, s>>>(a);
+    pack_i8_scalar_kernel<kTerms, kA, kOp><<<grid, kPackThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
 template <bool kTerms, bool kA>
-cudaError_t launch_i8_op(const PackI8Args& a, bool vec, dim3 grid, cudaStream_t s) {
-  return a.op == kXnor ? launch_i8_t<kTerms, kA, kXnor>(a, vec, grid, s) : launch_i8_t<kTerms, kA, kAnd>(a, vec, grid, s);
+cudaError_t launch_i8_op(const PackI8Args& a, int chunks, dim3 grid, cudaStream_t s) {
+  return a.op == kXnor ? launch_i8_t<kTerms, kA, kXnor>(a, chunks, grid, s)
+                       : launch_i8_t<kTerms, kA, kAnd>(a, chunks, grid, s);
 }
 
 }  // namespace
@@ -174,13 +248,16 @@ cudaError_t launch_i8_op(const PackI8Args& a, bool vec, dim3 grid, cudaStream_t 
 cudaError_t launch_pack_i8(const PackI8Args& a, cudaStream_t s) {
   if (a.npix == 0) return cudaSuccess;
   const int sms = current_sm_count();
+  const bool vec = (a.ni % 4) == 0 && (reinterpret_cast<uintptr_t>(a.in) & 15) == 0 &&
+                   (!a.in_scale || ((reinterpret_cast<uintptr_t>(a.in_scale) | reinterpret_cast<uintptr_t>(a.in_bias)) & 15) == 0);
+  const int chunks = vec ? a.cip / 128 : 0;  // 1, 2, 4 -> vector kernel; anything else -> scalar
   int64_t blocks = ceil_div(a.npix, kPackThreads / 32);
-  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  const int64_t cap = static_cast<int64_t>(sms) * 3;  // one wave at 3 CTAs per SM
   if (blocks > cap) blocks = cap;
   const dim3 grid(static_cast<unsigned>(blocks));
-  const bool vec = (a.ni % 4) == 0 && (reinterpret_cast<uintptr_t>(a.in) & 15) == 0;
-  if (a.in_scale) return a.A ? launch_i8_op<true, true>(a, vec, grid, s) : launch_i8_op<true, false>(a, vec, grid, s);
-  return a.A ? launch_i8_op<false, true>(a, vec, grid, s) : launch_i8_op<false, false>(a, vec, grid, s);
+  if (a.in_scale)
+    return a.A ? launch_i8_op<true, true>(a, chunks, grid, s) : launch_i8_op<true, false>(a, chunks, grid, s);
+  return a.A ? launch_i8_op<false, true>(a, chunks, grid, s) : launch_i8_op<false, false>(a, chunks, grid, s);
 }
 
 }  // namespace bconv

@@ -50,6 +50,7 @@ struct __align__(8) Barriers {
   uint64_t done;
   uint32_t tmem_base;
   uint32_t abort_flag;
+  float2 sb[256];  // (scale, bias) of the tile's output channels
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -191,10 +192,20 @@ __host__ __device__ constexpr uint32_t idesc_i8(int bn) {
 
 struct TileCoord {
   int n0, oy0, ox0, ntile, split;
+  int noff, bn;  // output channels [ntile*BN + noff, + bn) of this work item
 };
 
-__device__ __forceinline__ TileCoord tile_coord(const TcArgs& a, int t) {
+__device__ __forceinline__ TileCoord tile_coord(const TcArgs& a, int w) {
   TileCoord c;
+  int t = w;
+  c.noff = 0;
+  c.bn = a.BN;
+  if (w >= a.full_tiles) {  // a piece of a tail tile
+    const int i = w - a.full_tiles;
+    t = a.full_tiles + i / a.pieces;
+    c.bn = a.BN / a.pieces;
+    c.noff = (i % a.pieces) * c.bn;
+  }
   c.split = t % a.k_splits;
   t /= a.k_splits;
   c.ntile = t % a.n_tiles;
@@ -203,7 +214,7 @@ __device__ __forceinline__ TileCoord tile_coord(const TcArgs& a, int t) {
   t /= a.tiles_x;
   const int ty = t % a.tiles_y;
   t /= a.tiles_y;
-  c.n0 = t * a.Bn;
+  c.n0 = t * a.Bn * a.mt;
   c.oy0 = ty * a.R;
   c.ox0 = tx * a.Cw;
   return c;
@@ -212,17 +223,25 @@ __device__ __forceinline__ TileCoord tile_coord(const TcArgs& a, int t) {
 template <bool kSplit>
 __global__ void __launch_bounds__(kThreadsTc, 1)
     tc_conv_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmOut, const TcArgs a) {
+                   const __grid_constant__ CUtensorMap tmBp, const __grid_constant__ CUtensorMap tmOut,
+                   const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // 1024-byte aligned base for the swizzled tiles
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // The swizzled tiles need a 1024-byte aligned base, which the dynamic shared window has
+  // when the kernel declares no static shared memory; anything else is refused before any
+  // barrier, copy or TMEM allocation happens.
+  if ((smem_u32(smem_raw) & 1023u) != 0u) {
+    if (threadIdx.x == 0) atomicOr(a.err, kErrLayout);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   const int b_bytes = a.BN * 128;
-  const int stage_bytes = kABytes + b_bytes;
+  const int a_bytes = a.mt * kABytes;
+  const int stage_bytes = a_bytes + b_bytes;
   uint8_t* stage_out = smem + kStages * stage_bytes;  // 2 x 16 KB epilogue staging
   Barriers* B = reinterpret_cast<Barriers*>(stage_out + 2 * kStageOutBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int total_tiles = a.m_tiles * a.n_tiles * a.k_splits;
+  const int total_tiles = a.full_tiles + (a.m_tiles * a.n_tiles * a.k_splits - a.full_tiles) * a.pieces;
   const int kb_total = a.kh * a.kw * a.kb_per_tap;
   const int kb_per_split = (kb_total + a.k_splits - 1) / a.k_splits;
   const uint32_t tmem_cols = a.tmem_cols;
@@ -266,12 +285,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             break;
           }
           uint8_t* sa = smem + stage * stage_bytes;
-          uint8_t* sb = sa + kABytes;
-          mbar_expect_tx(&B->full[stage], static_cast<uint32_t>(stage_bytes));
+          uint8_t* sb = sa + a_bytes;
+          mbar_expect_tx(&B->full[stage], static_cast<uint32_t>(a_bytes + tc.bn * 128));
           const int tap = kb / a.kb_per_tap, cb = kb - tap * a.kb_per_tap;
           const int ky = tap / a.kw, kx = tap - ky * a.kw;
-          tma_load_4d(sa, &tmA, &B->full[stage], cb * 128, tc.ox0 + kx - a.kw / 2, tc.oy0 + ky - a.kh / 2, tc.n0);
-          tma_load_2d(sb, &tmB, &B->full[stage], kb * 128, tc.ntile * a.BN);
+          for (int h = 0; h < a.mt; ++h)
+            tma_load_4d(sa + h * kABytes, &tmA, &B->full[stage], cb * 128, tc.ox0 + kx - a.kw / 2,
+                        tc.oy0 + ky - a.kh / 2, tc.n0 + h * a.Bn);
+          if (tc.bn == a.BN)
+            tma_load_2d(sb, &tmB, &B->full[stage], kb * 128, tc.ntile * a.BN);
+          else
+            tma_load_2d(sb, &tmBp, &B->full[stage], kb * 128, tc.ntile * a.BN + tc.noff);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
@@ -287,14 +311,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      const uint32_t idesc = idesc_i8(a.BN);
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
         const TileCoord tc = tile_coord(a, t);
+        const uint32_t idesc = idesc_i8(tc.bn);
         const int kb0 = tc.split * kb_per_split;
         const int kb1 = min(kb0 + kb_per_split, kb_total);
         if (!mbar_wait(&B->tmem_empty[acc], acc_phase ^ 1u, B, a.err)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.mt * a.BN);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&B->full[stage], phase, B, a.err)) {
             ok = false;
@@ -302,10 +326,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           }
           tc_fence_after();
           uint8_t* sa = smem + stage * stage_bytes;
-          const uint64_t da = smem_desc_sw128(sa), db = smem_desc_sw128(sa + kABytes);
+          const uint64_t db = smem_desc_sw128(sa + a_bytes);
+          for (int h = 0; h < a.mt; ++h) {
+            const uint64_t da = smem_desc_sw128(sa + h * kABytes);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)  // four K=32 steps across the 128-byte row
-            tc_mma_i8(d_tmem, da + 2u * j, db + 2u * j, idesc, (kb > kb0 || j > 0) ? 1u : 0u);
+            for (int j = 0; j < 4; ++j)  // four K=32 steps across the 128-byte row
+              tc_mma_i8(d_tmem + static_cast<uint32_t>(h * a.BN), da + 2u * j, db + 2u * j, idesc,
+                        (kb > kb0 || j > 0) ? 1u : 0u);
+          }
           tc_commit(&B->empty[stage]);
           if (++stage == kStages) {
             stage = 0;
@@ -330,60 +358,100 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     int chunk_count = 0;
+    int loaded_ntile = -1;
     const int rc = a.R * a.Cw;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       const TileCoord tc = tile_coord(a, t);
+      if (!kSplit && tc.ntile != loaded_ntile) {  // this tile's (scale, bias) into shared memory
+        epi_barrier();
+        for (int j = et; j < a.BN; j += kEpiThreads) {
+          const int c = tc.ntile * a.BN + j;
+          B->sb[j] = c < a.No ? make_float2(__ldg(a.scale + c), __ldg(a.bias + c)) : make_float2(0.f, 0.f);
+        }
+        epi_barrier();
+        loaded_ntile = tc.ntile;
+      }
+      // beta of this thread's row in each sub-tile, formed before the accumulator is ready
+      const bool has_beta = a.A != nullptr || a.beta != nullptr;
+      float beta_h[2] = {1.f, 1.f};
+      for (int h = 0; h < a.mt; ++h) {
+        const int n = tc.n0 + h * a.Bn + row / rc, oy = tc.oy0 + (row / a.Cw) % a.R, ox = tc.ox0 + row % a.Cw;
+        const bool valid = n < a.N && oy < a.Ho && ox < a.Wo;
+        if (kSplit || !valid) continue;
+        if (a.A) {
+          // beta = sum of A over the in-image window / (kh*kw), in the order of the beta kernel
+          const float* An = a.A + static_cast<int64_t>(n) * a.H * a.W;
+          float s = 0.f;
+          for (int dy = -(a.kh / 2); dy <= (a.kh - 1) / 2; ++dy) {
+            const int y = oy + dy;
+            if (y < 0 || y >= a.H) continue;
+            for (int dx = -(a.kw / 2); dx <= (a.kw - 1) / 2; ++dx) {
+              const int x = ox + dx;
+              if (x < 0 || x >= a.W) continue;
+              s += __ldg(An + static_cast<int64_t>(y) * a.W + x);
+            }
+          }
+          beta_h[h] = s / static_cast<float>(a.kh * a.kw);
+        } else if (a.beta) {
+          beta_h[h] = __ldg(a.beta + (static_cast<int64_t>(n) * a.Ho + oy) * a.Wo + ox);
+        }
+      }
       if (!mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err)) break;
       tc_fence_after();
-      const int n = tc.n0 + row / rc, oy = tc.oy0 + (row / a.Cw) % a.R, ox = tc.ox0 + row % a.Cw;
-      const bool valid = n < a.N && oy < a.Ho && ox < a.Wo;
-      float beta = 1.f;
-      if (!kSplit && a.beta && valid) beta = __ldg(a.beta + (static_cast<int64_t>(n) * a.Ho + oy) * a.Wo + ox);
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
-      for (int ch = 0; ch < a.BN / 32; ++ch) {
-        uint32_t v[32];
-        tc_ld_32x32(tbase + static_cast<uint32_t>(ch * 32), v);
-        if (ch == a.BN / 32 - 1) {  // accumulator fully read: hand it back to the MMA warp
-          tc_fence_before();
-          if (lane == 0) mbar_arrive(&B->tmem_empty[acc]);
-        }
-        const int buf = chunk_count & 1;
-        ++chunk_count;
-        uint8_t* so = stage_out + buf * kStageOutBytes;
-        epi_barrier();  // the store that last read `so` has finished (waited below by et 0)
-        const int c0 = tc.ntile * a.BN + ch * 32;
-        float y[32];
-        if (kSplit) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) y[j] = static_cast<float>(static_cast<int32_t>(v[j]));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int c = c0 + j;
-            const float sc = c < a.No ? __ldg(a.scale + c) : 0.f;
-            const float bi = c < a.No ? __ldg(a.bias + c) : 0.f;
-            const float s = static_cast<float>(static_cast<int32_t>(v[j]));
-            float r = a.beta ? fmaf(s * sc, beta, bi) : fmaf(s, sc, bi);
-            if (a.relu) r = fmaxf(r, 0.f);
-            y[j] = r;
+      for (int h = 0; h < a.mt; ++h) {
+        const float beta = beta_h[h];
+        const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>((acc * a.mt + h) * a.BN);
+        for (int ch = 0; ch < tc.bn / 32; ++ch) {
+          uint32_t v[32];
+          tc_ld_32x32(tbase + static_cast<uint32_t>(ch * 32), v);
+          if (h == a.mt - 1 && ch == tc.bn / 32 - 1) {  // accumulator fully read: hand it back
+            tc_fence_before();
+            if (lane == 0) mbar_arrive(&B->tmem_empty[acc]);
           }
-        }
-        // 128-byte swizzled row: 16-byte chunk k of row r lives at chunk k ^ (r % 8)
-        float4* orow = reinterpret_cast<float4*>(so + row * 128);
+          const int buf = chunk_count & 1;
+          ++chunk_count;
+          uint8_t* so = stage_out + buf * kStageOutBytes;
+          epi_barrier();  // the store that last read `so` has finished (waited below by et 0)
+          const int c0 = tc.ntile * a.BN + tc.noff + ch * 32;
+          float y[32];
+          if (kSplit) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          orow[k ^ (row & 7)] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
-        fence_proxy_async();
-        epi_barrier();
-        if (et == 0) {
-          if (c0 < a.No) {  // a box past the last channel would write nothing; skip it
-            if (kSplit)
-              tma_reduce_add_4d(&tmOut, so, c0, tc.ox0, tc.oy0, tc.n0);
-            else
-              tma_store_4d(&tmOut, so, c0, tc.ox0, tc.oy0, tc.n0);
+            for (int j = 0; j < 32; ++j) y[j] = static_cast<float>(static_cast<int32_t>(v[j]));
+          } else {
+            const float4* sb4 = reinterpret_cast<const float4*>(&B->sb[tc.noff + ch * 32]);
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const float4 p = sb4[j / 2];  // (scale, bias) of channels j, j+1 (same for all lanes)
+              const float s0 = static_cast<float>(static_cast<int32_t>(v[j]));
+              const float s1 = static_cast<float>(static_cast<int32_t>(v[j + 1]));
+              float r0 = has_beta ? fmaf(s0 * p.x, beta, p.y) : fmaf(s0, p.x, p.y);
+              float r1 = has_beta ? fmaf(s1 * p.z, beta, p.w) : fmaf(s1, p.z, p.w);
+              if (a.relu) {
+                r0 = fmaxf(r0, 0.f);
+                r1 = fmaxf(r1, 0.f);
+              }
+              y[j] = r0;
+              y[j + 1] = r1;
+            }
           }
-          bulk_commit();  // one group per chunk (possibly empty) keeps the buffer accounting
-          bulk_wait_read_1();
+          // 128-byte swizzled row: 16-byte chunk k of row r lives at chunk k ^ (r % 8)
+          float4* orow = reinterpret_cast<float4*>(so + row * 128);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            orow[k ^ (row & 7)] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
+          fence_proxy_async();
+          epi_barrier();
+          if (et == 0) {
+            if (c0 < a.No) {  // a box past the last channel would write nothing; skip it
+              if (kSplit)
+                tma_reduce_add_4d(&tmOut, so, c0, tc.ox0, tc.oy0, tc.n0 + h * a.Bn);
+              else
+                tma_store_4d(&tmOut, so, c0, tc.ox0, tc.oy0, tc.n0 + h * a.Bn);
+            }
+            bulk_commit();  // one group per chunk (possibly empty) keeps the buffer accounting
+            bulk_wait_read_1();
+          }
         }
       }
       acc ^= 1;
@@ -416,24 +484,45 @@ __global__ void tc_finalize_kernel(const float* __restrict__ ws, float* __restri
 
 }  // namespace
 
-int tc_smem_bytes(int bn) { return kStages * (kABytes + bn * 128) + 2 * kStageOutBytes + 256 + 1024; }
+int tc_smem_bytes(int bn, int mt) {
+  return kStages * (mt * kABytes + bn * 128) + 2 * kStageOutBytes + static_cast<int>(sizeof(Barriers));
+}
 
-cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmOut, const TcArgs& a,
-                           cudaStream_t s) {
-  const int smem = tc_smem_bytes(a.BN);
-  const int total_tiles = a.m_tiles * a.n_tiles * a.k_splits;
-  if (total_tiles == 0) return cudaSuccess;
+int tc_plan(TcArgs& a, int sm_count) {
+  const int tiles = a.m_tiles * a.n_tiles * a.k_splits;
+  int grid = sm_count < tiles ? sm_count : tiles;
+  a.full_tiles = tiles;
+  a.pieces = 1;
+  const int tail = grid > 0 ? tiles % grid : 0;
+  if (a.k_splits == 1 && tiles > grid && tail > 0) {
+    // cut each tail tile into the most 32-channel-multiple pieces that still fit one wave
+    for (int p = a.BN / 32; p > 1; --p) {
+      if ((a.BN / 32) % p == 0 && tail * p <= grid) {
+        a.pieces = p;
+        break;
+      }
+    }
+    if (a.pieces > 1) a.full_tiles = tiles - tail;
+  }
+  return grid;
+}
+
+cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmBp,
+                           const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s) {
+  const int smem = tc_smem_bytes(a.BN, a.mt);
+  const int tiles = a.m_tiles * a.n_tiles * a.k_splits;
+  if (tiles == 0) return cudaSuccess;
   int grid = current_sm_count();
-  if (grid > total_tiles) grid = total_tiles;
+  if (grid > tiles) grid = tiles;
   cudaError_t e;
   if (a.k_splits > 1) {
     e = cudaFuncSetAttribute(tc_conv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    tc_conv_kernel<true><<<grid, kThreadsTc, smem, s>>>(*tmA, *tmB, *tmOut, a);
+    tc_conv_kernel<true><<<grid, kThreadsTc, smem, s>>>(*tmA, *tmB, *tmBp, *tmOut, a);
   } else {
     e = cudaFuncSetAttribute(tc_conv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    tc_conv_kernel<false><<<grid, kThreadsTc, smem, s>>>(*tmA, *tmB, *tmOut, a);
+    tc_conv_kernel<false><<<grid, kThreadsTc, smem, s>>>(*tmA, *tmB, *tmBp, *tmOut, a);
   }
   return cudaGetLastError();
 }

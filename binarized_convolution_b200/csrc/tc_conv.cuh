@@ -19,19 +19,30 @@ struct TcArgs {
   int m_tiles;         // tiles_y * tiles_x * ceil(N / Bn)
   int tiles_x, tiles_y;
   int R, Cw, Bn;
+  int mt;              // M sub-tiles per CTA tile sharing each weight stage: 1, or 2 for the FC
+                       // (the second sub-tile is the next Bn images; needs R = Cw = 1)
   int k_splits;        // > 1: partial sums reduced into an fp32 workspace
+  // Work list: tiles [0, full_tiles) whole, then the remaining tail tiles cut along N into
+  // `pieces` parts of BN / pieces channels each (so the last wave spreads over more SMs).
+  int full_tiles;
+  int pieces;
   int No;
   uint32_t tmem_cols;  // power of two >= 2*BN
   const float* scale;
   const float* bias;
-  const float* beta;   // [N][Ho][Wo] or nullptr
+  const float* beta;   // [N][Ho][Wo] or nullptr (ignored when A is given)
+  const float* A;      // [N][H][W] channel means: beta is then formed in the epilogue
+  int H, W;            // input extent (for the window of A)
   int relu;
   uint32_t* err;
 };
 
-int tc_smem_bytes(int bn);
-cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmOut, const TcArgs& a,
-                           cudaStream_t s);
+int tc_smem_bytes(int bn, int mt);
+// tmBp: the weight map with a box of BN / pieces rows (used for tail pieces).
+cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmBp,
+                           const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s);
+// Grid size and tail split for a launch on `sm_count` SMs (fills full_tiles / pieces).
+int tc_plan(TcArgs& a, int sm_count);
 cudaError_t launch_tc_finalize(const float* ws, float* out, const float* scale, const float* bias, const float* beta,
                                int64_t total, int no, int rows_per_beta, int relu, cudaStream_t s);
 

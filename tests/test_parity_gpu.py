@@ -38,6 +38,8 @@ MEDIUM = [
                      in_terms=False, seed=109),
     synth.small_case(batch=20, h=4, w=4, ni=33, no=70, kind="fc", op=synth.BINARY_WEIGHTS, use_beta=True,
                      relu=False, in_terms=True, seed=110),
+    synth.small_case(batch=300, h=2, w=3, ni=96, no=200, kind="fc", op=synth.XNOR, use_beta=True, relu=True,
+                     in_terms=True, seed=111),
 ]
 
 
