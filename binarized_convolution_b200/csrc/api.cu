@@ -119,6 +119,7 @@ struct Layer {
   uint32_t* err = nullptr;
   // tensor-core path: int8 codes [N][H][W][cip], int8 weights [no_tc][taps*cip], tensor maps
   bool tc_ok = false;
+  bool tc_pair = false;  // convolution on SM pairs (cta_group::2); the FC uses single SMs
   int cip = 0;
   int8_t* codes = nullptr;
   int8_t* wq = nullptr;
@@ -298,10 +299,24 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   }
   ok = ok && encode_2d(&L.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(kt),
                        static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128, static_cast<uint32_t>(t.BN));
-  tc_plan(t, current_sm_count());  // work list for this device: tail tiles cut along N
-  ok = ok && encode_2d(&L.tmBp, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(kt),
-                       static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128,
-                       static_cast<uint32_t>(t.BN / t.pieces));
+  // Convolutions run on SM pairs when two-CTA clusters fit; each CTA then loads half of
+  // every weight tile (boxes of BN/2 rows).
+  const int pairs = L.fc ? 0 : tc2_max_pairs(t.BN);
+  if (pairs > 0) {
+    L.tc_pair = true;
+    tc2_plan(t, pairs);
+    ok = ok && encode_2d(&L.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(kt),
+                         static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128,
+                         static_cast<uint32_t>(t.BN / 2));
+    ok = ok && encode_2d(&L.tmBp, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(kt),
+                         static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128,
+                         static_cast<uint32_t>(t.BN / t.pieces / 2));
+  } else {
+    t.grid_ctas = tc_plan(t, current_sm_count());  // work list: tail tiles cut along N
+    ok = ok && encode_2d(&L.tmBp, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(kt),
+                         static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128,
+                         static_cast<uint32_t>(t.BN / t.pieces));
+  }
   if (ok && t.k_splits > 1) ok = encode_out_map(L, &L.tmWs, L.ws);
   if (!ok) return BCONV_OK;  // the POPC path stays available
   L.tc_ok = true;
@@ -466,7 +481,7 @@ bconv_status_t run_forward_tc(Layer& L, const float* in, float* out, cudaStream_
   }
   const bool timed = L.prof.active && L.prof.used < static_cast<int>(L.prof.start.size());
   if (timed) cudaEventRecord(L.prof.start[L.prof.used], s);
-  e = launch_tc_conv(&L.tmA, &L.tmB, &L.tmBp, om, t, s);
+  e = L.tc_pair ? launch_tc_conv2(&L.tmA, &L.tmB, &L.tmBp, om, t, s) : launch_tc_conv(&L.tmA, &L.tmB, &L.tmBp, om, t, s);
   if (timed) cudaEventRecord(L.prof.stop[L.prof.used++], s);
   if (e != cudaSuccess) return from_cuda(e);
   if (t.k_splits > 1)
@@ -891,7 +906,7 @@ bconv_status_t bconv_pack_bits(const uint8_t* bits, int64_t rows, int32_t nbits,
 int32_t bconv_version(void) { return 100; }
 
 bconv_status_t bconv_measure_peak(int32_t kind, double* ops_per_s, double* sm_mhz) {
-  if (kind < 0 || kind > 2 || !ops_per_s) return BCONV_ERR_INVALID_ARG;
+  if (kind < 0 || kind > 4 || !ops_per_s) return BCONV_ERR_INVALID_ARG;
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
     cudaGetLastError();

@@ -5,11 +5,15 @@
 //   kind 1: LOP3 alone; reported as bit operations per second (32 per instruction).
 //   kind 2: b1 tensor MMA, mma.sync m16n8k256 .xor.popc; reported as bit
 //           multiply-accumulates per second (16*8*256 per instruction).
+//   kind 3: tcgen05.mma.cta_group::1.kind::i8, M=128 N=256 K=32, operands in shared memory,
+//           accumulator in TMEM; multiply-accumulates per second.
+//   kind 4: tcgen05.mma.cta_group::1.kind::f16 (bf16 operands), M=128 N=256 K=16.
 //
 // Every thread runs independent dependency chains so that issue rate, not latency, is the
 // limit.  Results are stored so the work cannot be removed.  The grid fills every SM with
 // four 256-thread CTAs.
 #include "common.cuh"
+#include "tc_device.cuh"
 
 namespace bconv {
 namespace {
@@ -96,9 +100,124 @@ __global__ void __launch_bounds__(kProbeThreads) b1mma_probe(int iters, uint32_t
   if ((threadIdx.x & 31) == 0) atomicMax(reinterpret_cast<unsigned long long*>(cycles), static_cast<unsigned long long>(t1 - t0));
 }
 
+// Back-to-back tcgen05 MMAs of one CTA per SM on zero operands (no data movement): the tensor
+// pipe's own rate.  One thread issues `iters` groups of 4 MMAs into one TMEM accumulator and
+// waits for them through tcgen05.commit (bounded wait).
+template <bool kI8>
+__global__ void __launch_bounds__(128, 1) tcgen05_probe(int iters, uint32_t* out, long long* cycles, uint32_t* err) {
+  using namespace tcdev;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  struct Bars {
+    uint64_t done;
+    uint32_t tmem_base;
+    uint32_t abort_flag;
+  };
+  if ((smem_u32(smem) & 1023u) != 0u) {
+    if (threadIdx.x == 0) atomicOr(err, kErrLayout);
+    return;
+  }
+  uint8_t* sa = smem;                  // 128 rows x 128 B
+  uint8_t* sb = smem + 128 * 128;      // 256 rows x 128 B
+  Bars* B = reinterpret_cast<Bars*>(smem + 128 * 128 + 256 * 128);
+  for (int i = threadIdx.x; i < (128 + 256) * 128 / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+  if (threadIdx.x == 0) {
+    mbar_init(&B->done, 1);
+    B->abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (threadIdx.x < 32) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&B->tmem_base)),
+                 "r"(256));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = B->tmem_base;
+  if (threadIdx.x == 0) {
+    // s32 (i8) or f32 (bf16) accumulator, K-major, M=128, N=256
+    const uint32_t idesc = kI8 ? ((2u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((128u >> 4) << 24))
+                               : ((1u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((128u >> 4) << 24));
+    const uint64_t da = smem_desc_sw128(sa), db = smem_desc_sw128(sb);
+    const long long t0 = clock64();
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t acc = (it > 0 || j > 0) ? 1u : 0u;
+        if (kI8)
+          asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+                       "l"(da + 2u * j), "l"(db + 2u * j), "r"(idesc), "r"(acc) : "memory");
+        else
+          asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+                       "l"(da + 2u * j), "l"(db + 2u * j), "r"(idesc), "r"(acc) : "memory");
+      }
+    }
+    tc_commit(&B->done);
+    mbar_wait(&B->done, 0, B, err, false);
+    const long long t1 = clock64();
+    atomicMax(reinterpret_cast<unsigned long long*>(cycles), static_cast<unsigned long long>(t1 - t0));
+    out[blockIdx.x] = 1u;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
+  }
+}
+
 }  // namespace
 
 cudaError_t probe_peak(int kind, double* ops_per_s, double* sm_mhz) {
+  if (kind == 3 || kind == 4) {
+    const int sms = current_sm_count();
+    const int iters = 2048;
+    const int smem = 120 * 1024;  // more than half an SM's shared memory: one CTA per SM
+    uint32_t* out = nullptr;
+    long long* cyc = nullptr;
+    uint32_t* err = nullptr;
+    cudaEvent_t e0 = nullptr, e1 = nullptr;
+    cudaError_t e = cudaMalloc(&out, sms * sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaMalloc(&cyc, sizeof(long long));
+    if (e == cudaSuccess) e = cudaMalloc(&err, sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaMemset(err, 0, sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaEventCreate(&e0);
+    if (e == cudaSuccess) e = cudaEventCreate(&e1);
+    auto kern = kind == 3 ? tcgen05_probe<true> : tcgen05_probe<false>;
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    float best = 0.f;
+    long long cycles = 0;
+    for (int rep = 0; rep < 4 && e == cudaSuccess; ++rep) {
+      cudaMemset(cyc, 0, sizeof(long long));
+      cudaEventRecord(e0, 0);
+      kern<<<sms, 128, smem>>>(iters, out, cyc, err);
+      e = cudaGetLastError();
+      cudaEventRecord(e1, 0);
+      if (e == cudaSuccess) e = cudaEventSynchronize(e1);
+      float ms = 0.f;
+      if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, e0, e1);
+      if (e == cudaSuccess && rep > 0 && (best == 0.f || ms < best)) {
+        best = ms;
+        cudaMemcpy(&cycles, cyc, sizeof(long long), cudaMemcpyDeviceToHost);
+      }
+    }
+    uint32_t herr = 0;
+    if (e == cudaSuccess) e = cudaMemcpy(&herr, err, sizeof(herr), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && herr) e = cudaErrorLaunchTimeout;
+    if (e == cudaSuccess && best > 0.f) {
+      const double macs = static_cast<double>(sms) * iters * 4.0 * 128.0 * 256.0 * (kind == 3 ? 32.0 : 16.0);
+      if (ops_per_s) *ops_per_s = macs / (best * 1e-3);
+      if (sm_mhz) *sm_mhz = static_cast<double>(cycles) / (best * 1e3);
+    }
+    if (e0) cudaEventDestroy(e0);
+    if (e1) cudaEventDestroy(e1);
+    if (out) cudaFree(out);
+    if (cyc) cudaFree(cyc);
+    if (err) cudaFree(err);
+    return e;
+  }
   const int sms = current_sm_count();
   const int blocks = sms * 4;
   const int64_t threads = static_cast<int64_t>(blocks) * kProbeThreads;

@@ -26,6 +26,7 @@ struct TcArgs {
   // `pieces` parts of BN / pieces channels each (so the last wave spreads over more SMs).
   int full_tiles;
   int pieces;
+  int grid_ctas;       // CTAs launched (pair kernel: 2 x co-resident clusters)
   int No;
   uint32_t tmem_cols;  // power of two >= 2*BN
   const float* scale;
@@ -43,6 +44,14 @@ cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmB, const
                            const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s);
 // Grid size and tail split for a launch on `sm_count` SMs (fills full_tiles / pieces).
 int tc_plan(TcArgs& a, int sm_count);
+
+// SM-pair kernel (tcgen05.mma.cta_group::2, M = 256 per cluster of two CTAs); convolutions only.
+// tmB / tmBp are weight maps with boxes of BN/2 and BN/pieces/2 rows.
+int tc2_smem_bytes(int bn);
+int tc2_plan(TcArgs& a, int pairs);  // pairs = clusters that can be resident at once
+int tc2_max_pairs(int bn);           // co-resident two-CTA clusters on the current device (0: none)
+cudaError_t launch_tc_conv2(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmBp,
+                            const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s);
 cudaError_t launch_tc_finalize(const float* ws, float* out, const float* scale, const float* bias, const float* beta,
                                int64_t total, int no, int rows_per_beta, int relu, cudaStream_t s);
 

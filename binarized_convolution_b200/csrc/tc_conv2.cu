@@ -1,0 +1,438 @@
+// Binary convolution on SM pairs: tcgen05.mma.cta_group::2 kind::i8 (M = 256 across two SMs).
+//
+// Same arithmetic as tc_conv.cu (exact int8 +-1 / {0,1} dot products accumulated in int32;
+// Apple page "MPSCNNBinaryConvolution", XNOR and AND bullets), with the operand traffic per SM
+// cut by a third: a cluster of two CTAs computes a 256 x BN output tile, each CTA holding its
+// own 128 output pixels of A and half (BN/2 rows) of the weight tile B.  The pair's MMA is
+// issued by one thread of the even CTA (the leader) and reads both CTAs' shared memory; each
+// CTA's TMEM receives its own 128 x BN accumulator rows.
+//
+// Per CTA: warp 0 loads its A box and its half of B with TMA into a 6-stage ring; both CTAs'
+// copies complete on the leader's `full` barrier, whose expected byte count covers the pair.
+// The leader's warp 1 issues the MMAs and releases each stage and each finished accumulator
+// with tcgen05.commit multicast to both CTAs.  Warps 2-5 of each CTA run the epilogue of its
+// 128 rows (as in tc_conv.cu) and release the accumulator on the leader's barrier.  TMEM is
+// allocated and freed with cta_group::2 in both CTAs; the pair synchronises (cluster barrier)
+// after set-up and before exit, so no copy or commit ever targets a CTA that has left.
+// Every mbarrier wait is bounded by one second of %globaltimer.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "tc_conv.cuh"
+#include "tc_device.cuh"
+
+namespace bconv {
+namespace {
+
+using namespace tcdev;
+
+constexpr int kStages2 = 6;
+constexpr int kABytes2 = 128 * 128;
+constexpr int kThreads2 = 192;
+constexpr int kEpi2 = 128;
+constexpr int kOutBytes2 = 128 * 128;
+
+struct __align__(8) Barriers2 {
+  uint64_t full[kStages2];   // used in the leader only
+  uint64_t empty[kStages2];  // both CTAs (multicast commit)
+  uint64_t tmem_full[2];     // both CTAs (multicast commit)
+  uint64_t tmem_empty[2];    // leader only: 4 epilogue warps x 2 CTAs
+  uint64_t done;             // both CTAs: every MMA of the pair has completed
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+  float2 sb[256];
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// shared::cluster address of a local shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
+                                                 int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
+                                                 int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on the barrier at this offset in both CTAs of the pair when the MMAs issued so far
+// by this thread have completed.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+// Instruction descriptor: s32 accumulator, signed int8 A and B, K-major, M = 256, N = bn.
+__host__ __device__ constexpr uint32_t idesc_i8_m256(int bn) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(bn >> 3) << 17) | ((256u >> 4) << 24);
+}
+
+struct PairCoord {
+  int n0, oy0, ox0, ntile;
+  int noff, bn;  // channels [ntile*BN + noff, + bn)
+  bool dummy;    // this CTA's M tile lies past the end (odd tile count): compute, do not store
+};
+
+// Work item w of the pair -> this CTA's M tile (2*pair + rank) and the N range.
+__device__ __forceinline__ PairCoord pair_coord(const TcArgs& a, int w, int rank) {
+  PairCoord c;
+  int t = w;
+  c.noff = 0;
+  c.bn = a.BN;
+  if (w >= a.full_tiles) {
+    const int i = w - a.full_tiles;
+    t = a.full_tiles + i / a.pieces;
+    c.bn = a.BN / a.pieces;
+    c.noff = (i % a.pieces) * c.bn;
+  }
+  c.ntile = t % a.n_tiles;
+  int m = (t / a.n_tiles) * 2 + rank;
+  c.dummy = m >= a.m_tiles;
+  if (c.dummy) m = a.m_tiles - 1;
+  const int tx = m % a.tiles_x;
+  m /= a.tiles_x;
+  const int ty = m % a.tiles_y;
+  m /= a.tiles_y;
+  c.n0 = m * a.Bn;
+  c.oy0 = ty * a.R;
+  c.ox0 = tx * a.Cw;
+  return c;
+}
+
+__global__ void __launch_bounds__(kThreads2, 1)
+    tc_conv2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmBp, const __grid_constant__ CUtensorMap tmOut,
+                    const TcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0u) {  // same in both CTAs: both leave before any set-up
+    if (threadIdx.x == 0) atomicOr(a.err, kErrLayout);
+    return;
+  }
+  const int half_b = a.BN / 2;  // weight rows this CTA holds
+  const int stage_bytes = kABytes2 + half_b * 128;
+  uint8_t* stage_out = smem + kStages2 * stage_bytes;
+  Barriers2* B = reinterpret_cast<Barriers2*>(stage_out + 2 * kOutBytes2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int pair_tiles = (a.m_tiles + 1) / 2 * a.n_tiles;
+  const int total = a.full_tiles + (pair_tiles - a.full_tiles) * a.pieces;
+  const int kb_total = a.kh * a.kw * a.kb_per_tap;
+  const uint32_t tmem_cols = a.tmem_cols;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages2; ++s) {
+      mbar_init(&B->full[s], 1);
+      mbar_init(&B->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&B->tmem_full[b], 1);
+      mbar_init(&B->tmem_empty[b], 2 * kEpi2 / 32);
+    }
+    mbar_init(&B->done, 1);
+    B->abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&B->tmem_base)),
+                 "r"(tmem_cols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any copy or commit crosses over
+  tc_fence_after();
+  const uint32_t tmem_base = B->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs) ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int w = pair; w < total && ok; w += npairs) {
+        const PairCoord pc = pair_coord(a, w, rank);
+        const uint32_t tx = static_cast<uint32_t>(2 * (kABytes2 + (pc.bn / 2) * 128));  // both CTAs' bytes
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait(&B->empty[stage], phase ^ 1u, B, a.err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * stage_bytes;
+          uint8_t* sb = sa + kABytes2;
+          const uint32_t full_leader = mapa(&B->full[stage], 0);
+          if (leader) mbar_expect_tx(&B->full[stage], tx);
+          const int tap = kb / a.kb_per_tap, cb = kb - tap * a.kb_per_tap;
+          const int ky = tap / a.kw, kx = tap - ky * a.kw;
+          tma_load_4d_pair(sa, &tmA, full_leader, cb * 128, pc.ox0 + kx - a.kw / 2, pc.oy0 + ky - a.kh / 2, pc.n0);
+          const int brow = pc.ntile * a.BN + pc.noff + static_cast<int>(rank) * (pc.bn / 2);
+          if (pc.bn == a.BN)
+            tma_load_2d_pair(sb, &tmB, full_leader, kb * 128, brow);
+          else
+            tma_load_2d_pair(sb, &tmBp, full_leader, kb * 128, brow);
+          if (++stage == kStages2) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (leader only) ----------------
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int w = pair; w < total && ok; w += npairs) {
+        const PairCoord pc = pair_coord(a, w, 0);
+        const uint32_t idesc = idesc_i8_m256(pc.bn);
+        if (!mbar_wait(&B->tmem_empty[acc], acc_phase ^ 1u, B, a.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait(&B->full[stage], phase, B, a.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint8_t* sa = smem + stage * stage_bytes;
+          const uint64_t da = smem_desc_sw128(sa), db = smem_desc_sw128(sa + kABytes2);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            tc_mma_i8_pair(d_tmem, da + 2u * j, db + 2u * j, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+          tc_commit_pair(&B->empty[stage]);
+          if (++stage == kStages2) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair(&B->tmem_full[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      tc_commit_pair(&B->done);  // fires in both CTAs once every MMA above has completed
+    }
+    if (lane == 0) mbar_wait(&B->done, 0, B, a.err, false);
+  } else {
+    // ---------------- epilogue (both CTAs, warps 2..5) ----------------
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int et = threadIdx.x - 64;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int chunk_count = 0;
+    int loaded_ntile = -1;
+    const int rc = a.R * a.Cw;
+    const uint32_t empty_leader0 = mapa(&B->tmem_empty[0], 0), empty_leader1 = mapa(&B->tmem_empty[1], 0);
+    for (int w = pair; w < total; w += npairs) {
+      const PairCoord pc = pair_coord(a, w, rank);
+      if (pc.ntile != loaded_ntile) {
+        epi_barrier();
+        for (int j = et; j < a.BN; j += kEpi2) {
+          const int c = pc.ntile * a.BN + j;
+          B->sb[j] = c < a.No ? make_float2(__ldg(a.scale + c), __ldg(a.bias + c)) : make_float2(0.f, 0.f);
+        }
+        epi_barrier();
+        loaded_ntile = pc.ntile;
+      }
+      const int n = pc.n0 + row / rc, oy = pc.oy0 + (row / a.Cw) % a.R, ox = pc.ox0 + row % a.Cw;
+      const bool valid = !pc.dummy && n < a.N && oy < a.Ho && ox < a.Wo;
+      const bool has_beta = a.A != nullptr || a.beta != nullptr;
+      float beta = 1.f;
+      if (valid && a.A) {
+        const float* An = a.A + static_cast<int64_t>(n) * a.H * a.W;
+        float s = 0.f;
+        for (int dy = -(a.kh / 2); dy <= (a.kh - 1) / 2; ++dy) {
+          const int y = oy + dy;
+          if (y < 0 || y >= a.H) continue;
+          for (int dx = -(a.kw / 2); dx <= (a.kw - 1) / 2; ++dx) {
+            const int x = ox + dx;
+            if (x < 0 || x >= a.W) continue;
+            s += __ldg(An + static_cast<int64_t>(y) * a.W + x);
+          }
+        }
+        beta = s / static_cast<float>(a.kh * a.kw);
+      } else if (valid && a.beta) {
+        beta = __ldg(a.beta + (static_cast<int64_t>(n) * a.Ho + oy) * a.Wo + ox);
+      }
+      if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err))) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
+      for (int ch = 0; ch < pc.bn / 32; ++ch) {
+        uint32_t v[32];
+        tc_ld_32x32(tbase + static_cast<uint32_t>(ch * 32), v);
+        if (ch == pc.bn / 32 - 1) {  // this CTA's rows are read: release them on the leader
+          tc_fence_before();
+          if (lane == 0) mbar_arrive_remote(acc == 0 ? empty_leader0 : empty_leader1);
+        }
+        const int buf = chunk_count & 1;
+        ++chunk_count;
+        uint8_t* so = stage_out + buf * kOutBytes2;
+        epi_barrier();
+        const int c0 = pc.ntile * a.BN + pc.noff + ch * 32;
+        const float4* sb4 = reinterpret_cast<const float4*>(&B->sb[pc.noff + ch * 32]);
+        float y[32];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float4 p = sb4[j / 2];
+          const float s0 = static_cast<float>(static_cast<int32_t>(v[j]));
+          const float s1 = static_cast<float>(static_cast<int32_t>(v[j + 1]));
+          float r0 = has_beta ? fmaf(s0 * p.x, beta, p.y) : fmaf(s0, p.x, p.y);
+          float r1 = has_beta ? fmaf(s1 * p.z, beta, p.w) : fmaf(s1, p.z, p.w);
+          if (a.relu) {
+            r0 = fmaxf(r0, 0.f);
+            r1 = fmaxf(r1, 0.f);
+          }
+          y[j] = r0;
+          y[j + 1] = r1;
+        }
+        float4* orow = reinterpret_cast<float4*>(so + row * 128);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          orow[k ^ (row & 7)] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
+        fence_proxy_async();
+        epi_barrier();
+        if (et == 0) {
+          if (c0 < a.No && !pc.dummy) tma_store_4d(&tmOut, so, c0, pc.ox0, pc.oy0, pc.n0);
+          bulk_commit();
+          bulk_wait_read_1();
+        }
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (et == 0) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer is done with this CTA's barriers and shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(tmem_cols));
+  }
+}
+
+}  // namespace
+
+int tc2_smem_bytes(int bn) {
+  return kStages2 * (kABytes2 + (bn / 2) * 128) + 2 * kOutBytes2 + static_cast<int>(sizeof(Barriers2));
+}
+
+int tc2_max_pairs(int bn) {
+  const int smem = tc2_smem_bytes(bn);
+  if (cudaFuncSetAttribute(tc_conv2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(kThreads2);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, tc_conv2_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+int tc2_plan(TcArgs& a, int pairs) {
+  const int pair_tiles = (a.m_tiles + 1) / 2 * a.n_tiles;
+  const int npairs = pairs;
+  a.full_tiles = pair_tiles;
+  a.pieces = 1;
+  const int grid_pairs = npairs < pair_tiles ? npairs : pair_tiles;
+  const int tail = grid_pairs > 0 ? pair_tiles % grid_pairs : 0;
+  if (pair_tiles > grid_pairs && tail > 0) {
+    for (int p = a.BN / 32; p > 1; --p) {
+      if ((a.BN / 32) % p == 0 && tail * p <= grid_pairs) {
+        a.pieces = p;
+        break;
+      }
+    }
+    if (a.pieces > 1) a.full_tiles = pair_tiles - tail;
+  }
+  a.grid_ctas = 2 * grid_pairs;
+  return a.grid_ctas;
+}
+
+cudaError_t launch_tc_conv2(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmBp,
+                            const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s) {
+  const int pair_tiles = (a.m_tiles + 1) / 2 * a.n_tiles;
+  if (pair_tiles == 0) return cudaSuccess;
+  const int smem = tc2_smem_bytes(a.BN);
+  const int npairs = a.grid_ctas / 2;
+  if (npairs <= 0) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(tc_conv2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * npairs));
+  cfg.blockDim = dim3(kThreads2);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, tc_conv2_kernel, *tmA, *tmB, *tmBp, *tmOut, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace bconv

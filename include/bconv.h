@@ -221,7 +221,9 @@ int32_t bconv_version(void);
  * Measured peak of an instruction the contraction kernels are bound by, on the current
  * device: kind 0 = POPC (32-bit population count, reported as bit-ops/s = 32 x
  * instructions/s), 1 = LOP3 (32-bit logic op, instructions/s x 32), 2 = b1 tensor MMA
- * mma.sync m16n8k256 .xor.popc (bit multiply-accumulates/s).  Runs a few short kernels
+ * mma.sync m16n8k256 .xor.popc (bit multiply-accumulates/s), 3 = tcgen05.mma kind::i8
+ * M128 N256 K32 from shared memory into TMEM (multiply-accumulates/s), 4 = tcgen05.mma
+ * kind::f16 with bf16 operands, M128 N256 K16 (multiply-accumulates/s).  Runs a few short kernels
  * (milliseconds) and waits for them.  *sm_mhz receives the SM clock the kernels saw,
  * derived from clock64() over the event-timed interval (may be NULL).
  */
