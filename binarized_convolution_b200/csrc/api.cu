@@ -172,10 +172,12 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // 4-D tiled map, dims innermost first, 128-byte swizzle, out-of-range elements read as 0.
 bool encode_4d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, const uint64_t dims[4],
-               const uint64_t strides_bytes[3], const uint32_t box[4]) {
+               const uint64_t strides_bytes[3], const uint32_t box[4], const uint32_t elem_strides[4] = nullptr) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  if (elem_strides)
+    for (int i = 0; i < 4; ++i) estr[i] = elem_strides[i];
   return enc(m, dt, 4, const_cast<void*>(base), reinterpret_cast<const cuuint64_t*>(dims),
              reinterpret_cast<const cuuint64_t*>(strides_bytes), reinterpret_cast<const cuuint32_t*>(box), estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -213,14 +215,19 @@ bool encode_out_map(Layer& L, CUtensorMap* m, const float* out) {
   return encode_4d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, out, d, strides, box);
 }
 
-// The tensor-core path covers XNOR/AND with stride 1 (or the FC) and No % 4 == 0 (16-byte
-// output rows for the TMA store).  Sets up its buffers, weights and maps.
+// The tensor-core path: XNOR/AND as int8 codes (kind 0) and binaryWeights as three exact
+// bf16 parts of x~ (kind 1), for No % 4 == 0 (16-byte output rows for the TMA store) and
+// strided windows whose TMA box (stride x tile extent) stays within 256 elements.
+// Sets up its buffers, weights and maps.
 bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
-  if (L.type == kBinaryWeights || L.No % 4 != 0 || (!L.fc && (L.sy != 1 || L.sx != 1)) || L.N == 0) return BCONV_OK;
+  if (L.No % 4 != 0 || L.N == 0) return BCONV_OK;
   if (!tensor_map_encoder()) return BCONV_OK;
   const int taps = L.kh * L.kw;
-  L.cip = round_up(L.Ni, 128);
   TcArgs& t = L.tc;
+  t.kind = L.type == kBinaryWeights ? 1 : 0;
+  // channels per part, padded to whole 128-byte rows; bytes of operand per pixel
+  L.cip = t.kind == 0 ? round_up(L.Ni, 128) : round_up(L.Ni, 64);
+  const int bpp = t.kind == 0 ? L.cip : 6 * L.cip;
   // The FC keeps a batch of up to 256 images in one CTA tile (two 128-row sub-tiles sharing
   // every weight stage), so its large weight matrix streams from memory once.
   t.mt = (L.fc && L.N > 128) ? 2 : 1;
@@ -234,18 +241,19 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   t.scale = L.scale;
   t.bias = L.bias;
   if (L.fc) {
-    t.Ho = 1; t.Wo = 1; t.kh = 1; t.kw = 1;
-    t.kb_per_tap = L.H * L.W * L.cip / 128;
+    t.Ho = 1; t.Wo = 1; t.kh = 1; t.kw = 1; t.sy = 1; t.sx = 1;
+    t.kb_per_tap = L.H * L.W * bpp / 128;
     t.R = 1; t.Cw = 1; t.Bn = 128;
     t.tiles_x = 1; t.tiles_y = 1;
   } else {
-    t.Ho = L.Ho; t.Wo = L.Wo; t.kh = L.kh; t.kw = L.kw;
-    t.kb_per_tap = L.cip / 128;
+    t.Ho = L.Ho; t.Wo = L.Wo; t.kh = L.kh; t.kw = L.kw; t.sy = L.sy; t.sx = L.sx;
+    t.kb_per_tap = bpp / 128;
     t.Cw = std::min(128, next_pow2(L.Wo));
     t.R = std::min(128 / t.Cw, next_pow2(L.Ho));
     t.Bn = 128 / (t.Cw * t.R);
     t.tiles_x = (L.Wo + t.Cw - 1) / t.Cw;
     t.tiles_y = (L.Ho + t.R - 1) / t.R;
+    if (t.sx * t.Cw > 256 || t.sy * t.R > 256) return BCONV_OK;  // box too wide for TMA
   }
   t.m_tiles = t.tiles_x * t.tiles_y * ((L.N + t.Bn * t.mt - 1) / (t.Bn * t.mt));
   const int kb_total = t.kh * t.kw * t.kb_per_tap;
@@ -254,48 +262,59 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
     const int sms = current_sm_count();
     const int64_t tiles = static_cast<int64_t>(t.m_tiles) * t.n_tiles;
     int64_t best = -1;
-    for (int s = 1; s <= 16 && kb_total / s >= 4; ++s) {
-      const int64_t cost = ceil_div(tiles * s, sms) * ceil_div(kb_total, s);
+    for (int sp = 1; sp <= 16 && kb_total / sp >= 4; ++sp) {
+      const int64_t cost = ceil_div(tiles * sp, sms) * ceil_div(kb_total, sp);
       if (best < 0 || cost < best) {
         best = cost;
-        t.k_splits = s;
+        t.k_splits = sp;
       }
     }
   }
 
-  // int8 weights [no_tc][taps*cip]: +-1 (XNOR) or 0/1 (AND) codes, 0 in every padding slot.
+  // Weights [no_tc][taps][bpp bytes]: kind 0 int8 +-1 (XNOR) or 0/1 (AND); kind 1 bf16 +-1
+  // repeated for the three parts.  Every padding slot is 0.
   const int no_tc = t.n_tiles * t.BN;
-  const int64_t kt = static_cast<int64_t>(taps) * L.cip;
+  const int64_t kt = static_cast<int64_t>(taps) * bpp;
   std::vector<int8_t> hq(static_cast<size_t>(no_tc) * kt, 0);
-  const int8_t one = 1, zero_code = (L.type == kXnor) ? -1 : 0;
+  const int8_t zero_code = (L.type == kXnor) ? -1 : 0;
   for (int c = 0; c < L.No; ++c)
     for (int tp = 0; tp < taps; ++tp)
       for (int f = 0; f < L.Ni; ++f) {
         const uint32_t word = packed[(static_cast<int64_t>(c) * taps + tp) * L.nw + f / kWordBits];
-        hq[static_cast<size_t>(c) * kt + static_cast<int64_t>(tp) * L.cip + f] =
-            ((word >> (f % kWordBits)) & 1u) ? one : zero_code;
+        const bool bit = ((word >> (f % kWordBits)) & 1u) != 0;
+        int8_t* row = hq.data() + static_cast<size_t>(c) * kt + static_cast<int64_t>(tp) * bpp;
+        if (t.kind == 0) {
+          row[f] = bit ? 1 : zero_code;
+        } else {
+          const uint16_t v = bit ? 0x3F80u : 0xBF80u;  // bf16 +1 / -1
+          for (int part = 0; part < 3; ++part) memcpy(row + 2 * (part * L.cip + f), &v, 2);
+        }
       }
   const int64_t npix = static_cast<int64_t>(L.N) * L.H * L.W;
   cudaError_t e = L.mem.alloc(&L.wq, hq.size());
   if (e == cudaSuccess) e = cudaMemcpy(L.wq, hq.data(), hq.size(), cudaMemcpyHostToDevice);
-  if (e == cudaSuccess) e = L.mem.alloc(&L.codes, static_cast<size_t>(npix) * L.cip);
+  if (e == cudaSuccess) e = L.mem.alloc(&L.codes, static_cast<size_t>(npix) * bpp);
   if (e == cudaSuccess && t.k_splits > 1) e = L.mem.alloc(&L.ws, static_cast<size_t>(L.N) * L.No);
   if (e != cudaSuccess) return from_cuda(e);
 
   bool ok = true;
   if (L.fc) {
-    const uint64_t K = static_cast<uint64_t>(L.H) * L.W * L.cip;
+    const uint64_t K = static_cast<uint64_t>(L.H) * L.W * bpp;
     const uint64_t dims[4] = {K, 1, 1, static_cast<uint64_t>(L.N)};
     const uint64_t strides[3] = {K, K, K};
     const uint32_t box[4] = {128, 1, 1, 128};
     ok = encode_4d(&L.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.codes, dims, strides, box);
   } else {
-    const uint64_t dims[4] = {static_cast<uint64_t>(L.cip), static_cast<uint64_t>(L.W), static_cast<uint64_t>(L.H),
+    // box: 128 bytes of channels x (stride x Cw) columns x (stride x R) rows x Bn images,
+    // stepping by the stride, so the copy lands Cw x R x Bn pixels = 128 rows
+    const uint64_t dims[4] = {static_cast<uint64_t>(bpp), static_cast<uint64_t>(L.W), static_cast<uint64_t>(L.H),
                               static_cast<uint64_t>(L.N)};
-    const uint64_t strides[3] = {static_cast<uint64_t>(L.cip), static_cast<uint64_t>(L.cip) * L.W,
-                                 static_cast<uint64_t>(L.cip) * L.W * L.H};
-    const uint32_t box[4] = {128, static_cast<uint32_t>(t.Cw), static_cast<uint32_t>(t.R), static_cast<uint32_t>(t.Bn)};
-    ok = encode_4d(&L.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.codes, dims, strides, box);
+    const uint64_t strides[3] = {static_cast<uint64_t>(bpp), static_cast<uint64_t>(bpp) * L.W,
+                                 static_cast<uint64_t>(bpp) * L.W * L.H};
+    const uint32_t box[4] = {128, static_cast<uint32_t>(t.sx * t.Cw), static_cast<uint32_t>(t.sy * t.R),
+                             static_cast<uint32_t>(t.Bn)};
+    const uint32_t estr[4] = {1, static_cast<uint32_t>(t.sx), static_cast<uint32_t>(t.sy), 1};
+    ok = encode_4d(&L.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.codes, dims, strides, box, estr);
   }
   ok = ok && encode_2d(&L.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(kt),
                        static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128, static_cast<uint32_t>(t.BN));
@@ -446,17 +465,31 @@ bool use_tc(const Layer& L) {
 // Tensor-core forward: int8 codes (+ A) -> [beta] -> tcgen05 contraction [-> finalize].
 bconv_status_t run_forward_tc(Layer& L, const float* in, float* out, cudaStream_t s) {
   const bool beta = L.use_beta();
-  PackI8Args p{};
-  p.in = in;
-  p.npix = static_cast<int64_t>(L.N) * L.H * L.W;
-  p.ni = L.Ni;
-  p.cip = L.cip;
-  p.in_scale = L.in_scale;
-  p.in_bias = L.in_bias;
-  p.codes = L.codes;
-  p.A = beta ? L.A : nullptr;
-  p.op = L.type;
-  cudaError_t e = launch_pack_i8(p, s);
+  cudaError_t e;
+  if (L.tc.kind == 0) {
+    PackI8Args p{};
+    p.in = in;
+    p.npix = static_cast<int64_t>(L.N) * L.H * L.W;
+    p.ni = L.Ni;
+    p.cip = L.cip;
+    p.in_scale = L.in_scale;
+    p.in_bias = L.in_bias;
+    p.codes = L.codes;
+    p.A = beta ? L.A : nullptr;
+    p.op = L.type;
+    e = launch_pack_i8(p, s);
+  } else {
+    PackBf16x3Args p{};
+    p.in = in;
+    p.npix = static_cast<int64_t>(L.N) * L.H * L.W;
+    p.ni = L.Ni;
+    p.cip = L.cip;
+    p.in_scale = L.in_scale;
+    p.in_bias = L.in_bias;
+    p.parts = reinterpret_cast<uint16_t*>(L.codes);
+    p.A = beta ? L.A : nullptr;
+    e = launch_pack_bf16x3(p, s);
+  }
   if (e != cudaSuccess) return from_cuda(e);
   if (beta && L.fc) {  // the convolution forms beta from A inside its epilogue
     BetaArgs b{L.A, L.beta, L.N, L.H, L.W, L.Ho, L.Wo, L.kh, L.kw, L.sy, L.sx};

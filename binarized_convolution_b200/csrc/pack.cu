@@ -10,6 +10,8 @@
 // one coalesced 128-byte line and __ballot_sync assembles the word in channel order
 // (LSB = lowest channel).  Eight words are loaded before any is used so that each warp
 // keeps a kilobyte in flight; the kernel is bound by the fp32 read.
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 
 namespace bconv {
@@ -258,6 +260,82 @@ cudaError_t launch_pack_i8(const PackI8Args& a, cudaStream_t s) {
   if (a.in_scale)
     return a.A ? launch_i8_op<true, true>(a, chunks, grid, s) : launch_i8_op<true, false>(a, chunks, grid, s);
   return a.A ? launch_i8_op<false, true>(a, chunks, grid, s) : launch_i8_op<false, false>(a, chunks, grid, s);
+}
+
+
+// ------------------------------------------------------------------------------------
+// binaryWeights operand: three exact bf16 parts of x~ per channel.  A warp per pixel; a
+// lane takes 2 consecutive channels per step (one 4-byte store per part).
+// ------------------------------------------------------------------------------------
+namespace {
+
+__device__ __forceinline__ uint32_t split3_pair(float x0, float x1, uint32_t (&w)[3]) {
+  const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+  const float r0 = x0 - __bfloat162float(h0), r1 = x1 - __bfloat162float(h1);  // exact
+  const __nv_bfloat16 m0 = __float2bfloat16_rn(r0), m1 = __float2bfloat16_rn(r1);
+  const float q0 = r0 - __bfloat162float(m0), q1 = r1 - __bfloat162float(m1);  // exact
+  const __nv_bfloat16 l0 = __float2bfloat16_rn(q0), l1 = __float2bfloat16_rn(q1);
+  w[0] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+  w[1] = static_cast<uint32_t>(__bfloat16_as_ushort(m0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(m1)) << 16);
+  w[2] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+  return 0;
+}
+
+template <bool kTerms, bool kA>
+__global__ void __launch_bounds__(kPackThreads) pack_bf16x3_kernel(PackBf16x3Args a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kPackThreads) >> 5;
+  const int ni = a.ni, cip = a.cip;
+  for (int64_t p = warp; p < a.npix; p += nwarps) {
+    const float* row = a.in + p * ni;
+    uint16_t* prow = a.parts + p * 3 * cip;
+    float asum = 0.f;
+    for (int f0 = 0; f0 < cip; f0 += 64) {
+      const int f = f0 + lane * 2;  // channels f, f+1
+      float x0 = 0.f, x1 = 0.f;
+      if (f < ni) {
+        x0 = __ldcs(row + f);
+        if (kTerms) x0 = fmaf(x0, __ldg(a.in_scale + f), __ldg(a.in_bias + f));
+      }
+      if (f + 1 < ni) {
+        x1 = __ldcs(row + f + 1);
+        if (kTerms) x1 = fmaf(x1, __ldg(a.in_scale + f + 1), __ldg(a.in_bias + f + 1));
+      }
+      if (kA) asum += fabsf(x0) + fabsf(x1);
+      uint32_t w[3];
+      split3_pair(x0, x1, w);
+#pragma unroll
+      for (int part = 0; part < 3; ++part) *reinterpret_cast<uint32_t*>(prow + part * cip + f) = w[part];
+    }
+    if (kA) {
+      asum = warp_sum(asum);
+      if (lane == 0) a.A[p] = asum / static_cast<float>(ni);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pack_bf16x3(const PackBf16x3Args& a, cudaStream_t s) {
+  if (a.npix == 0) return cudaSuccess;
+  const int sms = current_sm_count();
+  int64_t blocks = ceil_div(a.npix, kPackThreads / 32);
+  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  if (blocks > cap) blocks = cap;
+  const dim3 grid(static_cast<unsigned>(blocks));
+  if (a.in_scale) {
+    if (a.A)
+      pack_bf16x3_kernel<true, true><<<grid, kPackThreads, 0, s>>>(a);
+    else
+      pack_bf16x3_kernel<true, false><<<grid, kPackThreads, 0, s>>>(a);
+  } else {
+    if (a.A)
+      pack_bf16x3_kernel<false, true><<<grid, kPackThreads, 0, s>>>(a);
+    else
+      pack_bf16x3_kernel<false, false><<<grid, kPackThreads, 0, s>>>(a);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace bconv

@@ -155,8 +155,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           const int tap = kb / a.kb_per_tap, cb = kb - tap * a.kb_per_tap;
           const int ky = tap / a.kw, kx = tap - ky * a.kw;
           for (int h = 0; h < a.mt; ++h)
-            tma_load_4d(sa + h * kABytes, &tmA, &B->full[stage], cb * 128, tc.ox0 + kx - a.kw / 2,
-                        tc.oy0 + ky - a.kh / 2, tc.n0 + h * a.Bn);
+            tma_load_4d(sa + h * kABytes, &tmA, &B->full[stage], cb * 128, tc.ox0 * a.sx + kx - a.kw / 2,
+                        tc.oy0 * a.sy + ky - a.kh / 2, tc.n0 + h * a.Bn);
           if (tc.bn == a.BN)
             tma_load_2d(sb, &tmB, &B->full[stage], kb * 128, tc.ntile * a.BN);
           else
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
         const TileCoord tc = tile_coord(a, t);
-        const uint32_t idesc = idesc_i8(tc.bn);
+        const uint32_t idesc = idesc_for(a.kind, 128, tc.bn);
         const int kb0 = tc.split * kb_per_split;
         const int kb1 = min(kb0 + kb_per_split, kb_total);
         if (!mbar_wait(&B->tmem_empty[acc], acc_phase ^ 1u, B, a.err)) break;
@@ -195,9 +195,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           for (int h = 0; h < a.mt; ++h) {
             const uint64_t da = smem_desc_sw128(sa + h * kABytes);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)  // four K=32 steps across the 128-byte row
-              tc_mma_i8(d_tmem + static_cast<uint32_t>(h * a.BN), da + 2u * j, db + 2u * j, idesc,
-                        (kb > kb0 || j > 0) ? 1u : 0u);
+            for (int j = 0; j < 4; ++j) {  // four 32-byte K steps across the 128-byte row
+              const uint32_t accum = (kb > kb0 || j > 0) ? 1u : 0u;
+              if (a.kind)
+                tc_mma_bf16(d_tmem + static_cast<uint32_t>(h * a.BN), da + 2u * j, db + 2u * j, idesc, accum);
+              else
+                tc_mma_i8(d_tmem + static_cast<uint32_t>(h * a.BN), da + 2u * j, db + 2u * j, idesc, accum);
+            }
           }
           tc_commit(&B->empty[stage]);
           if (++stage == kStages) {
@@ -248,10 +252,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           const float* An = a.A + static_cast<int64_t>(n) * a.H * a.W;
           float s = 0.f;
           for (int dy = -(a.kh / 2); dy <= (a.kh - 1) / 2; ++dy) {
-            const int y = oy + dy;
+            const int y = oy * a.sy + dy;  // window centred on input (oy*sy, ox*sx)
             if (y < 0 || y >= a.H) continue;
             for (int dx = -(a.kw / 2); dx <= (a.kw - 1) / 2; ++dx) {
-              const int x = ox + dx;
+              const int x = ox * a.sx + dx;
               if (x < 0 || x >= a.W) continue;
               s += __ldg(An + static_cast<int64_t>(y) * a.W + x);
             }
@@ -282,14 +286,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           float y[32];
           if (kSplit) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) y[j] = static_cast<float>(static_cast<int32_t>(v[j]));
+            for (int j = 0; j < 32; ++j) y[j] = acc_value(a.kind, v[j]);
           } else {
             const float4* sb4 = reinterpret_cast<const float4*>(&B->sb[tc.noff + ch * 32]);
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
               const float4 p = sb4[j / 2];  // (scale, bias) of channels j, j+1 (same for all lanes)
-              const float s0 = static_cast<float>(static_cast<int32_t>(v[j]));
-              const float s1 = static_cast<float>(static_cast<int32_t>(v[j + 1]));
+              const float s0 = acc_value(a.kind, v[j]);
+              const float s1 = acc_value(a.kind, v[j + 1]);
               float r0 = has_beta ? fmaf(s0 * p.x, beta, p.y) : fmaf(s0, p.x, p.y);
               float r1 = has_beta ? fmaf(s1 * p.z, beta, p.w) : fmaf(s1, p.z, p.w);
               if (a.relu) {

@@ -13,6 +13,8 @@ namespace bconv {
 struct TcArgs {
   int N, Ho, Wo;
   int kh, kw;          // window (1 x 1 for the FC)
+  int sy, sx;          // stride (the activation map steps the box by it)
+  int kind;            // 0: int8 codes, s32 accumulator; 1: bf16 parts, f32 accumulator
   int kb_per_tap;      // 128-byte channel blocks per tap
   int BN;              // output channels per tile (multiple of 32, <= 256)
   int n_tiles;         // ceil(No / BN)
@@ -68,5 +70,20 @@ struct PackI8Args {
   int op;                 // kXnor or kAnd
 };
 cudaError_t launch_pack_i8(const PackI8Args& a, cudaStream_t s);
+
+// binaryWeights operand for the tensor cores: x~ split exactly into three bf16 parts,
+// x~ = hi + mid + lo (hi = bf16(x~), mid = bf16(x~ - hi), lo = bf16(x~ - hi - mid); each
+// difference is exact in fp32), stored per pixel as [part][cip] bf16; channels in [ni, cip) are 0.
+struct PackBf16x3Args {
+  const float* in;        // [npix][ni]
+  int64_t npix;
+  int ni;
+  int cip;                // channels per part (multiple of 64)
+  const float* in_scale;  // [ni] or nullptr
+  const float* in_bias;   // [ni] or nullptr
+  uint16_t* parts;        // [npix][3][cip] bf16 bits
+  float* A;               // [npix] or nullptr
+};
+cudaError_t launch_pack_bf16x3(const PackBf16x3Args& a, cudaStream_t s);
 
 }  // namespace bconv

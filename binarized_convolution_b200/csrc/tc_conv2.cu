@@ -82,6 +82,15 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                                uint32_t accumulate) {
   asm volatile(
@@ -100,11 +109,6 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
           smem_u32(bar)),
       "h"(mask)
       : "memory");
-}
-
-// Instruction descriptor: s32 accumulator, signed int8 A and B, K-major, M = 256, N = bn.
-__host__ __device__ constexpr uint32_t idesc_i8_m256(int bn) {
-  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(bn >> 3) << 17) | ((256u >> 4) << 24);
 }
 
 struct PairCoord {
@@ -206,7 +210,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
           if (leader) mbar_expect_tx(&B->full[stage], tx);
           const int tap = kb / a.kb_per_tap, cb = kb - tap * a.kb_per_tap;
           const int ky = tap / a.kw, kx = tap - ky * a.kw;
-          tma_load_4d_pair(sa, &tmA, full_leader, cb * 128, pc.ox0 + kx - a.kw / 2, pc.oy0 + ky - a.kh / 2, pc.n0);
+          tma_load_4d_pair(sa, &tmA, full_leader, cb * 128, pc.ox0 * a.sx + kx - a.kw / 2, pc.oy0 * a.sy + ky - a.kh / 2, pc.n0);
           const int brow = pc.ntile * a.BN + pc.noff + static_cast<int>(rank) * (pc.bn / 2);
           if (pc.bn == a.BN)
             tma_load_2d_pair(sb, &tmB, full_leader, kb * 128, brow);
@@ -229,7 +233,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
       bool ok = true;
       for (int w = pair; w < total && ok; w += npairs) {
         const PairCoord pc = pair_coord(a, w, 0);
-        const uint32_t idesc = idesc_i8_m256(pc.bn);
+        const uint32_t idesc = idesc_for(a.kind, 256, pc.bn);
         if (!mbar_wait(&B->tmem_empty[acc], acc_phase ^ 1u, B, a.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
@@ -242,8 +246,13 @@ __global__ void __launch_bounds__(kThreads2, 1)
           uint8_t* sa = smem + stage * stage_bytes;
           const uint64_t da = smem_desc_sw128(sa), db = smem_desc_sw128(sa + kABytes2);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tc_mma_i8_pair(d_tmem, da + 2u * j, db + 2u * j, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t accum = (kb > 0 || j > 0) ? 1u : 0u;
+            if (a.kind)
+              tc_mma_bf16_pair(d_tmem, da + 2u * j, db + 2u * j, idesc, accum);
+            else
+              tc_mma_i8_pair(d_tmem, da + 2u * j, db + 2u * j, idesc, accum);
+          }
           tc_commit_pair(&B->empty[stage]);
           if (++stage == kStages2) {
             stage = 0;
@@ -288,10 +297,10 @@ __global__ void __launch_bounds__(kThreads2, 1)
         const float* An = a.A + static_cast<int64_t>(n) * a.H * a.W;
         float s = 0.f;
         for (int dy = -(a.kh / 2); dy <= (a.kh - 1) / 2; ++dy) {
-          const int y = oy + dy;
+          const int y = oy * a.sy + dy;  // window centred on input (oy*sy, ox*sx)
           if (y < 0 || y >= a.H) continue;
           for (int dx = -(a.kw / 2); dx <= (a.kw - 1) / 2; ++dx) {
-            const int x = ox + dx;
+            const int x = ox * a.sx + dx;
             if (x < 0 || x >= a.W) continue;
             s += __ldg(An + static_cast<int64_t>(y) * a.W + x);
           }
@@ -320,8 +329,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const float4 p = sb4[j / 2];
-          const float s0 = static_cast<float>(static_cast<int32_t>(v[j]));
-          const float s1 = static_cast<float>(static_cast<int32_t>(v[j + 1]));
+          const float s0 = acc_value(a.kind, v[j]);
+          const float s1 = acc_value(a.kind, v[j + 1]);
           float r0 = has_beta ? fmaf(s0 * p.x, beta, p.y) : fmaf(s0, p.x, p.y);
           float r1 = has_beta ? fmaf(s1 * p.z, beta, p.w) : fmaf(s1, p.z, p.w);
           if (a.relu) {

@@ -131,6 +131,28 @@ __device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D[tmem] (+)= A * B^T with bf16 operands and an fp32 accumulator (kind::f16, K = 16).
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor for M = m, N = n, K-major operands: kind 0 = signed int8 with an s32
+// accumulator, kind 1 = bf16 with an f32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_for(int kind, int m, int n) {
+  return (kind == 0 ? ((2u << 4) | (1u << 7) | (1u << 10)) : ((1u << 4) | (1u << 7) | (1u << 10))) |
+         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// Accumulator word -> fp32 value of the window sum.
+__device__ __forceinline__ float acc_value(int kind, uint32_t v) {
+  return kind ? __uint_as_float(v) : static_cast<float>(static_cast<int32_t>(v));
+}
+
 // 32 consecutive 32-bit columns of this warp's 32 TMEM lanes.
 __device__ __forceinline__ void tc_ld_32x32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
@@ -156,10 +178,6 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
   return d;
 }
 
-// Instruction descriptor: s32 accumulator, signed int8 A and B, both K-major, M=128, N=bn.
-__host__ __device__ constexpr uint32_t idesc_i8(int bn) {
-  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(bn >> 3) << 17) | ((128u >> 4) << 24);
-}
 
 
 }  // namespace tcdev

@@ -72,9 +72,11 @@ typedef enum {
   BCONV_ALGO_AUTO = 0,
   BCONV_ALGO_POPC = 1,     /* XNOR/AND: LOP3 XOR/AND + POPC into int32 registers     */
   BCONV_ALGO_SIMT_F32 = 2, /* binaryWeights: FP32 signed-add contraction on the SIMT */
-  BCONV_ALGO_TCGEN05 = 3   /* XNOR/AND: +-1 / {0,1} int8 codes on the tcgen05 tensor
-                              cores, int32 accumulation in TMEM (stride 1 or the FC, and
-                              out_channels % 4 == 0); exact, like the POPC family */
+  BCONV_ALGO_TCGEN05 = 3   /* tcgen05 tensor cores, for out_channels % 4 == 0:
+                              XNOR/AND as +-1 / {0,1} int8 codes with int32 accumulation in
+                              TMEM (exact, like the POPC family); binaryWeights as three exact
+                              bf16 parts of the input against +-1 bf16 weights, fp32
+                              accumulation */
 } bconv_algo_t;
 
 /*

@@ -44,15 +44,14 @@ def make_layer(w: synth.Workload, inp: synth.Inputs, *, sums: bool = False):
 
 
 def algo_for(w: synth.Workload, name: str):
-    """Library algorithm code for a test parameter: 'auto', or 'popc' (XNOR/AND only; None
-    for binaryWeights, which has one kernel family)."""
+    """Library algorithm code for a test parameter: 'auto' (the library's choice: the tensor
+    cores where they apply) or 'alt' (the SIMT family: POPC for XNOR/AND, the FP32 signed-add
+    kernel for binaryWeights)."""
     import binarized_convolution_b200 as bc
 
     if name == "auto":
         return bc.ALGO_AUTO
-    if w.op == synth.BINARY_WEIGHTS:
-        return None
-    return bc.ALGO_POPC
+    return bc.ALGO_SIMT_F32 if w.op == synth.BINARY_WEIGHTS else bc.ALGO_POPC
 
 
 def run_device(w: synth.Workload, inp: synth.Inputs, *, sums: bool = False, algo=None):

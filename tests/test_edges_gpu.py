@@ -15,14 +15,17 @@ pytestmark = pytest.mark.gpu
 
 
 def _check(w, inp=None):
+    """Both kernel families (the library's choice and the SIMT one) against the oracle."""
     inp = inp if inp is not None else synth.make_inputs(w)
     S_ref, beta_ref, y_ref = pu.run_oracle(w, inp)
-    y = pu.run_device(w, inp)
-    pu.assert_outputs_close(w, inp, y, S_ref, beta_ref, y_ref)
-    if w.op != synth.BINARY_WEIGHTS:
-        S_dev = pu.run_device(w, inp, sums=True)
-        S_sum, _, _ = pu.run_oracle(w, inp, sums=True)
-        pu.assert_sums_exact(S_dev, S_sum)
+    S_sum, _, _ = pu.run_oracle(w, inp, sums=True)
+    for name in ("auto", "alt"):
+        a = pu.algo_for(w, name)
+        y = pu.run_device(w, inp, algo=a)
+        pu.assert_outputs_close(w, inp, y, S_ref, beta_ref, y_ref)
+        if w.op != synth.BINARY_WEIGHTS:
+            S_dev = pu.run_device(w, inp, sums=True, algo=a)
+            pu.assert_sums_exact(S_dev, S_sum)
 
 
 SWEEP = []

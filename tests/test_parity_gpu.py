@@ -43,12 +43,10 @@ MEDIUM = [
 ]
 
 
-@pytest.mark.parametrize("algo", ["auto", "popc"])
+@pytest.mark.parametrize("algo", ["auto", "alt"])
 @pytest.mark.parametrize("w", MEDIUM, ids=lambda w: w.name)
 def test_medium_all_outputs(w, algo, cuda_device):
     a = pu.algo_for(w, algo)
-    if a is None:
-        pytest.skip("binaryWeights has a single kernel family")
     inp = synth.make_inputs(w)
     S_ref, beta_ref, y_ref = pu.run_oracle(w, inp)
     y = pu.run_device(w, inp, algo=a)
@@ -63,13 +61,11 @@ def test_medium_all_outputs(w, algo, cuda_device):
         pu.assert_sums_exact(S_dev, S_sum)
 
 
-@pytest.mark.parametrize("algo", ["auto", "popc"])
+@pytest.mark.parametrize("algo", ["auto", "alt"])
 @pytest.mark.parametrize("idx", range(5), ids=lambda i: synth.WORKLOAD_ORDER[i])
 def test_workload_full_size(idx, algo, cuda_device):
     w = synth.workload(idx)
     a = pu.algo_for(w, algo)
-    if a is None:
-        pytest.skip("binaryWeights has a single kernel family")
     inp = synth.make_inputs(w)
     rows = pu.sample_rows(w, seed=idx)
     y = pu.run_device(w, inp, algo=a)
