@@ -14,6 +14,7 @@ from .oracle import (  # noqa: F401
     SOURCE_PATH,
     Variant,
     compile_source,
+    binarize,
     build,
     conv,
     conv_out_dims,

@@ -197,6 +197,33 @@ int oracle_bfc(int32_t batch, int32_t H, int32_t W, int32_t Ni, int32_t No, int3
   return 0;
 }
 
+/*
+ * The binarized form of an fp32 image, as the next binary layer sees it: per pixel and
+ * channel x~ = inScale[c] * x + inBias[c], the sign bit bin(x~) as 1 (x~ >= 0) or 0, and the
+ * per-pixel mean of |x~| over the channels (the "A" of the beta formula).  This is what a
+ * binary convolution does to its input before the sum (same page, same paragraphs as
+ * above); applied to one layer's output with the following layer's input terms it gives
+ * the following layer's view of that output.
+ *   x       [npix][C] fp32
+ *   bits    [npix][C] uint8 0/1, may be NULL
+ *   A       [npix] mean |x~|, may be NULL
+ *   xt      [npix][C] x~ in double (before the sign decision), may be NULL
+ */
+int oracle_binarize(const float* x, int64_t npix, int32_t C, const float* in_scale, const float* in_bias,
+                    uint8_t* bits, double* A, double* xt) {
+  if (!x || npix < 0 || C <= 0) return -1;
+#pragma omp parallel for schedule(static)
+  for (int64_t p = 0; p < npix; ++p) {
+    for (int32_t c = 0; c < C; ++c) {
+      const double v = transformed_input(x, in_scale, in_bias, p, C, c);
+      if (bits) bits[p * C + c] = (uint8_t)bin_01(v);
+      if (xt) xt[p * C + c] = v;
+    }
+    if (A) A[p] = channel_mean_abs(x, in_scale, in_bias, p, C);
+  }
+  return 0;
+}
+
 /* Number of threads an OpenMP parallel region of the oracle uses (1 without OpenMP). */
 int oracle_num_threads(void) {
   int n = 1;

@@ -57,6 +57,8 @@ def _bind(path: str):
     lib.oracle_bconv.argtypes = [ctypes.POINTER(_ConvDesc)] + [P] * 7 + [ctypes.c_int64] + [P] * 3
     lib.oracle_bfc.restype = ctypes.c_int
     lib.oracle_bfc.argtypes = [ctypes.c_int32] * 8 + [P] * 7 + [ctypes.c_int64] + [P] * 3
+    lib.oracle_binarize.restype = ctypes.c_int
+    lib.oracle_binarize.argtypes = [P, ctypes.c_int64, ctypes.c_int32] + [P] * 5
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
 
@@ -94,6 +96,9 @@ class Variant:
 
     def fc(self, *args, **kw):
         return fc(*args, _lib_override=self._lib, **kw)
+
+    def binarize(self, *args, **kw):
+        return binarize(*args, _lib_override=self._lib, **kw)
 
 
 def compile_source(src: str, out_path: str) -> str:
@@ -186,3 +191,22 @@ def fc(x, wbits, *, type: int, _lib_override=None, scale=None, scale_value: floa
     if rc != 0:
         raise ValueError("oracle_bfc rejected its arguments")
     return S, beta, y
+
+
+def binarize(x, *, _lib_override=None, in_scale=None, in_bias=None):
+    """Oracle binarization of an fp32 image as the next binary layer sees it.
+
+    x float32 [..., C] (any leading shape).  Returns (bits, A, xt): bits uint8 {0,1} with
+    x's shape, A float64 with the leading shape, xt float64 (the transformed values).
+    """
+    x = _f32(x)
+    lead, c = x.shape[:-1], x.shape[-1]
+    npix = int(np.prod(lead)) if lead else 1
+    bits = np.empty(x.shape, np.uint8)
+    A = np.empty(lead, np.float64)
+    xt = np.empty(x.shape, np.float64)
+    rc = (_lib_override or _load()).oracle_binarize(_ptr(x), npix, c, _ptr(_f32(in_scale)), _ptr(_f32(in_bias)),
+                                                    _ptr(bits), _ptr(A), _ptr(xt))
+    if rc != 0:
+        raise ValueError("oracle_binarize rejected its arguments")
+    return bits, A, xt

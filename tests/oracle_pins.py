@@ -353,8 +353,63 @@ def pin_epilogue(orc):
         np.testing.assert_allclose(y5, y1 * beta[:, None], rtol=1e-15)
 
 
+# ----------------------------------------------------------------------------------------
+# The binarized view of an image (what a following binary layer reads)
+# ----------------------------------------------------------------------------------------
+def pin_binarize_golden(orc):
+    """Hand-worked bits and A (tests/golden/binarize_examples.txt): input terms before the
+    sign, bin(+-0) = +1, the sign decided in fp32, A = mean |x~| (MPSCNNBinaryConvolution)."""
+    terms, xs, bits, As = {}, {}, {}, {}
+    for row in _rows("binarize_examples.txt"):
+        tag, idx, vals = row[0], int(row[1]), row[2:]
+        if tag == "T":
+            terms[idx] = (float(vals[0]), float(vals[1]))
+        elif tag == "P":
+            xs[idx] = [float(v) for v in vals]
+        elif tag == "B":
+            bits[idx] = [int(v) for v in vals]
+        elif tag == "A":
+            As[idx] = float(vals[0])
+    c = len(terms)
+    s = np.array([terms[i][0] for i in range(c)], np.float32)
+    b = np.array([terms[i][1] for i in range(c)], np.float32)
+    x = np.array([xs[p] for p in sorted(xs)], np.float32)
+    got_bits, got_A, _ = orc.binarize(x, in_scale=s, in_bias=b)
+    np.testing.assert_array_equal(got_bits, np.array([bits[p] for p in sorted(bits)], np.uint8))
+    np.testing.assert_allclose(got_A, np.array([As[p] for p in sorted(As)]), rtol=1e-12)
+
+
+def pin_binarize_is_the_conv_input(orc):
+    """The bits and A of the binarized view are exactly what the (separately pinned) binary
+    convolution sums and averages: brute-force XNOR/AND sums over the bits equal the conv's S,
+    and the window mean of A equals its beta."""
+    rng = np.random.default_rng(41)
+    n, h, w, ni, no = 2, 5, 6, 37, 4
+    x, wb = _rand_case(rng, n, h, w, ni, no, 3, 3)
+    in_scale = rng.uniform(-1.5, 1.5, ni).astype(np.float32)
+    in_bias = rng.normal(0, 0.5, ni).astype(np.float32)
+    bits, A, xt = orc.binarize(x, in_scale=in_scale, in_bias=in_bias)
+    assert bits.shape == x.shape and A.shape == x.shape[:3]
+    assert 0 < bits.mean() < 1
+    pad = ((0, 0), (1, 1), (1, 1), (0, 0))
+    for op in (XNOR, AND):
+        a = (2.0 * bits - 1.0) if op == XNOR else bits.astype(np.float64)
+        wv = (2.0 * wb - 1.0) if op == XNOR else wb.astype(np.float64)
+        ap = np.pad(a, pad)
+        ref = np.zeros((n, h, w, no))
+        for oy in range(h):
+            for ox in range(w):
+                ref[:, oy, ox, :] = np.einsum("nhwf,chwf->nc", ap[:, oy:oy + 3, ox:ox + 3, :], wv)
+        S, beta, _ = orc.conv(x, wb, type=op, in_scale=in_scale, in_bias=in_bias, use_beta=True)
+        np.testing.assert_array_equal(S, ref.reshape(-1, no))
+        Ap = np.pad(A, ((0, 0), (1, 1), (1, 1)))
+        bref = np.stack([Ap[:, oy:oy + 3, ox:ox + 3].sum(axis=(1, 2)) / 9.0 for oy in range(h) for ox in range(w)], 1)
+        np.testing.assert_allclose(beta, bref.reshape(-1), rtol=1e-12)
+    np.testing.assert_allclose(np.abs(xt).mean(axis=-1), A, rtol=1e-12)
+
+
 ALL_PINS = [
     pin_truth_table, pin_pm1_products, pin_word_results, pin_brute_force_tiny, pin_torch_conv2d,
     pin_signed_zero, pin_fc_matvec, pin_fc_is_conv_at_centre, pin_beta_closed_form, pin_input_terms,
-    pin_invariants, pin_epilogue,
+    pin_invariants, pin_epilogue, pin_binarize_golden, pin_binarize_is_the_conv_input,
 ]

@@ -34,6 +34,14 @@ MUTANTS = [
     ("fc_beta_divisor", "beta = acc / ((double)H * (double)W);", "beta = acc / ((double)H * (double)H);"),
     ("fc_weight_flatten", "const uint8_t* wrow = wbits + (int64_t)c * K;\n      double acc = 0.0;\n      for (int64_t k = 0; k < K; ++k) {\n        const int32_t f = (int32_t)(k % Ni);\n        acc += op_term(type, transformed_input(img, in_scale, in_bias, k / Ni, Ni, f), wrow[k]);",
      "const uint8_t* wrow = wbits + (int64_t)c * K;\n      double acc = 0.0;\n      for (int64_t k = 0; k < K; ++k) {\n        const int32_t f = (int32_t)(k % Ni);\n        acc += op_term(type, transformed_input(img, in_scale, in_bias, k / Ni, Ni, f), wrow[(k % Ni) * (K / Ni) + k / Ni]);"),
+    ("binarize_polarity", "if (bits) bits[p * C + c] = (uint8_t)bin_01(v);",
+     "if (bits) bits[p * C + c] = (uint8_t)(1.0 - bin_01(v));"),
+    ("binarize_sign_in_double", "if (bits) bits[p * C + c] = (uint8_t)bin_01(v);",
+     "if (bits) bits[p * C + c] = (uint8_t)(v < 0.0 ? 0 : 1);"),
+    ("binarize_without_terms", "const double v = transformed_input(x, in_scale, in_bias, p, C, c);",
+     "const double v = transformed_input(x, NULL, NULL, p, C, c);"),
+    ("binarize_A_of_first_pixel", "if (A) A[p] = channel_mean_abs(x, in_scale, in_bias, p, C);",
+     "if (A) A[p] = channel_mean_abs(x, in_scale, in_bias, 0, C);"),
 ]
 
 
