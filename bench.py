@@ -1,7 +1,7 @@
 """Throughput of the binary convolution on B200: one JSON line per run.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                    [--workload NAME|INDEX] [--no-e2e] [--no-cpu-baseline]
+                    [--workload NAME|INDEX] [--io f32|bits] [--no-e2e] [--no-cpu-baseline]
 
 A step is one forward of the layer (input transform + pack + A, beta, contraction and
 epilogue) over one batch of the workload: by default XNOR with beta scaling and input terms,
@@ -12,6 +12,10 @@ when it is next used (411 MB > the 126 MB L2).  ``e2e`` is the same metric throu
 bconv_forward_host with page-locked host buffers (host-to-device copy, forward,
 device-to-host copy inside every step).  Multi-GPU runs (torchrun) are independent replicas
 with a batch each (weak scaling); their time is the maximum over ranks.
+
+``--io bits`` times the same layer as the middle of a chain of such layers instead: it reads
+the bit-packed output of the previous layer (sign bits and A) and writes its own for the next
+(bconv_forward_io); the input terms move to the previous layer's epilogue.
 
 ``--impl reference`` times the oracle (the plain double-precision CPU loops) on the same
 workload, each step a bounded sample of output pixels, on rank 0 only.
@@ -40,6 +44,7 @@ DEFAULT_WORKLOAD = "xnor_beta_n16_56x56_c256_k256_3x3"
 METRIC = "binary conv TOPS (1 op = 1 bit MAC) and images/s on 1 B200; % of roofline"
 UNIT = "TOPS"
 ROTATE = 4
+ROTATE_BITS = 40  # bit-packed sets are 32x smaller: 40 of them exceed the L2
 POPC_PER_CLK_PER_SM = 16  # 32-bit POPC lanes per clock per SM
 FP32_PER_CLK_PER_SM = 128  # FFMA lanes per clock per SM
 
@@ -280,11 +285,46 @@ def run_native(args, w: synth.Workload):
     xs = [torch.from_numpy(inp.x).to(device)]
     for r in range(1, ROTATE):
         xs.append(torch.from_numpy(synth.make_batch(w, seed=replica_seed(w.seed, rank) * 1000 + r)).to(device))
-    ys = [torch.empty(out_shape, dtype=torch.float32, device=device) for _ in range(ROTATE)]
     stream = torch.cuda.current_stream(device)
+    bits_io = args.io == "bits"
+    if bits_io:
+        # A middle layer of a chain of identical layers: it reads the bit-packed output of the
+        # previous one (made here by the same layer with fp32 input) and writes its own for the
+        # next, whose input terms are this layer's.  The timed layer has no input terms.
+        if w.kind == "fc" or w.op == synth.BINARY_WEIGHTS or w.in_channels != w.out_channels or \
+                (w.stride_y, w.stride_x) != (1, 1):
+            raise SystemExit("--io bits needs an XNOR/AND convolution with in = out channels and stride 1")
+        layer.set_output_terms(inp.in_scale, inp.in_bias)
+        feeds = [layer.forward_to_bits(x) for x in xs]
+        del xs
+        for r in range(ROTATE, ROTATE_BITS):  # enough sets that one step's data has left L2
+            x = torch.from_numpy(synth.make_batch(w, seed=replica_seed(w.seed, rank) * 1000 + r)).to(device)
+            feeds.append(layer.forward_to_bits(x))
+            del x
+        torch.cuda.synchronize(device)
+        layer.close()
+        layer = bc.BinaryConv2d(w.batch, w.in_h, w.in_w, w.in_channels, w.out_channels, (w.kernel_h, w.kernel_w),
+                                (w.stride_y, w.stride_x), wbits=inp.wbits, op=w.op, scale=inp.scale, bias=inp.bias,
+                                use_beta=w.use_beta, relu=w.relu)
+        if args.algo != "auto":
+            layer.set_algo({"popc": bc.ALGO_POPC, "tcgen05": bc.ALGO_TCGEN05}[args.algo])
+        layer.set_output_terms(inp.in_scale, inp.in_bias)
+        bshape, ashape = layer.bits_shape()
+        outs = [(torch.empty(bshape, dtype=torch.int32, device=device), torch.empty(ashape, device=device))
+                for _ in range(ROTATE_BITS)]
+
+        def fwd(i):
+            xb, xa = feeds[i % ROTATE_BITS]
+            ob, oa = outs[i % ROTATE_BITS]
+            layer.forward_io(x_bits=xb, x_a=xa if w.use_beta else None, out_bits=ob, out_a=oa)
+    else:
+        ys = [torch.empty(out_shape, dtype=torch.float32, device=device) for _ in range(ROTATE)]
+
+        def fwd(i):
+            layer.forward_into(xs[i % ROTATE], ys[i % ROTATE])
 
     for i in range(args.warmup):
-        layer.forward_into(xs[i % ROTATE], ys[i % ROTATE])
+        fwd(i)
     layer.sync_status(stream.cuda_stream)
     torch.cuda.synchronize(device)
 
@@ -295,7 +335,7 @@ def run_native(args, w: synth.Workload):
     torch.cuda.synchronize(device)
     ev0.record(stream)
     for i in range(args.steps):
-        layer.forward_into(xs[i % ROTATE], ys[i % ROTATE])
+        fwd(i)
     ev1.record(stream)
     torch.cuda.synchronize(device)
     barrier(device)
@@ -346,8 +386,13 @@ def run_native(args, w: synth.Workload):
                    "kernel": [w.kernel_h, w.kernel_w], "stride": [w.stride_y, w.stride_x], "op": w.op,
                    "beta": w.use_beta, "relu": w.relu, "input_terms": w.in_terms,
                    "parallelism": f"replicas x{world}", "algo": kname,
-                   "l2": f"{ROTATE} rotating input/output sets, "
-                         f"{ROTATE * (inp.x.nbytes + int(np.prod(out_shape)) * 4) / 1e6:.0f} MB > 126 MB L2"},
+                   "io": "bit-packed in and out (chain middle layer)" if bits_io else "fp32 in and out",
+                   "l2": (f"{ROTATE} rotating input/output sets, "
+                          f"{ROTATE * (inp.x.nbytes + int(np.prod(out_shape)) * 4) / 1e6:.0f} MB > 126 MB L2")
+                   if not bits_io else
+                   f"{ROTATE_BITS} rotating bit-packed input/output sets, "
+                   f"{ROTATE_BITS * 2 * (int(np.prod(out_shape)) // 8 + int(np.prod(out_shape[:3])) * 4) / 1e6:.0f}"
+                   f" MB > 126 MB L2"},
         "images_per_s": images_s,
         "roofline": roof,
         "clocks": clock_info,
@@ -355,7 +400,7 @@ def run_native(args, w: synth.Workload):
     }
 
     # end to end through the C ABI with page-locked host buffers
-    if not args.no_e2e:
+    if not args.no_e2e and not bits_io:
         e2e_steps = max(3, min(args.steps, 20))
         hin = torch.from_numpy(inp.x).pin_memory()
         hout = torch.empty(out_shape, dtype=torch.float32).pin_memory()
@@ -445,6 +490,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--algo", choices=["auto", "popc", "tcgen05", "simt_f32"], default="auto",
                     help="kernel family of the contraction (auto = the library's choice)")
+    ap.add_argument("--io", choices=["f32", "bits"], default="f32",
+                    help="bits: time a middle layer of a chain (bit-packed input and output)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time of the cpu_baseline sample")

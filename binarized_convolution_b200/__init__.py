@@ -32,6 +32,11 @@ from ._native import (  # noqa: F401
     bconv_forward,
     bconv_forward_host,
     bconv_forward_noalloc,
+    bconv_forward_io,
+    bconv_set_output_terms,
+    bconv_io_t,
+    bfc_forward_io,
+    bfc_set_output_terms,
     NOALLOC_SCRATCH_BYTES,
     bconv_get_output_dims,
     bconv_input_feature_channels,

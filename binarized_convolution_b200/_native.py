@@ -46,6 +46,10 @@ class bfc_desc_t(ctypes.Structure):
                                               "stride_x", "groups", "neuron")] + [("scale_value", ctypes.c_float)]
 
 
+class bconv_io_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("in_", "in_bits", "in_a", "out", "out_bits", "out_a")]
+
+
 _lock = threading.Lock()
 _lib = None
 _P = ctypes.c_void_p
@@ -81,6 +85,10 @@ _SIGS = {
     "bconv_version": (_I32, []),
     "bconv_measure_peak": (_I32, [_I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
     "bconv_forward_noalloc": (_I32, [ctypes.POINTER(bconv_desc_t), _I32, ctypes.c_uint32] + [_P] * 8),
+    "bconv_set_output_terms": (_I32, [_P, _P, _P]),
+    "bconv_forward_io": (_I32, [_P, ctypes.POINTER(bconv_io_t), _P]),
+    "bfc_set_output_terms": (_I32, [_P, _P, _P]),
+    "bfc_forward_io": (_I32, [_P, ctypes.POINTER(bconv_io_t), _P]),
 }
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -169,6 +177,34 @@ def bfc_create(desc: bfc_desc_t, packed_weights, scale=None, bias=None, in_scale
 
 def bconv_forward(h, in_ptr: int, out_ptr: int, stream: int = 0):
     _check(load_library().bconv_forward(h, in_ptr, out_ptr, stream), "bconv_forward")
+
+
+def bconv_set_output_terms(h, next_in_scale=None, next_in_bias=None):
+    """Host arrays of out_channels floats (None: 1 / 0) for the layer that reads the bits."""
+    no = bconv_output_feature_channels(h)
+    s, b = _host_f32(next_in_scale, no, "next_in_scale"), _host_f32(next_in_bias, no, "next_in_bias")
+    _check(load_library().bconv_set_output_terms(h, _ptr(s), _ptr(b)), "bconv_set_output_terms")
+
+
+def bconv_forward_io(h, in_ptr: int | None = None, in_bits_ptr: int | None = None, in_a_ptr: int | None = None,
+                     out_ptr: int | None = None, out_bits_ptr: int | None = None, out_a_ptr: int | None = None,
+                     stream: int = 0):
+    """Forward with fp32 or bit-packed input and output (device addresses; see bconv_io_t)."""
+    io = bconv_io_t(in_ptr, in_bits_ptr, in_a_ptr, out_ptr, out_bits_ptr, out_a_ptr)
+    _check(load_library().bconv_forward_io(h, ctypes.byref(io), stream), "bconv_forward_io")
+
+
+def bfc_set_output_terms(h, next_in_scale=None, next_in_bias=None):
+    no = bfc_output_feature_channels(h)
+    s, b = _host_f32(next_in_scale, no, "next_in_scale"), _host_f32(next_in_bias, no, "next_in_bias")
+    _check(load_library().bfc_set_output_terms(h, _ptr(s), _ptr(b)), "bfc_set_output_terms")
+
+
+def bfc_forward_io(h, in_ptr: int | None = None, in_bits_ptr: int | None = None, in_a_ptr: int | None = None,
+                   out_ptr: int | None = None, out_bits_ptr: int | None = None, out_a_ptr: int | None = None,
+                   stream: int = 0):
+    io = bconv_io_t(in_ptr, in_bits_ptr, in_a_ptr, out_ptr, out_bits_ptr, out_a_ptr)
+    _check(load_library().bfc_forward_io(h, ctypes.byref(io), stream), "bfc_forward_io")
 
 
 def bfc_forward(h, in_ptr: int, out_ptr: int, stream: int = 0):

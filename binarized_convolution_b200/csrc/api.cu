@@ -127,6 +127,14 @@ struct Layer {
   TcArgs tc{};
   CUtensorMap tmA{}, tmB{}, tmBp{}, tmWs{}, tmOut{};
   const float* tm_out_ptr = nullptr;
+  // chained layers: the next layer's input terms (bit-packed output) and what emitting the
+  // bits needs -- the slice partials of A on the tensor-core path, an fp32 output buffer
+  // for the kernel families that binarize in a separate pass
+  bool has_next = false;
+  float *next_scale = nullptr, *next_bias = nullptr;
+  float* a_part = nullptr;
+  uint32_t* a_count = nullptr;
+  float* y_scratch = nullptr;
   // host-buffer forward staging (allocated on first use)
   float *stage_in = nullptr, *stage_out = nullptr;
   DevMem mem;
@@ -462,11 +470,29 @@ bool use_tc(const Layer& L) {
   return L.tc_ok && (L.algo == BCONV_ALGO_AUTO || L.algo == BCONV_ALGO_TCGEN05);
 }
 
+// The input and output forms of one forward: fp32 (in / out) or bit-packed (bits + A).
+struct Io {
+  const float* in = nullptr;
+  const uint32_t* in_bits = nullptr;
+  const float* in_a = nullptr;
+  float* out = nullptr;
+  uint32_t* out_bits = nullptr;
+  float* out_a = nullptr;
+};
+
+// Whether the tensor-core epilogue writes the bit-packed output itself.
+bool tc_emits_bits(const Layer& L) { return use_tc(L) && !L.fc && L.tc.k_splits == 1; }
+
 // Tensor-core forward: int8 codes (+ A) -> [beta] -> tcgen05 contraction [-> finalize].
-bconv_status_t run_forward_tc(Layer& L, const float* in, float* out, cudaStream_t s) {
+bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
+  const float* in = io.in;
+  float* out = io.out;
   const bool beta = L.use_beta();
+  const float* A = io.in_bits ? io.in_a : L.A;
   cudaError_t e;
-  if (L.tc.kind == 0) {
+  if (io.in_bits) {
+    e = launch_unpack_bits_i8(io.in_bits, static_cast<int64_t>(L.N) * L.H * L.W, L.Ni, L.cip, L.type, L.codes, s);
+  } else if (L.tc.kind == 0) {
     PackI8Args p{};
     p.in = in;
     p.npix = static_cast<int64_t>(L.N) * L.H * L.W;
@@ -492,17 +518,26 @@ bconv_status_t run_forward_tc(Layer& L, const float* in, float* out, cudaStream_
   }
   if (e != cudaSuccess) return from_cuda(e);
   if (beta && L.fc) {  // the convolution forms beta from A inside its epilogue
-    BetaArgs b{L.A, L.beta, L.N, L.H, L.W, L.Ho, L.Wo, L.kh, L.kw, L.sy, L.sx};
+    BetaArgs b{A, L.beta, L.N, L.H, L.W, L.Ho, L.Wo, L.kh, L.kw, L.sy, L.sx};
     e = launch_beta_image_mean(b, s);
     if (e != cudaSuccess) return from_cuda(e);
   }
   TcArgs t = L.tc;
   t.beta = beta ? L.beta : nullptr;
-  t.A = (beta && !L.fc) ? L.A : nullptr;
+  t.A = (beta && !L.fc) ? A : nullptr;
   t.H = L.H;
   t.W = L.W;
   const CUtensorMap* om = &L.tmWs;
-  if (t.k_splits > 1) {
+  if (io.out_bits) {  // the epilogue binarizes; the output map is not used
+    t.out_bits = io.out_bits;
+    t.out_a = io.out_a;
+    t.next_scale = L.next_scale;
+    t.next_bias = L.next_bias;
+    t.nwo = words_for(L.No);
+    t.a_part = L.a_part;
+    t.a_count = L.a_count;
+    om = &L.tmOut;
+  } else if (t.k_splits > 1) {
     e = cudaMemsetAsync(L.ws, 0, sizeof(float) * static_cast<size_t>(L.N) * L.No, s);
     if (e != cudaSuccess) return from_cuda(e);
   } else {
@@ -518,20 +553,24 @@ bconv_status_t run_forward_tc(Layer& L, const float* in, float* out, cudaStream_
   if (timed) cudaEventRecord(L.prof.stop[L.prof.used++], s);
   if (e != cudaSuccess) return from_cuda(e);
   if (t.k_splits > 1)
-    e = launch_tc_finalize(L.ws, out, L.scale, L.bias, t.beta, static_cast<int64_t>(L.N) * L.No, L.No, 1, L.relu, s);
+    e = launch_tc_finalize(L.ws, out, L.scale, L.bias, t.beta, L.N, L.No, L.relu, s);
   return from_cuda(e);
 }
 
-// The launch sequence of one forward.
-bconv_status_t run_forward(Layer& L, const float* in, float* out, cudaStream_t s) {
-  if (L.N > 0 && use_tc(L)) return run_forward_tc(L, in, out, s);
+// The launch sequence of one forward on the POPC / SIMT families (fp32 output).
+bconv_status_t run_forward_simt(Layer& L, const Io& io, cudaStream_t s) {
+  const float* in = io.in;
+  float* out = io.out;
   const int64_t npix = static_cast<int64_t>(L.N) * L.H * L.W;
-  if (L.N == 0) return BCONV_OK;
   cudaError_t e = cudaSuccess;
   const bool beta = L.use_beta();
+  const float* A = io.in_bits ? io.in_a : L.A;
 
-  // 1. input transform + sign + pack (+ A)
-  if (L.type != kBinaryWeights || beta) {
+  // 1. input transform + sign + pack (+ A), or the caller's bits into the padded layout
+  if (io.in_bits) {
+    e = launch_repack_bits(io.in_bits, npix, L.Ni, L.nw_pad, L.bits, s);
+    if (e != cudaSuccess) return from_cuda(e);
+  } else if (L.type != kBinaryWeights || beta) {
     PackArgs p{};
     p.in = in;
     p.npix = npix;
@@ -546,7 +585,7 @@ bconv_status_t run_forward(Layer& L, const float* in, float* out, cudaStream_t s
   }
   // 2. beta
   if (beta) {
-    BetaArgs b{L.A, L.beta, L.N, L.H, L.W, L.Ho, L.Wo, L.kh, L.kw, L.sy, L.sx};
+    BetaArgs b{A, L.beta, L.N, L.H, L.W, L.Ho, L.Wo, L.kh, L.kw, L.sy, L.sx};
     e = L.fc ? launch_beta_image_mean(b, s) : launch_beta_conv(b, s);
     if (e != cudaSuccess) return from_cuda(e);
   }
@@ -606,6 +645,89 @@ bconv_status_t run_forward(Layer& L, const float* in, float* out, cudaStream_t s
   return from_cuda(e);
 }
 
+// One forward with the given input and output forms.
+bconv_status_t run_io(Layer& L, const Io& io, cudaStream_t s) {
+  if (L.N == 0) return BCONV_OK;
+  if (io.out_bits && !tc_emits_bits(L)) {
+    // fp32 output into the handle's buffer, then the next layer's transform, sign and A
+    Io fp = io;
+    fp.out = L.y_scratch;
+    fp.out_bits = nullptr;
+    fp.out_a = nullptr;
+    bconv_status_t st = use_tc(L) ? run_forward_tc(L, fp, s) : run_forward_simt(L, fp, s);
+    if (st != BCONV_OK) return st;
+    PackArgs p{};
+    p.in = L.y_scratch;
+    p.npix = static_cast<int64_t>(L.N) * L.Ho * L.Wo;
+    p.ni = L.No;
+    p.nw_pad = words_for(L.No);
+    p.in_scale = L.next_scale;
+    p.in_bias = L.next_bias;
+    p.bits = io.out_bits;
+    p.A = io.out_a;
+    return from_cuda(launch_pack(p, s));
+  }
+  return use_tc(L) ? run_forward_tc(L, io, s) : run_forward_simt(L, io, s);
+}
+
+bconv_status_t run_forward(Layer& L, const float* in, float* out, cudaStream_t s) {
+  Io io;
+  io.in = in;
+  io.out = out;
+  return run_io(L, io, s);
+}
+
+// Buffers a bit-packed output needs with the current kernel family (kept until destroy).
+bconv_status_t ensure_bits_buffers(Layer& L) {
+  if (!L.has_next || L.N == 0) return BCONV_OK;
+  cudaError_t e = cudaSuccess;
+  if (tc_emits_bits(L)) {
+    const int slices = L.tc.n_tiles * L.tc.pieces;
+    if (slices > 1 && !L.a_part) {
+      e = L.mem.alloc(&L.a_part, static_cast<size_t>(slices) * L.N * L.Ho * L.Wo);
+      if (e == cudaSuccess) e = L.mem.alloc(&L.a_count, static_cast<size_t>(L.tc.m_tiles));
+      if (e == cudaSuccess) e = cudaMemset(L.a_count, 0, sizeof(uint32_t) * L.tc.m_tiles);
+    }
+  } else if (!L.y_scratch) {
+    e = L.mem.alloc(&L.y_scratch, static_cast<size_t>(L.out_elems()));
+  }
+  return from_cuda(e);
+}
+
+bconv_status_t set_output_terms(Layer& L, const float* next_scale, const float* next_bias) {
+  std::vector<float> hs(L.No, 1.f), hb(L.No, 0.f);
+  if (next_scale) memcpy(hs.data(), next_scale, sizeof(float) * L.No);
+  if (next_bias) memcpy(hb.data(), next_bias, sizeof(float) * L.No);
+  cudaError_t e = cudaSuccess;
+  if (!L.next_scale) e = L.mem.alloc(&L.next_scale, L.No);
+  if (e == cudaSuccess && !L.next_bias) e = L.mem.alloc(&L.next_bias, L.No);
+  if (e == cudaSuccess) e = cudaMemcpy(L.next_scale, hs.data(), sizeof(float) * L.No, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(L.next_bias, hb.data(), sizeof(float) * L.No, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return from_cuda(e);
+  L.has_next = true;
+  return ensure_bits_buffers(L);
+}
+
+bconv_status_t forward_io(Layer& L, const bconv_io_t* io, cudaStream_t s) {
+  if (!io) return BCONV_ERR_INVALID_ARG;
+  if ((io->in == nullptr) == (io->in_bits == nullptr)) return BCONV_ERR_INVALID_ARG;
+  if ((io->out == nullptr) == (io->out_bits == nullptr)) return BCONV_ERR_INVALID_ARG;
+  if (io->in_bits) {
+    if (L.type == kBinaryWeights) return BCONV_ERR_UNSUPPORTED;  // needs the full-precision input
+    if (L.in_scale) return BCONV_ERR_INVALID_ARG;  // the producer of the bits applied the input terms
+    if (L.use_beta() && !io->in_a) return BCONV_ERR_INVALID_ARG;
+  }
+  if (io->out_bits && (!io->out_a || !L.has_next)) return BCONV_ERR_INVALID_ARG;
+  Io v;
+  v.in = io->in;
+  v.in_bits = io->in_bits;
+  v.in_a = io->in_a;
+  v.out = io->out;
+  v.out_bits = io->out_bits;
+  v.out_a = io->out_a;
+  return run_io(L, v, s);
+}
+
 bconv_status_t forward_host(Layer& L, const float* hin, float* hout, cudaStream_t s) {
   if (!hin || !hout) return BCONV_ERR_INVALID_ARG;
   cudaError_t e = cudaSuccess;
@@ -629,6 +751,7 @@ bconv_status_t sync_status(Layer& L, cudaStream_t s) {
   if (e != cudaSuccess) return from_cuda(e);
   if (word) {
     cudaMemset(L.err, 0, sizeof(uint32_t));
+    if (L.a_count) cudaMemset(L.a_count, 0, sizeof(uint32_t) * L.tc.m_tiles);  // an aborted launch may leave counts
     if (word & kErrTimeout) return BCONV_ERR_TIMEOUT;
     return BCONV_ERR_CUDA;  // kErrLayout: a kernel refused an unexpected shared-memory layout
   }
@@ -636,21 +759,12 @@ bconv_status_t sync_status(Layer& L, cudaStream_t s) {
 }
 
 bconv_status_t set_algo(Layer& L, int algo) {
-  if (algo == BCONV_ALGO_AUTO) {
+  const bool ok = algo == BCONV_ALGO_AUTO || (algo == BCONV_ALGO_POPC && (L.type == kXnor || L.type == kAnd)) ||
+                  (algo == BCONV_ALGO_SIMT_F32 && L.type == kBinaryWeights) ||
+                  (algo == BCONV_ALGO_TCGEN05 && L.tc_ok);
+  if (ok) {
     L.algo = algo;
-    return BCONV_OK;
-  }
-  if (algo == BCONV_ALGO_POPC && (L.type == kXnor || L.type == kAnd)) {
-    L.algo = algo;
-    return BCONV_OK;
-  }
-  if (algo == BCONV_ALGO_SIMT_F32 && L.type == kBinaryWeights) {
-    L.algo = algo;
-    return BCONV_OK;
-  }
-  if (algo == BCONV_ALGO_TCGEN05 && L.tc_ok) {
-    L.algo = algo;
-    return BCONV_OK;
+    return ensure_bits_buffers(L);
   }
   if (algo < 0 || algo > BCONV_ALGO_TCGEN05) return BCONV_ERR_INVALID_ARG;
   return BCONV_ERR_UNSUPPORTED;
@@ -762,6 +876,20 @@ bconv_status_t bconv_forward(bconv_handle_t h, const float* in, float* out, stru
   return run_forward(h->L, in, out, stream);
 }
 
+bconv_status_t bconv_set_output_terms(bconv_handle_t h, const float* next_in_scale, const float* next_in_bias) {
+  if (!checked(h, kConvMagic)) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  if (!g.ok) return BCONV_ERR_CUDA;
+  return set_output_terms(h->L, next_in_scale, next_in_bias);
+}
+
+bconv_status_t bconv_forward_io(bconv_handle_t h, const bconv_io_t* io, struct CUstream_st* stream) {
+  if (!checked(h, kConvMagic)) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  if (!g.ok) return BCONV_ERR_CUDA;
+  return forward_io(h->L, io, stream);
+}
+
 bconv_status_t bconv_forward_host(bconv_handle_t h, const float* host_in, float* host_out,
                                   struct CUstream_st* stream) {
   if (!checked(h, kConvMagic)) return BCONV_ERR_INVALID_ARG;
@@ -862,6 +990,20 @@ bconv_status_t bfc_forward(bfc_handle_t h, const float* in, float* out, struct C
   DeviceGuard g(h->L.device);
   if (!g.ok) return BCONV_ERR_CUDA;
   return run_forward(h->L, in, out, stream);
+}
+
+bconv_status_t bfc_set_output_terms(bfc_handle_t h, const float* next_in_scale, const float* next_in_bias) {
+  if (!checked(h, kFcMagic)) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  if (!g.ok) return BCONV_ERR_CUDA;
+  return set_output_terms(h->L, next_in_scale, next_in_bias);
+}
+
+bconv_status_t bfc_forward_io(bfc_handle_t h, const bconv_io_t* io, struct CUstream_st* stream) {
+  if (!checked(h, kFcMagic)) return BCONV_ERR_INVALID_ARG;
+  DeviceGuard g(h->L.device);
+  if (!g.ok) return BCONV_ERR_CUDA;
+  return forward_io(h->L, io, stream);
 }
 
 bconv_status_t bfc_forward_host(bfc_handle_t h, const float* host_in, float* host_out, struct CUstream_st* stream) {

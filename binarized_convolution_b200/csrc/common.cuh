@@ -38,6 +38,14 @@ struct PackArgs {
 };
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s);
 
+// Bit-packed activations u32 [npix][ceil(ni/32)] (bits at or past ni ignored) into the POPC
+// layout [npix][nw_pad] (tail bits cleared, padding words 0), or into int8 operand codes
+// [npix][cip] (XNOR: bit 1 -> +1, 0 -> -1; AND: 1 -> 1, 0 -> 0; channels >= ni -> 0;
+// codes 16-byte aligned, cip a multiple of 16).
+cudaError_t launch_repack_bits(const uint32_t* bits, int64_t npix, int ni, int nw_pad, uint32_t* out, cudaStream_t s);
+cudaError_t launch_unpack_bits_i8(const uint32_t* bits, int64_t npix, int ni, int cip, int op, int8_t* codes,
+                                  cudaStream_t s);
+
 // ------------------------------------------------------------------------------------
 // Beta: box filter of A over the window (conv) or mean of A over the image (FC).
 // ------------------------------------------------------------------------------------

@@ -317,13 +317,102 @@ __global__ void __launch_bounds__(kPackThreads) pack_bf16x3_kernel(PackBf16x3Arg
 
 }  // namespace
 
+// Vector path: kC chunks of 64 channels per pixel (compile-time 1, 2, 4 or 8), a group of
+// 8 / kC pixels per warp step with all float2 loads issued first; lane l handles channels
+// chunk*64 + 2l, 2l+1 and keeps their input terms in registers.
+template <bool kTerms, bool kA, int kC>
+__global__ void __launch_bounds__(kPackThreads, 3) pack_bf16x3_vec_kernel(PackBf16x3Args a) {
+  constexpr int kG = kC >= 8 ? 1 : 8 / kC;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kPackThreads) >> 5;
+  const int ni = a.ni, cip = a.cip;
+  const float* __restrict__ in = a.in;
+  uint16_t* __restrict__ parts = a.parts;
+  float2 sc[kC], bi[kC];
+  bool live[kC];
+#pragma unroll
+  for (int c = 0; c < kC; ++c) {
+    const int f = c * 64 + lane * 2;
+    live[c] = f < ni;
+    sc[c] = make_float2(1.f, 1.f);
+    bi[c] = make_float2(0.f, 0.f);
+    if (kTerms && live[c]) {
+      sc[c] = __ldg(reinterpret_cast<const float2*>(a.in_scale + f));
+      bi[c] = __ldg(reinterpret_cast<const float2*>(a.in_bias + f));
+    }
+  }
+  for (int64_t p0 = warp * kG; p0 < a.npix; p0 += nwarps * kG) {
+    float2 v[kG][kC];
+#pragma unroll
+    for (int g = 0; g < kG; ++g)
+#pragma unroll
+      for (int c = 0; c < kC; ++c) {
+        const int64_t p = p0 + g;
+        v[g][c] = (p < a.npix && live[c]) ? __ldcs(reinterpret_cast<const float2*>(in + p * ni + c * 64 + lane * 2))
+                                          : make_float2(0.f, 0.f);
+      }
+#pragma unroll
+    for (int g = 0; g < kG; ++g) {
+      const int64_t p = p0 + g;
+      if (p >= a.npix) break;  // warp-uniform
+      uint16_t* prow = parts + p * 3 * cip;
+      float asum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kC; ++c) {
+        float2 t = v[g][c];
+        if (kTerms && live[c]) {
+          t.x = fmaf(t.x, sc[c].x, bi[c].x);
+          t.y = fmaf(t.y, sc[c].y, bi[c].y);
+        }
+        if (kA) asum += fabsf(t.x) + fabsf(t.y);
+        uint32_t w[3];
+        split3_pair(t.x, t.y, w);
+        const int f = c * 64 + lane * 2;
+#pragma unroll
+        for (int part = 0; part < 3; ++part) *reinterpret_cast<uint32_t*>(prow + part * cip + f) = w[part];
+      }
+      if (kA) {
+        asum = warp_sum(asum);
+        if (lane == 0) a.A[p] = asum / static_cast<float>(ni);
+      }
+    }
+  }
+}
+
+template <bool kTerms, bool kA>
+void launch_bf16x3_vec(const PackBf16x3Args& a, int chunks, dim3 grid, cudaStream_t s) {
+  if (chunks == 1)
+    pack_bf16x3_vec_kernel<kTerms, kA, 1><<<grid, kPackThreads, 0, s>>>(a);
+  else if (chunks == 2)
+    pack_bf16x3_vec_kernel<kTerms, kA, 2><<<grid, kPackThreads, 0, s>>>(a);
+  else if (chunks == 4)
+    pack_bf16x3_vec_kernel<kTerms, kA, 4><<<grid, kPackThreads, 0, s>>>(a);
+  else
+    pack_bf16x3_vec_kernel<kTerms, kA, 8><<<grid, kPackThreads, 0, s>>>(a);
+}
+
 cudaError_t launch_pack_bf16x3(const PackBf16x3Args& a, cudaStream_t s) {
   if (a.npix == 0) return cudaSuccess;
   const int sms = current_sm_count();
+  const int chunks = a.cip / 64;
+  const bool vec = (a.ni % 2) == 0 && (reinterpret_cast<uintptr_t>(a.in) & 7) == 0 &&
+                   (!a.in_scale || ((reinterpret_cast<uintptr_t>(a.in_scale) | reinterpret_cast<uintptr_t>(a.in_bias)) & 7) == 0) &&
+                   (chunks == 1 || chunks == 2 || chunks == 4 || chunks == 8);
   int64_t blocks = ceil_div(a.npix, kPackThreads / 32);
-  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  const int64_t cap = static_cast<int64_t>(sms) * (vec ? 3 : 8);
   if (blocks > cap) blocks = cap;
   const dim3 grid(static_cast<unsigned>(blocks));
+  if (vec) {
+    if (a.in_scale) {
+      if (a.A) launch_bf16x3_vec<true, true>(a, chunks, grid, s);
+      else launch_bf16x3_vec<true, false>(a, chunks, grid, s);
+    } else {
+      if (a.A) launch_bf16x3_vec<false, true>(a, chunks, grid, s);
+      else launch_bf16x3_vec<false, false>(a, chunks, grid, s);
+    }
+    return cudaGetLastError();
+  }
   if (a.in_scale) {
     if (a.A)
       pack_bf16x3_kernel<true, true><<<grid, kPackThreads, 0, s>>>(a);
@@ -335,6 +424,86 @@ cudaError_t launch_pack_bf16x3(const PackBf16x3Args& a, cudaStream_t s) {
     else
       pack_bf16x3_kernel<false, false><<<grid, kPackThreads, 0, s>>>(a);
   }
+  return cudaGetLastError();
+}
+
+}  // namespace bconv
+
+// ------------------------------------------------------------------------------------
+// Bit-packed activations (a previous layer's binarized output) into the operand layouts
+// of the contractions.  Input: u32 [npix][nw_in], channel c = bit c % 32 of word c / 32,
+// nw_in = ceil(ni / 32); bits at or past ni are ignored.
+// ------------------------------------------------------------------------------------
+namespace bconv {
+namespace {
+
+// One thread per 16 channels of a pixel: 16 code bytes as one 16-byte store.
+__global__ void __launch_bounds__(256) unpack_bits_i8_kernel(const uint32_t* __restrict__ bits, int64_t npix,
+                                                              int nw_in, int ni, int cip, int op,
+                                                              uint4* __restrict__ codes) {
+  const int groups = cip / 16;
+  const int64_t total = npix * groups;
+  const uint32_t neg = op == kXnor ? 0xFFu : 0x00u;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t p = i / groups;
+    const int g = static_cast<int>(i - p * groups);
+    const int c0 = g * 16;
+    uint32_t half = 0;
+    if (c0 < ni) half = (__ldg(bits + p * nw_in + c0 / 32) >> (c0 & 16)) & 0xFFFFu;
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t v = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int b = k * 4 + j;
+        const uint32_t code = (c0 + b < ni) ? (((half >> b) & 1u) ? 0x01u : neg) : 0x00u;
+        v |= code << (8 * j);
+      }
+      w[k] = v;
+    }
+    codes[i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// One thread per output word: copy, clear the bits past ni, zero the padding words.
+__global__ void __launch_bounds__(256) repack_bits_kernel(const uint32_t* __restrict__ bits, int64_t npix, int nw_in,
+                                                           int ni, int nw_pad, uint32_t* __restrict__ out) {
+  const int64_t total = npix * nw_pad;
+  const int tail = ni % 32;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t p = i / nw_pad;
+    const int w = static_cast<int>(i - p * nw_pad);
+    uint32_t v = 0;
+    if (w < nw_in) {
+      v = __ldg(bits + p * nw_in + w);
+      if (w == nw_in - 1 && tail != 0) v &= (1u << tail) - 1u;
+    }
+    out[i] = v;
+  }
+}
+
+unsigned grid_for(int64_t threads) {
+  int64_t blocks = ceil_div(threads, 256);
+  const int64_t cap = static_cast<int64_t>(current_sm_count()) * 8;
+  return static_cast<unsigned>(blocks < cap ? blocks : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_unpack_bits_i8(const uint32_t* bits, int64_t npix, int ni, int cip, int op, int8_t* codes,
+                                  cudaStream_t s) {
+  if (npix == 0) return cudaSuccess;
+  unpack_bits_i8_kernel<<<grid_for(npix * (cip / 16)), 256, 0, s>>>(bits, npix, words_for(ni), ni, cip, op,
+                                                                     reinterpret_cast<uint4*>(codes));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_repack_bits(const uint32_t* bits, int64_t npix, int ni, int nw_pad, uint32_t* out, cudaStream_t s) {
+  if (npix == 0) return cudaSuccess;
+  repack_bits_kernel<<<grid_for(npix * nw_pad), 256, 0, s>>>(bits, npix, words_for(ni), ni, nw_pad, out);
   return cudaGetLastError();
 }
 

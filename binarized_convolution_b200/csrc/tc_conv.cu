@@ -30,6 +30,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "tc_bits.cuh"
 #include "tc_conv.cuh"
 #include "tc_device.cuh"
 
@@ -58,6 +59,7 @@ struct __align__(8) Barriers {
 struct TileCoord {
   int n0, oy0, ox0, ntile, split;
   int noff, bn;  // output channels [ntile*BN + noff, + bn) of this work item
+  int mtile;     // M tile index
 };
 
 __device__ __forceinline__ TileCoord tile_coord(const TcArgs& a, int w) {
@@ -75,6 +77,7 @@ __device__ __forceinline__ TileCoord tile_coord(const TcArgs& a, int w) {
   t /= a.k_splits;
   c.ntile = t % a.n_tiles;
   t /= a.n_tiles;
+  c.mtile = t;
   const int tx = t % a.tiles_x;
   t /= a.tiles_x;
   const int ty = t % a.tiles_y;
@@ -85,7 +88,7 @@ __device__ __forceinline__ TileCoord tile_coord(const TcArgs& a, int w) {
   return c;
 }
 
-template <bool kSplit>
+template <bool kSplit, int kKind, bool kBits>
 __global__ void __launch_bounds__(kThreadsTc, 1)
     tc_conv_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmBp, const __grid_constant__ CUtensorMap tmOut,
@@ -178,7 +181,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
         const TileCoord tc = tile_coord(a, t);
-        const uint32_t idesc = idesc_for(a.kind, 128, tc.bn);
+        const uint32_t idesc = idesc_for(kKind, 128, tc.bn);
         const int kb0 = tc.split * kb_per_split;
         const int kb1 = min(kb0 + kb_per_split, kb_total);
         if (!mbar_wait(&B->tmem_empty[acc], acc_phase ^ 1u, B, a.err)) break;
@@ -197,7 +200,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {  // four 32-byte K steps across the 128-byte row
               const uint32_t accum = (kb > kb0 || j > 0) ? 1u : 0u;
-              if (a.kind)
+              if constexpr (kKind == 1)
                 tc_mma_bf16(d_tmem + static_cast<uint32_t>(h * a.BN), da + 2u * j, db + 2u * j, idesc, accum);
               else
                 tc_mma_i8(d_tmem + static_cast<uint32_t>(h * a.BN), da + 2u * j, db + 2u * j, idesc, accum);
@@ -229,6 +232,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     int chunk_count = 0;
     int loaded_ntile = -1;
     const int rc = a.R * a.Cw;
+    // bit-packed output: the next layer's terms and a flag live in the unused staging area
+    constexpr bool bits_out = kBits && !kSplit;
+    float2* next_t = reinterpret_cast<float2*>(stage_out);
+    uint32_t* bits_flag = reinterpret_cast<uint32_t*>(stage_out + kStageOutBytes);
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       const TileCoord tc = tile_coord(a, t);
       if (!kSplit && tc.ntile != loaded_ntile) {  // this tile's (scale, bias) into shared memory
@@ -236,6 +243,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         for (int j = et; j < a.BN; j += kEpiThreads) {
           const int c = tc.ntile * a.BN + j;
           B->sb[j] = c < a.No ? make_float2(__ldg(a.scale + c), __ldg(a.bias + c)) : make_float2(0.f, 0.f);
+          if (bits_out)
+            next_t[j] = c < a.No ? make_float2(__ldg(a.next_scale + c), __ldg(a.next_bias + c)) : make_float2(0.f, 0.f);
         }
         epi_barrier();
         loaded_ntile = tc.ntile;
@@ -267,6 +276,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       }
       if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err))) break;
       tc_fence_after();
+      float bits_asum = 0.f;
+      const int bits_n = tc.n0 + row / rc, bits_oy = tc.oy0 + (row / a.Cw) % a.R, bits_ox = tc.ox0 + row % a.Cw;
+      const bool bits_valid = bits_n < a.N && bits_oy < a.Ho && bits_ox < a.Wo;
+      const int64_t bits_pix = (static_cast<int64_t>(bits_n) * a.Ho + bits_oy) * a.Wo + bits_ox;
       for (int h = 0; h < a.mt; ++h) {
         const float beta = beta_h[h];
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
@@ -281,19 +294,19 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           const int buf = chunk_count & 1;
           ++chunk_count;
           uint8_t* so = stage_out + buf * kStageOutBytes;
-          epi_barrier();  // the store that last read `so` has finished (waited below by et 0)
+          if (!bits_out) epi_barrier();  // the store that last read `so` has finished (waited below by et 0)
           const int c0 = tc.ntile * a.BN + tc.noff + ch * 32;
           float y[32];
           if (kSplit) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) y[j] = acc_value(a.kind, v[j]);
+            for (int j = 0; j < 32; ++j) y[j] = acc_value(kKind, v[j]);
           } else {
             const float4* sb4 = reinterpret_cast<const float4*>(&B->sb[tc.noff + ch * 32]);
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
               const float4 p = sb4[j / 2];  // (scale, bias) of channels j, j+1 (same for all lanes)
-              const float s0 = acc_value(a.kind, v[j]);
-              const float s1 = acc_value(a.kind, v[j + 1]);
+              const float s0 = acc_value(kKind, v[j]);
+              const float s1 = acc_value(kKind, v[j + 1]);
               float r0 = has_beta ? fmaf(s0 * p.x, beta, p.y) : fmaf(s0, p.x, p.y);
               float r1 = has_beta ? fmaf(s1 * p.z, beta, p.w) : fmaf(s1, p.z, p.w);
               if (a.relu) {
@@ -303,6 +316,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
               y[j] = r0;
               y[j + 1] = r1;
             }
+          }
+          if (bits_out) {
+            const uint32_t word = bits_chunk(y, next_t + tc.noff + ch * 32, min(32, a.No - c0), bits_asum);
+            if (bits_valid && c0 < a.No) a.out_bits[bits_pix * a.nwo + c0 / 32] = word;
+            continue;
           }
           // 128-byte swizzled row: 16-byte chunk k of row r lives at chunk k ^ (r % 8)
           float4* orow = reinterpret_cast<float4*>(so + row * 128);
@@ -323,6 +341,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           }
         }
       }
+      if (bits_out)
+        bits_finish_item(a, bits_pix, bits_valid, bits_asum, tc.mtile, tc.mtile, tc.ntile,
+                         tc.ntile * a.pieces + tc.noff / tc.bn, bits_flag, et);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -337,18 +358,27 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   }
 }
 
-// y = act(S * scale[c] * beta[n] + bias[c]) over the fp32 partial-sum workspace [N][No].
-__global__ void tc_finalize_kernel(const float* __restrict__ ws, float* __restrict__ out, const float* __restrict__ scale,
-                                   const float* __restrict__ bias, const float* __restrict__ beta, int64_t total, int no,
-                                   int rows_per_beta, int relu) {
+// y = act(S * scale[c] * beta[n] + bias[c]) over the fp32 partial-sum workspace [N][No]; a
+// thread per 4 consecutive channels of one row (No % 4 == 0 on this path).
+__global__ void tc_finalize_kernel(const float4* __restrict__ ws, float4* __restrict__ out,
+                                   const float* __restrict__ scale, const float* __restrict__ bias,
+                                   const float* __restrict__ beta, int rows, int no4, int relu) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= total) return;
-  const int c = static_cast<int>(i % no);
-  const float s = ws[i];
-  float r = beta ? fmaf(s * __ldg(scale + c), __ldg(beta + (i / no) / rows_per_beta), __ldg(bias + c))
-                 : fmaf(s, __ldg(scale + c), __ldg(bias + c));
-  if (relu) r = fmaxf(r, 0.f);
-  out[i] = r;
+  if (i >= static_cast<int64_t>(rows) * no4) return;
+  const int r = static_cast<int>(i / no4), c = static_cast<int>(i - static_cast<int64_t>(r) * no4) * 4;
+  const float4 s = ws[i];
+  const float4 sc = __ldg(reinterpret_cast<const float4*>(scale + c));
+  const float4 bi = __ldg(reinterpret_cast<const float4*>(bias + c));
+  float4 y;
+  if (beta) {
+    const float b = __ldg(beta + r);
+    y = make_float4(fmaf(s.x * sc.x, b, bi.x), fmaf(s.y * sc.y, b, bi.y), fmaf(s.z * sc.z, b, bi.z),
+                    fmaf(s.w * sc.w, b, bi.w));
+  } else {
+    y = make_float4(fmaf(s.x, sc.x, bi.x), fmaf(s.y, sc.y, bi.y), fmaf(s.z, sc.z, bi.z), fmaf(s.w, sc.w, bi.w));
+  }
+  if (relu) y = make_float4(fmaxf(y.x, 0.f), fmaxf(y.y, 0.f), fmaxf(y.z, 0.f), fmaxf(y.w, 0.f));
+  out[i] = y;
 }
 
 }  // namespace
@@ -383,24 +413,22 @@ cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmB, const
   if (tiles == 0) return cudaSuccess;
   int grid = current_sm_count();
   if (grid > tiles) grid = tiles;
-  cudaError_t e;
-  if (a.k_splits > 1) {
-    e = cudaFuncSetAttribute(tc_conv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    tc_conv_kernel<true><<<grid, kThreadsTc, smem, s>>>(*tmA, *tmB, *tmBp, *tmOut, a);
-  } else {
-    e = cudaFuncSetAttribute(tc_conv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    tc_conv_kernel<false><<<grid, kThreadsTc, smem, s>>>(*tmA, *tmB, *tmBp, *tmOut, a);
-  }
+  if (a.out_bits && a.k_splits > 1) return cudaErrorInvalidValue;
+  auto kern = a.k_splits > 1 ? (a.kind ? tc_conv_kernel<true, 1, false> : tc_conv_kernel<true, 0, false>)
+              : a.out_bits   ? (a.kind ? tc_conv_kernel<false, 1, true> : tc_conv_kernel<false, 0, true>)
+                             : (a.kind ? tc_conv_kernel<false, 1, false> : tc_conv_kernel<false, 0, false>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreadsTc, smem, s>>>(*tmA, *tmB, *tmBp, *tmOut, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_tc_finalize(const float* ws, float* out, const float* scale, const float* bias, const float* beta,
-                               int64_t total, int no, int rows_per_beta, int relu, cudaStream_t s) {
-  if (total == 0) return cudaSuccess;
-  tc_finalize_kernel<<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(ws, out, scale, bias, beta, total, no,
-                                                                                 rows_per_beta, relu);
+                               int rows, int no, int relu, cudaStream_t s) {
+  const int64_t total4 = static_cast<int64_t>(rows) * (no / 4);
+  if (total4 == 0) return cudaSuccess;
+  tc_finalize_kernel<<<static_cast<unsigned>(ceil_div(total4, 256)), 256, 0, s>>>(
+      reinterpret_cast<const float4*>(ws), reinterpret_cast<float4*>(out), scale, bias, beta, rows, no / 4, relu);
   return cudaGetLastError();
 }
 

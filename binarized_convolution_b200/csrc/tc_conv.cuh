@@ -38,6 +38,19 @@ struct TcArgs {
   int H, W;            // input extent (for the window of A)
   int relu;
   uint32_t* err;
+  // Bit-packed output for a following binary layer (out_bits == nullptr: fp32 through the
+  // output tensor map).  Per output pixel p and channel c, x~ = next_scale[c] * y + next_bias[c]
+  // gives bit c % 32 of out_bits[p * nwo + c / 32] (1 for x~ >= 0) and out_a[p] = mean_c |x~|.
+  // When a pixel's channels span several work items, each item leaves its partial sum of
+  // |x~| in a_part[slice][p] and the last of them to finish (counted in a_count[m tile])
+  // adds the slices in slice order, so the result does not depend on timing.
+  uint32_t* out_bits;
+  float* out_a;
+  const float* next_scale;  // [No]
+  const float* next_bias;   // [No]
+  int nwo;                  // ceil(No / 32)
+  float* a_part;            // [n_tiles * pieces][N * Ho * Wo]
+  uint32_t* a_count;        // [m_tiles], zero between launches
 };
 
 int tc_smem_bytes(int bn, int mt);
@@ -54,8 +67,9 @@ int tc2_plan(TcArgs& a, int pairs);  // pairs = clusters that can be resident at
 int tc2_max_pairs(int bn);           // co-resident two-CTA clusters on the current device (0: none)
 cudaError_t launch_tc_conv2(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmBp,
                             const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s);
+// ws and out are 16-byte aligned, no % 4 == 0 (the tensor-core path's condition).
 cudaError_t launch_tc_finalize(const float* ws, float* out, const float* scale, const float* bias, const float* beta,
-                               int64_t total, int no, int rows_per_beta, int relu, cudaStream_t s);
+                               int rows, int no, int relu, cudaStream_t s);
 
 // int8 operand codes: XNOR -> bin(x~) in {-1,+1}, AND -> {0,1}; channels in [ni, cip) are 0.
 struct PackI8Args {

@@ -18,6 +18,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "tc_bits.cuh"
 #include "tc_conv.cuh"
 #include "tc_device.cuh"
 
@@ -115,6 +116,8 @@ struct PairCoord {
   int n0, oy0, ox0, ntile;
   int noff, bn;  // channels [ntile*BN + noff, + bn)
   bool dummy;    // this CTA's M tile lies past the end (odd tile count): compute, do not store
+  int ptile;     // the pair's M tile (index into the work list)
+  int mtile;     // this CTA's M tile
 };
 
 // Work item w of the pair -> this CTA's M tile (2*pair + rank) and the N range.
@@ -130,9 +133,11 @@ __device__ __forceinline__ PairCoord pair_coord(const TcArgs& a, int w, int rank
     c.noff = (i % a.pieces) * c.bn;
   }
   c.ntile = t % a.n_tiles;
-  int m = (t / a.n_tiles) * 2 + rank;
+  c.ptile = t / a.n_tiles;
+  int m = c.ptile * 2 + rank;
   c.dummy = m >= a.m_tiles;
   if (c.dummy) m = a.m_tiles - 1;
+  c.mtile = m;
   const int tx = m % a.tiles_x;
   m /= a.tiles_x;
   const int ty = m % a.tiles_y;
@@ -143,6 +148,7 @@ __device__ __forceinline__ PairCoord pair_coord(const TcArgs& a, int w, int rank
   return c;
 }
 
+template <int kKind, bool kBits>
 __global__ void __launch_bounds__(kThreads2, 1)
     tc_conv2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmBp, const __grid_constant__ CUtensorMap tmOut,
@@ -233,7 +239,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
       bool ok = true;
       for (int w = pair; w < total && ok; w += npairs) {
         const PairCoord pc = pair_coord(a, w, 0);
-        const uint32_t idesc = idesc_for(a.kind, 256, pc.bn);
+        const uint32_t idesc = idesc_for(kKind, 256, pc.bn);
         if (!mbar_wait(&B->tmem_empty[acc], acc_phase ^ 1u, B, a.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
@@ -248,7 +254,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint32_t accum = (kb > 0 || j > 0) ? 1u : 0u;
-            if (a.kind)
+            if constexpr (kKind == 1)
               tc_mma_bf16_pair(d_tmem, da + 2u * j, db + 2u * j, idesc, accum);
             else
               tc_mma_i8_pair(d_tmem, da + 2u * j, db + 2u * j, idesc, accum);
@@ -278,6 +284,10 @@ __global__ void __launch_bounds__(kThreads2, 1)
     int loaded_ntile = -1;
     const int rc = a.R * a.Cw;
     const uint32_t empty_leader0 = mapa(&B->tmem_empty[0], 0), empty_leader1 = mapa(&B->tmem_empty[1], 0);
+    // bit-packed output: the next layer's terms and a flag live in the unused staging area
+    constexpr bool bits_out = kBits;
+    float2* next_t = reinterpret_cast<float2*>(stage_out);
+    uint32_t* bits_flag = reinterpret_cast<uint32_t*>(stage_out + kOutBytes2);
     for (int w = pair; w < total; w += npairs) {
       const PairCoord pc = pair_coord(a, w, rank);
       if (pc.ntile != loaded_ntile) {
@@ -285,6 +295,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
         for (int j = et; j < a.BN; j += kEpi2) {
           const int c = pc.ntile * a.BN + j;
           B->sb[j] = c < a.No ? make_float2(__ldg(a.scale + c), __ldg(a.bias + c)) : make_float2(0.f, 0.f);
+          if (bits_out)
+            next_t[j] = c < a.No ? make_float2(__ldg(a.next_scale + c), __ldg(a.next_bias + c)) : make_float2(0.f, 0.f);
         }
         epi_barrier();
         loaded_ntile = pc.ntile;
@@ -311,6 +323,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
       }
       if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err))) break;
       tc_fence_after();
+      float bits_asum = 0.f;
+      const int64_t pix = (static_cast<int64_t>(n) * a.Ho + oy) * a.Wo + ox;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
       for (int ch = 0; ch < pc.bn / 32; ++ch) {
         uint32_t v[32];
@@ -322,15 +336,15 @@ __global__ void __launch_bounds__(kThreads2, 1)
         const int buf = chunk_count & 1;
         ++chunk_count;
         uint8_t* so = stage_out + buf * kOutBytes2;
-        epi_barrier();
+        if (!bits_out) epi_barrier();
         const int c0 = pc.ntile * a.BN + pc.noff + ch * 32;
         const float4* sb4 = reinterpret_cast<const float4*>(&B->sb[pc.noff + ch * 32]);
         float y[32];
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const float4 p = sb4[j / 2];
-          const float s0 = acc_value(a.kind, v[j]);
-          const float s1 = acc_value(a.kind, v[j + 1]);
+          const float s0 = acc_value(kKind, v[j]);
+          const float s1 = acc_value(kKind, v[j + 1]);
           float r0 = has_beta ? fmaf(s0 * p.x, beta, p.y) : fmaf(s0, p.x, p.y);
           float r1 = has_beta ? fmaf(s1 * p.z, beta, p.w) : fmaf(s1, p.z, p.w);
           if (a.relu) {
@@ -339,6 +353,11 @@ __global__ void __launch_bounds__(kThreads2, 1)
           }
           y[j] = r0;
           y[j + 1] = r1;
+        }
+        if (bits_out) {
+          const uint32_t word = bits_chunk(y, next_t + pc.noff + ch * 32, min(32, a.No - c0), bits_asum);
+          if (valid && c0 < a.No) a.out_bits[pix * a.nwo + c0 / 32] = word;
+          continue;
         }
         float4* orow = reinterpret_cast<float4*>(so + row * 128);
 #pragma unroll
@@ -352,6 +371,9 @@ __global__ void __launch_bounds__(kThreads2, 1)
           bulk_wait_read_1();
         }
       }
+      if (bits_out && !pc.dummy)
+        bits_finish_item(a, pix, valid, bits_asum, pc.ptile, pc.mtile, pc.ntile, pc.ntile * a.pieces + pc.noff / pc.bn,
+                         bits_flag, et);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -375,7 +397,10 @@ int tc2_smem_bytes(int bn) {
 
 int tc2_max_pairs(int bn) {
   const int smem = tc2_smem_bytes(bn);
-  if (cudaFuncSetAttribute(tc_conv2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+  if (cudaFuncSetAttribute(tc_conv2_kernel<0, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      cudaFuncSetAttribute(tc_conv2_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      cudaFuncSetAttribute(tc_conv2_kernel<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      cudaFuncSetAttribute(tc_conv2_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -391,7 +416,7 @@ int tc2_max_pairs(int bn) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, tc_conv2_kernel, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, tc_conv2_kernel<0, false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -425,7 +450,9 @@ cudaError_t launch_tc_conv2(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
   const int smem = tc2_smem_bytes(a.BN);
   const int npairs = a.grid_ctas / 2;
   if (npairs <= 0) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(tc_conv2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  auto kern = a.out_bits ? (a.kind ? tc_conv2_kernel<1, true> : tc_conv2_kernel<0, true>)
+                         : (a.kind ? tc_conv2_kernel<1, false> : tc_conv2_kernel<0, false>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * npairs));
@@ -439,7 +466,7 @@ cudaError_t launch_tc_conv2(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, tc_conv2_kernel, *tmA, *tmB, *tmBp, *tmOut, a);
+  e = cudaLaunchKernelEx(&cfg, kern, *tmA, *tmB, *tmBp, *tmOut, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

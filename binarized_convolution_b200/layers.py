@@ -41,6 +41,46 @@ class _Layer:
         except Exception:  # noqa: BLE001 -- interpreter shutdown
             pass
 
+    # ---- chained binary layers (bit-packed activations; see bconv_forward_io) ----
+    def set_output_terms(self, next_in_scale=None, next_in_bias=None):
+        """The input terms of the layer that will read this layer's bit-packed output."""
+        type(self)._set_output_terms(self.handle, next_in_scale, next_in_bias)
+
+    def bits_shape(self):
+        """Shapes of this layer's bit-packed output: (32-bit words, A)."""
+        *lead, c = self.out_dims
+        return (*lead, (c + 31) // 32), tuple(lead)
+
+    def forward_io(self, x=None, x_bits=None, x_a=None, out=None, out_bits=None, out_a=None):
+        """Device tensors in either form: fp32 ``x`` or ``x_bits`` (+ ``x_a``); fp32 ``out`` or
+        ``out_bits`` + ``out_a``.  Bit tensors hold the uint32 words (any 32-bit dtype)."""
+        import torch
+
+        def p(t):
+            return None if t is None else t.data_ptr()
+
+        type(self)._forward_io(self.handle, p(x), p(x_bits), p(x_a), p(out), p(out_bits), p(out_a),
+                               torch.cuda.current_stream().cuda_stream)
+
+    def forward_to_bits(self, x=None, x_bits=None, x_a=None):
+        """Run the layer and return its output as (bits, A) device tensors (bits as int32)."""
+        import torch
+
+        src = x if x is not None else x_bits
+        bshape, ashape = self.bits_shape()
+        bits = torch.empty(bshape, dtype=torch.int32, device=src.device)
+        a = torch.empty(ashape, dtype=torch.float32, device=src.device)
+        self.forward_io(x=x, x_bits=x_bits, x_a=x_a, out_bits=bits, out_a=a)
+        return bits, a
+
+    def forward_from_bits(self, x_bits, x_a=None):
+        """Run the layer on bit-packed input; returns the fp32 output tensor."""
+        import torch
+
+        out = torch.empty(self.out_dims, dtype=torch.float32, device=x_bits.device)
+        self.forward_io(x_bits=x_bits, x_a=x_a, out=out)
+        return out
+
     def __enter__(self):
         return self
 
@@ -56,6 +96,8 @@ class BinaryConv2d(_Layer):
     """
 
     _destroy = staticmethod(nat.bconv_destroy)
+    _set_output_terms = staticmethod(nat.bconv_set_output_terms)
+    _forward_io = staticmethod(nat.bconv_forward_io)
 
     def __init__(self, batch, in_h, in_w, in_channels, out_channels, kernel=(3, 3), stride=(1, 1), *,
                  wbits=None, packed=None, op="xnor", scale=None, scale_value=1.0, bias=None, in_scale=None,
@@ -121,6 +163,8 @@ class BinaryFC(_Layer):
     """
 
     _destroy = staticmethod(nat.bfc_destroy)
+    _set_output_terms = staticmethod(nat.bfc_set_output_terms)
+    _forward_io = staticmethod(nat.bfc_forward_io)
 
     def __init__(self, batch, in_h, in_w, in_channels, out_channels, *, wbits=None, packed=None, op="xnor",
                  scale=None, scale_value=1.0, bias=None, in_scale=None, in_bias=None, use_beta=False, relu=False,

@@ -132,3 +132,12 @@ def small_case(*, batch=1, h=5, w=5, ni=3, no=2, k=3, kw=None, stride=1, stride_
     return Workload(f"case_{kind}_{op}_{batch}x{h}x{w}x{ni}_k{no}_{k}x{kw}_s{stride}{sx}_{seed}", kind,
                     batch, h, w, ni, no, k, kw, stride, sx, op, use_beta, relu, in_terms, scale[0], scale[1],
                     p, seed)
+
+
+def next_terms(no: int, seed: int, bias_spread: float = 0.1) -> tuple[np.ndarray, np.ndarray]:
+    """Input terms of a following binary layer (chained layers): scales of random sign and
+    magnitude U(0.5, 1.5), biases N(0, bias_spread), as float32 [no] each."""
+    rng = np.random.default_rng(seed)
+    mag = rng.uniform(0.5, 1.5, no)
+    sign = np.where(rng.random(no) < 0.5, -1.0, 1.0)
+    return (mag * sign).astype(np.float32), rng.normal(0.0, bias_spread, no).astype(np.float32)

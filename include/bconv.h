@@ -131,6 +131,56 @@ bconv_status_t bconv_forward(bconv_handle_t h, const float* in, float* out, stru
 bconv_status_t bconv_forward_host(bconv_handle_t h, const float* host_in, float* host_out,
                                   struct CUstream_st* stream);
 
+/* ------------------------------------------------------------------------------------
+ * Chained binary layers.  A binary layer uses its input only through the step before the
+ * sum (MPSCNNBinaryConvolution Overview: the input terms act before binarization and
+ * before the beta image; bin(x) = x < 0 ? -1 : 1; A of the beta formula): per pixel and
+ * channel the sign of x~ = in_scale[c] * x + in_bias[c], and per pixel the mean over the
+ * channels of |x~|.  When one binary layer feeds another, the first can therefore emit
+ * that form from its epilogue and the second read it in place of fp32 activations: 32x
+ * fewer bytes per activation in each direction.  (The pages describe single layers; this
+ * form is what the next layer's definition reads of the previous layer's output.)
+ *
+ * Bit-packed activations of an [N][H][W][C] image:
+ *   bits  uint32 [N][H][W][ceil(C/32)]: channel c is bit c % 32 of word c / 32, 1 for
+ *         x~ >= 0 (bin = +1) and 0 for x~ < 0; bits past C in a pixel's last word are
+ *         written 0 and ignored on input.
+ *   a     float [N][H][W]: sum over the C channels of |x~|, divided by C.
+ * Signs are decided on x~ in fp32 (x~ = fmaf(y, in_scale, in_bias) of the fp32 output y).
+ * ------------------------------------------------------------------------------------ */
+
+/*
+ * The input terms of the layer that reads this layer's output: host float [out_channels]
+ * each, NULL meaning 1 (scale) or 0 (bias); copied.  Required before a forward with
+ * out_bits; may be called again to change them.  Allocates what the bit-packed output
+ * needs with the current kernel family (slice partials of A, or an fp32 output buffer
+ * for families that binarize in a separate pass; bconv_set_algo may allocate it later).
+ * Errors: INVALID_ARG, OOM, CUDA.
+ */
+bconv_status_t bconv_set_output_terms(bconv_handle_t h, const float* next_in_scale, const float* next_in_bias);
+
+/* Input and output forms of bconv_forward_io: exactly one of in / in_bits and exactly one
+ * of out / out_bits is non-NULL.  All pointers are device memory owned by the caller. */
+typedef struct {
+  const float* in;          /* fp32 [batch][in_h][in_w][in_channels] */
+  const uint32_t* in_bits;  /* bit-packed input, in_channels channels */
+  const float* in_a;        /* with in_bits: its A [batch][in_h][in_w]; required when the layer uses beta */
+  float* out;               /* fp32 [batch][Ho][Wo][out_channels] */
+  uint32_t* out_bits;       /* bit-packed output (binarized with the terms of bconv_set_output_terms) */
+  float* out_a;             /* with out_bits: its A [batch][Ho][Wo]; required */
+} bconv_io_t;
+
+/*
+ * bconv_forward with a choice of forms.  Bit-packed input: XNOR and AND layers created
+ * without input terms only (the producer applied them): UNSUPPORTED for binaryWeights,
+ * INVALID_ARG with input terms.  Bit-packed output: the layer output y (after the neuron)
+ * is binarized with the next layer's terms; INVALID_ARG before bconv_set_output_terms.
+ * Asynchronous on `stream`; allocates nothing.  When a pixel's output channels are
+ * computed by several work items, A is added in a fixed order, so results do not depend
+ * on timing.
+ */
+bconv_status_t bconv_forward_io(bconv_handle_t h, const bconv_io_t* io, struct CUstream_st* stream);
+
 /* Output dimensions (n, Ho, Wo, out_channels).  Any pointer may be NULL. */
 bconv_status_t bconv_get_output_dims(bconv_handle_t h, int32_t* n, int32_t* ho, int32_t* wo, int32_t* c);
 
@@ -191,6 +241,12 @@ bconv_status_t bfc_create(const bfc_desc_t* desc, const uint32_t* packed_weights
 /* in: device fp32 [batch][in_h][in_w][in_channels]; out: device fp32 [batch][out_channels]. */
 bconv_status_t bfc_forward(bfc_handle_t h, const float* in, float* out, struct CUstream_st* stream);
 bconv_status_t bfc_forward_host(bfc_handle_t h, const float* host_in, float* host_out, struct CUstream_st* stream);
+/* Chained layers (as bconv_set_output_terms / bconv_forward_io): the bit-packed input is
+ * [batch][in_h][in_w][ceil(in_channels/32)] words with A [batch][in_h][in_w] (a binary
+ * convolution's bit-packed output); the bit-packed output is [batch][ceil(out_channels/32)]
+ * words with A [batch]. */
+bconv_status_t bfc_set_output_terms(bfc_handle_t h, const float* next_in_scale, const float* next_in_bias);
+bconv_status_t bfc_forward_io(bfc_handle_t h, const bconv_io_t* io, struct CUstream_st* stream);
 int32_t bfc_input_feature_channels(bfc_handle_t h);
 int32_t bfc_output_feature_channels(bfc_handle_t h);
 bconv_status_t bfc_set_algo(bfc_handle_t h, bconv_algo_t algo);

@@ -105,7 +105,8 @@ def assert_sums_exact(S_dev, S_ref):
         f"device {S_dev[tuple(b[0] for b in bad)]} oracle {S_ref[tuple(b[0] for b in bad)]}")
 
 
-def relative_errors(w, inp, y_dev, S_ref, beta_ref, y_ref, rows=None):
+def error_scale(w, inp, S_ref, beta_ref, rows=None):
+    """D_i of the tolerance for each output (see the module docstring)."""
     scale = np.abs(inp.scale.astype(np.float64))[None, :]
     bias = np.abs(inp.bias.astype(np.float64))[None, :]
     beta = np.abs(beta_ref)[:, None]
@@ -113,7 +114,11 @@ def relative_errors(w, inp, y_dev, S_ref, beta_ref, y_ref, rows=None):
         mag = window_abs_sum(w, inp, rows)[:, None]
     else:
         mag = np.abs(S_ref)
-    D = scale * beta * mag + bias
+    return scale * beta * mag + bias
+
+
+def relative_errors(w, inp, y_dev, S_ref, beta_ref, y_ref, rows=None):
+    D = error_scale(w, inp, S_ref, beta_ref, rows)
     denom = np.maximum(np.abs(y_ref), D)
     denom = np.where(denom == 0, 1.0, denom)
     return np.abs(y_dev.astype(np.float64) - y_ref) / denom
