@@ -177,7 +177,8 @@ KERNEL_SOURCES = {
     "popc_gemm": ["binarized_convolution_b200/csrc/popc_gemm.cu", "binarized_convolution_b200/csrc/common.cuh"],
     "bw_conv": ["binarized_convolution_b200/csrc/bw_conv.cu", "binarized_convolution_b200/csrc/common.cuh"],
     "tc_conv": ["binarized_convolution_b200/csrc/tc_conv.cu", "binarized_convolution_b200/csrc/tc_conv2.cu",
-                "binarized_convolution_b200/csrc/tc_conv.cuh", "binarized_convolution_b200/csrc/tc_device.cuh"],
+                "binarized_convolution_b200/csrc/tc_conv.cuh", "binarized_convolution_b200/csrc/tc_device.cuh",
+                "binarized_convolution_b200/csrc/tc_bits.cuh"],
 }
 ALGO_KERNEL = {1: "popc_gemm", 2: "bw_conv", 3: "tc_conv"}
 BF16_FALLBACK_TFLOPS = 1590.0  # recipe fallback when MEASURED_PEAKS.json is absent

@@ -437,48 +437,44 @@ cudaError_t launch_pack_bf16x3(const PackBf16x3Args& a, cudaStream_t s) {
 namespace bconv {
 namespace {
 
-// One thread per 16 channels of a pixel: 16 code bytes as one 16-byte store.
-__global__ void __launch_bounds__(256) unpack_bits_i8_kernel(const uint32_t* __restrict__ bits, int64_t npix,
-                                                              int nw_in, int ni, int cip, int op,
+// Four channels' codes from their four bits (bit j -> byte j): the multiply places bit j of n
+// at bit 8j (and nowhere else inside the mask); XNOR turns 1 / 0 into 0x01 / 0xFF with no
+// carries between bytes, AND keeps 1 / 0; bytes of channels past ni are 0.
+template <int kOp>
+__device__ __forceinline__ uint32_t codes_of_nibble(uint32_t n, int nvalid) {
+  const uint32_t b = (n * 0x00204081u) & 0x01010101u;
+  uint32_t c = kOp == kXnor ? ~(b * 0xFEu) : b;
+  if (nvalid < 4) c &= nvalid <= 0 ? 0u : ((1u << (8 * nvalid)) - 1u);
+  return c;
+}
+
+// One thread per 16 channels of a pixel: 16 code bytes as one 16-byte store.  Index math in
+// 32 bits (the launcher checks that the chunk count fits).
+template <int kOp>
+__global__ void __launch_bounds__(256) unpack_bits_i8_kernel(const uint32_t* __restrict__ bits, uint32_t total,
+                                                              uint32_t groups, int nw_in, int ni,
                                                               uint4* __restrict__ codes) {
-  const int groups = cip / 16;
-  const int64_t total = npix * groups;
-  const uint32_t neg = op == kXnor ? 0xFFu : 0x00u;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t p = i / groups;
-    const int g = static_cast<int>(i - p * groups);
-    const int c0 = g * 16;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const uint32_t p = i / groups;
+    const int c0 = static_cast<int>(i - p * groups) * 16;
     uint32_t half = 0;
-    if (c0 < ni) half = (__ldg(bits + p * nw_in + c0 / 32) >> (c0 & 16)) & 0xFFFFu;
-    uint32_t w[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      uint32_t v = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int b = k * 4 + j;
-        const uint32_t code = (c0 + b < ni) ? (((half >> b) & 1u) ? 0x01u : neg) : 0x00u;
-        v |= code << (8 * j);
-      }
-      w[k] = v;
-    }
-    codes[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    if (c0 < ni) half = (__ldg(bits + static_cast<size_t>(p) * nw_in + c0 / 32) >> (c0 & 16)) & 0xFFFFu;
+    const int nv = ni - c0;
+    codes[i] = make_uint4(codes_of_nibble<kOp>(half & 0xFu, nv), codes_of_nibble<kOp>((half >> 4) & 0xFu, nv - 4),
+                          codes_of_nibble<kOp>((half >> 8) & 0xFu, nv - 8), codes_of_nibble<kOp>(half >> 12, nv - 12));
   }
 }
 
 // One thread per output word: copy, clear the bits past ni, zero the padding words.
-__global__ void __launch_bounds__(256) repack_bits_kernel(const uint32_t* __restrict__ bits, int64_t npix, int nw_in,
-                                                           int ni, int nw_pad, uint32_t* __restrict__ out) {
-  const int64_t total = npix * nw_pad;
+__global__ void __launch_bounds__(256) repack_bits_kernel(const uint32_t* __restrict__ bits, uint32_t total, int nw_in,
+                                                           int ni, uint32_t nw_pad, uint32_t* __restrict__ out) {
   const int tail = ni % 32;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t p = i / nw_pad;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const uint32_t p = i / nw_pad;
     const int w = static_cast<int>(i - p * nw_pad);
     uint32_t v = 0;
     if (w < nw_in) {
-      v = __ldg(bits + p * nw_in + w);
+      v = __ldg(bits + static_cast<size_t>(p) * nw_in + w);
       if (w == nw_in - 1 && tail != 0) v &= (1u << tail) - 1u;
     }
     out[i] = v;
@@ -496,14 +492,23 @@ unsigned grid_for(int64_t threads) {
 cudaError_t launch_unpack_bits_i8(const uint32_t* bits, int64_t npix, int ni, int cip, int op, int8_t* codes,
                                   cudaStream_t s) {
   if (npix == 0) return cudaSuccess;
-  unpack_bits_i8_kernel<<<grid_for(npix * (cip / 16)), 256, 0, s>>>(bits, npix, words_for(ni), ni, cip, op,
-                                                                     reinterpret_cast<uint4*>(codes));
+  const int64_t total = npix * (cip / 16);
+  if (total >= (int64_t{1} << 31)) return cudaErrorInvalidValue;
+  const uint32_t t = static_cast<uint32_t>(total), g = static_cast<uint32_t>(cip / 16);
+  uint4* out = reinterpret_cast<uint4*>(codes);
+  if (op == kXnor)
+    unpack_bits_i8_kernel<kXnor><<<grid_for(total), 256, 0, s>>>(bits, t, g, words_for(ni), ni, out);
+  else
+    unpack_bits_i8_kernel<kAnd><<<grid_for(total), 256, 0, s>>>(bits, t, g, words_for(ni), ni, out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_repack_bits(const uint32_t* bits, int64_t npix, int ni, int nw_pad, uint32_t* out, cudaStream_t s) {
   if (npix == 0) return cudaSuccess;
-  repack_bits_kernel<<<grid_for(npix * nw_pad), 256, 0, s>>>(bits, npix, words_for(ni), ni, nw_pad, out);
+  const int64_t total = npix * nw_pad;
+  if (total >= (int64_t{1} << 31)) return cudaErrorInvalidValue;
+  repack_bits_kernel<<<grid_for(total), 256, 0, s>>>(bits, static_cast<uint32_t>(total), words_for(ni), ni,
+                                                     static_cast<uint32_t>(nw_pad), out);
   return cudaGetLastError();
 }
 

@@ -27,6 +27,48 @@ __device__ __forceinline__ uint32_t bits_chunk(const float (&y)[32], const float
   return word;
 }
 
+// The sign words of one pixel's work item (up to 8 chunks of 32 channels), held in registers.
+struct Words8 {
+  uint4 lo, hi;
+};
+
+__device__ __forceinline__ void words_set(Words8& w, int i, uint32_t v) {
+  switch (i) {
+    case 0: w.lo.x = v; break;
+    case 1: w.lo.y = v; break;
+    case 2: w.lo.z = v; break;
+    case 3: w.lo.w = v; break;
+    case 4: w.hi.x = v; break;
+    case 5: w.hi.y = v; break;
+    case 6: w.hi.z = v; break;
+    default: w.hi.w = v; break;
+  }
+}
+
+__device__ __forceinline__ uint32_t words_get(const Words8& w, int i) {
+  switch (i) {
+    case 0: return w.lo.x;
+    case 1: return w.lo.y;
+    case 2: return w.lo.z;
+    case 3: return w.lo.w;
+    case 4: return w.hi.x;
+    case 5: return w.hi.y;
+    case 6: return w.hi.z;
+    default: return w.hi.w;
+  }
+}
+
+// Store the first n (<= 8) words at dst: 16-byte stores when dst is 16-byte aligned and n is
+// a multiple of 4 (one 32-byte sector per pixel for a 256-channel item), else word by word.
+__device__ __forceinline__ void words_store(uint32_t* dst, const Words8& w, int n) {
+  if ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0 && (n & 3) == 0) {
+    if (n >= 4) reinterpret_cast<uint4*>(dst)[0] = w.lo;
+    if (n == 8) reinterpret_cast<uint4*>(dst)[1] = w.hi;
+  } else {
+    for (int i = 0; i < n; ++i) dst[i] = words_get(w, i);
+  }
+}
+
 // Work items (slices of output channels) that cover M tile `mi` of the work list: tiles
 // before `full_tiles` are whole, later ones come in `pieces` parts.
 __device__ __forceinline__ int bits_slices_of(const TcArgs& a, int mi) {

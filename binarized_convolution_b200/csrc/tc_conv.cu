@@ -277,6 +277,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err))) break;
       tc_fence_after();
       float bits_asum = 0.f;
+      Words8 bits_w{};
       const int bits_n = tc.n0 + row / rc, bits_oy = tc.oy0 + (row / a.Cw) % a.R, bits_ox = tc.ox0 + row % a.Cw;
       const bool bits_valid = bits_n < a.N && bits_oy < a.Ho && bits_ox < a.Wo;
       const int64_t bits_pix = (static_cast<int64_t>(bits_n) * a.Ho + bits_oy) * a.Wo + bits_ox;
@@ -318,8 +319,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             }
           }
           if (bits_out) {
-            const uint32_t word = bits_chunk(y, next_t + tc.noff + ch * 32, min(32, a.No - c0), bits_asum);
-            if (bits_valid && c0 < a.No) a.out_bits[bits_pix * a.nwo + c0 / 32] = word;
+            words_set(bits_w, ch, bits_chunk(y, next_t + tc.noff + ch * 32, min(32, a.No - c0), bits_asum));
             continue;
           }
           // 128-byte swizzled row: 16-byte chunk k of row r lives at chunk k ^ (r % 8)
@@ -341,9 +341,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           }
         }
       }
-      if (bits_out)
+      if (bits_out) {
+        const int w0 = (tc.ntile * a.BN + tc.noff) / 32;  // first word of this item
+        if (bits_valid) words_store(a.out_bits + bits_pix * a.nwo + w0, bits_w, min(tc.bn / 32, a.nwo - w0));
         bits_finish_item(a, bits_pix, bits_valid, bits_asum, tc.mtile, tc.mtile, tc.ntile,
                          tc.ntile * a.pieces + tc.noff / tc.bn, bits_flag, et);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }

@@ -324,6 +324,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
       if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err))) break;
       tc_fence_after();
       float bits_asum = 0.f;
+      Words8 bits_w{};
       const int64_t pix = (static_cast<int64_t>(n) * a.Ho + oy) * a.Wo + ox;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
       for (int ch = 0; ch < pc.bn / 32; ++ch) {
@@ -355,8 +356,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
           y[j + 1] = r1;
         }
         if (bits_out) {
-          const uint32_t word = bits_chunk(y, next_t + pc.noff + ch * 32, min(32, a.No - c0), bits_asum);
-          if (valid && c0 < a.No) a.out_bits[pix * a.nwo + c0 / 32] = word;
+          words_set(bits_w, ch, bits_chunk(y, next_t + pc.noff + ch * 32, min(32, a.No - c0), bits_asum));
           continue;
         }
         float4* orow = reinterpret_cast<float4*>(so + row * 128);
@@ -371,9 +371,12 @@ __global__ void __launch_bounds__(kThreads2, 1)
           bulk_wait_read_1();
         }
       }
-      if (bits_out && !pc.dummy)
+      if (bits_out && !pc.dummy) {
+        const int w0 = (pc.ntile * a.BN + pc.noff) / 32;  // first word of this item
+        if (valid) words_store(a.out_bits + pix * a.nwo + w0, bits_w, min(pc.bn / 32, a.nwo - w0));
         bits_finish_item(a, pix, valid, bits_asum, pc.ptile, pc.mtile, pc.ntile, pc.ntile * a.pieces + pc.noff / pc.bn,
                          bits_flag, et);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
