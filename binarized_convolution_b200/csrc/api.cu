@@ -256,12 +256,28 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   } else {
     t.Ho = L.Ho; t.Wo = L.Wo; t.kh = L.kh; t.kw = L.kw; t.sy = L.sy; t.sx = L.sx;
     t.kb_per_tap = bpp / 128;
-    t.Cw = std::min(128, next_pow2(L.Wo));
-    t.R = std::min(128 / t.Cw, next_pow2(L.Ho));
+    // 128 output pixels per tile as Bn images x R rows x Cw columns (powers of two, so that
+    // every 32-row quarter is a box too): the shape with the fewest tiles, i.e. the least
+    // MMA work on pixels past the image edges (56 x 56 -> 8 x 8 x 2 images: none), then
+    // the smallest window footprint; the TMA box (stride x extent) stays within 256.
+    int64_t best_tiles = -1, best_halo = 0;
+    for (int cw = 1; cw <= 128; cw *= 2)
+      for (int r = 1; cw * r <= 128; r *= 2) {
+        const int bn = 128 / (cw * r);
+        if (t.sx * cw > 256 || t.sy * r > 256) continue;
+        const int64_t tiles = static_cast<int64_t>((L.Wo + cw - 1) / cw) * ((L.Ho + r - 1) / r) * ((L.N + bn - 1) / bn);
+        const int64_t halo = static_cast<int64_t>(cw * t.sx + L.kw - 1) * (r * t.sy + L.kh - 1) * bn;
+        if (best_tiles < 0 || tiles < best_tiles || (tiles == best_tiles && halo < best_halo)) {
+          best_tiles = tiles;
+          best_halo = halo;
+          t.Cw = cw;
+          t.R = r;
+        }
+      }
+    if (best_tiles < 0) return BCONV_OK;  // no box fits the TMA limits
     t.Bn = 128 / (t.Cw * t.R);
     t.tiles_x = (L.Wo + t.Cw - 1) / t.Cw;
     t.tiles_y = (L.Ho + t.R - 1) / t.R;
-    if (t.sx * t.Cw > 256 || t.sy * t.R > 256) return BCONV_OK;  // box too wide for TMA
   }
   t.m_tiles = t.tiles_x * t.tiles_y * ((L.N + t.Bn * t.mt - 1) / (t.Bn * t.mt));
   const int kb_total = t.kh * t.kw * t.kb_per_tap;
