@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace bconv {
 
 enum Op : int { kBinaryWeights = 0, kXnor = 1, kAnd = 2 };
@@ -22,6 +24,30 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Multiprocessor count of the current device (cached per device).
 int current_sm_count();
+
+// Programmatic dependent launch, used by the kernels of the tensor-core forward: a kernel
+// started with launch_overlapped may be scheduled while the previous kernel of the stream is
+// finishing.  It calls wait_prior_grid() before it touches global memory (the previous kernel
+// may be writing its input), and allow_next_grid() so that the next kernel can be scheduled
+// in turn.  Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_next_grid() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_overlapped(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // ------------------------------------------------------------------------------------
 // Input transform, sign and pack (one pass over the fp32 input).

@@ -131,11 +131,27 @@ __device__ __forceinline__ float4 transform4(float4 v, const float* __restrict__
 }
 
 // Vector path: kC chunks of 128 channels per pixel (a compile-time 1, 2 or 4), a group of
-// 8 / kC pixels per warp step with all 8 float4 loads per lane issued before any is used.
+// 8 / kC pixels per warp step (8 float4 loads per lane).  The loads of the next group are
+// issued before the current one is converted, so two groups per warp are in flight.
 // Lane l always handles channels chunk*128 + 4l .. 4l+3, so its input terms stay in registers.
+template <int kG, int kC>
+__device__ __forceinline__ void load_group(float4 (&v)[kG][kC], const float* __restrict__ in, int64_t p0, int64_t npix,
+                                           int ni, const bool (&live)[kC], int lane) {
+#pragma unroll
+  for (int g = 0; g < kG; ++g)
+#pragma unroll
+    for (int c = 0; c < kC; ++c) {
+      const int64_t p = p0 + g;
+      v[g][c] = (p < npix && live[c]) ? __ldcs(reinterpret_cast<const float4*>(in + p * ni + c * 128 + lane * 4))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
 template <bool kTerms, bool kA, int kOp, int kC>
-__global__ void __launch_bounds__(kPackThreads, 3) pack_i8_vec_kernel(PackI8Args a) {
+__global__ void __launch_bounds__(kPackThreads, 2) pack_i8_vec_kernel(PackI8Args a) {
   constexpr int kG = 8 / kC;  // pixels per warp step
+  wait_prior_grid();
+  allow_next_grid();
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kPackThreads) >> 5;
@@ -155,17 +171,13 @@ __global__ void __launch_bounds__(kPackThreads, 3) pack_i8_vec_kernel(PackI8Args
       bi[c] = __ldg(reinterpret_cast<const float4*>(a.in_bias + f));
     }
   }
-  for (int64_t p0 = warp * kG; p0 < a.npix; p0 += nwarps * kG) {
-    float4 v[kG][kC];
-#pragma unroll
-    for (int g = 0; g < kG; ++g)
-#pragma unroll
-      for (int c = 0; c < kC; ++c) {
-        const int64_t p = p0 + g;
-        v[g][c] = (p < a.npix && live[c])
-                      ? __ldcs(reinterpret_cast<const float4*>(in + p * ni + c * 128 + lane * 4))
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+  const int64_t step = nwarps * kG;
+  float4 v[kG][kC];
+  int64_t p0 = warp * kG;
+  if (p0 < a.npix) load_group<kG, kC>(v, in, p0, a.npix, ni, live, lane);
+  for (; p0 < a.npix; p0 += step) {
+    float4 nxt[kG][kC];
+    if (p0 + step < a.npix) load_group<kG, kC>(nxt, in, p0 + step, a.npix, ni, live, lane);
 #pragma unroll
     for (int g = 0; g < kG; ++g) {
       const int64_t p = p0 + g;
@@ -192,12 +204,18 @@ __global__ void __launch_bounds__(kPackThreads, 3) pack_i8_vec_kernel(PackI8Args
         if (lane == 0) a.A[p] = asum / static_cast<float>(ni);
       }
     }
+#pragma unroll
+    for (int g = 0; g < kG; ++g)
+#pragma unroll
+      for (int c = 0; c < kC; ++c) v[g][c] = nxt[g][c];
   }
 }
 
 // Any channel count: one byte per lane per step.
 template <bool kTerms, bool kA, int kOp>
 __global__ void __launch_bounds__(kPackThreads) pack_i8_scalar_kernel(PackI8Args a) {
+  wait_prior_grid();
+  allow_next_grid();
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kPackThreads) >> 5;
@@ -228,15 +246,11 @@ __global__ void __launch_bounds__(kPackThreads) pack_i8_scalar_kernel(PackI8Args
 
 template <bool kTerms, bool kA, int kOp>
 cudaError_t launch_i8_t(const PackI8Args& a, int chunks, dim3 grid, cudaStream_t s) {
-  if (chunks == 1)
-    pack_i8_vec_kernel<kTerms, kA, kOp, 1><<<grid, kPackThreads, 0, s>>>(a);
-  else if (chunks == 2)
-    pack_i8_vec_kernel<kTerms, kA, kOp, 2><<<grid, kPackThreads, 0, s>>>(a);
-  else if (chunks == 4)
-    pack_i8_vec_kernel<kTerms, kA, kOp, 4><<<grid, kPackThreads, 0, s>>>(a);
-  else
-    pack_i8_scalar_kernel<kTerms, kA, kOp><<<grid, kPackThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  auto kern = chunks == 1   ? pack_i8_vec_kernel<kTerms, kA, kOp, 1>
+              : chunks == 2 ? pack_i8_vec_kernel<kTerms, kA, kOp, 2>
+              : chunks == 4 ? pack_i8_vec_kernel<kTerms, kA, kOp, 4>
+                            : pack_i8_scalar_kernel<kTerms, kA, kOp>;
+  return launch_overlapped(kern, grid, dim3(kPackThreads), 0, s, a);
 }
 
 template <bool kTerms, bool kA>
@@ -254,7 +268,7 @@ cudaError_t launch_pack_i8(const PackI8Args& a, cudaStream_t s) {
                    (!a.in_scale || ((reinterpret_cast<uintptr_t>(a.in_scale) | reinterpret_cast<uintptr_t>(a.in_bias)) & 15) == 0);
   const int chunks = vec ? a.cip / 128 : 0;  // 1, 2, 4 -> vector kernel; anything else -> scalar
   int64_t blocks = ceil_div(a.npix, kPackThreads / 32);
-  const int64_t cap = static_cast<int64_t>(sms) * 3;  // one wave at 3 CTAs per SM
+  const int64_t cap = static_cast<int64_t>(sms) * (chunks ? 2 : 3);  // one wave
   if (blocks > cap) blocks = cap;
   const dim3 grid(static_cast<unsigned>(blocks));
   if (a.in_scale)
@@ -283,6 +297,8 @@ __device__ __forceinline__ uint32_t split3_pair(float x0, float x1, uint32_t (&w
 
 template <bool kTerms, bool kA>
 __global__ void __launch_bounds__(kPackThreads) pack_bf16x3_kernel(PackBf16x3Args a) {
+  wait_prior_grid();
+  allow_next_grid();
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kPackThreads) >> 5;
@@ -322,6 +338,8 @@ __global__ void __launch_bounds__(kPackThreads) pack_bf16x3_kernel(PackBf16x3Arg
 // chunk*64 + 2l, 2l+1 and keeps their input terms in registers.
 template <bool kTerms, bool kA, int kC>
 __global__ void __launch_bounds__(kPackThreads, 3) pack_bf16x3_vec_kernel(PackBf16x3Args a) {
+  wait_prior_grid();
+  allow_next_grid();
   constexpr int kG = kC >= 8 ? 1 : 8 / kC;
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
@@ -381,15 +399,12 @@ __global__ void __launch_bounds__(kPackThreads, 3) pack_bf16x3_vec_kernel(PackBf
 }
 
 template <bool kTerms, bool kA>
-void launch_bf16x3_vec(const PackBf16x3Args& a, int chunks, dim3 grid, cudaStream_t s) {
-  if (chunks == 1)
-    pack_bf16x3_vec_kernel<kTerms, kA, 1><<<grid, kPackThreads, 0, s>>>(a);
-  else if (chunks == 2)
-    pack_bf16x3_vec_kernel<kTerms, kA, 2><<<grid, kPackThreads, 0, s>>>(a);
-  else if (chunks == 4)
-    pack_bf16x3_vec_kernel<kTerms, kA, 4><<<grid, kPackThreads, 0, s>>>(a);
-  else
-    pack_bf16x3_vec_kernel<kTerms, kA, 8><<<grid, kPackThreads, 0, s>>>(a);
+cudaError_t launch_bf16x3_vec(const PackBf16x3Args& a, int chunks, dim3 grid, cudaStream_t s) {
+  auto kern = chunks == 1   ? pack_bf16x3_vec_kernel<kTerms, kA, 1>
+              : chunks == 2 ? pack_bf16x3_vec_kernel<kTerms, kA, 2>
+              : chunks == 4 ? pack_bf16x3_vec_kernel<kTerms, kA, 4>
+                            : pack_bf16x3_vec_kernel<kTerms, kA, 8>;
+  return launch_overlapped(kern, grid, dim3(kPackThreads), 0, s, a);
 }
 
 cudaError_t launch_pack_bf16x3(const PackBf16x3Args& a, cudaStream_t s) {
@@ -405,26 +420,16 @@ cudaError_t launch_pack_bf16x3(const PackBf16x3Args& a, cudaStream_t s) {
   const dim3 grid(static_cast<unsigned>(blocks));
   if (vec) {
     if (a.in_scale) {
-      if (a.A) launch_bf16x3_vec<true, true>(a, chunks, grid, s);
-      else launch_bf16x3_vec<true, false>(a, chunks, grid, s);
+      return a.A ? launch_bf16x3_vec<true, true>(a, chunks, grid, s) : launch_bf16x3_vec<true, false>(a, chunks, grid, s);
     } else {
-      if (a.A) launch_bf16x3_vec<false, true>(a, chunks, grid, s);
-      else launch_bf16x3_vec<false, false>(a, chunks, grid, s);
+      return a.A ? launch_bf16x3_vec<false, true>(a, chunks, grid, s)
+                 : launch_bf16x3_vec<false, false>(a, chunks, grid, s);
     }
     return cudaGetLastError();
   }
-  if (a.in_scale) {
-    if (a.A)
-      pack_bf16x3_kernel<true, true><<<grid, kPackThreads, 0, s>>>(a);
-    else
-      pack_bf16x3_kernel<true, false><<<grid, kPackThreads, 0, s>>>(a);
-  } else {
-    if (a.A)
-      pack_bf16x3_kernel<false, true><<<grid, kPackThreads, 0, s>>>(a);
-    else
-      pack_bf16x3_kernel<false, false><<<grid, kPackThreads, 0, s>>>(a);
-  }
-  return cudaGetLastError();
+  auto kern = a.in_scale ? (a.A ? pack_bf16x3_kernel<true, true> : pack_bf16x3_kernel<true, false>)
+                        : (a.A ? pack_bf16x3_kernel<false, true> : pack_bf16x3_kernel<false, false>);
+  return launch_overlapped(kern, grid, dim3(kPackThreads), 0, s, a);
 }
 
 }  // namespace bconv
@@ -454,6 +459,8 @@ template <int kOp>
 __global__ void __launch_bounds__(256) unpack_bits_i8_kernel(const uint32_t* __restrict__ bits, uint32_t total,
                                                               uint32_t groups, int nw_in, int ni,
                                                               uint4* __restrict__ codes) {
+  wait_prior_grid();
+  allow_next_grid();
   for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
     const uint32_t p = i / groups;
     const int c0 = static_cast<int>(i - p * groups) * 16;
@@ -496,11 +503,8 @@ cudaError_t launch_unpack_bits_i8(const uint32_t* bits, int64_t npix, int ni, in
   if (total >= (int64_t{1} << 31)) return cudaErrorInvalidValue;
   const uint32_t t = static_cast<uint32_t>(total), g = static_cast<uint32_t>(cip / 16);
   uint4* out = reinterpret_cast<uint4*>(codes);
-  if (op == kXnor)
-    unpack_bits_i8_kernel<kXnor><<<grid_for(total), 256, 0, s>>>(bits, t, g, words_for(ni), ni, out);
-  else
-    unpack_bits_i8_kernel<kAnd><<<grid_for(total), 256, 0, s>>>(bits, t, g, words_for(ni), ni, out);
-  return cudaGetLastError();
+  return launch_overlapped(op == kXnor ? unpack_bits_i8_kernel<kXnor> : unpack_bits_i8_kernel<kAnd>,
+                           dim3(grid_for(total)), dim3(256), 0, s, bits, t, g, words_for(ni), ni, out);
 }
 
 cudaError_t launch_repack_bits(const uint32_t* bits, int64_t npix, int ni, int nw_pad, uint32_t* out, cudaStream_t s) {

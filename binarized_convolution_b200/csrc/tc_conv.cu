@@ -136,6 +136,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = B->tmem_base;
+  wait_prior_grid();  // the codes, A and the output buffer are the previous kernels' business until here
+  allow_next_grid();
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -422,8 +424,7 @@ cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmB, const
                              : (a.kind ? tc_conv_kernel<false, 1, false> : tc_conv_kernel<false, 0, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreadsTc, smem, s>>>(*tmA, *tmB, *tmBp, *tmOut, a);
-  return cudaGetLastError();
+  return launch_overlapped(kern, dim3(grid), dim3(kThreadsTc), smem, s, *tmA, *tmB, *tmBp, *tmOut, a);
 }
 
 cudaError_t launch_tc_finalize(const float* ws, float* out, const float* scale, const float* bias, const float* beta,

@@ -195,6 +195,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
   cluster_sync();  // both CTAs' barriers exist before any copy or commit crosses over
   tc_fence_after();
   const uint32_t tmem_base = B->tmem_base;
+  wait_prior_grid();  // the codes, A and the output buffer are the previous kernels' business until here
+  allow_next_grid();
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
@@ -462,13 +464,15 @@ cudaError_t launch_tc_conv2(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
   cfg.blockDim = dim3(kThreads2);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may overlap the pack's tail
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, kern, *tmA, *tmB, *tmBp, *tmOut, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
