@@ -45,6 +45,7 @@ METRIC = "binary conv TOPS (1 op = 1 bit MAC) and images/s on 1 B200; % of roofl
 UNIT = "TOPS"
 ROTATE = 4
 ROTATE_BITS = 40  # bit-packed sets are 32x smaller: 40 of them exceed the L2
+PROFILE_EVERY = 8  # time the contraction of one step in 8 (at least 1 for any --steps)
 POPC_PER_CLK_PER_SM = 16  # 32-bit POPC lanes per clock per SM
 FP32_PER_CLK_PER_SM = 128  # FFMA lanes per clock per SM
 
@@ -275,11 +276,11 @@ def run_native(args, w: synth.Workload):
                     use_beta=w.use_beta, relu=w.relu)
     if w.kind == "fc":
         layer = bc.BinaryFC(w.batch, w.in_h, w.in_w, w.in_channels, w.out_channels, wbits=inp.wbits, **layer_kw)
-        prof_begin, prof_end = bc.bfc_profile_begin, bc.bfc_profile_end
+        prof_begin, prof_end, prof_stride = bc.bfc_profile_begin, bc.bfc_profile_end, bc.bfc_profile_stride
     else:
         layer = bc.BinaryConv2d(w.batch, w.in_h, w.in_w, w.in_channels, w.out_channels, (w.kernel_h, w.kernel_w),
                                 (w.stride_y, w.stride_x), wbits=inp.wbits, **layer_kw)
-        prof_begin, prof_end = bc.bconv_profile_begin, bc.bconv_profile_end
+        prof_begin, prof_end, prof_stride = bc.bconv_profile_begin, bc.bconv_profile_end, bc.bconv_profile_stride
     if args.algo != "auto":
         layer.set_algo({"popc": bc.ALGO_POPC, "tcgen05": bc.ALGO_TCGEN05, "simt_f32": bc.ALGO_SIMT_F32}[args.algo])
     out_shape = layer.out_dims
@@ -330,7 +331,10 @@ def run_native(args, w: synth.Workload):
     torch.cuda.synchronize(device)
 
     clocks = ClockSampler(local).start()
+    # the contraction of every PROFILE_EVERY-th step is timed with an event pair on the
+    # library's stream; the pairs serialise the stream around it, so they stay sparse
     prof_begin(layer.handle, args.steps)
+    prof_stride(layer.handle, PROFILE_EVERY)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(device)
     torch.cuda.synchronize(device)
@@ -362,6 +366,7 @@ def run_native(args, w: synth.Workload):
     traffic = measured_traffic(kname, w.name, KERNEL_SOURCES[kname])
     roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
             "traffic": traffic, "kernel": kname, "kernel_ms": kern_ms_max,
+            "kernel_launches_timed": kern_n, "timed_every": PROFILE_EVERY,
             "peak_source": how if bound == "tensor" else f"derived: {how}"}
     sm_mhz = clock_info.get("sm_mhz")
     if sm_mhz and bound == "alu":

@@ -46,6 +46,7 @@ from ._native import (  # noqa: F401
     bconv_pack_bits,
     bconv_profile_begin,
     bconv_profile_end,
+    bconv_profile_stride,
     bconv_set_algo,
     bconv_status_string,
     bconv_sync_status,
@@ -61,6 +62,7 @@ from ._native import (  # noqa: F401
     bfc_output_feature_channels,
     bfc_profile_begin,
     bfc_profile_end,
+    bfc_profile_stride,
     bfc_set_algo,
     bfc_sync_status,
     exported_symbols,

@@ -78,6 +78,8 @@ _SIGS = {
     "bfc_effective_algo": (_I32, [_P]),
     "bfc_sync_status": (_I32, [_P, _P]),
     "bfc_profile_begin": (_I32, [_P, _I32]),
+    "bfc_profile_stride": (_I32, [_P, _I32]),
+    "bconv_profile_stride": (_I32, [_P, _I32]),
     "bfc_profile_end": (_I32, [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_I32)]),
     "bfc_destroy": (_I32, [_P]),
     "bconv_status_string": (ctypes.c_char_p, [_I32]),
@@ -279,6 +281,14 @@ def bconv_profile_begin(h, max_launches: int):
 
 def bfc_profile_begin(h, max_launches: int):
     _check(load_library().bfc_profile_begin(h, int(max_launches)), "bfc_profile_begin")
+
+
+def bconv_profile_stride(h, every: int):
+    _check(load_library().bconv_profile_stride(h, int(every)), "bconv_profile_stride")
+
+
+def bfc_profile_stride(h, every: int):
+    _check(load_library().bfc_profile_stride(h, int(every)), "bfc_profile_stride")
 
 
 def _profile_end(fn, h):

@@ -76,6 +76,13 @@ struct Profile {
   std::vector<cudaEvent_t> start, stop;
   int used = 0;
   bool active = false;
+  int every = 1;  // time every `every`-th forward of the window
+  int seen = 0;
+  // Whether this forward's contraction is timed (advances the sampling counter).
+  bool take() {
+    if (!active || used >= static_cast<int>(start.size())) return false;
+    return (seen++ % every) == 0;
+  }
   void clear() {
     for (auto e : start) cudaEventDestroy(e);
     for (auto e : stop) cudaEventDestroy(e);
@@ -563,7 +570,7 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
     }
     om = &L.tmOut;
   }
-  const bool timed = L.prof.active && L.prof.used < static_cast<int>(L.prof.start.size());
+  const bool timed = L.prof.take();
   if (timed) cudaEventRecord(L.prof.start[L.prof.used], s);
   e = L.tc_pair ? launch_tc_conv2(&L.tmA, &L.tmB, &L.tmBp, om, t, s) : launch_tc_conv(&L.tmA, &L.tmB, &L.tmBp, om, t, s);
   if (timed) cudaEventRecord(L.prof.stop[L.prof.used++], s);
@@ -606,7 +613,7 @@ bconv_status_t run_forward_simt(Layer& L, const Io& io, cudaStream_t s) {
     if (e != cudaSuccess) return from_cuda(e);
   }
   // 3. contraction + epilogue (timed when profiling)
-  const bool timed = L.prof.active && L.prof.used < static_cast<int>(L.prof.start.size());
+  const bool timed = L.prof.take();
   if (timed) cudaEventRecord(L.prof.start[L.prof.used], s);
   if (L.type == kBinaryWeights) {
     BwArgs b{};
@@ -814,6 +821,15 @@ bconv_status_t profile_begin(Layer& L, int32_t n) {
     L.prof.stop.push_back(b);
   }
   L.prof.active = true;
+  L.prof.every = 1;
+  L.prof.seen = 0;
+  return BCONV_OK;
+}
+
+bconv_status_t profile_stride(Layer& L, int32_t every) {
+  if (every <= 0) return BCONV_ERR_INVALID_ARG;
+  L.prof.every = every;
+  L.prof.seen = 0;
   return BCONV_OK;
 }
 
@@ -949,6 +965,11 @@ bconv_status_t bconv_profile_begin(bconv_handle_t h, int32_t max_launches) {
   return profile_begin(h->L, max_launches);
 }
 
+bconv_status_t bconv_profile_stride(bconv_handle_t h, int32_t every) {
+  if (!checked(h, kConvMagic)) return BCONV_ERR_INVALID_ARG;
+  return profile_stride(h->L, every);
+}
+
 bconv_status_t bconv_profile_end(bconv_handle_t h, float* total_ms, int32_t* launches) {
   if (!checked(h, kConvMagic)) return BCONV_ERR_INVALID_ARG;
   DeviceGuard g(h->L.device);
@@ -1051,6 +1072,11 @@ bconv_status_t bfc_profile_begin(bfc_handle_t h, int32_t max_launches) {
   if (!checked(h, kFcMagic)) return BCONV_ERR_INVALID_ARG;
   DeviceGuard g(h->L.device);
   return profile_begin(h->L, max_launches);
+}
+
+bconv_status_t bfc_profile_stride(bfc_handle_t h, int32_t every) {
+  if (!checked(h, kFcMagic)) return BCONV_ERR_INVALID_ARG;
+  return profile_stride(h->L, every);
 }
 
 bconv_status_t bfc_profile_end(bfc_handle_t h, float* total_ms, int32_t* launches) {

@@ -136,6 +136,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = B->tmem_base;
+  if (threadIdx.x == 0) {
+    prefetch_tensor_map(&tmA);
+    prefetch_tensor_map(&tmB);
+    prefetch_tensor_map(&tmBp);
+    if (!kBits) prefetch_tensor_map(&tmOut);  // a bit-packed output never uses (or encodes) it
+  }
   wait_prior_grid();  // the codes, A and the output buffer are the previous kernels' business until here
   allow_next_grid();
 

@@ -211,6 +211,14 @@ bconv_status_t bconv_sync_status(bconv_handle_t h, struct CUstream_st* stream);
  */
 bconv_status_t bconv_profile_begin(bconv_handle_t h, int32_t max_launches);
 bconv_status_t bconv_profile_end(bconv_handle_t h, float* total_ms, int32_t* launches);
+/*
+ * Called after bconv_profile_begin: time only every `every`-th forward (>= 1; each window
+ * starts at 1) of that window, beginning with the next one; max_launches still counts the
+ * timed ones.  Each event pair serialises the stream
+ * around the timed kernel (several microseconds per forward), so a sparse sample keeps the
+ * measurement out of the back-to-back throughput.  INVALID_ARG for every < 1.
+ */
+bconv_status_t bconv_profile_stride(bconv_handle_t h, int32_t every);
 
 /* Free everything the handle owns (waits for the device first).  NULL is a no-op (OK). */
 bconv_status_t bconv_destroy(bconv_handle_t h);
@@ -255,6 +263,7 @@ int32_t bfc_effective_algo(bfc_handle_t h);
 bconv_status_t bfc_sync_status(bfc_handle_t h, struct CUstream_st* stream);
 bconv_status_t bfc_profile_begin(bfc_handle_t h, int32_t max_launches);
 bconv_status_t bfc_profile_end(bfc_handle_t h, float* total_ms, int32_t* launches);
+bconv_status_t bfc_profile_stride(bfc_handle_t h, int32_t every);
 bconv_status_t bfc_destroy(bfc_handle_t h);
 
 /* ------------------------------------------------------------------------------------

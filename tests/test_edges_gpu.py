@@ -109,3 +109,29 @@ def test_properties_and_algo(cuda_device):
         layer.set_algo(bc.ALGO_SIMT_F32)
     assert layer.launches_per_forward() == 2
     layer.close()
+
+
+def test_profile_window_and_stride(cuda_device):
+    """bconv_profile_begin(n) times the contraction of the next n forwards; with
+    bconv_profile_stride(k) only every k-th forward of the window is timed."""
+    import torch
+
+    w = synth.small_case(batch=1, h=8, w=8, ni=64, no=32, k=3, op=synth.XNOR, seed=16)
+    inp = synth.make_inputs(w)
+    layer = pu.make_layer(w, inp)
+    x = torch.from_numpy(inp.x).cuda()
+    bc.bconv_profile_begin(layer.handle, 100)
+    for _ in range(5):
+        layer(x)
+    ms, n = bc.bconv_profile_end(layer.handle)
+    assert n == 5 and ms > 0
+    bc.bconv_profile_begin(layer.handle, 100)
+    bc.bconv_profile_stride(layer.handle, 3)
+    for _ in range(7):
+        layer(x)
+    ms, n = bc.bconv_profile_end(layer.handle)
+    assert n == 3 and ms > 0  # forwards 0, 3 and 6
+    with pytest.raises(bc.BconvError):
+        bc.bconv_profile_stride(layer.handle, 0)
+    layer.sync_status()
+    layer.close()
