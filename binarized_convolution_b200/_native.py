@@ -336,7 +336,8 @@ def bconv_version() -> int:
 
 def bconv_measure_peak(kind: int):
     """Returns (ops per second, SM MHz) for probe kind 0 (POPC), 1 (LOP3), 2 (b1 mma.sync),
-    3 (tcgen05 kind::i8 M128 N256) or 4 (tcgen05 kind::f16 bf16 M128 N256)."""
+    3 (tcgen05 kind::i8 M128 N256) or 4 (tcgen05 kind::f16 bf16 M128 N256) on zero operands,
+    5 or 6 (kinds 3 and 4 on pseudo-random +-1 operands)."""
     ops, mhz = ctypes.c_double(), ctypes.c_double()
     _check(load_library().bconv_measure_peak(int(kind), ctypes.byref(ops), ctypes.byref(mhz)), "bconv_measure_peak")
     return ops.value, mhz.value

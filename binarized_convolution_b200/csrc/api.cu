@@ -355,6 +355,13 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   if (pairs > 0) {
     L.tc_pair = true;
     tc2_plan(t, pairs);
+    if (t.sk) {  // partial sums of the items cut between pairs, and their ready flags
+      const int cuts = t.grid_ctas / 2 - 1;
+      cudaError_t e2 = L.mem.alloc(&t.sk_part, static_cast<size_t>(cuts) * 2 * t.BN * 128);
+      if (e2 == cudaSuccess) e2 = L.mem.alloc(&t.sk_flag, static_cast<size_t>(cuts) * 2);
+      if (e2 == cudaSuccess) e2 = cudaMemset(t.sk_flag, 0, sizeof(uint32_t) * cuts * 2);
+      if (e2 != cudaSuccess) return from_cuda(e2);
+    }
     ok = ok && encode_2d(&L.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(kt),
                          static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128,
                          static_cast<uint32_t>(t.BN / 2));
@@ -775,6 +782,7 @@ bconv_status_t sync_status(Layer& L, cudaStream_t s) {
   if (word) {
     cudaMemset(L.err, 0, sizeof(uint32_t));
     if (L.a_count) cudaMemset(L.a_count, 0, sizeof(uint32_t) * L.tc.m_tiles);  // an aborted launch may leave counts
+    if (L.tc.sk_flag) cudaMemset(L.tc.sk_flag, 0, sizeof(uint32_t) * (L.tc.grid_ctas / 2 - 1) * 2);  // and flags
     if (word & kErrTimeout) return BCONV_ERR_TIMEOUT;
     return BCONV_ERR_CUDA;  // kErrLayout: a kernel refused an unexpected shared-memory layout
   }
@@ -1123,7 +1131,7 @@ bconv_status_t bconv_pack_bits(const uint8_t* bits, int64_t rows, int32_t nbits,
 int32_t bconv_version(void) { return 100; }
 
 bconv_status_t bconv_measure_peak(int32_t kind, double* ops_per_s, double* sm_mhz) {
-  if (kind < 0 || kind > 4 || !ops_per_s) return BCONV_ERR_INVALID_ARG;
+  if (kind < 0 || kind > 6 || !ops_per_s) return BCONV_ERR_INVALID_ARG;
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
     cudaGetLastError();

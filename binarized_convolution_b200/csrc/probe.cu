@@ -8,6 +8,7 @@
 //   kind 3: tcgen05.mma.cta_group::1.kind::i8, M=128 N=256 K=32, operands in shared memory,
 //           accumulator in TMEM; multiply-accumulates per second.
 //   kind 4: tcgen05.mma.cta_group::1.kind::f16 (bf16 operands), M=128 N=256 K=16.
+//   kinds 5, 6: kinds 3 and 4 on pseudo-random +-1 operands instead of zeros.
 //
 // Every thread runs independent dependency chains so that issue rate, not latency, is the
 // limit.  Results are stored so the work cannot be removed.  The grid fills every SM with
@@ -100,10 +101,11 @@ __global__ void __launch_bounds__(kProbeThreads) b1mma_probe(int iters, uint32_t
   if ((threadIdx.x & 31) == 0) atomicMax(reinterpret_cast<unsigned long long*>(cycles), static_cast<unsigned long long>(t1 - t0));
 }
 
-// Back-to-back tcgen05 MMAs of one CTA per SM on zero operands (no data movement): the tensor
-// pipe's own rate.  One thread issues `iters` groups of 4 MMAs into one TMEM accumulator and
-// waits for them through tcgen05.commit (bounded wait).
-template <bool kI8>
+// Back-to-back tcgen05 MMAs of one CTA per SM (no data movement): the tensor pipe's own rate,
+// on zero operands or (kRandom) on pseudo-random +-1 operands -- int8 0x01 / 0xFF, bf16 +1 / -1
+// -- like the contraction's.  One thread issues `iters` groups of 4 MMAs into one TMEM
+// accumulator and waits for them through tcgen05.commit (bounded wait).
+template <bool kI8, bool kRandom>
 __global__ void __launch_bounds__(128, 1) tcgen05_probe(int iters, uint32_t* out, long long* cycles, uint32_t* err) {
   using namespace tcdev;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -119,8 +121,21 @@ __global__ void __launch_bounds__(128, 1) tcgen05_probe(int iters, uint32_t* out
   uint8_t* sa = smem;                  // 128 rows x 128 B
   uint8_t* sb = smem + 128 * 128;      // 256 rows x 128 B
   Bars* B = reinterpret_cast<Bars*>(smem + 128 * 128 + 256 * 128);
-  for (int i = threadIdx.x; i < (128 + 256) * 128 / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = threadIdx.x; i < (128 + 256) * 128 / 4; i += blockDim.x) {
+    uint32_t w = 0;
+    if (kRandom) {
+      uint32_t h = (static_cast<uint32_t>(i) + 0x9E3779B9u * (blockIdx.x + 1)) * 0x85EBCA6Bu;
+      h ^= h >> 13;
+      h *= 0xC2B2AE35u;
+      h ^= h >> 16;
+      if (kI8) {
+        for (int b = 0; b < 4; ++b) w |= (((h >> b) & 1u) ? 0x01u : 0xFFu) << (8 * b);
+      } else {
+        w = (((h & 1u) ? 0x3F80u : 0xBF80u)) | (((h & 2u) ? 0x3F80u : 0xBF80u) << 16);
+      }
+    }
+    reinterpret_cast<uint32_t*>(smem)[i] = w;
+  }
   if (threadIdx.x == 0) {
     mbar_init(&B->done, 1);
     B->abort_flag = 0;
@@ -171,7 +186,7 @@ __global__ void __launch_bounds__(128, 1) tcgen05_probe(int iters, uint32_t* out
 }  // namespace
 
 cudaError_t probe_peak(int kind, double* ops_per_s, double* sm_mhz) {
-  if (kind == 3 || kind == 4) {
+  if (kind == 3 || kind == 4 || kind == 5 || kind == 6) {
     const int sms = current_sm_count();
     const int iters = 2048;
     const int smem = 120 * 1024;  // more than half an SM's shared memory: one CTA per SM
@@ -185,7 +200,10 @@ cudaError_t probe_peak(int kind, double* ops_per_s, double* sm_mhz) {
     if (e == cudaSuccess) e = cudaMemset(err, 0, sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaEventCreate(&e0);
     if (e == cudaSuccess) e = cudaEventCreate(&e1);
-    auto kern = kind == 3 ? tcgen05_probe<true> : tcgen05_probe<false>;
+    auto kern = kind == 3   ? tcgen05_probe<true, false>
+                : kind == 4 ? tcgen05_probe<false, false>
+                : kind == 5 ? tcgen05_probe<true, true>
+                            : tcgen05_probe<false, true>;
     if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     float best = 0.f;
     long long cycles = 0;
@@ -207,7 +225,7 @@ cudaError_t probe_peak(int kind, double* ops_per_s, double* sm_mhz) {
     if (e == cudaSuccess) e = cudaMemcpy(&herr, err, sizeof(herr), cudaMemcpyDeviceToHost);
     if (e == cudaSuccess && herr) e = cudaErrorLaunchTimeout;
     if (e == cudaSuccess && best > 0.f) {
-      const double macs = static_cast<double>(sms) * iters * 4.0 * 128.0 * 256.0 * (kind == 3 ? 32.0 : 16.0);
+      const double macs = static_cast<double>(sms) * iters * 4.0 * 128.0 * 256.0 * ((kind == 3 || kind == 5) ? 32.0 : 16.0);
       if (ops_per_s) *ops_per_s = macs / (best * 1e-3);
       if (sm_mhz) *sm_mhz = static_cast<double>(cycles) / (best * 1e3);
     }

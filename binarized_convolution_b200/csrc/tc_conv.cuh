@@ -51,6 +51,14 @@ struct TcArgs {
   int nwo;                  // ceil(No / 32)
   float* a_part;            // [n_tiles * pieces][N * Ho * Wo]
   uint32_t* a_count;        // [m_tiles], zero between launches
+  // Balanced split of the reduction (SM-pair kernel; sk != 0): the work list's items x
+  // k-blocks are cut into equal contiguous shares, one per pair.  An item cut between pairs
+  // p and p+1 is finished by p (which computes its first k-blocks, last in its share); p+1
+  // computes the rest first and leaves its raw partial sums in sk_part[p][rank] with
+  // sk_flag[p][rank] = 1, which p adds (int32 exactly, fp32 in a fixed order) and resets.
+  int sk;
+  uint32_t* sk_part;        // [pairs - 1][2][BN / 32][32][128] accumulator words
+  uint32_t* sk_flag;        // [pairs - 1][2], zero between launches
 };
 
 int tc_smem_bytes(int bn, int mt);

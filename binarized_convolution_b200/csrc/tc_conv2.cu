@@ -148,7 +148,48 @@ __device__ __forceinline__ PairCoord pair_coord(const TcArgs& a, int w, int rank
   return c;
 }
 
-template <int kKind, bool kBits>
+// A pair's work: the items w = pair, pair + npairs, ... with all k-blocks, or (kSk) the
+// contiguous share [U*pair/npairs, U*(pair+1)/npairs) of the U = items x kb_total
+// reduction units, as segments (item, k0, k1).
+template <bool kSk>
+struct PairWork {
+  int64_t u, uend;
+  int w;
+  __device__ PairWork(int pair, int npairs, int items, int kb_total) {
+    const int64_t U = static_cast<int64_t>(items) * kb_total;
+    u = kSk ? U * pair / npairs : 0;
+    uend = kSk ? U * (pair + 1) / npairs : 0;
+    w = pair;
+  }
+  __device__ bool next(int npairs, int items, int kb_total, int& item, int& k0, int& k1) {
+    if (!kSk) {
+      if (w >= items) return false;
+      item = w;
+      k0 = 0;
+      k1 = kb_total;
+      w += npairs;
+      return true;
+    }
+    if (u >= uend) return false;
+    item = static_cast<int>(u / kb_total);
+    k0 = static_cast<int>(u - static_cast<int64_t>(item) * kb_total);
+    k1 = static_cast<int>(min(static_cast<int64_t>(kb_total), k0 + (uend - u)));
+    u += k1 - k0;
+    return true;
+  }
+};
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+template <int kKind, bool kBits, bool kSk>
 __global__ void __launch_bounds__(kThreads2, 1)
     tc_conv2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmBp, const __grid_constant__ CUtensorMap tmOut,
@@ -210,10 +251,12 @@ __global__ void __launch_bounds__(kThreads2, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int w = pair; w < total && ok; w += npairs) {
+      PairWork<kSk> work(pair, npairs, total, kb_total);
+      int w, k0, k1;
+      while (ok && work.next(npairs, total, kb_total, w, k0, k1)) {
         const PairCoord pc = pair_coord(a, w, rank);
         const uint32_t tx = static_cast<uint32_t>(2 * (kABytes2 + (pc.bn / 2) * 128));  // both CTAs' bytes
-        for (int kb = 0; kb < kb_total; ++kb) {
+        for (int kb = k0; kb < k1; ++kb) {
           if (!mbar_wait(&B->empty[stage], phase ^ 1u, B, a.err)) {
             ok = false;
             break;
@@ -245,13 +288,15 @@ __global__ void __launch_bounds__(kThreads2, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int w = pair; w < total && ok; w += npairs) {
+      PairWork<kSk> work(pair, npairs, total, kb_total);
+      int w, k0, k1;
+      while (ok && work.next(npairs, total, kb_total, w, k0, k1)) {
         const PairCoord pc = pair_coord(a, w, 0);
         const uint32_t idesc = idesc_for(kKind, 256, pc.bn);
         if (!mbar_wait(&B->tmem_empty[acc], acc_phase ^ 1u, B, a.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
-        for (int kb = 0; kb < kb_total; ++kb) {
+        for (int kb = k0; kb < k1; ++kb) {
           if (!mbar_wait(&B->full[stage], phase, B, a.err)) {
             ok = false;
             break;
@@ -261,7 +306,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
           const uint64_t da = smem_desc_sw128(sa), db = smem_desc_sw128(sa + kABytes2);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint32_t accum = (kb > 0 || j > 0) ? 1u : 0u;
+            const uint32_t accum = (kb > k0 || j > 0) ? 1u : 0u;
             if constexpr (kKind == 1)
               tc_mma_bf16_pair(d_tmem, da + 2u * j, db + 2u * j, idesc, accum);
             else
@@ -296,8 +341,34 @@ __global__ void __launch_bounds__(kThreads2, 1)
     constexpr bool bits_out = kBits;
     float2* next_t = reinterpret_cast<float2*>(stage_out);
     uint32_t* bits_flag = reinterpret_cast<uint32_t*>(stage_out + kOutBytes2);
-    for (int w = pair; w < total; w += npairs) {
+    PairWork<kSk> work(pair, npairs, total, kb_total);
+    int w, k0, k1;
+    while (work.next(npairs, total, kb_total, w, k0, k1)) {
       const PairCoord pc = pair_coord(a, w, rank);
+      if (kSk && k0 > 0) {
+        // the later k-blocks of an item that pair - 1 finishes: leave the raw sums for it
+        if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err))) break;
+        tc_fence_after();
+        uint32_t* part = a.sk_part + static_cast<size_t>((pair - 1) * 2 + static_cast<int>(rank)) * a.BN * 128;
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
+        for (int ch = 0; ch < pc.bn / 32; ++ch) {
+          uint32_t v[32];
+          tc_ld_32x32(tb + static_cast<uint32_t>(ch * 32), v);
+          if (ch == pc.bn / 32 - 1) {
+            tc_fence_before();
+            if (lane == 0) mbar_arrive_remote(acc == 0 ? empty_leader0 : empty_leader1);
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) part[(ch * 32 + j) * 128 + row] = v[j];  // lanes write 128 B rows
+        }
+        __threadfence();
+        epi_barrier();
+        if (et == 0) st_release(a.sk_flag + (pair - 1) * 2 + rank, 1u);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+        continue;
+      }
+      const bool owner = kSk && k1 < kb_total;  // pair + 1 computes this item's remaining k-blocks
       if (pc.ntile != loaded_ntile) {
         epi_barrier();
         for (int j = et; j < a.BN; j += kEpi2) {
@@ -331,6 +402,25 @@ __global__ void __launch_bounds__(kThreads2, 1)
       }
       if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err))) break;
       tc_fence_after();
+      const uint32_t* part = nullptr;
+      if (owner) {  // wait (bounded) for the partial sums of this item's remaining k-blocks
+        bool ready = true;
+        if (et == 0) {
+          const uint32_t* flag = a.sk_flag + pair * 2 + rank;
+          const uint64_t t0 = globaltimer();
+          while (ld_acquire(flag) == 0u) {
+            if (*reinterpret_cast<volatile uint32_t*>(&B->abort_flag) || globaltimer() - t0 > kTimeoutNs) {
+              atomicOr(a.err, kErrTimeout);
+              atomicExch(&B->abort_flag, 1u);
+              ready = false;
+              break;
+            }
+          }
+        }
+        if (!epi_all(ready)) break;
+        __threadfence();
+        part = a.sk_part + static_cast<size_t>(pair * 2 + static_cast<int>(rank)) * a.BN * 128;
+      }
       float bits_asum = 0.f;
       Words8 bits_w{};
       const int64_t pix = (static_cast<int64_t>(n) * a.Ho + oy) * a.Wo + ox;
@@ -341,6 +431,14 @@ __global__ void __launch_bounds__(kThreads2, 1)
         if (ch == pc.bn / 32 - 1) {  // this CTA's rows are read: release them on the leader
           tc_fence_before();
           if (lane == 0) mbar_arrive_remote(acc == 0 ? empty_leader0 : empty_leader1);
+        }
+        if (part) {  // + the other pair's sums: int32 exactly, fp32 in this fixed order
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const uint32_t o = __ldcg(part + (ch * 32 + j) * 128 + row);
+            v[j] = kKind == 1 ? __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(o))
+                              : static_cast<uint32_t>(static_cast<int32_t>(v[j]) + static_cast<int32_t>(o));
+          }
         }
         const int buf = chunk_count & 1;
         ++chunk_count;
@@ -379,6 +477,10 @@ __global__ void __launch_bounds__(kThreads2, 1)
           bulk_wait_read_1();
         }
       }
+      if (owner) {  // every thread has read the partial sums: the slot is free for the next launch
+        epi_barrier();
+        if (et == 0) a.sk_flag[pair * 2 + rank] = 0u;
+      }
       if (bits_out && !pc.dummy) {
         const int w0 = (pc.ntile * a.BN + pc.noff) / 32;  // first word of this item
         if (valid) words_store(a.out_bits + pix * a.nwo + w0, bits_w, min(pc.bn / 32, a.nwo - w0));
@@ -408,10 +510,15 @@ int tc2_smem_bytes(int bn) {
 
 int tc2_max_pairs(int bn) {
   const int smem = tc2_smem_bytes(bn);
-  if (cudaFuncSetAttribute(tc_conv2_kernel<0, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-      cudaFuncSetAttribute(tc_conv2_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-      cudaFuncSetAttribute(tc_conv2_kernel<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-      cudaFuncSetAttribute(tc_conv2_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+  const void* kerns[] = {
+      reinterpret_cast<const void*>(tc_conv2_kernel<0, false, false>), reinterpret_cast<const void*>(tc_conv2_kernel<1, false, false>),
+      reinterpret_cast<const void*>(tc_conv2_kernel<0, true, false>), reinterpret_cast<const void*>(tc_conv2_kernel<1, true, false>),
+      reinterpret_cast<const void*>(tc_conv2_kernel<0, false, true>), reinterpret_cast<const void*>(tc_conv2_kernel<1, false, true>),
+      reinterpret_cast<const void*>(tc_conv2_kernel<0, true, true>), reinterpret_cast<const void*>(tc_conv2_kernel<1, true, true>)};
+  bool attr_ok = true;
+  for (const void* k : kerns)
+    attr_ok = attr_ok && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+  if (!attr_ok) {
     cudaGetLastError();
     return 0;
   }
@@ -427,7 +534,7 @@ int tc2_max_pairs(int bn) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, tc_conv2_kernel<0, false>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, tc_conv2_kernel<0, false, false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -439,16 +546,17 @@ int tc2_plan(TcArgs& a, int pairs) {
   const int npairs = pairs;
   a.full_tiles = pair_tiles;
   a.pieces = 1;
+  a.sk = 0;
   const int grid_pairs = npairs < pair_tiles ? npairs : pair_tiles;
   const int tail = grid_pairs > 0 ? pair_tiles % grid_pairs : 0;
+  // More items than pairs and a last wave so ragged that whole-item waves would keep more
+  // than a fifth of the pairs idle on average: give every pair an equal share of the
+  // items x k-blocks instead (each share then spans at least one whole item, so an item is
+  // cut between two pairs at most).  Measured: 98 items on 74 pairs (waves 66 % full) go from
+  // 53.2 to 46.3 us; 196 items (88 % full) run slower split than whole (36.5 -> 49.9 us).
   if (pair_tiles > grid_pairs && tail > 0) {
-    for (int p = a.BN / 32; p > 1; --p) {
-      if ((a.BN / 32) % p == 0 && tail * p <= grid_pairs) {
-        a.pieces = p;
-        break;
-      }
-    }
-    if (a.pieces > 1) a.full_tiles = pair_tiles - tail;
+    const int waves = (pair_tiles + grid_pairs - 1) / grid_pairs;
+    if (static_cast<double>(pair_tiles) / (static_cast<double>(waves) * grid_pairs) < 0.8) a.sk = 1;
   }
   a.grid_ctas = 2 * grid_pairs;
   return a.grid_ctas;
@@ -461,8 +569,10 @@ cudaError_t launch_tc_conv2(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
   const int smem = tc2_smem_bytes(a.BN);
   const int npairs = a.grid_ctas / 2;
   if (npairs <= 0) return cudaErrorInvalidConfiguration;
-  auto kern = a.out_bits ? (a.kind ? tc_conv2_kernel<1, true> : tc_conv2_kernel<0, true>)
-                         : (a.kind ? tc_conv2_kernel<1, false> : tc_conv2_kernel<0, false>);
+  auto kern = a.sk ? (a.out_bits ? (a.kind ? tc_conv2_kernel<1, true, true> : tc_conv2_kernel<0, true, true>)
+                                 : (a.kind ? tc_conv2_kernel<1, false, true> : tc_conv2_kernel<0, false, true>))
+                   : (a.out_bits ? (a.kind ? tc_conv2_kernel<1, true, false> : tc_conv2_kernel<0, true, false>)
+                                 : (a.kind ? tc_conv2_kernel<1, false, false> : tc_conv2_kernel<0, false, false>));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};

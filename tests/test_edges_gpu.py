@@ -135,3 +135,23 @@ def test_profile_window_and_stride(cuda_device):
         bc.bconv_profile_stride(layer.handle, 0)
     layer.sync_status()
     layer.close()
+
+
+@pytest.mark.parametrize("op,ni", [(synth.XNOR, 32), (synth.AND, 160), (synth.BINARY_WEIGHTS, 32)])
+def test_reduction_split_between_sm_pairs(op, ni, cuda_device):
+    """162 tiles of 128 pixels on the SM pairs (more pair items than pairs, a ragged last wave):
+    the reduction is shared out evenly and items cut between two pairs are summed from both
+    halves.  Every output is checked, and two runs must agree bit for bit."""
+    import torch
+
+    w = synth.small_case(batch=4, h=70, w=70, ni=ni, no=32, k=3, op=op, use_beta=True, relu=True, in_terms=True,
+                         seed=17)
+    inp = synth.make_inputs(w)
+    _check(w, inp)
+    layer = pu.make_layer(w, inp)
+    x = torch.from_numpy(inp.x).cuda()
+    y1 = layer(x)
+    y2 = layer(x)
+    layer.sync_status()
+    layer.close()
+    assert torch.equal(y1, y2)
