@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       // all MMAs issued by this thread have completed once `done` fires (waited even after an
       // abort, so that TMEM is never released under a running MMA)
       tc_commit(&B->done);
-      mbar_wait(&B->done, 0, B, a.err, false);
+      mbar_wait(&B->done, 0, B, a.err, false, true);
     }
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           beta_h[h] = __ldg(a.beta + (static_cast<int64_t>(n) * a.Ho + oy) * a.Wo + ox);
         }
       }
-      if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err))) break;
+      if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err, true, true))) break;
       tc_fence_after();
       float bits_asum = 0.f;
       Words8 bits_w{};

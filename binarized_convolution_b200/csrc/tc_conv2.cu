@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
       }
       tc_commit_pair(&B->done);  // fires in both CTAs once every MMA above has completed
     }
-    if (lane == 0) mbar_wait(&B->done, 0, B, a.err, false);
+    if (lane == 0) mbar_wait(&B->done, 0, B, a.err, false, true);
   } else {
     // ---------------- epilogue (both CTAs, warps 2..5) ----------------
     const int q = warp & 3;
@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
       const PairCoord pc = pair_coord(a, w, rank);
       if (kSk && k0 > 0) {
         // the later k-blocks of an item that pair - 1 finishes: leave the raw sums for it
-        if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err))) break;
+        if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err, true, true))) break;
         tc_fence_after();
         uint32_t* part = a.sk_part + static_cast<size_t>((pair - 1) * 2 + static_cast<int>(rank)) * a.BN * 128;
         const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
       } else if (valid && a.beta) {
         beta = __ldg(a.beta + (static_cast<int64_t>(n) * a.Ho + oy) * a.Wo + ox);
       }
-      if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err))) break;
+      if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err, true, true))) break;
       tc_fence_after();
       const uint32_t* part = nullptr;
       if (owner) {  // wait (bounded) for the partial sums of this item's remaining k-blocks

@@ -44,15 +44,28 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that may suspend the thread (up to `hint_ns`) until the phase completes, so that a
+// waiting warp takes no issue slots from the warps that share its scheduler.
+__device__ __forceinline__ bool mbar_try_suspend(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete; false after the time limit or, when
-// `follow_abort`, as soon as another role has given up (the caller then stops).
+// `follow_abort`, as soon as another role has given up (the caller then stops).  `idle`
+// waits (the epilogue's wait for an accumulator, the final drain) suspend between checks.
 template <class Bars>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Bars* B, uint32_t* err,
-                                          bool follow_abort = true) {
+                                          bool follow_abort = true, bool idle = false) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try(bar, parity)) return true;
+    if (idle ? mbar_try_suspend(bar, parity, 20000u) : mbar_try(bar, parity)) return true;
     if (follow_abort && *reinterpret_cast<volatile uint32_t*>(&B->abort_flag)) return false;
     if (globaltimer() - t0 > kTimeoutNs) {
       atomicOr(err, kErrTimeout);
