@@ -7,8 +7,9 @@ A step is one forward of the layer (input transform + pack + A, beta, contractio
 epilogue) over one batch of the workload: by default XNOR with beta scaling and input terms,
 batch 16, 56x56, 256 -> 256 channels, 3x3, ReLU.  ``value`` is nominal bit multiply-
 accumulates (every window tap, 1 op = 1 bit MAC) per second over all ranks, with inputs
-resident in HBM; four input/output buffer sets rotate so that one step's data is not in L2
-when it is next used (411 MB > the 126 MB L2).  ``e2e`` is the same metric through
+resident in HBM; input/output buffer sets rotate so that one step's data is not in L2 when it
+is next used (at least four sets and together more than 1.5 x the L2: 411 MB for the default
+workload).  ``e2e`` is the same metric through
 bconv_forward_host with page-locked host buffers (host-to-device copy, forward,
 device-to-host copy inside every step).  Multi-GPU runs (torchrun) are independent replicas
 with a batch each (weak scaling); their time is the maximum over ranks.
@@ -43,8 +44,14 @@ from binarized_convolution_b200 import synth  # noqa: E402
 DEFAULT_WORKLOAD = "xnor_beta_n16_56x56_c256_k256_3x3"
 METRIC = "binary conv TOPS (1 op = 1 bit MAC) and images/s on 1 B200; % of roofline"
 UNIT = "TOPS"
-ROTATE = 4
-ROTATE_BITS = 40  # bit-packed sets are 32x smaller: 40 of them exceed the L2
+ROTATE_MIN = 4
+L2_BYTES = 126 * 1024 * 1024  # B200 L2 (the device property is used when available)
+
+
+def rotation_count(set_bytes: int, l2_bytes: int, minimum: int = ROTATE_MIN) -> int:
+    """Input/output sets to rotate through so that together they exceed 1.5 x the L2: a
+    step's data has then been evicted by the time the step comes round again."""
+    return max(minimum, -(-int(1.5 * l2_bytes) // max(int(set_bytes), 1)))
 PROFILE_EVERY = 8  # time the contraction of one step in 8 (at least 1 for any --steps)
 POPC_PER_CLK_PER_SM = 16  # 32-bit POPC lanes per clock per SM
 FP32_PER_CLK_PER_SM = 128  # FFMA lanes per clock per SM
@@ -284,8 +291,13 @@ def run_native(args, w: synth.Workload):
     if args.algo != "auto":
         layer.set_algo({"popc": bc.ALGO_POPC, "tcgen05": bc.ALGO_TCGEN05, "simt_f32": bc.ALGO_SIMT_F32}[args.algo])
     out_shape = layer.out_dims
+    l2_bytes = getattr(torch.cuda.get_device_properties(device), "L2_cache_size", 0) or L2_BYTES
+    set_bytes = inp.x.nbytes + int(np.prod(out_shape)) * 4
+    bits_set_bytes = 2 * ((int(np.prod(out_shape)) + 31) // 32 * 4 + int(np.prod(out_shape[:-1])) * 4)
+    ROTATE = rotation_count(set_bytes, l2_bytes)
+    ROTATE_BITS = rotation_count(bits_set_bytes, l2_bytes)
     xs = [torch.from_numpy(inp.x).to(device)]
-    for r in range(1, ROTATE):
+    for r in range(1, min(ROTATE, ROTATE_BITS) if args.io == "bits" else ROTATE):
         xs.append(torch.from_numpy(synth.make_batch(w, seed=replica_seed(w.seed, rank) * 1000 + r)).to(device))
     stream = torch.cuda.current_stream(device)
     bits_io = args.io == "bits"
@@ -393,12 +405,11 @@ def run_native(args, w: synth.Workload):
                    "beta": w.use_beta, "relu": w.relu, "input_terms": w.in_terms,
                    "parallelism": f"replicas x{world}", "algo": kname,
                    "io": "bit-packed in and out (chain middle layer)" if bits_io else "fp32 in and out",
-                   "l2": (f"{ROTATE} rotating input/output sets, "
-                          f"{ROTATE * (inp.x.nbytes + int(np.prod(out_shape)) * 4) / 1e6:.0f} MB > 126 MB L2")
+                   "l2": (f"{ROTATE} rotating input/output sets, {ROTATE * set_bytes / 1e6:.0f} MB > "
+                          f"{l2_bytes / 1e6:.0f} MB L2")
                    if not bits_io else
-                   f"{ROTATE_BITS} rotating bit-packed input/output sets, "
-                   f"{ROTATE_BITS * 2 * (int(np.prod(out_shape)) // 8 + int(np.prod(out_shape[:3])) * 4) / 1e6:.0f}"
-                   f" MB > 126 MB L2"},
+                   f"{ROTATE_BITS} rotating bit-packed input/output sets, {ROTATE_BITS * bits_set_bytes / 1e6:.0f}"
+                   f" MB > {l2_bytes / 1e6:.0f} MB L2"},
         "images_per_s": images_s,
         "roofline": roof,
         "clocks": clock_info,

@@ -243,9 +243,12 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   // channels per part, padded to whole 128-byte rows; bytes of operand per pixel
   L.cip = t.kind == 0 ? round_up(L.Ni, 128) : round_up(L.Ni, 64);
   const int bpp = t.kind == 0 ? L.cip : 6 * L.cip;
-  // The FC keeps a batch of up to 256 images in one CTA tile (two 128-row sub-tiles sharing
-  // every weight stage), so its large weight matrix streams from memory once.
-  t.mt = (L.fc && L.N > 128) ? 2 : 1;
+  // The FC runs on SM pairs when its batch fills both CTAs of a pair (256 images per pair
+  // tile, so the weight matrix streams from memory once, with half of every weight tile per
+  // SM); otherwise a single SM keeps up to 256 images in one tile (two 128-row sub-tiles
+  // sharing every weight stage).
+  const bool fc_pair = L.fc && L.N > 128 && tc2_max_pairs(std::min(256, round_up(L.No, 32))) > 0;
+  t.mt = (L.fc && L.N > 128 && !fc_pair) ? 2 : 1;
   t.BN = std::min(t.mt == 2 ? 128 : 256, round_up(L.No, 32));
   t.n_tiles = (L.No + t.BN - 1) / t.BN;
   t.No = L.No;
@@ -289,12 +292,12 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   t.m_tiles = t.tiles_x * t.tiles_y * ((L.N + t.Bn * t.mt - 1) / (t.Bn * t.mt));
   const int kb_total = t.kh * t.kw * t.kb_per_tap;
   t.k_splits = 1;
-  if (L.fc) {  // spread the reduction so that the tiles fill the GPU
-    const int sms = current_sm_count();
-    const int64_t tiles = static_cast<int64_t>(t.m_tiles) * t.n_tiles;
+  if (L.fc) {  // spread the reduction so that the tiles fill the GPU (or its SM pairs)
+    const int workers = fc_pair ? tc2_max_pairs(t.BN) : current_sm_count();
+    const int64_t tiles = static_cast<int64_t>(fc_pair ? (t.m_tiles + 1) / 2 : t.m_tiles) * t.n_tiles;
     int64_t best = -1;
     for (int sp = 1; sp <= 16 && kb_total / sp >= 4; ++sp) {
-      const int64_t cost = ceil_div(tiles * sp, sms) * ceil_div(kb_total, sp);
+      const int64_t cost = ceil_div(tiles * sp, workers) * ceil_div(kb_total, sp);
       if (best < 0 || cost < best) {
         best = cost;
         t.k_splits = sp;
@@ -351,7 +354,7 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
                        static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128, static_cast<uint32_t>(t.BN));
   // Convolutions run on SM pairs when two-CTA clusters fit; each CTA then loads half of
   // every weight tile (boxes of BN/2 rows).
-  const int pairs = L.fc ? 0 : tc2_max_pairs(t.BN);
+  const int pairs = (L.fc && !fc_pair) ? 0 : tc2_max_pairs(t.BN);
   if (pairs > 0) {
     L.tc_pair = true;
     tc2_plan(t, pairs);

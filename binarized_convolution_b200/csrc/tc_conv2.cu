@@ -154,19 +154,23 @@ __device__ __forceinline__ PairCoord pair_coord(const TcArgs& a, int w, int rank
 template <bool kSk>
 struct PairWork {
   int64_t u, uend;
-  int w;
-  __device__ PairWork(int pair, int npairs, int items, int kb_total) {
+  int w, ks;
+  __device__ PairWork(int pair, int npairs, int items, int kb_total, int k_splits = 1) {
     const int64_t U = static_cast<int64_t>(items) * kb_total;
     u = kSk ? U * pair / npairs : 0;
     uend = kSk ? U * (pair + 1) / npairs : 0;
     w = pair;
+    ks = k_splits;
   }
+  // items are (tile, split) pairs, split fastest; a tile's split s covers k-blocks
+  // [s * ceil(kb_total / ks), ...) -- ks = 1 without a split reduction
   __device__ bool next(int npairs, int items, int kb_total, int& item, int& k0, int& k1) {
     if (!kSk) {
       if (w >= items) return false;
-      item = w;
-      k0 = 0;
-      k1 = kb_total;
+      item = w / ks;
+      const int per = (kb_total + ks - 1) / ks;
+      k0 = (w - item * ks) * per;
+      k1 = min(k0 + per, kb_total);
       w += npairs;
       return true;
     }
@@ -189,7 +193,7 @@ __device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-template <int kKind, bool kBits, bool kSk>
+template <int kKind, bool kBits, bool kSk, bool kSplit>
 __global__ void __launch_bounds__(kThreads2, 1)
     tc_conv2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmBp, const __grid_constant__ CUtensorMap tmOut,
@@ -208,7 +212,9 @@ __global__ void __launch_bounds__(kThreads2, 1)
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int pair_tiles = (a.m_tiles + 1) / 2 * a.n_tiles;
+  // work items: pair tiles (x k splits for a split reduction, with its partial sums added into
+  // an fp32 workspace by TMA reduce-add; a separate kernel applies the epilogue)
+  const int pair_tiles = (a.m_tiles + 1) / 2 * a.n_tiles * a.k_splits;
   const int total = a.full_tiles + (pair_tiles - a.full_tiles) * a.pieces;
   const int kb_total = a.kh * a.kw * a.kb_per_tap;
   const uint32_t tmem_cols = a.tmem_cols;
@@ -251,7 +257,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      PairWork<kSk> work(pair, npairs, total, kb_total);
+      PairWork<kSk> work(pair, npairs, total, kb_total, a.k_splits);
       int w, k0, k1;
       while (ok && work.next(npairs, total, kb_total, w, k0, k1)) {
         const PairCoord pc = pair_coord(a, w, rank);
@@ -288,7 +294,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      PairWork<kSk> work(pair, npairs, total, kb_total);
+      PairWork<kSk> work(pair, npairs, total, kb_total, a.k_splits);
       int w, k0, k1;
       while (ok && work.next(npairs, total, kb_total, w, k0, k1)) {
         const PairCoord pc = pair_coord(a, w, 0);
@@ -341,7 +347,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
     constexpr bool bits_out = kBits;
     float2* next_t = reinterpret_cast<float2*>(stage_out);
     uint32_t* bits_flag = reinterpret_cast<uint32_t*>(stage_out + kOutBytes2);
-    PairWork<kSk> work(pair, npairs, total, kb_total);
+    PairWork<kSk> work(pair, npairs, total, kb_total, a.k_splits);
     int w, k0, k1;
     while (work.next(npairs, total, kb_total, w, k0, k1)) {
       const PairCoord pc = pair_coord(a, w, rank);
@@ -447,19 +453,24 @@ __global__ void __launch_bounds__(kThreads2, 1)
         const int c0 = pc.ntile * a.BN + pc.noff + ch * 32;
         const float4* sb4 = reinterpret_cast<const float4*>(&B->sb[pc.noff + ch * 32]);
         float y[32];
+        if (kSplit) {  // raw partial sums for the workspace (integers below 2^24 add exactly)
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float4 p = sb4[j / 2];
-          const float s0 = acc_value(kKind, v[j]);
-          const float s1 = acc_value(kKind, v[j + 1]);
-          float r0 = has_beta ? fmaf(s0 * p.x, beta, p.y) : fmaf(s0, p.x, p.y);
-          float r1 = has_beta ? fmaf(s1 * p.z, beta, p.w) : fmaf(s1, p.z, p.w);
-          if (a.relu) {
-            r0 = fmaxf(r0, 0.f);
-            r1 = fmaxf(r1, 0.f);
+          for (int j = 0; j < 32; ++j) y[j] = acc_value(kKind, v[j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float4 p = sb4[j / 2];
+            const float s0 = acc_value(kKind, v[j]);
+            const float s1 = acc_value(kKind, v[j + 1]);
+            float r0 = has_beta ? fmaf(s0 * p.x, beta, p.y) : fmaf(s0, p.x, p.y);
+            float r1 = has_beta ? fmaf(s1 * p.z, beta, p.w) : fmaf(s1, p.z, p.w);
+            if (a.relu) {
+              r0 = fmaxf(r0, 0.f);
+              r1 = fmaxf(r1, 0.f);
+            }
+            y[j] = r0;
+            y[j + 1] = r1;
           }
-          y[j] = r0;
-          y[j + 1] = r1;
         }
         if (bits_out) {
           words_set(bits_w, ch, bits_chunk(y, next_t + pc.noff + ch * 32, min(32, a.No - c0), bits_asum));
@@ -472,7 +483,12 @@ __global__ void __launch_bounds__(kThreads2, 1)
         fence_proxy_async();
         epi_barrier();
         if (et == 0) {
-          if (c0 < a.No && !pc.dummy) tma_store_4d(&tmOut, so, c0, pc.ox0, pc.oy0, pc.n0);
+          if (c0 < a.No && !pc.dummy) {
+            if (kSplit)
+              tma_reduce_add_4d(&tmOut, so, c0, pc.ox0, pc.oy0, pc.n0);
+            else
+              tma_store_4d(&tmOut, so, c0, pc.ox0, pc.oy0, pc.n0);
+          }
           bulk_commit();
           bulk_wait_read_1();
         }
@@ -511,10 +527,16 @@ int tc2_smem_bytes(int bn) {
 int tc2_max_pairs(int bn) {
   const int smem = tc2_smem_bytes(bn);
   const void* kerns[] = {
-      reinterpret_cast<const void*>(tc_conv2_kernel<0, false, false>), reinterpret_cast<const void*>(tc_conv2_kernel<1, false, false>),
-      reinterpret_cast<const void*>(tc_conv2_kernel<0, true, false>), reinterpret_cast<const void*>(tc_conv2_kernel<1, true, false>),
-      reinterpret_cast<const void*>(tc_conv2_kernel<0, false, true>), reinterpret_cast<const void*>(tc_conv2_kernel<1, false, true>),
-      reinterpret_cast<const void*>(tc_conv2_kernel<0, true, true>), reinterpret_cast<const void*>(tc_conv2_kernel<1, true, true>)};
+      reinterpret_cast<const void*>(tc_conv2_kernel<0, false, false, false>),
+      reinterpret_cast<const void*>(tc_conv2_kernel<1, false, false, false>),
+      reinterpret_cast<const void*>(tc_conv2_kernel<0, true, false, false>),
+      reinterpret_cast<const void*>(tc_conv2_kernel<1, true, false, false>),
+      reinterpret_cast<const void*>(tc_conv2_kernel<0, false, true, false>),
+      reinterpret_cast<const void*>(tc_conv2_kernel<1, false, true, false>),
+      reinterpret_cast<const void*>(tc_conv2_kernel<0, true, true, false>),
+      reinterpret_cast<const void*>(tc_conv2_kernel<1, true, true, false>),
+      reinterpret_cast<const void*>(tc_conv2_kernel<0, false, false, true>),
+      reinterpret_cast<const void*>(tc_conv2_kernel<1, false, false, true>)};
   bool attr_ok = true;
   for (const void* k : kerns)
     attr_ok = attr_ok && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
@@ -534,7 +556,7 @@ int tc2_max_pairs(int bn) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, tc_conv2_kernel<0, false, false>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, tc_conv2_kernel<0, false, false, false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -542,7 +564,7 @@ int tc2_max_pairs(int bn) {
 }
 
 int tc2_plan(TcArgs& a, int pairs) {
-  const int pair_tiles = (a.m_tiles + 1) / 2 * a.n_tiles;
+  const int pair_tiles = (a.m_tiles + 1) / 2 * a.n_tiles * a.k_splits;
   const int npairs = pairs;
   a.full_tiles = pair_tiles;
   a.pieces = 1;
@@ -554,7 +576,7 @@ int tc2_plan(TcArgs& a, int pairs) {
   // items x k-blocks instead (each share then spans at least one whole item, so an item is
   // cut between two pairs at most).  Measured: 98 items on 74 pairs (waves 66 % full) go from
   // 53.2 to 46.3 us; 196 items (88 % full) run slower split than whole (36.5 -> 49.9 us).
-  if (pair_tiles > grid_pairs && tail > 0) {
+  if (a.k_splits == 1 && pair_tiles > grid_pairs && tail > 0) {
     const int waves = (pair_tiles + grid_pairs - 1) / grid_pairs;
     if (static_cast<double>(pair_tiles) / (static_cast<double>(waves) * grid_pairs) < 0.8) a.sk = 1;
   }
@@ -564,15 +586,18 @@ int tc2_plan(TcArgs& a, int pairs) {
 
 cudaError_t launch_tc_conv2(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmBp,
                             const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s) {
-  const int pair_tiles = (a.m_tiles + 1) / 2 * a.n_tiles;
+  const int pair_tiles = (a.m_tiles + 1) / 2 * a.n_tiles * a.k_splits;
   if (pair_tiles == 0) return cudaSuccess;
   const int smem = tc2_smem_bytes(a.BN);
   const int npairs = a.grid_ctas / 2;
   if (npairs <= 0) return cudaErrorInvalidConfiguration;
-  auto kern = a.sk ? (a.out_bits ? (a.kind ? tc_conv2_kernel<1, true, true> : tc_conv2_kernel<0, true, true>)
-                                 : (a.kind ? tc_conv2_kernel<1, false, true> : tc_conv2_kernel<0, false, true>))
-                   : (a.out_bits ? (a.kind ? tc_conv2_kernel<1, true, false> : tc_conv2_kernel<0, true, false>)
-                                 : (a.kind ? tc_conv2_kernel<1, false, false> : tc_conv2_kernel<0, false, false>));
+  if (a.k_splits > 1 && (a.out_bits || a.sk)) return cudaErrorInvalidValue;
+  auto kern =
+      a.k_splits > 1 ? (a.kind ? tc_conv2_kernel<1, false, false, true> : tc_conv2_kernel<0, false, false, true>)
+      : a.sk ? (a.out_bits ? (a.kind ? tc_conv2_kernel<1, true, true, false> : tc_conv2_kernel<0, true, true, false>)
+                           : (a.kind ? tc_conv2_kernel<1, false, true, false> : tc_conv2_kernel<0, false, true, false>))
+             : (a.out_bits ? (a.kind ? tc_conv2_kernel<1, true, false, false> : tc_conv2_kernel<0, true, false, false>)
+                           : (a.kind ? tc_conv2_kernel<1, false, false, false> : tc_conv2_kernel<0, false, false, false>));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
