@@ -67,7 +67,7 @@ enum { BCONV_FLAG_NONE = 0u, BCONV_FLAG_USE_BETA_SCALING = 1u };
 /* The activation neuron applied last (the closing sentence of the Overview). */
 typedef enum { BCONV_NEURON_NONE = 0, BCONV_NEURON_RELU = 1 } bconv_neuron_t;
 
-/* Kernel family used for the contraction.  AUTO picks the fastest one this build has. */
+/* Kernel family used for the contraction.  AUTO picks the fastest one available for the layer. */
 typedef enum {
   BCONV_ALGO_AUTO = 0,
   BCONV_ALGO_POPC = 1,     /* XNOR/AND: LOP3 XOR/AND + POPC into int32 registers     */
