@@ -329,6 +329,7 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   if (e == cudaSuccess) e = cudaMemcpy(L.wq, hq.data(), hq.size(), cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = L.mem.alloc(&L.codes, static_cast<size_t>(npix) * bpp);
   if (e == cudaSuccess && t.k_splits > 1) e = L.mem.alloc(&L.ws, static_cast<size_t>(L.N) * L.No);
+  if (e == cudaSuccess && t.k_splits > 1) e = cudaMemset(L.ws, 0, sizeof(float) * static_cast<size_t>(L.N) * L.No);
   if (e != cudaSuccess) return from_cuda(e);
 
   bool ok = true;
@@ -550,7 +551,8 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
     e = launch_pack_bf16x3(p, s);
   }
   if (e != cudaSuccess) return from_cuda(e);
-  if (beta && L.fc) {  // the convolution forms beta from A inside its epilogue
+  // the convolution forms beta from A inside its epilogue, a split FC inside the finalize
+  if (beta && L.fc && L.tc.k_splits == 1) {
     BetaArgs b{A, L.beta, L.N, L.H, L.W, L.Ho, L.Wo, L.kh, L.kw, L.sy, L.sx};
     e = launch_beta_image_mean(b, s);
     if (e != cudaSuccess) return from_cuda(e);
@@ -571,8 +573,7 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
     t.a_count = L.a_count;
     om = &L.tmOut;
   } else if (t.k_splits > 1) {
-    e = cudaMemsetAsync(L.ws, 0, sizeof(float) * static_cast<size_t>(L.N) * L.No, s);
-    if (e != cudaSuccess) return from_cuda(e);
+    // the workspace is zero: at allocation, then as each finalize reads it
   } else {
     if (out != L.tm_out_ptr) {
       if (!encode_out_map(L, &L.tmOut, out)) return BCONV_ERR_CUDA;
@@ -586,7 +587,7 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
   if (timed) cudaEventRecord(L.prof.stop[L.prof.used++], s);
   if (e != cudaSuccess) return from_cuda(e);
   if (t.k_splits > 1)
-    e = launch_tc_finalize(L.ws, out, L.scale, L.bias, t.beta, L.N, L.No, L.relu, s);
+    e = launch_tc_finalize(L.ws, out, L.scale, L.bias, beta ? A : nullptr, L.H * L.W, L.N, L.No, L.relu, s);
   return from_cuda(e);
 }
 
@@ -786,6 +787,7 @@ bconv_status_t sync_status(Layer& L, cudaStream_t s) {
     cudaMemset(L.err, 0, sizeof(uint32_t));
     if (L.a_count) cudaMemset(L.a_count, 0, sizeof(uint32_t) * L.tc.m_tiles);  // an aborted launch may leave counts
     if (L.tc.sk_flag) cudaMemset(L.tc.sk_flag, 0, sizeof(uint32_t) * (L.tc.grid_ctas / 2 - 1) * 2);  // and flags
+    if (L.ws) cudaMemset(L.ws, 0, sizeof(float) * static_cast<size_t>(L.N) * L.No);  // and partial sums
     if (word & kErrTimeout) return BCONV_ERR_TIMEOUT;
     return BCONV_ERR_CUDA;  // kErrLayout: a kernel refused an unexpected shared-memory layout
   }
@@ -805,8 +807,8 @@ bconv_status_t set_algo(Layer& L, int algo) {
 }
 
 int launches_per_forward(const Layer& L) {
-  if (L.N > 0 && use_tc(L))  // pack, contraction; the FC adds beta, memset and finalize
-    return 2 + ((L.fc && L.use_beta()) ? 1 : 0) + (L.tc.k_splits > 1 ? 2 : 0);
+  if (L.N > 0 && use_tc(L))  // pack, contraction; a split FC adds the finalize, an unsplit FC with beta its mean
+    return 2 + (L.tc.k_splits > 1 ? 1 : ((L.fc && L.use_beta()) ? 1 : 0));
   int n = 1;  // contraction
   if (L.type != kBinaryWeights || L.use_beta()) n += 1;  // pack
   if (L.use_beta()) n += 1;                              // beta

@@ -143,7 +143,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (!kBits) prefetch_tensor_map(&tmOut);  // a bit-packed output never uses (or encodes) it
   }
   wait_prior_grid();  // the codes, A and the output buffer are the previous kernels' business until here
-  allow_next_grid();
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -363,33 +362,69 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 
   tc_fence_before();
   __syncthreads();
+  // only now may the next kernel's blocks be scheduled: launched at the start they would sit
+  // beside this kernel's CTAs for its whole run, waiting for it, and take issue slots from it
+  allow_next_grid();
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(tmem_cols));
   }
 }
 
-// y = act(S * scale[c] * beta[n] + bias[c]) over the fp32 partial-sum workspace [N][No]; a
-// thread per 4 consecutive channels of one row (No % 4 == 0 on this path).
-__global__ void tc_finalize_kernel(const float4* __restrict__ ws, float4* __restrict__ out,
-                                   const float* __restrict__ scale, const float* __restrict__ bias,
-                                   const float* __restrict__ beta, int rows, int no4, int relu) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= static_cast<int64_t>(rows) * no4) return;
-  const int r = static_cast<int>(i / no4), c = static_cast<int>(i - static_cast<int64_t>(r) * no4) * 4;
-  const float4 s = ws[i];
-  const float4 sc = __ldg(reinterpret_cast<const float4*>(scale + c));
-  const float4 bi = __ldg(reinterpret_cast<const float4*>(bias + c));
-  float4 y;
-  if (beta) {
-    const float b = __ldg(beta + r);
-    y = make_float4(fmaf(s.x * sc.x, b, bi.x), fmaf(s.y * sc.y, b, bi.y), fmaf(s.z * sc.z, b, bi.z),
-                    fmaf(s.w * sc.w, b, bi.w));
-  } else {
-    y = make_float4(fmaf(s.x, sc.x, bi.x), fmaf(s.y, sc.y, bi.y), fmaf(s.z, sc.z, bi.z), fmaf(s.w, sc.w, bi.w));
+// y = act(S * scale[c] * beta[n] + bias[c]) from the fp32 partial-sum workspace [N][No]; a block
+// per 256 x 4 channels of one row n.  With beta, each block first forms beta[n] = sum over the
+// image of A / (H*W) (the FC's window is the whole image; the same reduction as
+// beta_image_mean_kernel, so every block of a row gets the same value).  Every workspace entry
+// is zeroed once read, so the next forward's reduce-add starts from zero.
+constexpr int kFinThreads = 256;
+__global__ void __launch_bounds__(kFinThreads) tc_finalize_kernel(float4* __restrict__ ws, float4* __restrict__ out,
+                                                                 const float* __restrict__ scale,
+                                                                 const float* __restrict__ bias,
+                                                                 const float* __restrict__ A, int hw, int no4,
+                                                                 int relu) {
+  wait_prior_grid();
+  allow_next_grid();
+  __shared__ float part[kFinThreads / 32];
+  __shared__ float beta_s;
+  const int chunks = (no4 + kFinThreads - 1) / kFinThreads;
+  const int r = blockIdx.x / chunks, i0 = (blockIdx.x - r * chunks) * kFinThreads;
+  float b = 1.f;
+  if (A) {
+    const float* Ar = A + static_cast<int64_t>(r) * hw;
+    float acc = 0.f;
+    for (int p = threadIdx.x; p < hw; p += kFinThreads) acc += __ldg(Ar + p);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      acc = threadIdx.x < kFinThreads / 32 ? part[threadIdx.x] : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (threadIdx.x == 0) beta_s = acc / static_cast<float>(hw);
+    }
+    __syncthreads();
+    b = beta_s;
   }
-  if (relu) y = make_float4(fmaxf(y.x, 0.f), fmaxf(y.y, 0.f), fmaxf(y.z, 0.f), fmaxf(y.w, 0.f));
-  out[i] = y;
+  const int i = i0 + threadIdx.x;
+  if (i < no4) {
+    const int64_t k = static_cast<int64_t>(r) * no4 + i;
+    const float4 sv = ws[k];
+    ws[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int c = i * 4;
+    const float4 sc = __ldg(reinterpret_cast<const float4*>(scale + c));
+    const float4 bi = __ldg(reinterpret_cast<const float4*>(bias + c));
+    float4 y;
+    if (A) {
+      y = make_float4(fmaf(sv.x * sc.x, b, bi.x), fmaf(sv.y * sc.y, b, bi.y), fmaf(sv.z * sc.z, b, bi.z),
+                      fmaf(sv.w * sc.w, b, bi.w));
+    } else {
+      y = make_float4(fmaf(sv.x, sc.x, bi.x), fmaf(sv.y, sc.y, bi.y), fmaf(sv.z, sc.z, bi.z),
+                      fmaf(sv.w, sc.w, bi.w));
+    }
+    if (relu) y = make_float4(fmaxf(y.x, 0.f), fmaxf(y.y, 0.f), fmaxf(y.z, 0.f), fmaxf(y.w, 0.f));
+    out[k] = y;
+  }
 }
 
 }  // namespace
@@ -433,13 +468,12 @@ cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmB, const
   return launch_overlapped(kern, dim3(grid), dim3(kThreadsTc), smem, s, *tmA, *tmB, *tmBp, *tmOut, a);
 }
 
-cudaError_t launch_tc_finalize(const float* ws, float* out, const float* scale, const float* bias, const float* beta,
+cudaError_t launch_tc_finalize(float* ws, float* out, const float* scale, const float* bias, const float* A, int hw,
                                int rows, int no, int relu, cudaStream_t s) {
-  const int64_t total4 = static_cast<int64_t>(rows) * (no / 4);
-  if (total4 == 0) return cudaSuccess;
-  tc_finalize_kernel<<<static_cast<unsigned>(ceil_div(total4, 256)), 256, 0, s>>>(
-      reinterpret_cast<const float4*>(ws), reinterpret_cast<float4*>(out), scale, bias, beta, rows, no / 4, relu);
-  return cudaGetLastError();
+  if (rows == 0 || no == 0) return cudaSuccess;
+  const int chunks = (no / 4 + kFinThreads - 1) / kFinThreads;
+  return launch_overlapped(tc_finalize_kernel, dim3(rows * chunks), dim3(kFinThreads), 0, s, reinterpret_cast<float4*>(ws),
+                           reinterpret_cast<float4*>(out), scale, bias, A, hw, no / 4, relu);
 }
 
 }  // namespace bconv

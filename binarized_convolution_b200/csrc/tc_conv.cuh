@@ -75,8 +75,10 @@ int tc2_plan(TcArgs& a, int pairs);  // pairs = clusters that can be resident at
 int tc2_max_pairs(int bn);           // co-resident two-CTA clusters on the current device (0: none)
 cudaError_t launch_tc_conv2(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmBp,
                             const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s);
-// ws and out are 16-byte aligned, no % 4 == 0 (the tensor-core path's condition).
-cudaError_t launch_tc_finalize(const float* ws, float* out, const float* scale, const float* bias, const float* beta,
+// The epilogue of a split reduction: y from the fp32 workspace [rows][no] (zeroed as it is
+// read), with beta = mean of A [rows][hw] over each image when A is given.  ws and out are
+// 16-byte aligned, no % 4 == 0 (the tensor-core path's condition).
+cudaError_t launch_tc_finalize(float* ws, float* out, const float* scale, const float* bias, const float* A, int hw,
                                int rows, int no, int relu, cudaStream_t s);
 
 // int8 operand codes: XNOR -> bin(x~) in {-1,+1}, AND -> {0,1}; channels in [ni, cip) are 0.

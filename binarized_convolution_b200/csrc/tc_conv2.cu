@@ -249,7 +249,6 @@ __global__ void __launch_bounds__(kThreads2, 1)
     if (!kBits) prefetch_tensor_map(&tmOut);  // a bit-packed output never uses (or encodes) it
   }
   wait_prior_grid();  // the codes, A and the output buffer are the previous kernels' business until here
-  allow_next_grid();
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
@@ -511,6 +510,9 @@ __global__ void __launch_bounds__(kThreads2, 1)
 
   tc_fence_before();
   __syncthreads();
+  // only now may the next kernel's blocks be scheduled: launched at the start they would sit
+  // beside this kernel's CTAs for its whole run, waiting for it, and take issue slots from it
+  allow_next_grid();
   cluster_sync();  // the peer is done with this CTA's barriers and shared memory
   if (warp == 1) {
     tc_fence_after();

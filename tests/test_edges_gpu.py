@@ -155,3 +155,31 @@ def test_reduction_split_between_sm_pairs(op, ni, cuda_device):
     layer.sync_status()
     layer.close()
     assert torch.equal(y1, y2)
+
+
+def test_fc_split_reduction_repeated(cuda_device):
+    """The FC's split reduction adds partial sums into a workspace that its last kernel zeroes
+    as it reads it: consecutive forwards on different inputs must each match the oracle."""
+    import torch
+
+    w = synth.small_case(batch=130, h=7, w=7, ni=256, no=64, kind="fc", op=synth.XNOR, use_beta=True, relu=True,
+                         in_terms=True, seed=18)
+    inp = synth.make_inputs(w)
+    layer = pu.make_layer(w, inp)
+    sums = pu.make_layer(w, inp, sums=True)
+    try:
+        for seed in (18, 19, 20):
+            x = synth.make_batch(w, seed)
+            cur = synth.Inputs(x, inp.wbits, inp.scale, inp.bias, inp.in_scale, inp.in_bias)
+            xt = torch.from_numpy(x).cuda()
+            y = layer(xt).reshape(-1, w.out_channels).cpu().numpy()
+            S = sums(xt).reshape(-1, w.out_channels).cpu().numpy()
+            S_ref, beta_ref, y_ref = pu.run_oracle(w, cur)
+            S_sum, _, _ = pu.run_oracle(w, cur, sums=True)
+            pu.assert_sums_exact(S, S_sum)
+            pu.assert_outputs_close(w, cur, y, S_ref, beta_ref, y_ref)
+        layer.sync_status()
+        sums.sync_status()
+    finally:
+        layer.close()
+        sums.close()
