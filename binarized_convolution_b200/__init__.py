@@ -33,6 +33,7 @@ from ._native import (  # noqa: F401
     bconv_forward_host,
     bconv_forward_noalloc,
     bconv_forward_io,
+    bconv_check_wait_timeout,
     bconv_set_output_terms,
     bconv_io_t,
     bfc_forward_io,

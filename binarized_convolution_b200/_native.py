@@ -88,6 +88,7 @@ _SIGS = {
     "bconv_measure_peak": (_I32, [_I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
     "bconv_forward_noalloc": (_I32, [ctypes.POINTER(bconv_desc_t), _I32, ctypes.c_uint32] + [_P] * 8),
     "bconv_set_output_terms": (_I32, [_P, _P, _P]),
+    "bconv_check_wait_timeout": (_I32, [ctypes.c_double]),
     "bconv_forward_io": (_I32, [_P, ctypes.POINTER(bconv_io_t), _P]),
     "bfc_set_output_terms": (_I32, [_P, _P, _P]),
     "bfc_forward_io": (_I32, [_P, ctypes.POINTER(bconv_io_t), _P]),
@@ -332,6 +333,11 @@ def bconv_pack_bits(bits) -> np.ndarray:
 
 def bconv_version() -> int:
     return load_library().bconv_version()
+
+
+def bconv_check_wait_timeout(limit_ms: float = 20.0) -> int:
+    """Status of the bounded-wait check (BCONV_ERR_TIMEOUT = 5 is the expected outcome)."""
+    return int(load_library().bconv_check_wait_timeout(float(limit_ms)))
 
 
 def bconv_measure_peak(kind: int):

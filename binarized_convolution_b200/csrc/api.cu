@@ -1135,6 +1135,19 @@ bconv_status_t bconv_pack_bits(const uint8_t* bits, int64_t rows, int32_t nbits,
 
 int32_t bconv_version(void) { return 100; }
 
+bconv_status_t bconv_check_wait_timeout(double limit_ms) {
+  if (!(limit_ms > 0.0) || limit_ms > 1000.0) return BCONV_ERR_INVALID_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+    cudaGetLastError();
+    return BCONV_ERR_NO_DEVICE;
+  }
+  uint32_t word = 0;
+  const cudaError_t e = wait_check(limit_ms, &word);
+  if (e != cudaSuccess) return from_cuda(e);
+  return (word & kErrTimeout) ? BCONV_ERR_TIMEOUT : BCONV_OK;
+}
+
 bconv_status_t bconv_measure_peak(int32_t kind, double* ops_per_s, double* sm_mhz) {
   if (kind < 0 || kind > 6 || !ops_per_s) return BCONV_ERR_INVALID_ARG;
   int ndev = 0;

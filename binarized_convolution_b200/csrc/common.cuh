@@ -134,5 +134,8 @@ constexpr int kTileN = 128;     // output channels per CTA tile (both contractio
 // Peak probes.
 // ------------------------------------------------------------------------------------
 cudaError_t probe_peak(int kind, double* ops_per_s, double* sm_mhz);
+// Runs the kernels' bounded mbarrier wait on a barrier nothing completes, with the given limit;
+// *status receives the error word it left (kErrTimeout expected).
+cudaError_t wait_check(double limit_ms, uint32_t* status);
 
 }  // namespace bconv

@@ -183,7 +183,37 @@ __global__ void __launch_bounds__(128, 1) tcgen05_probe(int iters, uint32_t* out
   }
 }
 
+// The bounded-wait path of the tensor-core kernels, on its own: one thread waits (with the
+// kernels' wait routine) on an mbarrier that nothing arrives on, gives up after `limit_ns`,
+// records kErrTimeout in the error word and returns -- the device stays usable.
+__global__ void wait_check_kernel(uint32_t* err, unsigned long long limit_ns) {
+  using namespace tcdev;
+  __shared__ struct {
+    uint64_t bar;
+    uint32_t abort_flag;
+  } B;
+  if (threadIdx.x != 0) return;
+  mbar_init(&B.bar, 1);
+  B.abort_flag = 0;
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  mbar_wait(&B.bar, 0, &B, err, true, false, limit_ns);
+}
+
 }  // namespace
+
+cudaError_t wait_check(double limit_ms, uint32_t* status) {
+  uint32_t* err = nullptr;
+  cudaError_t e = cudaMalloc(&err, sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMemset(err, 0, sizeof(uint32_t));
+  if (e == cudaSuccess) {
+    wait_check_kernel<<<1, 32>>>(err, static_cast<unsigned long long>(limit_ms * 1e6));
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(status, err, sizeof(uint32_t), cudaMemcpyDeviceToHost);
+  if (err) cudaFree(err);
+  return e;
+}
 
 cudaError_t probe_peak(int kind, double* ops_per_s, double* sm_mhz) {
   if (kind == 3 || kind == 4 || kind == 5 || kind == 6) {

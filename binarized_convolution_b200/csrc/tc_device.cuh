@@ -61,13 +61,14 @@ __device__ __forceinline__ bool mbar_try_suspend(uint64_t* bar, uint32_t parity,
 // waits (the epilogue's wait for an accumulator, the final drain) suspend between checks.
 template <class Bars>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Bars* B, uint32_t* err,
-                                          bool follow_abort = true, bool idle = false) {
+                                          bool follow_abort = true, bool idle = false,
+                                          uint64_t limit_ns = kTimeoutNs) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (idle ? mbar_try_suspend(bar, parity, 20000u) : mbar_try(bar, parity)) return true;
     if (follow_abort && *reinterpret_cast<volatile uint32_t*>(&B->abort_flag)) return false;
-    if (globaltimer() - t0 > kTimeoutNs) {
+    if (globaltimer() - t0 > limit_ns) {
       atomicOr(err, kErrTimeout);
       atomicExch(&B->abort_flag, 1u);
       return false;

@@ -297,6 +297,15 @@ int32_t bconv_version(void);
  */
 bconv_status_t bconv_measure_peak(int32_t kind, double* ops_per_s, double* sm_mhz);
 
+/*
+ * Check of the failure path every tensor-core kernel relies on (no counterpart on the pages):
+ * a kernel waits, with the kernels' own bounded-wait routine, on an mbarrier that nothing
+ * completes; after limit_ms (0 < limit_ms <= 1000) it gives up and records a timeout, and the
+ * device stays usable.  Returns TIMEOUT when the wait ended as designed, OK if it did not
+ * (which would mean the barrier completed), INVALID_ARG, NO_DEVICE or CUDA.
+ */
+bconv_status_t bconv_check_wait_timeout(double limit_ms);
+
 /* ------------------------------------------------------------------------------------
  * Forward without any allocation.  (The pages have no counterpart to this entry point; it
  * exists for callers of this library that cannot allocate device memory when they run a

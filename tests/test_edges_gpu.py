@@ -183,3 +183,11 @@ def test_fc_split_reduction_repeated(cuda_device):
     finally:
         layer.close()
         sums.close()
+
+
+def test_bounded_wait_gives_up_and_device_stays_usable(cuda_device):
+    """The kernels' mbarrier waits are bounded: a wait on a barrier that nothing completes ends
+    with a timeout status (not a hang), and the device keeps working afterwards."""
+    assert bc.bconv_check_wait_timeout(20.0) == 5  # BCONV_ERR_TIMEOUT
+    w = synth.small_case(batch=1, h=6, w=6, ni=64, no=32, k=3, op=synth.XNOR, seed=19)
+    _check(w)
