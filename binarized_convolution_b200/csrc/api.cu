@@ -13,6 +13,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <memory>
 #include <mutex>
 #include <new>
 #include <vector>
@@ -144,6 +145,15 @@ struct Layer {
   float* y_scratch = nullptr;
   // host-buffer forward staging (allocated on first use)
   float *stage_in = nullptr, *stage_out = nullptr;
+  // The host-buffer forward runs the batch as image chunks, so that one chunk's copy in, the
+  // previous chunk's compute and the one before's copy out overlap: the creation parameters
+  // (kept on the host), one layer per chunk (made on first use), two copy streams and events.
+  std::vector<uint32_t> h_packed;
+  std::vector<float> h_scale, h_bias, h_in_scale, h_in_bias;
+  float h_scale_value = 1.f;
+  std::vector<std::unique_ptr<struct Layer>> chunks;
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;
+  std::vector<cudaEvent_t> chunk_events;
   DevMem mem;
   Profile prof;
 
@@ -480,6 +490,20 @@ bconv_status_t alloc_workspace(Layer& L) {
   return from_cuda(e);
 }
 
+// Keep what creating the layer took, for the chunk layers of the host-buffer forward.
+void keep_host_params(Layer& L, const uint32_t* packed, const float* scale, const float* bias,
+                      const float* in_scale, const float* in_bias, float scale_value) {
+  const int64_t taps = L.fc ? 1 : static_cast<int64_t>(L.kh) * L.kw;
+  const int64_t words = L.fc ? static_cast<int64_t>(L.No) * L.H * L.W * words_for(L.Ni)
+                             : static_cast<int64_t>(L.No) * taps * words_for(L.Ni);
+  L.h_packed.assign(packed, packed + words);
+  if (scale) L.h_scale.assign(scale, scale + L.No);
+  if (bias) L.h_bias.assign(bias, bias + L.No);
+  if (in_scale) L.h_in_scale.assign(in_scale, in_scale + L.Ni);
+  if (in_bias) L.h_in_bias.assign(in_bias, in_bias + L.Ni);
+  L.h_scale_value = scale_value;
+}
+
 bconv_status_t finish_create(Layer& L, const uint32_t* packed, const float* scale, const float* bias,
                              const float* in_scale, const float* in_bias, float scale_value) {
   int ndev = 0;
@@ -762,12 +786,87 @@ bconv_status_t forward_io(Layer& L, const bconv_io_t* io, cudaStream_t s) {
   return run_io(L, v, s);
 }
 
+// The chunk layers: the same layer on batch N / k (k = 4, or 2, when it divides N and the
+// copies are large enough to be worth overlapping); their errors go to the parent's word.
+int host_chunks(const Layer& L) {
+  const int64_t bytes = (L.in_elems() + L.out_elems()) * static_cast<int64_t>(sizeof(float));
+  if (L.h_packed.empty() || bytes < (int64_t{8} << 20)) return 1;
+  for (int k : {4, 2})
+    if (L.N % k == 0) return k;
+  return 1;
+}
+
+bconv_status_t make_chunks(Layer& L, int k) {
+  L.chunks.clear();
+  for (int i = 0; i < k; ++i) {
+    std::unique_ptr<Layer> c(new (std::nothrow) Layer());
+    if (!c) return BCONV_ERR_OOM;
+    c->type = L.type;
+    c->flags = L.flags;
+    c->relu = L.relu;
+    c->fc = L.fc;
+    c->N = L.N / k; c->H = L.H; c->W = L.W; c->Ni = L.Ni; c->No = L.No;
+    c->kh = L.kh; c->kw = L.kw; c->sy = L.sy; c->sx = L.sx; c->Ho = L.Ho; c->Wo = L.Wo;
+    auto opt = [](const std::vector<float>& v) { return v.empty() ? nullptr : v.data(); };
+    const bconv_status_t st = finish_create(*c, L.h_packed.data(), opt(L.h_scale), opt(L.h_bias), opt(L.h_in_scale),
+                                            opt(L.h_in_bias), L.h_scale_value);
+    if (st != BCONV_OK) {
+      L.chunks.clear();
+      return st;
+    }
+    c->err = L.err;  // one error word for the layer
+    c->tc.err = L.err;
+    L.chunks.push_back(std::move(c));
+  }
+  cudaError_t e = cudaSuccess;
+  if (!L.copy_in) e = cudaStreamCreateWithFlags(&L.copy_in, cudaStreamNonBlocking);
+  if (e == cudaSuccess && !L.copy_out) e = cudaStreamCreateWithFlags(&L.copy_out, cudaStreamNonBlocking);
+  while (e == cudaSuccess && L.chunk_events.size() < static_cast<size_t>(2 * k + 1)) {
+    cudaEvent_t ev;
+    e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+    if (e == cudaSuccess) L.chunk_events.push_back(ev);
+  }
+  return from_cuda(e);
+}
+
 bconv_status_t forward_host(Layer& L, const float* hin, float* hout, cudaStream_t s) {
   if (!hin || !hout) return BCONV_ERR_INVALID_ARG;
   cudaError_t e = cudaSuccess;
   if (!L.stage_in) e = L.mem.alloc(&L.stage_in, L.in_elems());
   if (e == cudaSuccess && !L.stage_out) e = L.mem.alloc(&L.stage_out, L.out_elems());
   if (e != cudaSuccess) return from_cuda(e);
+  const int k = host_chunks(L);
+  if (k > 1 && L.chunks.size() != static_cast<size_t>(k) && make_chunks(L, k) != BCONV_OK) L.chunks.clear();
+  if (k > 1 && L.chunks.size() == static_cast<size_t>(k)) {
+    // copy in on one stream, compute on `stream`, copy out on another, chunk by chunk
+    const int64_t in_c = L.in_elems() / k, out_c = L.out_elems() / k;
+    cudaEvent_t start = L.chunk_events[2 * k];
+    e = cudaEventRecord(start, s);  // the staging buffers are free once earlier work on `stream` is done
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(L.copy_in, start, 0);
+    for (int i = 0; i < k && e == cudaSuccess; ++i) {
+      Layer& c = *L.chunks[i];
+      c.algo = L.algo;
+      e = cudaMemcpyAsync(L.stage_in + i * in_c, hin + i * in_c, in_c * sizeof(float), cudaMemcpyHostToDevice,
+                          L.copy_in);
+      if (e == cudaSuccess) e = cudaEventRecord(L.chunk_events[2 * i], L.copy_in);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s, L.chunk_events[2 * i], 0);
+      if (e != cudaSuccess) break;
+      const bconv_status_t st = run_forward(c, L.stage_in + i * in_c, L.stage_out + i * out_c, s);
+      if (st != BCONV_OK) {
+        cudaStreamSynchronize(L.copy_in);
+        cudaStreamSynchronize(L.copy_out);
+        return st;
+      }
+      e = cudaEventRecord(L.chunk_events[2 * i + 1], s);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(L.copy_out, L.chunk_events[2 * i + 1], 0);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(hout + i * out_c, L.stage_out + i * out_c, out_c * sizeof(float), cudaMemcpyDeviceToHost,
+                            L.copy_out);
+    }
+    const cudaError_t e1 = cudaStreamSynchronize(L.copy_out);
+    const cudaError_t e2 = cudaStreamSynchronize(s);
+    return from_cuda(e != cudaSuccess ? e : (e1 != cudaSuccess ? e1 : e2));
+  }
   e = cudaMemcpyAsync(L.stage_in, hin, L.in_elems() * sizeof(float), cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return from_cuda(e);
   bconv_status_t st = run_forward(L, L.stage_in, L.stage_out, s);
@@ -863,6 +962,13 @@ bconv_status_t profile_end(Layer& L, float* total_ms, int32_t* launches) {
 void destroy(Layer& L) {
   DeviceGuard g(L.device);
   L.prof.clear();
+  for (auto& c : L.chunks) c->mem.release();
+  L.chunks.clear();
+  for (cudaEvent_t ev : L.chunk_events) cudaEventDestroy(ev);
+  L.chunk_events.clear();
+  if (L.copy_in) cudaStreamDestroy(L.copy_in);
+  if (L.copy_out) cudaStreamDestroy(L.copy_out);
+  L.copy_in = L.copy_out = nullptr;
   L.mem.release();
 }
 
@@ -905,6 +1011,7 @@ bconv_status_t bconv_create(const bconv_desc_t* d, const uint32_t* packed_weight
   L.Ho = (L.H + L.sy - 1) / L.sy;
   L.Wo = (L.W + L.sx - 1) / L.sx;
   const bconv_status_t st = finish_create(L, packed_weights, scale, bias, in_scale, in_bias, d->scale_value);
+  if (st == BCONV_OK) keep_host_params(L, packed_weights, scale, bias, in_scale, in_bias, d->scale_value);
   if (st != BCONV_OK) {
     h->magic = 0;
     delete h;
@@ -1026,6 +1133,7 @@ bconv_status_t bfc_create(const bfc_desc_t* d, const uint32_t* packed_weights, c
   L.Ho = 1;
   L.Wo = 1;
   const bconv_status_t st = finish_create(L, packed_weights, scale, bias, in_scale, in_bias, d->scale_value);
+  if (st == BCONV_OK) keep_host_params(L, packed_weights, scale, bias, in_scale, in_bias, d->scale_value);
   if (st != BCONV_OK) {
     h->magic = 0;
     delete h;

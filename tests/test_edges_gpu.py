@@ -191,3 +191,25 @@ def test_bounded_wait_gives_up_and_device_stays_usable(cuda_device):
     assert bc.bconv_check_wait_timeout(20.0) == 5  # BCONV_ERR_TIMEOUT
     w = synth.small_case(batch=1, h=6, w=6, ni=64, no=32, k=3, op=synth.XNOR, seed=19)
     _check(w)
+
+
+@pytest.mark.parametrize("op", [synth.XNOR, synth.BINARY_WEIGHTS])
+def test_forward_host_in_chunks_matches_device(op, cuda_device):
+    """A batch large enough for the host-buffer forward to run as image chunks (copies and
+    compute overlapped on three streams) gives the device forward's result bit for bit."""
+    import torch
+
+    w = synth.small_case(batch=8, h=64, w=64, ni=64, no=64, k=3, op=op, use_beta=True, relu=True, in_terms=True,
+                         seed=21)
+    inp = synth.make_inputs(w)
+    y_dev = pu.run_device(w, inp)
+    layer = pu.make_layer(w, inp)
+    try:
+        hin = torch.from_numpy(inp.x).pin_memory()
+        hout = torch.empty(layer.out_dims, dtype=torch.float32).pin_memory()
+        for _ in range(2):  # the first call creates the chunk layers
+            bc.bconv_forward_host(layer.handle, hin.data_ptr(), hout.data_ptr(), 0)
+            np.testing.assert_array_equal(hout.numpy().reshape(y_dev.shape), y_dev)
+        layer.sync_status()
+    finally:
+        layer.close()
