@@ -94,3 +94,36 @@ def test_workload_full_size(idx, algo, cuda_device):
         assert np.all((S_dev - nbits) % 2 == 0)
     else:
         assert np.all(S_dev >= 0) and np.all(S_dev <= nbits)
+
+
+LARGE = [
+    # wide reductions: 4096 input channels x 9 taps = 36864 terms per output (|S| < 2^24,
+    # so the fp32 reduce-add and epilogue stay exact for the integer part)
+    synth.small_case(batch=2, h=9, w=10, ni=4096, no=64, k=3, op=synth.XNOR, use_beta=True, relu=True,
+                     in_terms=True, seed=31),
+    # many output channels: 1024 -> four 256-channel tiles per pixel
+    synth.small_case(batch=1, h=12, w=12, ni=128, no=1024, k=3, op=synth.AND, use_beta=True, seed=32),
+    # a large window: 11 x 11 taps on a 20 x 20 image
+    synth.small_case(batch=2, h=20, w=20, ni=96, no=32, k=11, op=synth.XNOR, use_beta=True, seed=33),
+    # a long FC reduction: 14 x 14 x 1024 = 200704 terms per output, split over many SMs
+    synth.small_case(batch=160, h=14, w=14, ni=1024, no=64, kind="fc", op=synth.XNOR, use_beta=True, seed=34),
+    # binaryWeights with a wide reduction (fp32 sums of 9 x 2048 terms)
+    synth.small_case(batch=1, h=8, w=8, ni=2048, no=32, k=3, op=synth.BINARY_WEIGHTS, use_beta=True, in_terms=True,
+                     seed=35),
+]
+
+
+@pytest.mark.parametrize("algo", ["auto", "alt"])
+@pytest.mark.parametrize("w", LARGE, ids=lambda w: w.name)
+def test_large_reductions_and_tiles(w, algo, cuda_device):
+    """Sizes at the large end of what the kernels plan for, on sampled outputs."""
+    a = pu.algo_for(w, algo)
+    inp = synth.make_inputs(w)
+    rows = pu.sample_rows(w, seed=w.seed, ops_budget=2e8)
+    y = pu.run_device(w, inp, algo=a)
+    S_ref, beta_ref, y_ref = pu.run_oracle(w, inp, rows=rows)
+    pu.assert_outputs_close(w, inp, y[rows], S_ref, beta_ref, y_ref, rows=rows)
+    if w.op != synth.BINARY_WEIGHTS:
+        S_dev = pu.run_device(w, inp, sums=True, algo=a)
+        S_sum, _, _ = pu.run_oracle(w, inp, rows=rows, sums=True)
+        pu.assert_sums_exact(S_dev[rows], S_sum)
