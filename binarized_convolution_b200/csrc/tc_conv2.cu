@@ -405,9 +405,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
       } else if (valid && a.beta) {
         beta = __ldg(a.beta + (static_cast<int64_t>(n) * a.Ho + oy) * a.Wo + ox);
       }
-      if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err, true, true))) break;
-      tc_fence_after();
       const uint32_t* part = nullptr;
+      uint32_t pnext[32];  // the other pair's sums for the next chunk, loaded a chunk ahead
       if (owner) {  // wait (bounded) for the partial sums of this item's remaining k-blocks
         bool ready = true;
         if (et == 0) {
@@ -425,7 +424,11 @@ __global__ void __launch_bounds__(kThreads2, 1)
         if (!epi_all(ready)) break;
         __threadfence();
         part = a.sk_part + static_cast<size_t>(pair * 2 + static_cast<int>(rank)) * a.BN * 128;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) pnext[j] = __ldcg(part + j * 128 + row);  // while the MMAs finish
       }
+      if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err, true, true))) break;
+      tc_fence_after();
       float bits_asum = 0.f;
       Words8 bits_w{};
       const int64_t pix = (static_cast<int64_t>(n) * a.Ho + oy) * a.Wo + ox;
@@ -438,12 +441,17 @@ __global__ void __launch_bounds__(kThreads2, 1)
           if (lane == 0) mbar_arrive_remote(acc == 0 ? empty_leader0 : empty_leader1);
         }
         if (part) {  // + the other pair's sums: int32 exactly, fp32 in this fixed order
+          uint32_t o[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const uint32_t o = __ldcg(part + (ch * 32 + j) * 128 + row);
-            v[j] = kKind == 1 ? __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(o))
-                              : static_cast<uint32_t>(static_cast<int32_t>(v[j]) + static_cast<int32_t>(o));
+          for (int j = 0; j < 32; ++j) o[j] = pnext[j];
+          if (ch + 1 < pc.bn / 32) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) pnext[j] = __ldcg(part + ((ch + 1) * 32 + j) * 128 + row);
           }
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            v[j] = kKind == 1 ? __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(o[j]))
+                              : static_cast<uint32_t>(static_cast<int32_t>(v[j]) + static_cast<int32_t>(o[j]));
         }
         const int buf = chunk_count & 1;
         ++chunk_count;
