@@ -279,6 +279,7 @@ def run_native(args, w: synth.Workload):
     dist_init("nccl")
 
     inp = synth.make_inputs(w, seed=replica_seed(w.seed, rank))
+    bc.bconv_set_cta_mode({"auto": bc.CTA_AUTO, "single": bc.CTA_SINGLE, "pair": bc.CTA_PAIR}[args.cta])
     layer_kw = dict(op=w.op, scale=inp.scale, bias=inp.bias, in_scale=inp.in_scale, in_bias=inp.in_bias,
                     use_beta=w.use_beta, relu=w.relu)
     if w.kind == "fc":
@@ -380,6 +381,9 @@ def run_native(args, w: synth.Workload):
             "traffic": traffic, "kernel": kname, "kernel_ms": kern_ms_max,
             "kernel_launches_timed": kern_n, "timed_every": PROFILE_EVERY,
             "peak_source": how if bound == "tensor" else f"derived: {how}"}
+    if kname == "tc_conv":
+        roof["spread"] = {bc.CTA_SINGLE: "one SM per tile", bc.CTA_PAIR: "SM pairs (cta_group::2)"}.get(
+            layer.cta_mode(), "?")
     sm_mhz = clock_info.get("sm_mhz")
     if sm_mhz and bound == "alu":
         p_obs, _, _ = derived_peak(w, sms, sm_mhz, kname)
@@ -507,6 +511,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--algo", choices=["auto", "popc", "tcgen05", "simt_f32"], default="auto",
                     help="kernel family of the contraction (auto = the library's choice)")
+    ap.add_argument("--cta", choices=["auto", "single", "pair"], default="auto",
+                    help="tensor-core contraction on one SM per tile or on SM pairs (auto = the library's choice)")
     ap.add_argument("--io", choices=["f32", "bits"], default="f32",
                     help="bits: time a middle layer of a chain (bit-packed input and output)")
     ap.add_argument("--no-e2e", action="store_true")

@@ -17,6 +17,9 @@ from ._native import (  # noqa: F401
     ALGO_POPC,
     ALGO_SIMT_F32,
     ALGO_TCGEN05,
+    CTA_AUTO,
+    CTA_PAIR,
+    CTA_SINGLE,
     FLAG_NONE,
     FLAG_USE_BETA_SCALING,
     NEURON_NONE,
@@ -26,6 +29,8 @@ from ._native import (  # noqa: F401
     TYPE_XNOR,
     BconvError,
     bconv_create,
+    bconv_cta_mode,
+    bconv_set_cta_mode,
     bconv_desc_t,
     bconv_destroy,
     bconv_effective_algo,
@@ -53,6 +58,7 @@ from ._native import (  # noqa: F401
     bconv_sync_status,
     bconv_version,
     bfc_create,
+    bfc_cta_mode,
     bfc_desc_t,
     bfc_destroy,
     bfc_effective_algo,

@@ -24,6 +24,7 @@ TYPE_BINARY_WEIGHTS, TYPE_XNOR, TYPE_AND = 0, 1, 2
 FLAG_NONE, FLAG_USE_BETA_SCALING = 0, 1
 NEURON_NONE, NEURON_RELU = 0, 1
 ALGO_AUTO, ALGO_POPC, ALGO_SIMT_F32, ALGO_TCGEN05 = 0, 1, 2, 3
+CTA_AUTO, CTA_SINGLE, CTA_PAIR = 0, 1, 2
 
 _STATUS = {0: "BCONV_OK", 1: "BCONV_ERR_INVALID_ARG", 2: "BCONV_ERR_UNSUPPORTED", 3: "BCONV_ERR_CUDA",
            4: "BCONV_ERR_OOM", 5: "BCONV_ERR_TIMEOUT", 6: "BCONV_ERR_NO_DEVICE"}
@@ -92,6 +93,9 @@ _SIGS = {
     "bconv_forward_io": (_I32, [_P, ctypes.POINTER(bconv_io_t), _P]),
     "bfc_set_output_terms": (_I32, [_P, _P, _P]),
     "bfc_forward_io": (_I32, [_P, ctypes.POINTER(bconv_io_t), _P]),
+    "bconv_set_cta_mode": (_I32, [_I32]),
+    "bconv_cta_mode": (_I32, [_P]),
+    "bfc_cta_mode": (_I32, [_P]),
 }
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -266,6 +270,19 @@ def bconv_effective_algo(h) -> int:
 
 def bfc_effective_algo(h) -> int:
     return load_library().bfc_effective_algo(h)
+
+
+def bconv_set_cta_mode(mode: int):
+    """Spread of the tensor-core contraction for layers created from now on (CTA_*)."""
+    _check(load_library().bconv_set_cta_mode(int(mode)), "bconv_set_cta_mode")
+
+
+def bconv_cta_mode(h) -> int:
+    return load_library().bconv_cta_mode(h)
+
+
+def bfc_cta_mode(h) -> int:
+    return load_library().bfc_cta_mode(h)
 
 
 def bconv_sync_status(h, stream: int = 0):

@@ -13,6 +13,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <memory>
 #include <mutex>
 #include <new>
@@ -127,7 +128,7 @@ struct Layer {
   uint32_t* err = nullptr;
   // tensor-core path: int8 codes [N][H][W][cip], int8 weights [no_tc][taps*cip], tensor maps
   bool tc_ok = false;
-  bool tc_pair = false;  // convolution on SM pairs (cta_group::2); the FC uses single SMs
+  bool tc_pair = false;  // contraction on SM pairs (cta_group::2), else one SM per tile
   int cip = 0;
   int8_t* codes = nullptr;
   int8_t* wq = nullptr;
@@ -244,6 +245,28 @@ bool encode_out_map(Layer& L, CUtensorMap* m, const float* out) {
 // bf16 parts of x~ (kind 1), for No % 4 == 0 (16-byte output rows for the TMA store) and
 // strided windows whose TMA box (stride x tile extent) stays within 256 elements.
 // Sets up its buffers, weights and maps.
+// Kernel family for layers created from now on (BCONV_CTA_*).
+std::atomic<int> g_cta_mode{BCONV_CTA_AUTO};
+
+// k-block stages on the busiest SM under each family's plan (the plans' own work lists).
+double plan_stages_single(TcArgs t, int sms) {
+  const int kb = t.kh * t.kw * t.kb_per_tap;
+  const int tiles = t.m_tiles * t.n_tiles;
+  const int grid = tc_plan(t, sms);
+  if (grid <= 0) return 0.0;
+  if (t.pieces > 1) return (static_cast<double>(t.full_tiles / grid) + 1.0 / t.pieces) * kb;
+  return static_cast<double>((tiles + grid - 1) / grid) * kb;
+}
+
+double plan_stages_pair(TcArgs t, int pairs) {
+  const int kb = t.kh * t.kw * t.kb_per_tap;
+  const int grid_pairs = tc2_plan(t, pairs) / 2;
+  if (grid_pairs <= 0) return 0.0;
+  const int64_t items = t.full_tiles;
+  if (t.sk) return static_cast<double>((items * kb + grid_pairs - 1) / grid_pairs);
+  return static_cast<double>((items + grid_pairs - 1) / grid_pairs) * kb;
+}
+
 bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   if (L.No % 4 != 0 || L.N == 0) return BCONV_OK;
   if (!tensor_map_encoder()) return BCONV_OK;
@@ -257,7 +280,9 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   // tile, so the weight matrix streams from memory once, with half of every weight tile per
   // SM); otherwise a single SM keeps up to 256 images in one tile (two 128-row sub-tiles
   // sharing every weight stage).
-  const bool fc_pair = L.fc && L.N > 128 && tc2_max_pairs(std::min(256, round_up(L.No, 32))) > 0;
+  const int mode = g_cta_mode.load();
+  const bool fc_pair =
+      L.fc && L.N > 128 && mode != BCONV_CTA_SINGLE && tc2_max_pairs(std::min(256, round_up(L.No, 32))) > 0;
   t.mt = (L.fc && L.N > 128 && !fc_pair) ? 2 : 1;
   t.BN = std::min(t.mt == 2 ? 128 : 256, round_up(L.No, 32));
   t.n_tiles = (L.No + t.BN - 1) / t.BN;
@@ -315,6 +340,22 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
     }
   }
 
+  // Kernel family.  The FC follows fc_pair.  A convolution runs on SM pairs only when their
+  // plan is clearly shorter: at equal k-block stages per SM the one-SM kernel measured faster
+  // (batch 16, 56 x 56, 256 -> 256, 3 x 3: 54 stages per SM either way, 44.2 us per forward on
+  // single SMs against 48.3 us on pairs), while the pairs' balanced split wins where whole
+  // tiles leave a ragged last wave (batch 8, 112 x 112, 128 -> 128, stride 2, binaryWeights:
+  // 61.9 us on pairs against 69.3 us).
+  int pairs = 0;
+  if (L.fc) {
+    pairs = fc_pair ? tc2_max_pairs(t.BN) : 0;
+  } else if (mode != BCONV_CTA_SINGLE) {
+    pairs = tc2_max_pairs(t.BN);
+    if (pairs > 0 && mode == BCONV_CTA_AUTO &&
+        !(plan_stages_pair(t, pairs) < 0.95 * plan_stages_single(t, current_sm_count())))
+      pairs = 0;
+  }
+
   // Weights [no_tc][taps][bpp bytes]: kind 0 int8 +-1 (XNOR) or 0/1 (AND); kind 1 bf16 +-1
   // repeated for the three parts.  Every padding slot is 0.
   const int no_tc = t.n_tiles * t.BN;
@@ -334,6 +375,20 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
           for (int part = 0; part < 3; ++part) memcpy(row + 2 * (part * L.cip + f), &v, 2);
         }
       }
+  if (pairs == 0) {
+    // the one-SM kernel copies each (N tile, k-block) stage of BN rows x 128 bytes as one
+    // block: lay the blocks out contiguously with the 128-byte swizzle already applied
+    const int kbt = static_cast<int>(kt / 128);
+    std::vector<int8_t> tiles(hq.size());
+    for (int nt = 0; nt < t.n_tiles; ++nt)
+      for (int kb = 0; kb < kbt; ++kb)
+        for (int r = 0; r < t.BN; ++r) {
+          const int8_t* src = hq.data() + static_cast<size_t>(nt * t.BN + r) * kt + static_cast<int64_t>(kb) * 128;
+          int8_t* dst = tiles.data() + (static_cast<size_t>(nt) * kbt + kb) * t.BN * 128 + static_cast<size_t>(r) * 128;
+          for (int c = 0; c < 8; ++c) memcpy(dst + 16 * (c ^ (r & 7)), src + 16 * c, 16);
+        }
+    hq.swap(tiles);
+  }
   const int64_t npix = static_cast<int64_t>(L.N) * L.H * L.W;
   cudaError_t e = L.mem.alloc(&L.wq, hq.size());
   if (e == cudaSuccess) e = cudaMemcpy(L.wq, hq.data(), hq.size(), cudaMemcpyHostToDevice);
@@ -361,11 +416,7 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
     const uint32_t estr[4] = {1, static_cast<uint32_t>(t.sx), static_cast<uint32_t>(t.sy), 1};
     ok = encode_4d(&L.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.codes, dims, strides, box, estr);
   }
-  ok = ok && encode_2d(&L.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(kt),
-                       static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128, static_cast<uint32_t>(t.BN));
-  // Convolutions run on SM pairs when two-CTA clusters fit; each CTA then loads half of
-  // every weight tile (boxes of BN/2 rows).
-  const int pairs = (L.fc && !fc_pair) ? 0 : tc2_max_pairs(t.BN);
+  // On SM pairs each CTA loads half of every weight tile (boxes of BN/2 rows).
   if (pairs > 0) {
     L.tc_pair = true;
     tc2_plan(t, pairs);
@@ -384,9 +435,7 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
                          static_cast<uint32_t>(t.BN / t.pieces / 2));
   } else {
     t.grid_ctas = tc_plan(t, current_sm_count());  // work list: tail tiles cut along N
-    ok = ok && encode_2d(&L.tmBp, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(kt),
-                         static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128,
-                         static_cast<uint32_t>(t.BN / t.pieces));
+    t.b_tiles = L.wq;
   }
   if (ok && t.k_splits > 1) ok = encode_out_map(L, &L.tmWs, L.ws);
   if (!ok) return BCONV_OK;  // the POPC path stays available
@@ -607,7 +656,7 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
   }
   const bool timed = L.prof.take();
   if (timed) cudaEventRecord(L.prof.start[L.prof.used], s);
-  e = L.tc_pair ? launch_tc_conv2(&L.tmA, &L.tmB, &L.tmBp, om, t, s) : launch_tc_conv(&L.tmA, &L.tmB, &L.tmBp, om, t, s);
+  e = L.tc_pair ? launch_tc_conv2(&L.tmA, &L.tmB, &L.tmBp, om, t, s) : launch_tc_conv(&L.tmA, om, t, s);
   if (timed) cudaEventRecord(L.prof.stop[L.prof.used++], s);
   if (e != cudaSuccess) return from_cuda(e);
   if (t.k_splits > 1)
@@ -1242,6 +1291,22 @@ bconv_status_t bconv_pack_bits(const uint8_t* bits, int64_t rows, int32_t nbits,
 }
 
 int32_t bconv_version(void) { return 100; }
+
+bconv_status_t bconv_set_cta_mode(bconv_cta_mode_t mode) {
+  if (mode != BCONV_CTA_AUTO && mode != BCONV_CTA_SINGLE && mode != BCONV_CTA_PAIR) return BCONV_ERR_INVALID_ARG;
+  bconv::g_cta_mode.store(mode);
+  return BCONV_OK;
+}
+
+int32_t bconv_cta_mode(bconv_handle_t h) {
+  if (!checked(h, kConvMagic)) return -1;
+  return h->L.tc_ok ? (h->L.tc_pair ? BCONV_CTA_PAIR : BCONV_CTA_SINGLE) : 0;
+}
+
+int32_t bfc_cta_mode(bfc_handle_t h) {
+  if (!checked(h, kFcMagic)) return -1;
+  return h->L.tc_ok ? (h->L.tc_pair ? BCONV_CTA_PAIR : BCONV_CTA_SINGLE) : 0;
+}
 
 bconv_status_t bconv_check_wait_timeout(double limit_ms) {
   if (!(limit_ms > 0.0) || limit_ms > 1000.0) return BCONV_ERR_INVALID_ARG;

@@ -90,8 +90,7 @@ __device__ __forceinline__ TileCoord tile_coord(const TcArgs& a, int w) {
 
 template <bool kSplit, int kKind, bool kBits>
 __global__ void __launch_bounds__(kThreadsTc, 1)
-    tc_conv_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmBp, const __grid_constant__ CUtensorMap tmOut,
+    tc_conv_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmOut,
                    const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The swizzled tiles need a 1024-byte aligned base, which the dynamic shared window has
@@ -138,8 +137,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const uint32_t tmem_base = B->tmem_base;
   if (threadIdx.x == 0) {
     prefetch_tensor_map(&tmA);
-    prefetch_tensor_map(&tmB);
-    prefetch_tensor_map(&tmBp);
     if (!kBits) prefetch_tensor_map(&tmOut);  // a bit-packed output never uses (or encodes) it
   }
   wait_prior_grid();  // the codes, A and the output buffer are the previous kernels' business until here
@@ -167,10 +164,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           for (int h = 0; h < a.mt; ++h)
             tma_load_4d(sa + h * kABytes, &tmA, &B->full[stage], cb * 128, tc.ox0 * a.sx + kx - a.kw / 2,
                         tc.oy0 * a.sy + ky - a.kh / 2, tc.n0 + h * a.Bn);
-          if (tc.bn == a.BN)
-            tma_load_2d(sb, &tmB, &B->full[stage], kb * 128, tc.ntile * a.BN);
-          else
-            tma_load_2d(sb, &tmBp, &B->full[stage], kb * 128, tc.ntile * a.BN + tc.noff);
+          // the weight stage is one contiguous, already swizzled block of bn rows
+          bulk_load(sb, a.b_tiles + ((static_cast<int64_t>(tc.ntile) * kb_total + kb) * a.BN + tc.noff) * 128,
+                    static_cast<uint32_t>(tc.bn * 128), &B->full[stage]);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
@@ -452,20 +448,19 @@ int tc_plan(TcArgs& a, int sm_count) {
   return grid;
 }
 
-cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmBp,
-                           const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s) {
+cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s) {
   const int smem = tc_smem_bytes(a.BN, a.mt);
   const int tiles = a.m_tiles * a.n_tiles * a.k_splits;
   if (tiles == 0) return cudaSuccess;
   int grid = current_sm_count();
   if (grid > tiles) grid = tiles;
-  if (a.out_bits && a.k_splits > 1) return cudaErrorInvalidValue;
+  if ((a.out_bits && a.k_splits > 1) || !a.b_tiles) return cudaErrorInvalidValue;
   auto kern = a.k_splits > 1 ? (a.kind ? tc_conv_kernel<true, 1, false> : tc_conv_kernel<true, 0, false>)
               : a.out_bits   ? (a.kind ? tc_conv_kernel<false, 1, true> : tc_conv_kernel<false, 0, true>)
                              : (a.kind ? tc_conv_kernel<false, 1, false> : tc_conv_kernel<false, 0, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  return launch_overlapped(kern, dim3(grid), dim3(kThreadsTc), smem, s, *tmA, *tmB, *tmBp, *tmOut, a);
+  return launch_overlapped(kern, dim3(grid), dim3(kThreadsTc), smem, s, *tmA, *tmOut, a);
 }
 
 cudaError_t launch_tc_finalize(float* ws, float* out, const float* scale, const float* bias, const float* A, int hw,

@@ -59,12 +59,16 @@ struct TcArgs {
   int sk;
   uint32_t* sk_part;        // [pairs - 1][2][BN / 32][32][128] accumulator words
   uint32_t* sk_flag;        // [pairs - 1][2], zero between launches
+  // Weights for the one-SM kernel: [n_tiles][kh * kw * kb_per_tap][BN][128] bytes, one
+  // contiguous block per (N tile, k-block) already in the shared-memory order of the 128-byte
+  // swizzle (16-byte chunk c of row r stored at chunk c ^ (r % 8)), so that each stage is one
+  // bulk copy.  The pair kernel reads row-major weights through tensor maps instead.
+  const int8_t* b_tiles;
 };
 
 int tc_smem_bytes(int bn, int mt);
-// tmBp: the weight map with a box of BN / pieces rows (used for tail pieces).
-cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmBp,
-                           const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s);
+// One CTA per tile; weights from a.b_tiles.
+cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s);
 // Grid size and tail split for a launch on `sm_count` SMs (fills full_tiles / pieces).
 int tc_plan(TcArgs& a, int sm_count);
 

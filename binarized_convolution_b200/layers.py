@@ -132,6 +132,9 @@ class BinaryConv2d(_Layer):
     def effective_algo(self) -> int:
         return nat.bconv_effective_algo(self.handle)
 
+    def cta_mode(self) -> int:
+        return nat.bconv_cta_mode(self.handle)
+
     def forward_into(self, x, out):
         import torch
 
@@ -197,6 +200,9 @@ class BinaryFC(_Layer):
 
     def effective_algo(self) -> int:
         return nat.bfc_effective_algo(self.handle)
+
+    def cta_mode(self) -> int:
+        return nat.bfc_cta_mode(self.handle)
 
     def forward_into(self, x, out):
         import torch

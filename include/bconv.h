@@ -201,6 +201,26 @@ int32_t bconv_launches_per_forward(bconv_handle_t h);
 int32_t bconv_effective_algo(bconv_handle_t h);
 
 /*
+ * How the tensor-core contraction spreads over the SMs, for layers created after the call
+ * (process-wide; a layer keeps what it was created with, and its weights are laid out for it).
+ *   SINGLE  one CTA per 128-pixel tile on one SM; each weight stage is one bulk copy.
+ *   PAIR    a cluster of two CTAs per 256-pixel tile (tcgen05 cta_group::2), each CTA
+ *           loading half of every weight stage; an FC needs batch > 128 for it.
+ *   AUTO    PAIR for an FC with batch > 128; PAIR for a convolution when the busiest SM of
+ *           the pair plan runs under 95 % of the k-block stages of the busiest SM of the
+ *           one-SM plan (e.g. where the pairs' balanced split evens out a ragged last wave);
+ *           otherwise SINGLE.
+ * A forced family that the layer or device cannot use falls back to the other one.
+ * Returns INVALID_ARG for an unknown mode.
+ */
+typedef enum { BCONV_CTA_AUTO = 0, BCONV_CTA_SINGLE = 1, BCONV_CTA_PAIR = 2 } bconv_cta_mode_t;
+bconv_status_t bconv_set_cta_mode(bconv_cta_mode_t mode);
+
+/* The spread a layer's tensor-core contraction runs with (BCONV_CTA_SINGLE or BCONV_CTA_PAIR);
+ * 0 when the layer has no tensor-core path, -1 for a bad handle. */
+int32_t bconv_cta_mode(bconv_handle_t h);
+
+/*
  * Wait for `stream`, then read and clear the handle's device error word.  Returns OK,
  * TIMEOUT (a kernel gave up a bounded wait), or CUDA (a pending CUDA error).
  */
@@ -263,6 +283,7 @@ int32_t bfc_output_feature_channels(bfc_handle_t h);
 bconv_status_t bfc_set_algo(bfc_handle_t h, bconv_algo_t algo);
 int32_t bfc_launches_per_forward(bfc_handle_t h);
 int32_t bfc_effective_algo(bfc_handle_t h);
+int32_t bfc_cta_mode(bfc_handle_t h);
 bconv_status_t bfc_sync_status(bfc_handle_t h, struct CUstream_st* stream);
 bconv_status_t bfc_profile_begin(bfc_handle_t h, int32_t max_launches);
 bconv_status_t bfc_profile_end(bfc_handle_t h, float* total_ms, int32_t* launches);

@@ -32,3 +32,13 @@ def pytest_sessionstart(session):
     import oracle
 
     oracle.build()
+
+
+@pytest.fixture(autouse=True)
+def _default_cta_mode():
+    """Tests may force the tensor-core spread of the layers they create; put it back."""
+    yield
+    from binarized_convolution_b200 import _native
+
+    if _native._lib is not None:
+        _native.bconv_set_cta_mode(_native.CTA_AUTO)

@@ -43,15 +43,23 @@ def make_layer(w: synth.Workload, inp: synth.Inputs, *, sums: bool = False):
                         (w.stride_y, w.stride_x), wbits=inp.wbits, **kw)
 
 
+# Kernel families a parity case runs on: the library's choice, the SIMT family, and the
+# tensor cores with the contraction forced onto one SM per tile or onto SM pairs.
+FAMILIES = ["auto", "alt", "single", "pair"]
+
+
 def algo_for(w: synth.Workload, name: str):
     """Library algorithm code for a test parameter: 'auto' (the library's choice: the tensor
-    cores where they apply) or 'alt' (the SIMT family: POPC for XNOR/AND, the FP32 signed-add
-    kernel for binaryWeights)."""
+    cores where they apply), 'alt' (the SIMT family: POPC for XNOR/AND, the FP32 signed-add
+    kernel for binaryWeights), or 'single' / 'pair' (the library's choice, with the
+    tensor-core contraction of the layers created after this call forced onto one SM per
+    tile or onto SM pairs; the test fixture puts the process-wide setting back to AUTO)."""
     import binarized_convolution_b200 as bc
 
-    if name == "auto":
-        return bc.ALGO_AUTO
-    return bc.ALGO_SIMT_F32 if w.op == synth.BINARY_WEIGHTS else bc.ALGO_POPC
+    bc.bconv_set_cta_mode({"single": bc.CTA_SINGLE, "pair": bc.CTA_PAIR}.get(name, bc.CTA_AUTO))
+    if name == "alt":
+        return bc.ALGO_SIMT_F32 if w.op == synth.BINARY_WEIGHTS else bc.ALGO_POPC
+    return bc.ALGO_AUTO
 
 
 def run_device(w: synth.Workload, inp: synth.Inputs, *, sums: bool = False, algo=None):

@@ -116,6 +116,16 @@ def test_calls_on_null_or_foreign_handles_return_errors():
     assert lib.bconv_forward(ctypes.cast(junk, ctypes.c_void_p), None, None, None) == 1
     assert lib.bconv_destroy(ctypes.cast(junk, ctypes.c_void_p)) == 1
     assert lib.bconv_pack_bits(None, 1, 1, None) == 1
+    assert lib.bconv_cta_mode(None) == -1
+    assert lib.bfc_cta_mode(None) == -1
+
+
+def test_cta_mode_setting_is_validated():
+    lib = bc.load_library()
+    for bad in (-1, 3, 100):
+        assert lib.bconv_set_cta_mode(bad) == 1  # INVALID_ARG
+    for good in (bc.CTA_SINGLE, bc.CTA_PAIR, bc.CTA_AUTO):
+        assert lib.bconv_set_cta_mode(good) == 0
 
 
 def test_create_without_a_device_reports_no_device():

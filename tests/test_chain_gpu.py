@@ -97,7 +97,7 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("algo", ["auto", "alt"])
+@pytest.mark.parametrize("algo", pu.FAMILIES)
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
 def test_bits_out(w, algo, cuda_device):
     inp = synth.make_inputs(w)
@@ -129,7 +129,7 @@ def _bits_input(w, inp, rows=None):
     return _pack(bits), A.astype(np.float32)
 
 
-@pytest.mark.parametrize("algo", ["auto", "alt"])
+@pytest.mark.parametrize("algo", pu.FAMILIES)
 @pytest.mark.parametrize("w", [c for c in CASES if c.op != synth.BINARY_WEIGHTS] + [
     synth.small_case(batch=2, h=6, w=7, ni=31, no=8, k=5, op=synth.XNOR, use_beta=True, in_terms=True, seed=57),
     synth.small_case(batch=1, h=9, w=9, ni=200, no=12, k=3, stride=2, op=synth.AND, use_beta=True, seed=58),
@@ -147,10 +147,11 @@ def test_bits_in(w, algo, cuda_device):
     bare = replace(inp, in_scale=None, in_bias=None)  # the consumer has no input terms
     xb = torch.from_numpy(words.view(np.int32)).cuda()
     xa = torch.from_numpy(A).cuda()
+    a = pu.algo_for(w, algo)
     for sums in (True, False):
         layer = pu.make_layer(w, bare, sums=sums)
         try:
-            layer.set_algo(pu.algo_for(w, algo))
+            layer.set_algo(a)
             y = layer.forward_from_bits(xb, xa if (w.use_beta and not sums) else None)
             layer.sync_status()
             y = y.reshape(-1, w.out_channels).cpu().numpy()
@@ -255,7 +256,7 @@ FC_CASES = [
 ]
 
 
-@pytest.mark.parametrize("algo", ["auto", "alt"])
+@pytest.mark.parametrize("algo", pu.FAMILIES)
 @pytest.mark.parametrize("w", FC_CASES + [synth.small_case(batch=3, h=2, w=2, ni=24, no=40, kind="fc",
                                                            op=synth.BINARY_WEIGHTS, use_beta=True, in_terms=True,
                                                            seed=84)], ids=lambda w: w.name)
@@ -265,7 +266,7 @@ def test_fc_bits_out(w, algo, cuda_device):
     _check_bits_out(w, inp, ns, nb, pu.algo_for(w, algo))
 
 
-@pytest.mark.parametrize("algo", ["auto", "alt"])
+@pytest.mark.parametrize("algo", pu.FAMILIES)
 @pytest.mark.parametrize("w", FC_CASES, ids=lambda w: w.name)
 def test_fc_bits_in(w, algo, cuda_device):
     """The FC reads a convolution's bit-packed output ([N][H][W][words] and A [N][H][W])."""
@@ -276,10 +277,11 @@ def test_fc_bits_in(w, algo, cuda_device):
     bare = replace(inp, in_scale=None, in_bias=None)
     xb = torch.from_numpy(words.view(np.int32)).cuda()
     xa = torch.from_numpy(A).cuda()
+    a = pu.algo_for(w, algo)
     for sums in (True, False):
         layer = pu.make_layer(w, bare, sums=sums)
         try:
-            layer.set_algo(pu.algo_for(w, algo))
+            layer.set_algo(a)
             y = layer.forward_from_bits(xb, xa if (w.use_beta and not sums) else None)
             layer.sync_status()
             y = y.reshape(-1, w.out_channels).cpu().numpy()

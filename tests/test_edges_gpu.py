@@ -19,13 +19,14 @@ def _check(w, inp=None):
     inp = inp if inp is not None else synth.make_inputs(w)
     S_ref, beta_ref, y_ref = pu.run_oracle(w, inp)
     S_sum, _, _ = pu.run_oracle(w, inp, sums=True)
-    for name in ("auto", "alt"):
+    for name in pu.FAMILIES:
         a = pu.algo_for(w, name)
         y = pu.run_device(w, inp, algo=a)
         pu.assert_outputs_close(w, inp, y, S_ref, beta_ref, y_ref)
         if w.op != synth.BINARY_WEIGHTS:
             S_dev = pu.run_device(w, inp, sums=True, algo=a)
             pu.assert_sums_exact(S_dev, S_sum)
+    bc.bconv_set_cta_mode(bc.CTA_AUTO)
 
 
 SWEEP = []
@@ -213,3 +214,38 @@ def test_forward_host_in_chunks_matches_device(op, cuda_device):
         layer.sync_status()
     finally:
         layer.close()
+
+
+def _spread(w, mode=None):
+    """The tensor-core spread a layer of this shape is created with."""
+    inp = synth.make_inputs(w)
+    if mode is not None:
+        bc.bconv_set_cta_mode(mode)
+    try:
+        layer = pu.make_layer(w, inp)
+    finally:
+        bc.bconv_set_cta_mode(bc.CTA_AUTO)
+    try:
+        return layer.cta_mode()
+    finally:
+        layer.close()
+
+
+def test_spread_choice(cuda_device):
+    """AUTO: one SM per tile where the pair plan is not clearly shorter (equal waves), SM
+    pairs where their balanced split evens out a ragged last wave and for the FC with batch
+    > 128; forced modes are kept where the layer allows them."""
+    assert _spread(synth.workload("xnor_beta_n16_56x56_c256_k256_3x3")) == bc.CTA_SINGLE
+    assert _spread(synth.workload("and_n32_28x28_c512_k512_3x3")) == bc.CTA_SINGLE
+    assert _spread(synth.workload("binw_n8_112x112_c128_k128_3x3_s2")) == bc.CTA_PAIR
+    assert _spread(synth.workload("fc_xnor_beta_n256_7x7x512_k4096")) == bc.CTA_PAIR
+    small = synth.small_case(batch=1, h=8, w=8, ni=64, no=32, k=3, op=synth.XNOR, seed=22)
+    assert _spread(small) == bc.CTA_SINGLE
+    assert _spread(small, bc.CTA_PAIR) == bc.CTA_PAIR
+    fc = synth.small_case(batch=200, h=2, w=2, ni=64, no=64, kind="fc", op=synth.AND, seed=23)
+    assert _spread(fc) == bc.CTA_PAIR
+    assert _spread(fc, bc.CTA_SINGLE) == bc.CTA_SINGLE
+    fc_small = synth.small_case(batch=100, h=2, w=2, ni=64, no=64, kind="fc", op=synth.AND, seed=24)
+    assert _spread(fc_small, bc.CTA_PAIR) == bc.CTA_SINGLE  # the FC's pair tile needs batch > 128
+    odd = synth.small_case(batch=1, h=5, w=5, ni=64, no=6, k=3, op=synth.XNOR, seed=25)
+    assert _spread(odd) == 0  # out_channels % 4 != 0: no tensor-core path

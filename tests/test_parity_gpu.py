@@ -43,7 +43,7 @@ MEDIUM = [
 ]
 
 
-@pytest.mark.parametrize("algo", ["auto", "alt"])
+@pytest.mark.parametrize("algo", pu.FAMILIES)
 @pytest.mark.parametrize("w", MEDIUM, ids=lambda w: w.name)
 def test_medium_all_outputs(w, algo, cuda_device):
     a = pu.algo_for(w, algo)
@@ -61,7 +61,7 @@ def test_medium_all_outputs(w, algo, cuda_device):
         pu.assert_sums_exact(S_dev, S_sum)
 
 
-@pytest.mark.parametrize("algo", ["auto", "alt"])
+@pytest.mark.parametrize("algo", pu.FAMILIES)
 @pytest.mark.parametrize("idx", range(5), ids=lambda i: synth.WORKLOAD_ORDER[i])
 def test_workload_full_size(idx, algo, cuda_device):
     w = synth.workload(idx)
@@ -113,7 +113,7 @@ LARGE = [
 ]
 
 
-@pytest.mark.parametrize("algo", ["auto", "alt"])
+@pytest.mark.parametrize("algo", pu.FAMILIES)
 @pytest.mark.parametrize("w", LARGE, ids=lambda w: w.name)
 def test_large_reductions_and_tiles(w, algo, cuda_device):
     """Sizes at the large end of what the kernels plan for, on sampled outputs."""
