@@ -125,11 +125,13 @@ bconv_status_t bconv_forward(bconv_handle_t h, const float* in, float* out, stru
 /*
  * Same as bconv_forward with HOST buffers: copies host_in to the device, runs the layer
  * and copies the result into host_out, then waits for all of it.  Batches of 8 MB or more
- * run as 2 or 4 image chunks: a chunk's copy in (on an internal stream), its compute (on
+ * (input plus output) run as 4 (else 2) image chunks where that divides the batch and keeps
+ * 2 MB or more per chunk: a chunk's copy in (on an internal stream), its compute (on
  * `stream`, after the work already queued there) and its copy out (on a second internal
  * stream) overlap with the neighbouring chunks'.  Use page-locked host memory for full copy
  * bandwidth.  The first call on a handle allocates the device staging buffers and the chunk
- * layers (about the layer's own working memory again) and keeps them until bconv_destroy.
+ * layers (about the layer's own working memory again, plus one more copy of its device
+ * weights, which all chunks share) and keeps them until bconv_destroy.
  */
 bconv_status_t bconv_forward_host(bconv_handle_t h, const float* host_in, float* host_out,
                                   struct CUstream_st* stream);

@@ -194,22 +194,50 @@ def test_bounded_wait_gives_up_and_device_stays_usable(cuda_device):
     _check(w)
 
 
+@pytest.mark.parametrize("family", pu.FAMILIES)
 @pytest.mark.parametrize("op", [synth.XNOR, synth.BINARY_WEIGHTS])
-def test_forward_host_in_chunks_matches_device(op, cuda_device):
+def test_forward_host_in_chunks_matches_device(op, family, cuda_device):
     """A batch large enough for the host-buffer forward to run as image chunks (copies and
-    compute overlapped on three streams) gives the device forward's result bit for bit."""
+    compute overlapped on three streams; four two-image chunks that share the first chunk's
+    weights) gives the device forward's result bit for bit, on every kernel family."""
     import torch
 
     w = synth.small_case(batch=8, h=64, w=64, ni=64, no=64, k=3, op=op, use_beta=True, relu=True, in_terms=True,
                          seed=21)
     inp = synth.make_inputs(w)
-    y_dev = pu.run_device(w, inp)
+    a = pu.algo_for(w, family)
+    y_dev = pu.run_device(w, inp, algo=a)
     layer = pu.make_layer(w, inp)
     try:
+        layer.set_algo(a)
         hin = torch.from_numpy(inp.x).pin_memory()
         hout = torch.empty(layer.out_dims, dtype=torch.float32).pin_memory()
         for _ in range(2):  # the first call creates the chunk layers
             bc.bconv_forward_host(layer.handle, hin.data_ptr(), hout.data_ptr(), 0)
+            np.testing.assert_array_equal(hout.numpy().reshape(y_dev.shape), y_dev)
+        layer.sync_status()
+    finally:
+        layer.close()
+
+
+def test_fc_forward_host_in_chunks_matches_device(cuda_device):
+    """The FC's host-buffer forward in image chunks (each chunk a split-reduction FC of its
+    own, all reading the first chunk's weights) against the device forward."""
+    import torch
+
+    # 128 images of 7 x 7 x 512: four chunks of 32 images
+    w = synth.small_case(batch=128, h=7, w=7, ni=512, no=512, kind="fc", op=synth.XNOR, use_beta=True, relu=True,
+                         in_terms=True, seed=26)
+    inp = synth.make_inputs(w)
+    y_dev = pu.run_device(w, inp)
+    S_ref, beta_ref, y_ref = pu.run_oracle(w, inp)
+    pu.assert_outputs_close(w, inp, y_dev, S_ref, beta_ref, y_ref)
+    layer = pu.make_layer(w, inp)
+    try:
+        hin = torch.from_numpy(inp.x).pin_memory()
+        hout = torch.empty(layer.out_dims, dtype=torch.float32).pin_memory()
+        for _ in range(2):  # exact integer sums and the same beta: equal bit for bit
+            bc.bfc_forward_host(layer.handle, hin.data_ptr(), hout.data_ptr(), 0)
             np.testing.assert_array_equal(hout.numpy().reshape(y_dev.shape), y_dev)
         layer.sync_status()
     finally:
