@@ -276,17 +276,23 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   const int taps = L.kh * L.kw;
   TcArgs& t = L.tc;
   t.kind = L.type == kBinaryWeights ? 1 : 0;
-  // channels per part, padded to whole 128-byte rows; bytes of operand per pixel
+  // channels per part, padded to whole 128-byte rows; bytes of activation operand per pixel
+  // (kind 1: three bf16 parts) and of weights per output channel and tap (kind 1: one bf16
+  // copy, which every part is multiplied with)
   L.cip = t.kind == 0 ? round_up(L.Ni, 128) : round_up(L.Ni, 64);
   const int bpp = t.kind == 0 ? L.cip : 6 * L.cip;
+  const int bpb = t.kind == 0 ? L.cip : 2 * L.cip;
+  t.kb_px = bpb / 128;
+  t.px_bytes = bpp;
+  t.part_bytes = t.kind == 0 ? 0 : 2 * L.cip;
   // The FC runs on SM pairs when its batch fills both CTAs of a pair (256 images per pair
   // tile, so the weight matrix streams from memory once, with half of every weight tile per
   // SM); otherwise a single SM keeps up to 256 images in one tile (two 128-row sub-tiles
   // sharing every weight stage).
   const int mode = g_cta_mode.load();
   const bool fc_pair =
-      L.fc && L.N > 128 && mode != BCONV_CTA_SINGLE && tc2_max_pairs(std::min(256, round_up(L.No, 32))) > 0;
-  t.mt = (L.fc && L.N > 128 && !fc_pair) ? 2 : 1;
+      L.fc && L.N > 128 && mode != BCONV_CTA_SINGLE && tc2_max_pairs(t.kind, std::min(256, round_up(L.No, 32))) > 0;
+  t.mt = (L.fc && L.N > 128 && !fc_pair && t.kind == 0) ? 2 : 1;
   t.BN = std::min(t.mt == 2 ? 128 : 256, round_up(L.No, 32));
   t.n_tiles = (L.No + t.BN - 1) / t.BN;
   t.No = L.No;
@@ -298,12 +304,12 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   t.bias = L.bias;
   if (L.fc) {
     t.Ho = 1; t.Wo = 1; t.kh = 1; t.kw = 1; t.sy = 1; t.sx = 1;
-    t.kb_per_tap = L.H * L.W * bpp / 128;
+    t.kb_per_tap = L.H * L.W * bpb / 128;
     t.R = 1; t.Cw = 1; t.Bn = 128;
     t.tiles_x = 1; t.tiles_y = 1;
   } else {
     t.Ho = L.Ho; t.Wo = L.Wo; t.kh = L.kh; t.kw = L.kw; t.sy = L.sy; t.sx = L.sx;
-    t.kb_per_tap = bpp / 128;
+    t.kb_per_tap = bpb / 128;
     // 128 output pixels per tile as Bn images x R rows x Cw columns (powers of two, so that
     // every 32-row quarter is a box too): the shape with the fewest tiles, i.e. the least
     // MMA work on pixels past the image edges (56 x 56 -> 8 x 8 x 2 images: none), then
@@ -331,7 +337,7 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   const int kb_total = t.kh * t.kw * t.kb_per_tap;
   t.k_splits = 1;
   if (L.fc) {  // spread the reduction so that the tiles fill the GPU (or its SM pairs)
-    const int workers = fc_pair ? tc2_max_pairs(t.BN) : current_sm_count();
+    const int workers = fc_pair ? tc2_max_pairs(t.kind, t.BN) : current_sm_count();
     const int64_t tiles = static_cast<int64_t>(fc_pair ? (t.m_tiles + 1) / 2 : t.m_tiles) * t.n_tiles;
     int64_t best = -1;
     for (int sp = 1; sp <= 16 && kb_total / sp >= 4; ++sp) {
@@ -344,25 +350,31 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   }
 
   // Kernel family.  The FC follows fc_pair.  A convolution runs on SM pairs only when their
-  // plan is clearly shorter: at equal k-block stages per SM the one-SM kernel measured faster
-  // (batch 16, 56 x 56, 256 -> 256, 3 x 3: 54 stages per SM either way, 44.2 us per forward on
-  // single SMs against 48.3 us on pairs), while the pairs' balanced split wins where whole
-  // tiles leave a ragged last wave (batch 8, 112 x 112, 128 -> 128, stride 2, binaryWeights:
-  // 61.9 us on pairs against 69.3 us).
+  // plan needs clearly fewer k-block stages on the busiest SM: under 95 % of the one-SM plan's
+  // for int8 codes, under 80 % for binaryWeights, whose stages cost the pairs relatively more
+  // (each CTA still loads all three 16 KB activation parts per stage, and the balanced split
+  // adds its exchange).  Measured on B200: batch 16, 56 x 56, 256 -> 256, 3 x 3 (54 stages per
+  // SM either way) 44.2 us per forward on single SMs against 48.3 us on pairs; batch 8,
+  // 112 x 112, 128 -> 128, stride 2, binaryWeights (27 stages on single SMs with the tail cut
+  // in halves, 24 on pairs with the balanced split) 46.9 us against 53.7 us.
+  const double pair_factor = t.kind == 1 ? 0.80 : 0.95;
   int pairs = 0;
   if (L.fc) {
-    pairs = fc_pair ? tc2_max_pairs(t.BN) : 0;
+    pairs = fc_pair ? tc2_max_pairs(t.kind, t.BN) : 0;
   } else if (mode != BCONV_CTA_SINGLE) {
-    pairs = tc2_max_pairs(t.BN);
+    pairs = tc2_max_pairs(t.kind, t.BN);
     if (pairs > 0 && mode == BCONV_CTA_AUTO &&
-        !(plan_stages_pair(t, pairs) < 0.95 * plan_stages_single(t, current_sm_count())))
+        !(plan_stages_pair(t, pairs) < pair_factor * plan_stages_single(t, current_sm_count())))
       pairs = 0;
   }
 
-  // Weights [no_tc][taps][bpp bytes]: kind 0 int8 +-1 (XNOR) or 0/1 (AND); kind 1 bf16 +-1
-  // repeated for the three parts.  Every padding slot is 0.
+  t.stages = pairs > 0 ? tc2_stages(t.kind, t.BN) : tc_stages(t.kind, t.BN, t.mt);
+  if (t.stages < 2) return BCONV_OK;  // no room for a pipeline: the SIMT family stays
+
+  // Weights [no_tc][taps][bpb bytes]: kind 0 int8 +-1 (XNOR) or 0/1 (AND); kind 1 bf16 +-1.
+  // Every padding slot is 0.
   const int no_tc = t.n_tiles * t.BN;
-  const int64_t kt = static_cast<int64_t>(taps) * bpp;
+  const int64_t kt = static_cast<int64_t>(taps) * bpb;
   const Layer* src = L.weights_from;
   const bool borrowed = src && src->tc_ok && src->wq && src->tc_pair == (pairs > 0) && src->tc.BN == t.BN &&
                         src->tc.kind == t.kind && src->tc.n_tiles == t.n_tiles && src->cip == L.cip;
@@ -373,12 +385,12 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
       for (int f = 0; f < L.Ni; ++f) {
         const uint32_t word = packed[(static_cast<int64_t>(c) * taps + tp) * L.nw + f / kWordBits];
         const bool bit = ((word >> (f % kWordBits)) & 1u) != 0;
-        int8_t* row = hq.data() + static_cast<size_t>(c) * kt + static_cast<int64_t>(tp) * bpp;
+        int8_t* row = hq.data() + static_cast<size_t>(c) * kt + static_cast<int64_t>(tp) * bpb;
         if (t.kind == 0) {
           row[f] = bit ? 1 : zero_code;
         } else {
           const uint16_t v = bit ? 0x3F80u : 0xBF80u;  // bf16 +1 / -1
-          for (int part = 0; part < 3; ++part) memcpy(row + 2 * (part * L.cip + f), &v, 2);
+          memcpy(row + 2 * f, &v, 2);
         }
       }
   if (pairs == 0 && !borrowed) {

@@ -102,9 +102,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   }
   uint8_t* smem = smem_raw;
   const int b_bytes = a.BN * 128;
-  const int a_bytes = a.mt * kABytes;
+  const int a_bytes = (kKind == 1 ? 3 : a.mt) * kABytes;  // kind 1: the three parts of x~
   const int stage_bytes = a_bytes + b_bytes;
-  uint8_t* stage_out = smem + kStages * stage_bytes;  // 2 x 16 KB epilogue staging
+  // kind 0 always fits kStages (a 48 KB stage at most); kind 1 stages are larger
+  const int stages = kKind == 1 ? a.stages : kStages;
+  uint8_t* stage_out = smem + stages * stage_bytes;  // 2 x 16 KB epilogue staging
   Barriers* B = reinterpret_cast<Barriers*>(stage_out + 2 * kStageOutBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -114,7 +116,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const uint32_t tmem_cols = a.tmem_cols;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < stages; ++s) {
       mbar_init(&B->full[s], 1);
       mbar_init(&B->empty[s], 1);
     }
@@ -161,13 +163,19 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           mbar_expect_tx(&B->full[stage], static_cast<uint32_t>(a_bytes + tc.bn * 128));
           const int tap = kb / a.kb_per_tap, cb = kb - tap * a.kb_per_tap;
           const int ky = tap / a.kw, kx = tap - ky * a.kw;
-          for (int h = 0; h < a.mt; ++h)
-            tma_load_4d(sa + h * kABytes, &tmA, &B->full[stage], cb * 128, tc.ox0 * a.sx + kx - a.kw / 2,
-                        tc.oy0 * a.sy + ky - a.kh / 2, tc.n0 + h * a.Bn);
+          if constexpr (kKind == 1) {
+            for (int part = 0; part < 3; ++part)
+              tma_load_4d(sa + part * kABytes, &tmA, &B->full[stage], act_x(cb, part, a.kb_px, a.px_bytes, a.part_bytes),
+                          tc.ox0 * a.sx + kx - a.kw / 2, tc.oy0 * a.sy + ky - a.kh / 2, tc.n0);
+          } else {
+            for (int h = 0; h < a.mt; ++h)  // kind 0: k-blocks are consecutive 128-byte blocks
+              tma_load_4d(sa + h * kABytes, &tmA, &B->full[stage], cb * 128, tc.ox0 * a.sx + kx - a.kw / 2,
+                          tc.oy0 * a.sy + ky - a.kh / 2, tc.n0 + h * a.Bn);
+          }
           // the weight stage is one contiguous, already swizzled block of bn rows
           bulk_load(sb, a.b_tiles + ((static_cast<int64_t>(tc.ntile) * kb_total + kb) * a.BN + tc.noff) * 128,
                     static_cast<uint32_t>(tc.bn * 128), &B->full[stage]);
-          if (++stage == kStages) {
+          if (++stage == stages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -198,19 +206,28 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           tc_fence_after();
           uint8_t* sa = smem + stage * stage_bytes;
           const uint64_t db = smem_desc_sw128(sa + a_bytes);
-          for (int h = 0; h < a.mt; ++h) {
-            const uint64_t da = smem_desc_sw128(sa + h * kABytes);
+          if constexpr (kKind == 1) {
+            // the three parts of x~ against the same weight block, into one accumulator
+            for (int part = 0; part < 3; ++part) {
+              const uint64_t da = smem_desc_sw128(sa + part * kABytes);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {  // four 32-byte K steps across the 128-byte row
-              const uint32_t accum = (kb > kb0 || j > 0) ? 1u : 0u;
-              if constexpr (kKind == 1)
-                tc_mma_bf16(d_tmem + static_cast<uint32_t>(h * a.BN), da + 2u * j, db + 2u * j, idesc, accum);
-              else
+              for (int j = 0; j < 4; ++j) {  // four 32-byte K steps across the 128-byte row
+                const uint32_t accum = (kb > kb0 || part > 0 || j > 0) ? 1u : 0u;
+                tc_mma_bf16(d_tmem, da + 2u * j, db + 2u * j, idesc, accum);
+              }
+            }
+          } else {
+            for (int h = 0; h < a.mt; ++h) {
+              const uint64_t da = smem_desc_sw128(sa + h * kABytes);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {  // four 32-byte K steps across the 128-byte row
+                const uint32_t accum = (kb > kb0 || j > 0) ? 1u : 0u;
                 tc_mma_i8(d_tmem + static_cast<uint32_t>(h * a.BN), da + 2u * j, db + 2u * j, idesc, accum);
+              }
             }
           }
           tc_commit(&B->empty[stage]);
-          if (++stage == kStages) {
+          if (++stage == stages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -425,8 +442,17 @@ __global__ void __launch_bounds__(kFinThreads) tc_finalize_kernel(float4* __rest
 
 }  // namespace
 
-int tc_smem_bytes(int bn, int mt) {
-  return kStages * (mt * kABytes + bn * 128) + 2 * kStageOutBytes + static_cast<int>(sizeof(Barriers));
+constexpr int kSmemMax = 227 * 1024;  // dynamic shared memory one CTA may opt in to
+
+int tc_stages(int kind, int bn, int mt) {
+  const int stage = (kind == 1 ? 3 : mt) * kABytes + bn * 128;
+  const int s = (kSmemMax - 2 * kStageOutBytes - static_cast<int>(sizeof(Barriers))) / stage;
+  return s < kStages ? s : kStages;
+}
+
+int tc_smem_bytes(const TcArgs& a) {
+  return a.stages * ((a.kind == 1 ? 3 : a.mt) * kABytes + a.BN * 128) + 2 * kStageOutBytes +
+         static_cast<int>(sizeof(Barriers));
 }
 
 int tc_plan(TcArgs& a, int sm_count) {
@@ -449,7 +475,8 @@ int tc_plan(TcArgs& a, int sm_count) {
 }
 
 cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s) {
-  const int smem = tc_smem_bytes(a.BN, a.mt);
+  if (a.stages < 2 || a.stages > kStages || (a.kind == 1 && a.mt != 1)) return cudaErrorInvalidValue;
+  const int smem = tc_smem_bytes(a);
   const int tiles = a.m_tiles * a.n_tiles * a.k_splits;
   if (tiles == 0) return cudaSuccess;
   int grid = current_sm_count();

@@ -15,7 +15,14 @@ struct TcArgs {
   int kh, kw;          // window (1 x 1 for the FC)
   int sy, sx;          // stride (the activation map steps the box by it)
   int kind;            // 0: int8 codes, s32 accumulator; 1: bf16 parts, f32 accumulator
-  int kb_per_tap;      // 128-byte channel blocks per tap
+  int kb_per_tap;      // k-blocks per tap (a k-block is 128 bytes of weights per output channel)
+  // Where k-block cb of a tap sits in a pixel of the activation map: kb_px k-blocks per pixel,
+  // px_bytes bytes per pixel; kind 1 keeps the three bf16 parts of x~ part_bytes apart, and a
+  // pipeline stage holds all three parts of one k-block against its single weight block.
+  int kb_px;
+  int px_bytes;
+  int part_bytes;
+  int stages;          // pipeline stages in shared memory (as many as fit, at most 4 / 6)
   int BN;              // output channels per tile (multiple of 32, <= 256)
   int n_tiles;         // ceil(No / BN)
   int m_tiles;         // tiles_y * tiles_x * ceil(N / Bn)
@@ -66,7 +73,8 @@ struct TcArgs {
   const int8_t* b_tiles;
 };
 
-int tc_smem_bytes(int bn, int mt);
+int tc_stages(int kind, int bn, int mt);  // stages that fit; < 2: the layout does not fit
+int tc_smem_bytes(const TcArgs& a);
 // One CTA per tile; weights from a.b_tiles.
 cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s);
 // Grid size and tail split for a launch on `sm_count` SMs (fills full_tiles / pieces).
@@ -74,9 +82,10 @@ int tc_plan(TcArgs& a, int sm_count);
 
 // SM-pair kernel (tcgen05.mma.cta_group::2, M = 256 per cluster of two CTAs); convolutions only.
 // tmB / tmBp are weight maps with boxes of BN/2 and BN/pieces/2 rows.
-int tc2_smem_bytes(int bn);
-int tc2_plan(TcArgs& a, int pairs);  // pairs = clusters that can be resident at once
-int tc2_max_pairs(int bn);           // co-resident two-CTA clusters on the current device (0: none)
+int tc2_stages(int kind, int bn);
+int tc2_smem_bytes(int kind, int bn, int stages);
+int tc2_plan(TcArgs& a, int pairs);      // pairs = clusters that can be resident at once
+int tc2_max_pairs(int kind, int bn);     // co-resident two-CTA clusters on the current device (0: none)
 cudaError_t launch_tc_conv2(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmBp,
                             const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s);
 // The epilogue of a split reduction: y from the fp32 workspace [rows][no] (zeroed as it is

@@ -204,8 +204,11 @@ __global__ void __launch_bounds__(kThreads2, 1)
     return;
   }
   const int half_b = a.BN / 2;  // weight rows this CTA holds
-  const int stage_bytes = kABytes2 + half_b * 128;
-  uint8_t* stage_out = smem + kStages2 * stage_bytes;
+  constexpr int kParts = kKind == 1 ? 3 : 1;  // kind 1: the three parts of x~ per stage
+  const int stage_bytes = kParts * kABytes2 + half_b * 128;
+  // kind 0 always fits kStages2 (a 32 KB stage at most); kind 1 stages are larger
+  const int stages = kKind == 1 ? a.stages : kStages2;
+  uint8_t* stage_out = smem + stages * stage_bytes;
   Barriers2* B = reinterpret_cast<Barriers2*>(stage_out + 2 * kOutBytes2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -220,7 +223,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
   const uint32_t tmem_cols = a.tmem_cols;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages2; ++s) {
+    for (int s = 0; s < stages; ++s) {
       mbar_init(&B->full[s], 1);
       mbar_init(&B->empty[s], 1);
     }
@@ -260,25 +263,28 @@ __global__ void __launch_bounds__(kThreads2, 1)
       int w, k0, k1;
       while (ok && work.next(npairs, total, kb_total, w, k0, k1)) {
         const PairCoord pc = pair_coord(a, w, rank);
-        const uint32_t tx = static_cast<uint32_t>(2 * (kABytes2 + (pc.bn / 2) * 128));  // both CTAs' bytes
+        const uint32_t tx = static_cast<uint32_t>(2 * (kParts * kABytes2 + (pc.bn / 2) * 128));  // both CTAs' bytes
         for (int kb = k0; kb < k1; ++kb) {
           if (!mbar_wait(&B->empty[stage], phase ^ 1u, B, a.err)) {
             ok = false;
             break;
           }
           uint8_t* sa = smem + stage * stage_bytes;
-          uint8_t* sb = sa + kABytes2;
+          uint8_t* sb = sa + kParts * kABytes2;
           const uint32_t full_leader = mapa(&B->full[stage], 0);
           if (leader) mbar_expect_tx(&B->full[stage], tx);
           const int tap = kb / a.kb_per_tap, cb = kb - tap * a.kb_per_tap;
           const int ky = tap / a.kw, kx = tap - ky * a.kw;
-          tma_load_4d_pair(sa, &tmA, full_leader, cb * 128, pc.ox0 * a.sx + kx - a.kw / 2, pc.oy0 * a.sy + ky - a.kh / 2, pc.n0);
+          for (int part = 0; part < kParts; ++part)  // kind 0: k-blocks are consecutive 128-byte blocks
+            tma_load_4d_pair(sa + part * kABytes2, &tmA, full_leader,
+                             kKind == 1 ? act_x(cb, part, a.kb_px, a.px_bytes, a.part_bytes) : cb * 128,
+                             pc.ox0 * a.sx + kx - a.kw / 2, pc.oy0 * a.sy + ky - a.kh / 2, pc.n0);
           const int brow = pc.ntile * a.BN + pc.noff + static_cast<int>(rank) * (pc.bn / 2);
           if (pc.bn == a.BN)
             tma_load_2d_pair(sb, &tmB, full_leader, kb * 128, brow);
           else
             tma_load_2d_pair(sb, &tmBp, full_leader, kb * 128, brow);
-          if (++stage == kStages2) {
+          if (++stage == stages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -308,17 +314,20 @@ __global__ void __launch_bounds__(kThreads2, 1)
           }
           tc_fence_after();
           uint8_t* sa = smem + stage * stage_bytes;
-          const uint64_t da = smem_desc_sw128(sa), db = smem_desc_sw128(sa + kABytes2);
+          const uint64_t db = smem_desc_sw128(sa + kParts * kABytes2);
+          for (int part = 0; part < kParts; ++part) {  // kind 1: the parts against one weight block
+            const uint64_t da = smem_desc_sw128(sa + part * kABytes2);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t accum = (kb > k0 || j > 0) ? 1u : 0u;
-            if constexpr (kKind == 1)
-              tc_mma_bf16_pair(d_tmem, da + 2u * j, db + 2u * j, idesc, accum);
-            else
-              tc_mma_i8_pair(d_tmem, da + 2u * j, db + 2u * j, idesc, accum);
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t accum = (kb > k0 || part > 0 || j > 0) ? 1u : 0u;
+              if constexpr (kKind == 1)
+                tc_mma_bf16_pair(d_tmem, da + 2u * j, db + 2u * j, idesc, accum);
+              else
+                tc_mma_i8_pair(d_tmem, da + 2u * j, db + 2u * j, idesc, accum);
+            }
           }
           tc_commit_pair(&B->empty[stage]);
-          if (++stage == kStages2) {
+          if (++stage == stages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -530,12 +539,23 @@ __global__ void __launch_bounds__(kThreads2, 1)
 
 }  // namespace
 
-int tc2_smem_bytes(int bn) {
-  return kStages2 * (kABytes2 + (bn / 2) * 128) + 2 * kOutBytes2 + static_cast<int>(sizeof(Barriers2));
+constexpr int kSmemMax2 = 227 * 1024;  // dynamic shared memory one CTA may opt in to
+
+int tc2_stages(int kind, int bn) {
+  const int stage = (kind == 1 ? 3 : 1) * kABytes2 + (bn / 2) * 128;
+  const int s = (kSmemMax2 - 2 * kOutBytes2 - static_cast<int>(sizeof(Barriers2))) / stage;
+  return s < kStages2 ? s : kStages2;
 }
 
-int tc2_max_pairs(int bn) {
-  const int smem = tc2_smem_bytes(bn);
+int tc2_smem_bytes(int kind, int bn, int stages) {
+  return stages * ((kind == 1 ? 3 : 1) * kABytes2 + (bn / 2) * 128) + 2 * kOutBytes2 +
+         static_cast<int>(sizeof(Barriers2));
+}
+
+int tc2_max_pairs(int kind, int bn) {
+  const int stages = tc2_stages(kind, bn);
+  if (stages < 2) return 0;
+  const int smem = tc2_smem_bytes(kind, bn, stages);
   const void* kerns[] = {
       reinterpret_cast<const void*>(tc_conv2_kernel<0, false, false, false>),
       reinterpret_cast<const void*>(tc_conv2_kernel<1, false, false, false>),
@@ -598,7 +618,8 @@ cudaError_t launch_tc_conv2(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
                             const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s) {
   const int pair_tiles = (a.m_tiles + 1) / 2 * a.n_tiles * a.k_splits;
   if (pair_tiles == 0) return cudaSuccess;
-  const int smem = tc2_smem_bytes(a.BN);
+  if (a.stages < 2 || a.stages > kStages2) return cudaErrorInvalidValue;
+  const int smem = tc2_smem_bytes(a.kind, a.BN, a.stages);
   const int npairs = a.grid_ctas / 2;
   if (npairs <= 0) return cudaErrorInvalidConfiguration;
   if (a.k_splits > 1 && (a.out_bits || a.sk)) return cudaErrorInvalidValue;

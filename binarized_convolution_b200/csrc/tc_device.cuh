@@ -177,6 +177,13 @@ __host__ __device__ constexpr uint32_t idesc_for(int kind, int m, int n) {
 }
 
 // Accumulator word -> fp32 value of the window sum.
+// Byte offset, within a pixel row of the activation map, of part `part` of k-block `cb` of a
+// tap (kind 0 has one part).
+__device__ __forceinline__ int act_x(int cb, int part, int kb_px, int px_bytes, int part_bytes) {
+  if (cb < kb_px) return part * part_bytes + cb * 128;  // a convolution tap: one pixel
+  return (cb / kb_px) * px_bytes + part * part_bytes + (cb % kb_px) * 128;
+}
+
 __device__ __forceinline__ float acc_value(int kind, uint32_t v) {
   return kind ? __uint_as_float(v) : static_cast<float>(static_cast<int32_t>(v));
 }

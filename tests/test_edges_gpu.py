@@ -260,12 +260,15 @@ def _spread(w, mode=None):
 
 
 def test_spread_choice(cuda_device):
-    """AUTO: one SM per tile where the pair plan is not clearly shorter (equal waves), SM
-    pairs where their balanced split evens out a ragged last wave and for the FC with batch
-    > 128; forced modes are kept where the layer allows them."""
+    """AUTO: one SM per tile where the pair plan is not clearly shorter (equal waves; the
+    binaryWeights layer's 24 against 27 stages is not enough for it), SM pairs where their
+    balanced split evens out a ragged last wave by more and for the FC with batch > 128;
+    forced modes are kept where the layer allows them."""
     assert _spread(synth.workload("xnor_beta_n16_56x56_c256_k256_3x3")) == bc.CTA_SINGLE
     assert _spread(synth.workload("and_n32_28x28_c512_k512_3x3")) == bc.CTA_SINGLE
-    assert _spread(synth.workload("binw_n8_112x112_c128_k128_3x3_s2")) == bc.CTA_PAIR
+    assert _spread(synth.workload("binw_n8_112x112_c128_k128_3x3_s2")) == bc.CTA_SINGLE
+    ragged = synth.small_case(batch=4, h=70, w=70, ni=32, no=32, k=3, op=synth.XNOR, seed=27)
+    assert _spread(ragged) == bc.CTA_PAIR  # 162 tiles: 18 stages on single SMs, 10 on pairs
     assert _spread(synth.workload("fc_xnor_beta_n256_7x7x512_k4096")) == bc.CTA_PAIR
     small = synth.small_case(batch=1, h=8, w=8, ni=64, no=32, k=3, op=synth.XNOR, seed=22)
     assert _spread(small) == bc.CTA_SINGLE
