@@ -12,10 +12,14 @@
 // tap spanning the flattened image.
 //
 // Structure: a persistent kernel, one CTA per SM, 6 warps.
-//   warp 0      TMA producer: per k-block, one 128-row x 128-byte activation tile (a box of
-//               Bn images x R rows x Cw columns of the int8 NHWC codes, shifted by the tap
-//               offset; out-of-image coordinates read zeros) and one BN x 128-byte weight
-//               tile, both 128-byte swizzled, into a 4-stage ring guarded by mbarriers.
+//   warp 0      producer: per k-block, one 128-row x 128-byte activation tile by TMA (a box
+//               of Bn images x R rows x Cw columns of the int8 NHWC codes, shifted by the tap
+//               offset; out-of-image coordinates read zeros; 128-byte swizzled) and one
+//               BN x 128-byte weight block by a single bulk copy (laid out already swizzled),
+//               into a ring of 4 stages guarded by mbarriers.  binaryWeights (kind::f16): the
+//               stage holds the three bf16 parts of x~ for one 64-channel block against one
+//               weight block, and the three parts' MMAs go into the same accumulator (2-3
+//               stages fit).
 //   warp 1      allocates TMEM (two BN-column int32 accumulators) and, from one thread,
 //               issues tcgen05.mma M=128 x N=BN x K=32 per 32-byte step; tcgen05.commit frees
 //               each stage and publishes each finished accumulator.

@@ -7,7 +7,8 @@
 // issued by one thread of the even CTA (the leader) and reads both CTAs' shared memory; each
 // CTA's TMEM receives its own 128 x BN accumulator rows.
 //
-// Per CTA: warp 0 loads its A box and its half of B with TMA into a 6-stage ring; both CTAs'
+// Per CTA: warp 0 loads its A box and its half of B with TMA into a 6-stage ring (binaryWeights:
+// three A boxes, the parts of x~, per stage against one half weight block; 3 stages); both CTAs'
 // copies complete on the leader's `full` barrier, whose expected byte count covers the pair.
 // The leader's warp 1 issues the MMAs and releases each stage and each finished accumulator
 // with tcgen05.commit multicast to both CTAs.  Warps 2-5 of each CTA run the epilogue of its
