@@ -189,6 +189,7 @@ KERNEL_SOURCES = {
                 "binarized_convolution_b200/csrc/tc_bits.cuh"],
 }
 ALGO_KERNEL = {1: "popc_gemm", 2: "bw_conv", 3: "tc_conv"}
+CODES_FP4 = 2  # bconv_tc_codes: e2m1 operand codes
 BF16_FALLBACK_TFLOPS = 1590.0  # recipe fallback when MEASURED_PEAKS.json is absent
 
 
@@ -210,9 +211,13 @@ def tensor_peak() -> tuple[float, str]:
     return BF16_FALLBACK_TFLOPS, "of fallback: 1590 TFLOP/s bf16 x 2 / 2 ops per MAC"
 
 
-def derived_peak(w: synth.Workload, sms: int, sm_mhz: float, kernel: str = "") -> tuple[float, str, str]:
+def derived_peak(w: synth.Workload, sms: int, sm_mhz: float, kernel: str = "", codes: int = 0) -> tuple[float, str, str]:
     """(peak in TOPS of the method's own operations, bound, how it was derived) for the
-    contraction's instruction mix."""
+    contraction's instruction mix (`codes`: the tensor-core operand codes, CODES_*)."""
+    if kernel == "tc_conv" and codes == CODES_FP4:
+        v, how = tensor_peak()
+        # block-scaled fp4 runs at twice the int8 rate (nominal 9 / 4.5 PFLOP/s dense)
+        return 2 * v, "tensor", how.replace("x 2 (int8/bf16 nominal)", "x 4 (fp4/bf16 nominal)")
     if kernel == "tc_conv" and w.op == synth.BINARY_WEIGHTS:
         p = measured_peaks()
         bf16 = float(p.get("bf16_tflops", BF16_FALLBACK_TFLOPS))
@@ -280,6 +285,7 @@ def run_native(args, w: synth.Workload):
 
     inp = synth.make_inputs(w, seed=replica_seed(w.seed, rank))
     bc.bconv_set_cta_mode({"auto": bc.CTA_AUTO, "single": bc.CTA_SINGLE, "pair": bc.CTA_PAIR}[args.cta])
+    bc.bconv_set_tc_codes({"auto": bc.CODES_AUTO, "int8": bc.CODES_INT8, "fp4": bc.CODES_FP4}[args.codes])
     layer_kw = dict(op=w.op, scale=inp.scale, bias=inp.bias, in_scale=inp.in_scale, in_bias=inp.in_bias,
                     use_beta=w.use_beta, relu=w.relu)
     if w.kind == "fc":
@@ -374,9 +380,12 @@ def run_native(args, w: synth.Workload):
     sms = props.multi_processor_count
     max_mhz = clock_info.get("sm_max_mhz") or 1965.0
     kname = ALGO_KERNEL[layer.effective_algo()]
-    peak, bound, how = derived_peak(w, sms, max_mhz, kname)
+    codes = layer.tc_codes() if kname == "tc_conv" else 0
+    peak, bound, how = derived_peak(w, sms, max_mhz, kname, codes)
     achieved = ops_step / (kern_ms_max * 1e-3) / 1e12
-    traffic = measured_traffic(kname, w.name, KERNEL_SOURCES[kname])
+    # the captured traffic is that of the library's own choice of spread and codes
+    traffic = (measured_traffic(kname, w.name, KERNEL_SOURCES[kname])
+               if args.cta == "auto" and args.codes == "auto" else None)
     roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
             "traffic": traffic, "kernel": kname, "kernel_ms": kern_ms_max,
             "kernel_launches_timed": kern_n, "timed_every": PROFILE_EVERY,
@@ -384,9 +393,11 @@ def run_native(args, w: synth.Workload):
     if kname == "tc_conv":
         roof["spread"] = {bc.CTA_SINGLE: "one SM per tile", bc.CTA_PAIR: "SM pairs (cta_group::2)"}.get(
             layer.cta_mode(), "?")
+        roof["codes"] = {bc.CODES_INT8: "int8", bc.CODES_FP4: "e2m1 (fp4), kind::mxf4",
+                         bc.CODES_BF16X3: "bf16 x3"}.get(codes, "?")
     sm_mhz = clock_info.get("sm_mhz")
     if sm_mhz and bound == "alu":
-        p_obs, _, _ = derived_peak(w, sms, sm_mhz, kname)
+        p_obs, _, _ = derived_peak(w, sms, sm_mhz, kname, codes)
         roof["frac_at_observed_clock"] = achieved / p_obs
     try:
         probe = 0 if kname == "popc_gemm" else None
@@ -401,6 +412,7 @@ def run_native(args, w: synth.Workload):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": ("bf16x3 / f32" if (kname == "tc_conv" and w.op == synth.BINARY_WEIGHTS) else
+                  "e2m1 (fp4) codes / f32" if codes == CODES_FP4 else
                   {"popc_gemm": "u32 bits / int32", "tc_conv": "int8 codes / int32", "bw_conv": "f32"}[kname]),
         "data": "synthetic (seeded N(0,1) inputs, Bernoulli weight bits)",
         "config": {"workload": w.name, "batch_per_gpu": w.batch, "global_batch": w.batch * world,
@@ -513,6 +525,8 @@ def main(argv=None):
                     help="kernel family of the contraction (auto = the library's choice)")
     ap.add_argument("--cta", choices=["auto", "single", "pair"], default="auto",
                     help="tensor-core contraction on one SM per tile or on SM pairs (auto = the library's choice)")
+    ap.add_argument("--codes", choices=["auto", "int8", "fp4"], default="auto",
+                    help="operand codes of the XNOR/AND tensor-core path (auto = the library's choice)")
     ap.add_argument("--io", choices=["f32", "bits"], default="f32",
                     help="bits: time a middle layer of a chain (bit-packed input and output)")
     ap.add_argument("--no-e2e", action="store_true")

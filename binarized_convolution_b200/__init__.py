@@ -17,6 +17,10 @@ from ._native import (  # noqa: F401
     ALGO_POPC,
     ALGO_SIMT_F32,
     ALGO_TCGEN05,
+    CODES_AUTO,
+    CODES_BF16X3,
+    CODES_FP4,
+    CODES_INT8,
     CTA_AUTO,
     CTA_PAIR,
     CTA_SINGLE,
@@ -31,6 +35,8 @@ from ._native import (  # noqa: F401
     bconv_create,
     bconv_cta_mode,
     bconv_set_cta_mode,
+    bconv_set_tc_codes,
+    bconv_tc_codes,
     bconv_desc_t,
     bconv_destroy,
     bconv_effective_algo,
@@ -59,6 +65,7 @@ from ._native import (  # noqa: F401
     bconv_version,
     bfc_create,
     bfc_cta_mode,
+    bfc_tc_codes,
     bfc_desc_t,
     bfc_destroy,
     bfc_effective_algo,

@@ -25,6 +25,7 @@ FLAG_NONE, FLAG_USE_BETA_SCALING = 0, 1
 NEURON_NONE, NEURON_RELU = 0, 1
 ALGO_AUTO, ALGO_POPC, ALGO_SIMT_F32, ALGO_TCGEN05 = 0, 1, 2, 3
 CTA_AUTO, CTA_SINGLE, CTA_PAIR = 0, 1, 2
+CODES_AUTO, CODES_INT8, CODES_FP4, CODES_BF16X3 = 0, 1, 2, 3
 
 _STATUS = {0: "BCONV_OK", 1: "BCONV_ERR_INVALID_ARG", 2: "BCONV_ERR_UNSUPPORTED", 3: "BCONV_ERR_CUDA",
            4: "BCONV_ERR_OOM", 5: "BCONV_ERR_TIMEOUT", 6: "BCONV_ERR_NO_DEVICE"}
@@ -96,6 +97,9 @@ _SIGS = {
     "bconv_set_cta_mode": (_I32, [_I32]),
     "bconv_cta_mode": (_I32, [_P]),
     "bfc_cta_mode": (_I32, [_P]),
+    "bconv_set_tc_codes": (_I32, [_I32]),
+    "bconv_tc_codes": (_I32, [_P]),
+    "bfc_tc_codes": (_I32, [_P]),
 }
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -275,6 +279,19 @@ def bfc_effective_algo(h) -> int:
 def bconv_set_cta_mode(mode: int):
     """Spread of the tensor-core contraction for layers created from now on (CTA_*)."""
     _check(load_library().bconv_set_cta_mode(int(mode)), "bconv_set_cta_mode")
+
+
+def bconv_set_tc_codes(codes: int):
+    """Operand codes of the XNOR/AND tensor-core path for layers created from now on (CODES_*)."""
+    _check(load_library().bconv_set_tc_codes(int(codes)), "bconv_set_tc_codes")
+
+
+def bconv_tc_codes(h) -> int:
+    return load_library().bconv_tc_codes(h)
+
+
+def bfc_tc_codes(h) -> int:
+    return load_library().bfc_tc_codes(h)
 
 
 def bconv_cta_mode(h) -> int:

@@ -71,6 +71,10 @@ cudaError_t launch_pack(const PackArgs& a, cudaStream_t s);
 cudaError_t launch_repack_bits(const uint32_t* bits, int64_t npix, int ni, int nw_pad, uint32_t* out, cudaStream_t s);
 cudaError_t launch_unpack_bits_i8(const uint32_t* bits, int64_t npix, int ni, int cip, int op, int8_t* codes,
                                   cudaStream_t s);
+// ... or into e2m1 (fp4) codes [npix][cip / 2] bytes, two channels per byte (XNOR: 1 -> +1.0
+// = 0x2, 0 -> -1.0 = 0xA; AND: 1 -> 0x2, 0 -> 0; channels >= ni -> 0; cip a multiple of 32).
+cudaError_t launch_unpack_bits_f4(const uint32_t* bits, int64_t npix, int ni, int cip, int op, int8_t* codes,
+                                  cudaStream_t s);
 
 // ------------------------------------------------------------------------------------
 // Beta: box filter of A over the window (conv) or mean of A over the image (FC).

@@ -116,6 +116,16 @@ __device__ __forceinline__ uint32_t codes4(const float4& v) {
          (((v.w < 0.f) ? kNeg : kPos) << 24);
 }
 
+// The same 4 values as e2m1 (fp4) codes in one 16-bit word, element j in bits 4j..4j+3:
+// +1.0 = 0x2; -1.0 = 0xA (XNOR) or 0 (AND).
+template <int kOp>
+__device__ __forceinline__ uint32_t nibbles4(const float4& v) {
+  constexpr uint32_t kPos = 0x2u;
+  constexpr uint32_t kNeg = kOp == kXnor ? 0xAu : 0x0u;
+  return ((v.x < 0.f) ? kNeg : kPos) | (((v.y < 0.f) ? kNeg : kPos) << 4) | (((v.z < 0.f) ? kNeg : kPos) << 8) |
+         (((v.w < 0.f) ? kNeg : kPos) << 12);
+}
+
 template <bool kTerms>
 __device__ __forceinline__ float4 transform4(float4 v, const float* __restrict__ sc, const float* __restrict__ bi,
                                              int f) {
@@ -147,7 +157,7 @@ __device__ __forceinline__ void load_group(float4 (&v)[kG][kC], const float* __r
     }
 }
 
-template <bool kTerms, bool kA, int kOp, int kC>
+template <bool kTerms, bool kA, int kOp, int kC, bool kF4>
 __global__ void __launch_bounds__(kPackThreads, 2) pack_i8_vec_kernel(PackI8Args a) {
   constexpr int kG = 8 / kC;  // pixels per warp step
   wait_prior_grid();
@@ -195,9 +205,12 @@ __global__ void __launch_bounds__(kPackThreads, 2) pack_i8_vec_kernel(PackI8Args
             t.w = fmaf(t.w, sc[c].w, bi[c].w);
           }
           if (kA) asum += (fabsf(t.x) + fabsf(t.y)) + (fabsf(t.z) + fabsf(t.w));
-          word = codes4<kOp>(t);
+          word = kF4 ? nibbles4<kOp>(t) : codes4<kOp>(t);
         }
-        *reinterpret_cast<uint32_t*>(codes + p * a.cip + c * 128 + lane * 4) = word;
+        if (kF4)  // e2m1 codes: cip / 2 bytes per pixel, 64 bytes per 128-channel chunk
+          *reinterpret_cast<uint16_t*>(codes + p * (a.cip / 2) + c * 64 + lane * 2) = static_cast<uint16_t>(word);
+        else
+          *reinterpret_cast<uint32_t*>(codes + p * a.cip + c * 128 + lane * 4) = word;
       }
       if (kA) {
         asum = warp_sum(asum);
@@ -211,8 +224,8 @@ __global__ void __launch_bounds__(kPackThreads, 2) pack_i8_vec_kernel(PackI8Args
   }
 }
 
-// Any channel count: one byte per lane per step.
-template <bool kTerms, bool kA, int kOp>
+// Any channel count: one byte per lane per step (one channel as int8, two as e2m1 nibbles).
+template <bool kTerms, bool kA, int kOp, bool kF4>
 __global__ void __launch_bounds__(kPackThreads) pack_i8_scalar_kernel(PackI8Args a) {
   wait_prior_grid();
   allow_next_grid();
@@ -220,22 +233,28 @@ __global__ void __launch_bounds__(kPackThreads) pack_i8_scalar_kernel(PackI8Args
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kPackThreads) >> 5;
   const int ni = a.ni;
-  constexpr uint32_t kPos = 0x01u;
-  constexpr uint32_t kNeg = kOp == kXnor ? 0xFFu : 0x00u;
+  constexpr uint32_t kPos = kF4 ? 0x2u : 0x01u;
+  constexpr uint32_t kNeg = kOp == kXnor ? (kF4 ? 0xAu : 0xFFu) : 0x00u;
+  constexpr int kPer = kF4 ? 2 : 1;  // channels per lane and step
   for (int64_t p = warp; p < a.npix; p += nwarps) {
     const float* row = a.in + p * ni;
-    int8_t* crow = a.codes + p * a.cip;
+    int8_t* crow = a.codes + p * (a.cip / kPer);
     float asum = 0.f;
-    for (int f0 = 0; f0 < a.cip; f0 += 32) {
-      const int f = f0 + lane;
-      uint32_t code = 0u;
-      if (f < ni) {
-        float v = __ldcs(row + f);
-        if (kTerms) v = fmaf(v, __ldg(a.in_scale + f), __ldg(a.in_bias + f));
-        if (kA) asum += fabsf(v);
-        code = (v < 0.f) ? kNeg : kPos;
+    for (int f0 = 0; f0 < a.cip; f0 += 32 * kPer) {
+      uint32_t byte = 0u;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int f = f0 + lane * kPer + u;
+        uint32_t code = 0u;
+        if (f < ni) {
+          float v = __ldcs(row + f);
+          if (kTerms) v = fmaf(v, __ldg(a.in_scale + f), __ldg(a.in_bias + f));
+          if (kA) asum += fabsf(v);
+          code = (v < 0.f) ? kNeg : kPos;
+        }
+        byte |= code << (4 * u);
       }
-      crow[f] = static_cast<int8_t>(code);
+      crow[f0 / kPer + lane] = static_cast<int8_t>(byte);
     }
     if (kA) {
       asum = warp_sum(asum);
@@ -244,13 +263,19 @@ __global__ void __launch_bounds__(kPackThreads) pack_i8_scalar_kernel(PackI8Args
   }
 }
 
+template <bool kTerms, bool kA, int kOp, bool kF4>
+cudaError_t launch_i8_f(const PackI8Args& a, int chunks, dim3 grid, cudaStream_t s) {
+  auto kern = chunks == 1   ? pack_i8_vec_kernel<kTerms, kA, kOp, 1, kF4>
+              : chunks == 2 ? pack_i8_vec_kernel<kTerms, kA, kOp, 2, kF4>
+              : chunks == 4 ? pack_i8_vec_kernel<kTerms, kA, kOp, 4, kF4>
+                            : pack_i8_scalar_kernel<kTerms, kA, kOp, kF4>;
+  return launch_overlapped(kern, grid, dim3(kPackThreads), 0, s, a);
+}
+
 template <bool kTerms, bool kA, int kOp>
 cudaError_t launch_i8_t(const PackI8Args& a, int chunks, dim3 grid, cudaStream_t s) {
-  auto kern = chunks == 1   ? pack_i8_vec_kernel<kTerms, kA, kOp, 1>
-              : chunks == 2 ? pack_i8_vec_kernel<kTerms, kA, kOp, 2>
-              : chunks == 4 ? pack_i8_vec_kernel<kTerms, kA, kOp, 4>
-                            : pack_i8_scalar_kernel<kTerms, kA, kOp>;
-  return launch_overlapped(kern, grid, dim3(kPackThreads), 0, s, a);
+  return a.f4 ? launch_i8_f<kTerms, kA, kOp, true>(a, chunks, grid, s)
+              : launch_i8_f<kTerms, kA, kOp, false>(a, chunks, grid, s);
 }
 
 template <bool kTerms, bool kA>
@@ -472,6 +497,37 @@ __global__ void __launch_bounds__(256) unpack_bits_i8_kernel(const uint32_t* __r
   }
 }
 
+// e2m1 codes of 8 channels (bits of `b`, LSB first) as 8 nibbles; nibbles at or past nvalid are 0.
+template <int kOp>
+__device__ __forceinline__ uint32_t f4_codes_of_byte(uint32_t b, int nvalid) {
+  uint32_t x = b & 0xFFu;  // bit i -> bit 4i
+  x = (x | (x << 12)) & 0x000F000Fu;
+  x = (x | (x << 6)) & 0x03030303u;
+  x = (x | (x << 3)) & 0x11111111u;
+  uint32_t c = kOp == kXnor ? (0xAAAAAAAAu ^ (x * 8u)) : (x * 2u);  // 1 -> 0x2; 0 -> 0xA or 0
+  if (nvalid < 8) c &= nvalid <= 0 ? 0u : ((1u << (4 * nvalid)) - 1u);
+  return c;
+}
+
+// One thread per 32 channels of a pixel: 32 e2m1 codes (16 bytes) as one 16-byte store.
+template <int kOp>
+__global__ void __launch_bounds__(256) unpack_bits_f4_kernel(const uint32_t* __restrict__ bits, uint32_t total,
+                                                              uint32_t groups, int nw_in, int ni,
+                                                              uint4* __restrict__ codes) {
+  wait_prior_grid();
+  allow_next_grid();
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const uint32_t p = i / groups;
+    const int g = static_cast<int>(i - p * groups);
+    const int c0 = g * 32;
+    uint32_t word = 0;
+    if (c0 < ni) word = __ldg(bits + static_cast<size_t>(p) * nw_in + g);
+    const int nv = ni - c0;
+    codes[i] = make_uint4(f4_codes_of_byte<kOp>(word, nv), f4_codes_of_byte<kOp>(word >> 8, nv - 8),
+                          f4_codes_of_byte<kOp>(word >> 16, nv - 16), f4_codes_of_byte<kOp>(word >> 24, nv - 24));
+  }
+}
+
 // One thread per output word: copy, clear the bits past ni, zero the padding words.
 __global__ void __launch_bounds__(256) repack_bits_kernel(const uint32_t* __restrict__ bits, uint32_t total, int nw_in,
                                                            int ni, uint32_t nw_pad, uint32_t* __restrict__ out) {
@@ -495,6 +551,17 @@ unsigned grid_for(int64_t threads) {
 }
 
 }  // namespace
+
+cudaError_t launch_unpack_bits_f4(const uint32_t* bits, int64_t npix, int ni, int cip, int op, int8_t* codes,
+                                  cudaStream_t s) {
+  if (npix == 0) return cudaSuccess;
+  const int64_t total = npix * (cip / 32);
+  if (total >= (int64_t{1} << 31)) return cudaErrorInvalidValue;
+  const uint32_t t = static_cast<uint32_t>(total), g = static_cast<uint32_t>(cip / 32);
+  uint4* out = reinterpret_cast<uint4*>(codes);
+  return launch_overlapped(op == kXnor ? unpack_bits_f4_kernel<kXnor> : unpack_bits_f4_kernel<kAnd>,
+                           dim3(grid_for(total)), dim3(256), 0, s, bits, t, g, words_for(ni), ni, out);
+}
 
 cudaError_t launch_unpack_bits_i8(const uint32_t* bits, int64_t npix, int ni, int cip, int op, int8_t* codes,
                                   cudaStream_t s) {

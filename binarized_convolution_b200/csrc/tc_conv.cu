@@ -1,4 +1,5 @@
-// Binary convolution on the 5th-generation tensor cores (tcgen05.mma kind::i8).
+// Binary convolution on the 5th-generation tensor cores (tcgen05.mma kind::i8, kind::mxf4 and,
+// for binaryWeights, kind::f16).
 //
 // What it computes (Apple page "MPSCNNBinaryConvolution", Overview, XNOR and AND bullets):
 // a product of two binarized values is +-1 (XNOR) or 0/1 (AND), so the window sum
@@ -7,7 +8,9 @@
 // w in {-1,+1}; AND codes a, w in {0,1}.  With int32 accumulation the result equals the
 // popcount form 32 - 2*popcount(x^y) (resp. popcount(x&y)) summed over the words, bit for
 // bit.  Out-of-image taps and padding channels are zero codes, which add exactly 0, so no
-// border correction is needed.  The epilogue is out = act(S * scale[c] * beta + bias[c]).
+// border correction is needed.  The same codes as e2m1 (fp4) values (+1.0, -1.0, 0) with every
+// block scale 1.0 (kind::mxf4, kind 2) give the same products exactly, summed in fp32 -- exact
+// for sums below 2^24.  The epilogue is out = act(S * scale[c] * beta + bias[c]).
 // The fully-connected layer (page "MPSCNNFullyConnected") is the same contraction with one
 // tap spanning the flattened image.
 //
@@ -43,15 +46,16 @@ namespace {
 
 using namespace tcdev;
 
-constexpr int kStages = 4;
+constexpr int kStages = 4;     // kind 0 (48 KB stages at most)
+constexpr int kMaxStages = 6;  // kinds 1 and 2: as many as fit
 constexpr int kABytes = 128 * 128;  // 128 rows x 128 bytes
 constexpr int kThreadsTc = 192;
 constexpr int kEpiThreads = 128;
 constexpr int kStageOutBytes = 128 * 128;  // 128 rows x 32 fp32
 
 struct __align__(8) Barriers {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t done;
@@ -108,8 +112,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const int b_bytes = a.BN * 128;
   const int a_bytes = (kKind == 1 ? 3 : a.mt) * kABytes;  // kind 1: the three parts of x~
   const int stage_bytes = a_bytes + b_bytes;
-  // kind 0 always fits kStages (a 48 KB stage at most); kind 1 stages are larger
-  const int stages = kKind == 1 ? a.stages : kStages;
+  // kind 0 always fits kStages (a 48 KB stage at most); kinds 1 and 2 take what fits
+  const int stages = kKind == 0 ? kStages : a.stages;
   uint8_t* stage_out = smem + stages * stage_bytes;  // 2 x 16 KB epilogue staging
   Barriers* B = reinterpret_cast<Barriers*>(stage_out + 2 * kStageOutBytes);
 
@@ -141,6 +145,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = B->tmem_base;
+  // kind 2: the block scale factors live in TMEM after the two accumulators, 16 columns for A
+  // and 16 for B; every factor is 1.0 (ue8m0 0x7F), so the epilogue warps fill all 32 columns
+  // of their lanes once and every MMA reads them in whatever arrangement it uses
+  const uint32_t sf_col = static_cast<uint32_t>(2 * a.BN);
+  if constexpr (kKind == 2) {
+    if (warp >= 2) tc_fill_32x32(tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + sf_col, 0x7F7F7F7Fu);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
   if (threadIdx.x == 0) {
     prefetch_tensor_map(&tmA);
     if (!kBits) prefetch_tensor_map(&tmOut);  // a bit-packed output never uses (or encodes) it
@@ -219,6 +233,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 const uint32_t accum = (kb > kb0 || part > 0 || j > 0) ? 1u : 0u;
                 tc_mma_bf16(d_tmem, da + 2u * j, db + 2u * j, idesc, accum);
               }
+            }
+          } else if constexpr (kKind == 2) {
+            const uint64_t da = smem_desc_sw128(sa);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {  // four 32-byte (64-code) K steps across the 128-byte row
+              const uint32_t accum = (kb > kb0 || j > 0) ? 1u : 0u;
+              tc_mma_f4(d_tmem, da + 2u * j, db + 2u * j, idesc, accum, tmem_base + sf_col, tmem_base + sf_col + 16u);
             }
           } else {
             for (int h = 0; h < a.mt; ++h) {
@@ -451,7 +472,8 @@ constexpr int kSmemMax = 227 * 1024;  // dynamic shared memory one CTA may opt i
 int tc_stages(int kind, int bn, int mt) {
   const int stage = (kind == 1 ? 3 : mt) * kABytes + bn * 128;
   const int s = (kSmemMax - 2 * kStageOutBytes - static_cast<int>(sizeof(Barriers))) / stage;
-  return s < kStages ? s : kStages;
+  const int cap = kind == 0 ? kStages : kMaxStages;
+  return s < cap ? s : cap;
 }
 
 int tc_smem_bytes(const TcArgs& a) {
@@ -479,16 +501,22 @@ int tc_plan(TcArgs& a, int sm_count) {
 }
 
 cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s) {
-  if (a.stages < 2 || a.stages > kStages || (a.kind == 1 && a.mt != 1)) return cudaErrorInvalidValue;
+  if (a.stages < 2 || a.stages > (a.kind == 0 ? kStages : kMaxStages) || (a.kind != 0 && a.mt != 1) ||
+      (a.kind == 0 && a.stages != kStages) || (a.kind == 2 && 2 * a.BN + 32 > static_cast<int>(a.tmem_cols)))
+    return cudaErrorInvalidValue;
   const int smem = tc_smem_bytes(a);
   const int tiles = a.m_tiles * a.n_tiles * a.k_splits;
   if (tiles == 0) return cudaSuccess;
   int grid = current_sm_count();
   if (grid > tiles) grid = tiles;
   if ((a.out_bits && a.k_splits > 1) || !a.b_tiles) return cudaErrorInvalidValue;
-  auto kern = a.k_splits > 1 ? (a.kind ? tc_conv_kernel<true, 1, false> : tc_conv_kernel<true, 0, false>)
-              : a.out_bits   ? (a.kind ? tc_conv_kernel<false, 1, true> : tc_conv_kernel<false, 0, true>)
-                             : (a.kind ? tc_conv_kernel<false, 1, false> : tc_conv_kernel<false, 0, false>);
+  auto pick = [](auto k0, auto k1, auto k2, int kind) { return kind == 2 ? k2 : kind == 1 ? k1 : k0; };
+  auto kern = a.k_splits > 1 ? pick(tc_conv_kernel<true, 0, false>, tc_conv_kernel<true, 1, false>,
+                                    tc_conv_kernel<true, 2, false>, a.kind)
+              : a.out_bits   ? pick(tc_conv_kernel<false, 0, true>, tc_conv_kernel<false, 1, true>,
+                                    tc_conv_kernel<false, 2, true>, a.kind)
+                             : pick(tc_conv_kernel<false, 0, false>, tc_conv_kernel<false, 1, false>,
+                                    tc_conv_kernel<false, 2, false>, a.kind);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   return launch_overlapped(kern, dim3(grid), dim3(kThreadsTc), smem, s, *tmA, *tmOut, a);

@@ -95,6 +95,9 @@ cudaError_t launch_tc_finalize(float* ws, float* out, const float* scale, const 
                                int rows, int no, int relu, cudaStream_t s);
 
 // int8 operand codes: XNOR -> bin(x~) in {-1,+1}, AND -> {0,1}; channels in [ni, cip) are 0.
+// With f4 the codes are e2m1 (fp4) values, two per byte (channel 2j in the low nibble):
+// +1.0 = 0x2, -1.0 = 0xA (XNOR) or 0 (AND), padding 0; the code buffer then holds cip / 2
+// bytes per pixel and cip is a multiple of 256.
 struct PackI8Args {
   const float* in;        // [npix][ni]
   int64_t npix;
@@ -102,9 +105,10 @@ struct PackI8Args {
   int cip;                // channels per pixel in the code buffer (multiple of 128)
   const float* in_scale;  // [ni] or nullptr
   const float* in_bias;   // [ni] or nullptr
-  int8_t* codes;          // [npix][cip]
+  int8_t* codes;          // [npix][cip] (f4: [npix][cip / 2] bytes)
   float* A;               // [npix] or nullptr
   int op;                 // kXnor or kAnd
+  int f4;
 };
 cudaError_t launch_pack_i8(const PackI8Args& a, cudaStream_t s);
 

@@ -172,11 +172,37 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, ui
 // Instruction descriptor for M = m, N = n, K-major operands: kind 0 = signed int8 with an s32
 // accumulator, kind 1 = bf16 with an f32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_for(int kind, int m, int n) {
-  return (kind == 0 ? ((2u << 4) | (1u << 7) | (1u << 10)) : ((1u << 4) | (1u << 7) | (1u << 10))) |
+  // kind 2, kind::mxf4 with block scales: A and B e2m1 (format 1 at bits 7 and 10), K-major,
+  // scale factors ue8m0 (bit 23), scale-factor ids 0 (bits 4-5, 29-30), K = 64 (bit 31 = 0);
+  // no accumulator-format field (always fp32).
+  return (kind == 2   ? ((1u << 7) | (1u << 10) | (1u << 23))
+          : kind == 0 ? ((2u << 4) | (1u << 7) | (1u << 10))
+                      : ((1u << 4) | (1u << 7) | (1u << 10))) |
          (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
 
-// Accumulator word -> fp32 value of the window sum.
+// D[tmem] (+)= A * B^T with e2m1 operands, every 32 elements scaled by the ue8m0 factors at
+// TMEM addresses sfa / sfb (kind::mxf4, K = 64, fp32 accumulator).  With codes +-1 / 0 and
+// unit scales every product is exact and so is the fp32 sum of up to 2^24 of them.
+__device__ __forceinline__ void tc_mma_f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate, uint32_t sfa, uint32_t sfb) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this warp's 32 lanes set to `value`.
+__device__ __forceinline__ void tc_fill_32x32(uint32_t taddr, uint32_t value) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+      "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
+      "r"(value)
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // Byte offset, within a pixel row of the activation map, of part `part` of k-block `cb` of a
 // tap (kind 0 has one part).
 __device__ __forceinline__ int act_x(int cb, int part, int kb_px, int px_bytes, int part_bytes) {
@@ -184,6 +210,7 @@ __device__ __forceinline__ int act_x(int cb, int part, int kb_px, int px_bytes, 
   return (cb / kb_px) * px_bytes + part * part_bytes + (cb % kb_px) * 128;
 }
 
+// Accumulator word -> fp32 value of the window sum (kind 0: int32; kinds 1 and 2: fp32).
 __device__ __forceinline__ float acc_value(int kind, uint32_t v) {
   return kind ? __uint_as_float(v) : static_cast<float>(static_cast<int32_t>(v));
 }

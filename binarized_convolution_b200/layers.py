@@ -135,6 +135,9 @@ class BinaryConv2d(_Layer):
     def cta_mode(self) -> int:
         return nat.bconv_cta_mode(self.handle)
 
+    def tc_codes(self) -> int:
+        return nat.bconv_tc_codes(self.handle)
+
     def forward_into(self, x, out):
         import torch
 
@@ -203,6 +206,9 @@ class BinaryFC(_Layer):
 
     def cta_mode(self) -> int:
         return nat.bfc_cta_mode(self.handle)
+
+    def tc_codes(self) -> int:
+        return nat.bfc_tc_codes(self.handle)
 
     def forward_into(self, x, out):
         import torch

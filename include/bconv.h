@@ -223,6 +223,24 @@ bconv_status_t bconv_set_cta_mode(bconv_cta_mode_t mode);
 int32_t bconv_cta_mode(bconv_handle_t h);
 
 /*
+ * Operand codes of the XNOR / AND tensor-core contraction, for layers created after the call
+ * (process-wide, like bconv_set_cta_mode).
+ *   FP4   e2m1 values, two per byte: +-1.0 (XNOR) or 1.0 / 0 (AND), multiplied by
+ *         tcgen05.mma kind::mxf4 with unit block scales and summed in fp32 -- exact, since
+ *         every product is -1, 0 or 1 and the sums stay below 2^24; half the operand bytes
+ *         and twice the MMA rate of INT8; one SM per tile, tiles of up to 128 channels.
+ *   INT8  int8 codes, kind::i8, int32 sums (single SMs or pairs).
+ *   AUTO  FP4, unless the spread is forced onto SM pairs (then INT8).
+ * binaryWeights layers always use three bf16 parts.  Returns INVALID_ARG for an unknown value.
+ */
+typedef enum { BCONV_CODES_AUTO = 0, BCONV_CODES_INT8 = 1, BCONV_CODES_FP4 = 2, BCONV_CODES_BF16X3 = 3 } bconv_tc_codes_t;
+bconv_status_t bconv_set_tc_codes(bconv_tc_codes_t codes);
+
+/* The codes a layer's tensor-core contraction uses (BCONV_CODES_INT8 / FP4 / BF16X3); 0 when
+ * the layer has no tensor-core path, -1 for a bad handle. */
+int32_t bconv_tc_codes(bconv_handle_t h);
+
+/*
  * Wait for `stream`, then read and clear the handle's device error word.  Returns OK,
  * TIMEOUT (a kernel gave up a bounded wait), or CUDA (a pending CUDA error).
  */
@@ -286,6 +304,7 @@ bconv_status_t bfc_set_algo(bfc_handle_t h, bconv_algo_t algo);
 int32_t bfc_launches_per_forward(bfc_handle_t h);
 int32_t bfc_effective_algo(bfc_handle_t h);
 int32_t bfc_cta_mode(bfc_handle_t h);
+int32_t bfc_tc_codes(bfc_handle_t h);
 bconv_status_t bfc_sync_status(bfc_handle_t h, struct CUstream_st* stream);
 bconv_status_t bfc_profile_begin(bfc_handle_t h, int32_t max_launches);
 bconv_status_t bfc_profile_end(bfc_handle_t h, float* total_ms, int32_t* launches);

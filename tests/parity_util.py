@@ -43,8 +43,8 @@ def make_layer(w: synth.Workload, inp: synth.Inputs, *, sums: bool = False):
                         (w.stride_y, w.stride_x), wbits=inp.wbits, **kw)
 
 
-# Kernel families a parity case runs on: the library's choice, the SIMT family, and the
-# tensor cores with the contraction forced onto one SM per tile or onto SM pairs.
+# Kernel families a parity case runs on: the library's choice (e2m1 codes for XNOR/AND), the
+# SIMT family, and the tensor cores with int8 codes forced onto one SM per tile or onto SM pairs.
 FAMILIES = ["auto", "alt", "single", "pair"]
 
 
@@ -53,10 +53,12 @@ def algo_for(w: synth.Workload, name: str):
     cores where they apply), 'alt' (the SIMT family: POPC for XNOR/AND, the FP32 signed-add
     kernel for binaryWeights), or 'single' / 'pair' (the library's choice, with the
     tensor-core contraction of the layers created after this call forced onto one SM per
-    tile or onto SM pairs; the test fixture puts the process-wide setting back to AUTO)."""
+    tile or onto SM pairs, XNOR/AND with int8 codes; the test fixture puts the process-wide
+    settings back to AUTO)."""
     import binarized_convolution_b200 as bc
 
     bc.bconv_set_cta_mode({"single": bc.CTA_SINGLE, "pair": bc.CTA_PAIR}.get(name, bc.CTA_AUTO))
+    bc.bconv_set_tc_codes(bc.CODES_INT8 if name in ("single", "pair") else bc.CODES_AUTO)
     if name == "alt":
         return bc.ALGO_SIMT_F32 if w.op == synth.BINARY_WEIGHTS else bc.ALGO_POPC
     return bc.ALGO_AUTO

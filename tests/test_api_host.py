@@ -118,6 +118,8 @@ def test_calls_on_null_or_foreign_handles_return_errors():
     assert lib.bconv_pack_bits(None, 1, 1, None) == 1
     assert lib.bconv_cta_mode(None) == -1
     assert lib.bfc_cta_mode(None) == -1
+    assert lib.bconv_tc_codes(None) == -1
+    assert lib.bfc_tc_codes(None) == -1
 
 
 def test_cta_mode_setting_is_validated():
@@ -126,6 +128,10 @@ def test_cta_mode_setting_is_validated():
         assert lib.bconv_set_cta_mode(bad) == 1  # INVALID_ARG
     for good in (bc.CTA_SINGLE, bc.CTA_PAIR, bc.CTA_AUTO):
         assert lib.bconv_set_cta_mode(good) == 0
+    for bad in (-1, 3, 7):  # BF16X3 is reported, not chosen
+        assert lib.bconv_set_tc_codes(bad) == 1
+    for good in (bc.CODES_INT8, bc.CODES_FP4, bc.CODES_AUTO):
+        assert lib.bconv_set_tc_codes(good) == 0
 
 
 def test_create_without_a_device_reports_no_device():

@@ -27,6 +27,7 @@ def _check(w, inp=None):
             S_dev = pu.run_device(w, inp, sums=True, algo=a)
             pu.assert_sums_exact(S_dev, S_sum)
     bc.bconv_set_cta_mode(bc.CTA_AUTO)
+    bc.bconv_set_tc_codes(bc.CODES_AUTO)
 
 
 SWEEP = []
@@ -244,39 +245,71 @@ def test_fc_forward_host_in_chunks_matches_device(cuda_device):
         layer.close()
 
 
-def _spread(w, mode=None):
-    """The tensor-core spread a layer of this shape is created with."""
+def _spread(w, mode=None, codes=None):
+    """(spread, operand codes) a layer of this shape is created with."""
     inp = synth.make_inputs(w)
     if mode is not None:
         bc.bconv_set_cta_mode(mode)
+    if codes is not None:
+        bc.bconv_set_tc_codes(codes)
     try:
         layer = pu.make_layer(w, inp)
     finally:
         bc.bconv_set_cta_mode(bc.CTA_AUTO)
+        bc.bconv_set_tc_codes(bc.CODES_AUTO)
     try:
-        return layer.cta_mode()
+        return layer.cta_mode(), layer.tc_codes()
     finally:
         layer.close()
 
 
 def test_spread_choice(cuda_device):
-    """AUTO: one SM per tile where the pair plan is not clearly shorter (equal waves; the
-    binaryWeights layer's 24 against 27 stages is not enough for it), SM pairs where their
-    balanced split evens out a ragged last wave by more and for the FC with batch > 128;
-    forced modes are kept where the layer allows them."""
-    assert _spread(synth.workload("xnor_beta_n16_56x56_c256_k256_3x3")) == bc.CTA_SINGLE
-    assert _spread(synth.workload("and_n32_28x28_c512_k512_3x3")) == bc.CTA_SINGLE
-    assert _spread(synth.workload("binw_n8_112x112_c128_k128_3x3_s2")) == bc.CTA_SINGLE
+    """AUTO: XNOR/AND on e2m1 codes, one SM per tile; with int8 codes one SM per tile where the
+    pair plan is not clearly shorter (equal waves), SM pairs where their balanced split evens
+    out a ragged last wave by more and for the FC with batch > 128; binaryWeights on bf16 parts
+    (its 24 against 27 stages on pairs is not enough for them); forced modes are kept where the
+    layer allows them."""
+    S, P, I8, F4, BF = bc.CTA_SINGLE, bc.CTA_PAIR, bc.CODES_INT8, bc.CODES_FP4, bc.CODES_BF16X3
+    c2 = synth.workload("xnor_beta_n16_56x56_c256_k256_3x3")
+    assert _spread(c2) == (S, F4)
+    assert _spread(c2, codes=I8) == (S, I8)
+    assert _spread(c2, mode=P) == (P, I8)  # SM pairs take int8 codes
+    assert _spread(synth.workload("and_n32_28x28_c512_k512_3x3")) == (S, F4)
+    assert _spread(synth.workload("binw_n8_112x112_c128_k128_3x3_s2")) == (S, BF)
+    assert _spread(synth.workload("fc_xnor_beta_n256_7x7x512_k4096"), codes=I8) == (P, I8)
     ragged = synth.small_case(batch=4, h=70, w=70, ni=32, no=32, k=3, op=synth.XNOR, seed=27)
-    assert _spread(ragged) == bc.CTA_PAIR  # 162 tiles: 18 stages on single SMs, 10 on pairs
-    assert _spread(synth.workload("fc_xnor_beta_n256_7x7x512_k4096")) == bc.CTA_PAIR
+    assert _spread(ragged, codes=I8) == (P, I8)  # 162 tiles: 18 stages on single SMs, 10 on pairs
+    assert _spread(ragged) == (S, F4)
     small = synth.small_case(batch=1, h=8, w=8, ni=64, no=32, k=3, op=synth.XNOR, seed=22)
-    assert _spread(small) == bc.CTA_SINGLE
-    assert _spread(small, bc.CTA_PAIR) == bc.CTA_PAIR
+    assert _spread(small, codes=I8) == (S, I8)
+    assert _spread(small, mode=P) == (P, I8)
     fc = synth.small_case(batch=200, h=2, w=2, ni=64, no=64, kind="fc", op=synth.AND, seed=23)
-    assert _spread(fc) == bc.CTA_PAIR
-    assert _spread(fc, bc.CTA_SINGLE) == bc.CTA_SINGLE
+    assert _spread(fc, codes=I8) == (P, I8)
+    assert _spread(fc, mode=S, codes=I8) == (S, I8)
     fc_small = synth.small_case(batch=100, h=2, w=2, ni=64, no=64, kind="fc", op=synth.AND, seed=24)
-    assert _spread(fc_small, bc.CTA_PAIR) == bc.CTA_SINGLE  # the FC's pair tile needs batch > 128
+    assert _spread(fc_small, mode=P) == (S, I8)  # the FC's pair tile needs batch > 128
     odd = synth.small_case(batch=1, h=5, w=5, ni=64, no=6, k=3, op=synth.XNOR, seed=25)
-    assert _spread(odd) == 0  # out_channels % 4 != 0: no tensor-core path
+    assert _spread(odd) == (0, 0)  # out_channels % 4 != 0: no tensor-core path
+
+
+def test_bit_output_replans_wide_e2m1_layer_on_int8(cuda_device):
+    """A convolution on e2m1 codes with more than one 128-channel tile takes int8 codes (one
+    256-channel tile) once it is asked for a bit-packed output, and still matches the oracle."""
+    w = synth.small_case(batch=1, h=9, w=10, ni=96, no=256, k=3, op=synth.XNOR, use_beta=True, relu=True,
+                         in_terms=True, seed=28)
+    inp = synth.make_inputs(w)
+    layer = pu.make_layer(w, inp)
+    try:
+        assert layer.tc_codes() == bc.CODES_FP4
+        ns, nb = synth.next_terms(w.out_channels, 5)
+        layer.set_output_terms(ns, nb)
+        assert layer.tc_codes() == bc.CODES_INT8 and layer.cta_mode() == bc.CTA_SINGLE
+    finally:
+        layer.close()
+    narrow = synth.small_case(batch=1, h=9, w=10, ni=96, no=64, k=3, op=synth.XNOR, seed=29)
+    layer = pu.make_layer(narrow, synth.make_inputs(narrow))
+    try:
+        layer.set_output_terms(*synth.next_terms(64, 6))
+        assert layer.tc_codes() == bc.CODES_FP4  # one tile: nothing to add across items
+    finally:
+        layer.close()
