@@ -909,8 +909,6 @@ bconv_status_t forward_io(Layer& L, const bconv_io_t* io, cudaStream_t s) {
   return run_io(L, v, s);
 }
 
-// The chunk layers: the same layer on batch N / k (k = 4, or 2, when it divides N and the
-// copies are large enough to be worth overlapping); their errors go to the parent's word.
 // Image chunks of a host-buffer forward: 4 (else 2) when that divides the batch and keeps
 // every chunk's copies at 2 MB or more.  With k chunks the copies in and out overlap except
 // for about 1/k of the transfer at either end, and each chunk adds its launch and copy
@@ -933,6 +931,8 @@ void clear_chunks(Layer& L) {
   L.chunks.clear();
 }
 
+// The chunk layers: the same layer on batch N / k, set up from the kept host parameters; the
+// first owns the device weights, the others read them, and all report to the parent's error word.
 bconv_status_t make_chunks(Layer& L, int k) {
   clear_chunks(L);
   for (int i = 0; i < k; ++i) {
