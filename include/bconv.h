@@ -207,11 +207,12 @@ int32_t bconv_effective_algo(bconv_handle_t h);
  * (process-wide; a layer keeps what it was created with, and its weights are laid out for it).
  *   SINGLE  one CTA per 128-pixel tile on one SM; each weight stage is one bulk copy.
  *   PAIR    a cluster of two CTAs per 256-pixel tile (tcgen05 cta_group::2), each CTA
- *           loading half of every weight stage; an FC needs batch > 128 for it.
- *   AUTO    PAIR for an FC with batch > 128; PAIR for a convolution when the busiest SM of
- *           the pair plan runs under 95 % of the k-block stages of the busiest SM of the
- *           one-SM plan (e.g. where the pairs' balanced split evens out a ragged last wave);
- *           otherwise SINGLE.
+ *           loading half of every weight stage; an FC needs batch > 128 for it.  XNOR/AND
+ *           layers then use int8 codes (see bconv_set_tc_codes).
+ *   AUTO    SINGLE for e2m1 codes.  Otherwise PAIR for an FC with batch > 128, and PAIR for a
+ *           convolution when the busiest SM of the pair plan runs under 95 % (binaryWeights:
+ *           80 %) of the k-block stages of the busiest SM of the one-SM plan (e.g. where the
+ *           pairs' balanced split evens out a ragged last wave); otherwise SINGLE.
  * A forced family that the layer or device cannot use falls back to the other one.
  * Returns INVALID_ARG for an unknown mode.
  */
