@@ -1427,7 +1427,7 @@ bconv_status_t bconv_check_wait_timeout(double limit_ms) {
 }
 
 bconv_status_t bconv_measure_peak(int32_t kind, double* ops_per_s, double* sm_mhz) {
-  if (kind < 0 || kind > 6 || !ops_per_s) return BCONV_ERR_INVALID_ARG;
+  if (kind < 0 || kind > 7 || !ops_per_s) return BCONV_ERR_INVALID_ARG;
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
     cudaGetLastError();

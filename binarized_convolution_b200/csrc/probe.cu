@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(kProbeThreads) b1mma_probe(int iters, uint32_t
 // on zero operands or (kRandom) on pseudo-random +-1 operands -- int8 0x01 / 0xFF, bf16 +1 / -1
 // -- like the contraction's.  One thread issues `iters` groups of 4 MMAs into one TMEM
 // accumulator and waits for them through tcgen05.commit (bounded wait).
-template <bool kI8, bool kRandom>
+template <bool kI8, bool kRandom, bool kF4 = false>
 __global__ void __launch_bounds__(128, 1) tcgen05_probe(int iters, uint32_t* out, long long* cycles, uint32_t* err) {
   using namespace tcdev;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -128,7 +128,9 @@ __global__ void __launch_bounds__(128, 1) tcgen05_probe(int iters, uint32_t* out
       h ^= h >> 13;
       h *= 0xC2B2AE35u;
       h ^= h >> 16;
-      if (kI8) {
+      if (kF4) {  // e2m1 +1.0 / -1.0 nibbles
+        for (int b = 0; b < 8; ++b) w |= (((h >> b) & 1u) ? 0x2u : 0xAu) << (4 * b);
+      } else if (kI8) {
         for (int b = 0; b < 4; ++b) w |= (((h >> b) & 1u) ? 0x01u : 0xFFu) << (8 * b);
       } else {
         w = (((h & 1u) ? 0x3F80u : 0xBF80u)) | (((h & 2u) ? 0x3F80u : 0xBF80u) << 16);
@@ -151,7 +153,28 @@ __global__ void __launch_bounds__(128, 1) tcgen05_probe(int iters, uint32_t* out
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = B->tmem_base;
-  if (threadIdx.x == 0) {
+  if (kF4) {  // unit block scale factors in the columns after the M128 x N128 accumulator
+    tc_fill_32x32(tmem + (static_cast<uint32_t>((threadIdx.x >> 5) * 32) << 16) + 128u, 0x7F7F7F7Fu);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  if (threadIdx.x == 0 && kF4) {
+    // kind::mxf4, e2m1 operands, M=128, N=128, K=64 per instruction
+    const uint32_t idesc = idesc_for(2, 128, 128);
+    const uint64_t da = smem_desc_sw128(sa), db = smem_desc_sw128(sb);
+    const long long t0 = clock64();
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        tc_mma_f4(tmem, da + 2u * j, db + 2u * j, idesc, (it > 0 || j > 0) ? 1u : 0u, tmem + 128u, tmem + 144u);
+    }
+    tc_commit(&B->done);
+    mbar_wait(&B->done, 0, B, err, false);
+    const long long t1 = clock64();
+    atomicMax(reinterpret_cast<unsigned long long*>(cycles), static_cast<unsigned long long>(t1 - t0));
+    out[blockIdx.x] = 1u;
+  } else if (threadIdx.x == 0) {
     // s32 (i8) or f32 (bf16) accumulator, K-major, M=128, N=256
     const uint32_t idesc = kI8 ? ((2u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((128u >> 4) << 24))
                                : ((1u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((128u >> 4) << 24));
@@ -216,7 +239,7 @@ cudaError_t wait_check(double limit_ms, uint32_t* status) {
 }
 
 cudaError_t probe_peak(int kind, double* ops_per_s, double* sm_mhz) {
-  if (kind == 3 || kind == 4 || kind == 5 || kind == 6) {
+  if (kind >= 3 && kind <= 7) {
     const int sms = current_sm_count();
     const int iters = 2048;
     const int smem = 120 * 1024;  // more than half an SM's shared memory: one CTA per SM
@@ -233,7 +256,8 @@ cudaError_t probe_peak(int kind, double* ops_per_s, double* sm_mhz) {
     auto kern = kind == 3   ? tcgen05_probe<true, false>
                 : kind == 4 ? tcgen05_probe<false, false>
                 : kind == 5 ? tcgen05_probe<true, true>
-                            : tcgen05_probe<false, true>;
+                : kind == 6 ? tcgen05_probe<false, true>
+                            : tcgen05_probe<false, true, true>;
     if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     float best = 0.f;
     long long cycles = 0;
@@ -255,7 +279,9 @@ cudaError_t probe_peak(int kind, double* ops_per_s, double* sm_mhz) {
     if (e == cudaSuccess) e = cudaMemcpy(&herr, err, sizeof(herr), cudaMemcpyDeviceToHost);
     if (e == cudaSuccess && herr) e = cudaErrorLaunchTimeout;
     if (e == cudaSuccess && best > 0.f) {
-      const double macs = static_cast<double>(sms) * iters * 4.0 * 128.0 * 256.0 * ((kind == 3 || kind == 5) ? 32.0 : 16.0);
+      const double macs = kind == 7 ? static_cast<double>(sms) * iters * 4.0 * 128.0 * 128.0 * 64.0
+                                    : static_cast<double>(sms) * iters * 4.0 * 128.0 * 256.0 *
+                                          ((kind == 3 || kind == 5) ? 32.0 : 16.0);
       if (ops_per_s) *ops_per_s = macs / (best * 1e-3);
       if (sm_mhz) *sm_mhz = static_cast<double>(cycles) / (best * 1e3);
     }

@@ -337,7 +337,9 @@ int32_t bconv_version(void);
  * mma.sync m16n8k256 .xor.popc (bit multiply-accumulates/s), 3 = tcgen05.mma kind::i8
  * M128 N256 K32 from shared memory into TMEM (multiply-accumulates/s), 4 = tcgen05.mma
  * kind::f16 with bf16 operands, M128 N256 K16 (multiply-accumulates/s); kinds 3 and 4 run on
- * zero operands, 5 and 6 are the same on pseudo-random +-1 operands.  Runs a few short kernels
+ * zero operands, 5 and 6 are the same on pseudo-random +-1 operands; 7 = tcgen05.mma
+ * kind::mxf4 on pseudo-random e2m1 +-1.0 operands with unit block scales, M128 N128 K64
+ * (multiply-accumulates/s).  Runs a few short kernels
  * (milliseconds) and waits for them.  *sm_mhz receives the SM clock the kernels saw,
  * derived from clock64() over the event-timed interval (may be NULL).
  */
