@@ -313,3 +313,27 @@ def test_bit_output_replans_wide_e2m1_layer_on_int8(cuda_device):
         assert layer.tc_codes() == bc.CODES_FP4  # one tile: nothing to add across items
     finally:
         layer.close()
+
+
+E2M1_CASES = [
+    # channel counts around the e2m1 layout (two codes per byte, 256-channel rows) and the
+    # 128-channel e2m1 tiles: a full row, two rows, the byte-wise path, mostly padding
+    synth.small_case(batch=2, h=20, w=20, ni=256, no=96, k=3, op=synth.XNOR, use_beta=True, relu=True, in_terms=True,
+                     seed=61),
+    synth.small_case(batch=1, h=15, w=15, ni=512, no=128, k=1, op=synth.AND, use_beta=True, seed=62),
+    synth.small_case(batch=1, h=7, w=9, ni=1000, no=40, k=3, op=synth.XNOR, in_terms=True, seed=63),
+    synth.small_case(batch=2, h=11, w=13, ni=20, no=200, k=5, stride=2, op=synth.AND, use_beta=True, relu=True,
+                     in_terms=True, seed=64),
+]
+
+
+@pytest.mark.parametrize("w", E2M1_CASES, ids=lambda w: w.name)
+def test_e2m1_code_layouts(w, cuda_device):
+    """Layers whose codes take the e2m1 layout's different paths, against the oracle on every
+    family (the library's choice is e2m1 here)."""
+    layer = pu.make_layer(w, synth.make_inputs(w))
+    try:
+        assert layer.tc_codes() == bc.CODES_FP4
+    finally:
+        layer.close()
+    _check(w)
