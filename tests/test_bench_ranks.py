@@ -70,3 +70,27 @@ def test_warmup_below_three_is_rejected():
 
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2"])
+
+
+def test_forcing_options_are_validated():
+    """--cta and --codes take only the library's settings (checked before any device work)."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    for bad in (["--cta", "both"], ["--codes", "int4"]):
+        with pytest.raises(SystemExit):
+            bench.main(bad)
+
+
+def test_fp4_peak_is_twice_the_int8_peak():
+    """The e2m1 (kind::mxf4) roofline is the int8 one doubled (nominal 9 / 4.5 PFLOP/s)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from binarized_convolution_b200 import synth
+
+    w = synth.workload("xnor_beta_n16_56x56_c256_k256_3x3")
+    p_int8, bound8, _ = bench.derived_peak(w, 148, 1965.0, "tc_conv", 1)
+    p_fp4, bound4, how = bench.derived_peak(w, 148, 1965.0, "tc_conv", bench.CODES_FP4)
+    assert bound8 == bound4 == "tensor"
+    assert p_fp4 == pytest.approx(2 * p_int8)
+    assert "fp4" in how
