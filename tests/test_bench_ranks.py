@@ -94,3 +94,34 @@ def test_fp4_peak_is_twice_the_int8_peak():
     assert bound8 == bound4 == "tensor"
     assert p_fp4 == pytest.approx(2 * p_int8)
     assert "fp4" in how
+
+
+def test_timed_region_fills_the_seconds_whatever_the_step_count():
+    """The timed region holds at least --steps steps and enough to fill the requested device time;
+    the contraction sampling keeps at least three timed launches."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert bench.timed_step_count(20, 0.044, 2.0) == 45455  # 2 s of 44 us steps
+    assert bench.timed_step_count(100000, 0.044, 2.0) == 100000
+    assert bench.timed_step_count(20, 50.0, 2.0) == 40
+    assert bench.profile_stride(45455) == bench.PROFILE_EVERY
+    assert bench.profile_stride(9) == 3 and bench.profile_stride(2) == 1
+
+
+def test_forward_roofline_is_the_slower_of_bytes_and_ops():
+    """Whole-step roofline: algorithmic bytes (fp32 in + packed weight bits + fp32 out) over HBM
+    against nominal ops over the pipe's peak."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from binarized_convolution_b200 import synth
+
+    w = synth.workload("xnor_beta_n16_56x56_c256_k256_3x3")
+    b = bench.algorithmic_bytes(w)
+    assert b == 16 * 56 * 56 * 256 * 4 * 2 + 256 * 9 * 8 * 4
+    gbs, _ = bench.hbm_peak()
+    r = bench.forward_roofline(w, step_ms=0.05, pipe_peak_tops=1e6)  # ops cost nothing: HBM-bound
+    assert r["bound"] == "hbm" and r["t_roof_us"] == pytest.approx(b / (gbs * 1e3))
+    assert r["frac"] == pytest.approx(r["t_roof_us"] / 50.0)
+    r = bench.forward_roofline(w, step_ms=1.0, pipe_peak_tops=1.0)  # 1 TOPS: ops-bound
+    assert r["bound"] == "tensor" and r["t_roof_us"] == pytest.approx(w.nominal_ops / 1e12 * 1e6)
