@@ -27,6 +27,9 @@ whole step with max(algorithmic bytes / HBM bandwidth, ops / pipe peak).  ``cloc
 from NVML reads every 5 ms during the timed region (read only; no setting is changed).
 ``e2e`` is the same metric through bconv_forward_host / bfc_forward_host with page-locked
 host buffers (host-to-device copy, forward, device-to-host copy inside every step).
+Two CPU figures sit beside it: ``cpu_baseline``, the oracle (plain double-precision loops) on
+a sample of output rows, and ``cpu_simd_baseline``, the vectorised CPU implementation in
+cpu_simd/ (bit-packed XOR / AND + popcount on AVX-512 or AVX2 registers) on the whole workload.
 
 ``--io bits`` times one workload as the middle of a chain of such layers instead: it reads
 the bit-packed output of the previous layer (sign bits and A) and writes its own for the next
@@ -361,6 +364,37 @@ def oracle_sample_rate(w: synth.Workload, inp, target_s: float, rng_seed: int = 
     return n * ops_per_row / dt / 1e12, dt, n, threads
 
 
+def simd_baseline_record(w: synth.Workload, inp, seconds: float) -> dict:
+    """The vectorised CPU baseline (cpu_simd/: bit-packed XOR / AND + popcount on AVX-512 or AVX2,
+    OpenMP) on the whole workload, repeated for about `seconds`."""
+    import binarized_convolution_b200 as bc
+    import cpu_simd
+
+    t = {synth.XNOR: cpu_simd.XNOR, synth.AND: cpu_simd.AND, synth.BINARY_WEIGHTS: cpu_simd.BINARY_WEIGHTS}[w.op]
+    packed = bc.bconv_pack_bits(inp.wbits.reshape(-1, w.in_channels)).reshape(*inp.wbits.shape[:3], -1)
+    kw = dict(type=t, scale=inp.scale, bias=inp.bias, in_scale=inp.in_scale, in_bias=inp.in_bias,
+              use_beta=w.use_beta, relu=w.relu)
+
+    def run():
+        if w.kind == "fc":
+            cpu_simd.fc(inp.x, packed, **kw)
+        else:
+            cpu_simd.conv(inp.x, packed, stride=(w.stride_y, w.stride_x), **kw)
+
+    run()  # first call builds and warms up
+    t0 = time.perf_counter()
+    run()
+    one = time.perf_counter() - t0
+    reps = max(1, int(seconds / max(one, 1e-6)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        run()
+    dt = time.perf_counter() - t0
+    return {"value": w.nominal_ops * reps / dt / 1e12, "unit": UNIT, "cores": cpu_simd.num_threads(),
+            "kind": f"simd ({cpu_simd.ISA_NAMES[cpu_simd.best_isa()]})", "ms_per_step": dt * 1e3 / reps,
+            "sample": f"the whole workload x {reps}, {dt:.1f} s"}
+
+
 def cpu_baseline_record(w: synth.Workload, inp, seconds: float) -> dict:
     v, dt, n, thr = oracle_sample_rate(w, inp, target_s=seconds)
     return {"value": v, "unit": UNIT, "cores": thr, "kind": "oracle",
@@ -562,6 +596,7 @@ def measure_workload(args, w: synth.Workload, device, bits_io: bool = False, cpu
 
     if rank == 0 and world == 1 and cpu_seconds > 0:
         rec["cpu_baseline"] = cpu_baseline_record(w, inp, cpu_seconds)
+        rec["cpu_simd_baseline"] = simd_baseline_record(w, inp, args.simd_seconds)
     torch.cuda.empty_cache()
     return rec
 
@@ -601,13 +636,14 @@ def run_native(args):
         "config": h["config"], "images_per_s": h["images_per_s"], "roofline": h["roofline"],
         "forward_roofline": h["forward_roofline"], "clocks": h["clocks"], "gpu_launches": h["gpu_launches"],
     }
-    for k in ("e2e", "cpu_baseline"):
+    for k in ("e2e", "cpu_baseline", "cpu_simd_baseline"):
         if k in h:
             result[k] = h[k]
     if len(recs) > 1:
         result["workloads"] = {
             n: {k: r[k] for k in ("value", "ms_per_step", "steps", "images_per_s", "dtype", "roofline",
-                                  "forward_roofline", "clocks", "gpu_launches", "e2e", "cpu_baseline") if k in r}
+                                  "forward_roofline", "clocks", "gpu_launches", "e2e", "cpu_baseline",
+                                  "cpu_simd_baseline") if k in r}
             for n, r in recs.items()}
         result["total_gpu_launches"] = sum(r["gpu_launches"] for r in recs.values())
     if rank == 0:
@@ -689,6 +725,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time of the headline's cpu_baseline")
     ap.add_argument("--cpu-seconds-other", type=float, default=3.0,
                     help="oracle time of the other workloads' cpu_baseline")
+    ap.add_argument("--simd-seconds", type=float, default=2.0,
+                    help="time of each workload's vectorised CPU baseline (cpu_simd_baseline)")
     ap.add_argument("--reference-seconds", type=float, default=120.0, help="oracle time budget of --impl reference")
     args = ap.parse_args(argv)
     if args.warmup < 3:
