@@ -137,6 +137,17 @@ struct Layer {
   int8_t* wq = nullptr;
   float* ws = nullptr;  // FC split-K partial sums [N][No]
   TcArgs tc{};
+  // Rows-staged contraction (tc_halo_kernel): codes in a zero-bordered grid, its plan
+  bool halo = false;
+  bool halo2 = false;     // the rows-staged contraction on SM pairs (tc_halo2_kernel)
+  bool halo_off = false;  // set when a bit-packed output needs the per-tap kernel instead
+  HaloArgs hx{};
+  PadMap pad{};
+  float* A_pad = nullptr;  // A in the zero-bordered grid (rows-staged layers with beta)
+  // Fully-connected contraction with 256-channel items (tc_fc_kernel): its plan and counters
+  bool fcb = false;
+  FcArgs fx{};
+  uint32_t* fc_count = nullptr;
   CUtensorMap tmA{}, tmB{}, tmBp{}, tmWs{}, tmOut{};
   const float* tm_out_ptr = nullptr;
   // chained layers: the next layer's input terms (bit-packed output) and what emitting the
@@ -186,6 +197,29 @@ namespace {
 
 bool valid_type(int t) { return t == kBinaryWeights || t == kXnor || t == kAnd; }
 
+}  // namespace
+
+bconv_status_t check_conv_shape(const bconv_desc_t* d) {
+  if (d->neuron != BCONV_NEURON_NONE && d->neuron != BCONV_NEURON_RELU) return BCONV_ERR_INVALID_ARG;
+  if (d->batch < 0 || d->in_h <= 0 || d->in_w <= 0 || d->in_channels <= 0 || d->out_channels <= 0 ||
+      d->kernel_h <= 0 || d->kernel_w <= 0 || d->stride_y <= 0 || d->stride_x <= 0 || d->groups <= 0)
+    return BCONV_ERR_INVALID_ARG;
+  if (d->groups != 1) return BCONV_ERR_UNSUPPORTED;
+  // a window wider than twice the image plus one has taps that no output can reach; the bounds
+  // are tested one by one (in 64 bits) before any product is formed
+  if (static_cast<int64_t>(d->kernel_h) > 2 * static_cast<int64_t>(d->in_h) + 1 ||
+      static_cast<int64_t>(d->kernel_w) > 2 * static_cast<int64_t>(d->in_w) + 1 || d->kernel_h > 4096 ||
+      d->kernel_w > 4096)
+    return BCONV_ERR_UNSUPPORTED;
+  const int64_t taps = static_cast<int64_t>(d->kernel_h) * d->kernel_w;
+  if (taps > 4096 || d->in_channels > (1 << 20) || d->out_channels > (1 << 20)) return BCONV_ERR_UNSUPPORTED;
+  // the integer window sums (at most taps x in_channels in magnitude) must fit int32
+  if (taps * d->in_channels > INT32_MAX) return BCONV_ERR_UNSUPPORTED;
+  return BCONV_OK;
+}
+
+namespace {
+
 // cuTensorMapEncodeTiled from the driver, found through the runtime (the library does not
 // link the driver library, so it loads on machines without one).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -203,7 +237,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // 4-D tiled map, dims innermost first, 128-byte swizzle, out-of-range elements read as 0.
 bool encode_4d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, const uint64_t dims[4],
-               const uint64_t strides_bytes[3], const uint32_t box[4], const uint32_t elem_strides[4] = nullptr) {
+               const uint64_t strides_bytes[3], const uint32_t box[4], const uint32_t elem_strides[4] = nullptr,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint32_t estr[4] = {1, 1, 1, 1};
@@ -211,20 +246,20 @@ bool encode_4d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, const u
     for (int i = 0; i < 4; ++i) estr[i] = elem_strides[i];
   return enc(m, dt, 4, const_cast<void*>(base), reinterpret_cast<const cuuint64_t*>(dims),
              reinterpret_cast<const cuuint64_t*>(strides_bytes), reinterpret_cast<const cuuint32_t*>(box), estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1, uint64_t stride1,
-               uint32_t b0, uint32_t b1) {
+               uint32_t b0, uint32_t b1, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t dims[2] = {d0, d1};
   const cuuint64_t strides[1] = {stride1};
   const cuuint32_t box[2] = {b0, b1};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -234,11 +269,10 @@ int next_pow2(int v) {
   return p;
 }
 
-// Output map over `out` ([N][Ho][Wo][No] fp32) with the tile's box.
+// Output map over `out` ([N][Ho][Wo][No] fp32) with the tile's box: 32 channels x Cw x R x Bn.
 bool encode_out_map(Layer& L, CUtensorMap* m, const float* out) {
-  const uint64_t dims[4] = {static_cast<uint64_t>(L.No), static_cast<uint64_t>(L.Ho), static_cast<uint64_t>(L.Wo),
-                            static_cast<uint64_t>(L.N)};
-  uint64_t d[4] = {dims[0], dims[2], dims[1], dims[3]};  // {No, Wo, Ho, N}
+  const uint64_t d[4] = {static_cast<uint64_t>(L.No), static_cast<uint64_t>(L.Wo), static_cast<uint64_t>(L.Ho),
+                         static_cast<uint64_t>(L.N)};
   const uint64_t row = static_cast<uint64_t>(L.No) * 4;
   const uint64_t strides[3] = {row, row * L.Wo, row * L.Wo * L.Ho};
   const uint32_t box[4] = {32, static_cast<uint32_t>(L.tc.Cw), static_cast<uint32_t>(L.tc.R),
@@ -253,6 +287,7 @@ bool encode_out_map(Layer& L, CUtensorMap* m, const float* out) {
 // Kernel family and operand codes for layers created from now on (BCONV_CTA_*, BCONV_CODES_*).
 std::atomic<int> g_cta_mode{BCONV_CTA_AUTO};
 std::atomic<int> g_tc_codes{BCONV_CODES_AUTO};
+std::atomic<int> g_staging{BCONV_STAGING_AUTO};
 
 // k-block stages on the busiest SM under each family's plan (the plans' own work lists).
 double plan_stages_single(TcArgs t, int sms) {
@@ -273,6 +308,74 @@ double plan_stages_pair(TcArgs t, int pairs) {
   return static_cast<double>((items + grid_pairs - 1) / grid_pairs) * kb;
 }
 
+// The FC on e2m1 codes with 256-channel items (tc_fc_kernel).  Weight row c (output channel,
+// rows padded to 256 per tile) holds, per pixel, cip codes as cip / 2 bytes: the layer's bits as
+// +1.0 / -1.0 (XNOR) or 1.0 / 0 (AND), channel 2j in the low nibble, zero codes past Ni.
+bconv_status_t setup_fc(Layer& L, const uint32_t* packed) {
+  FcArgs& f = L.fx;
+  f = FcArgs{};
+  const int hw = L.H * L.W;
+  const int64_t px_bytes = L.cip / 2;
+  f.N = L.N;
+  f.No = L.No;
+  f.hw = hw;
+  f.kb_total = hw * (L.cip / 256);
+  tc_fc_plan(f, current_sm_count());
+  const int64_t rows = static_cast<int64_t>(f.n_tiles) * 256;
+  const int64_t row_bytes = static_cast<int64_t>(hw) * px_bytes;
+  const Layer* src = L.weights_from;
+  const bool borrowed = src && src->fcb && src->wq && src->fx.n_tiles == f.n_tiles && src->fx.kb_total == f.kb_total;
+  cudaError_t e = cudaSuccess;
+  if (borrowed) {
+    L.wq = src->wq;
+  } else {
+    const uint8_t neg = (L.type == kXnor) ? 0xAu : 0x0u;  // e2m1 -1.0, or 0
+    std::vector<uint8_t> hb(static_cast<size_t>(rows * row_bytes), 0u);
+    for (int c = 0; c < L.No; ++c)
+      for (int p = 0; p < hw; ++p) {
+        uint8_t* dst = hb.data() + static_cast<size_t>(c) * row_bytes + static_cast<int64_t>(p) * px_bytes;
+        for (int f0 = 0; f0 < L.Ni; ++f0) {
+          const uint32_t word = packed[(static_cast<int64_t>(c) * hw + p) * L.nw + f0 / kWordBits];
+          const uint8_t code = ((word >> (f0 % kWordBits)) & 1u) ? 0x2u : neg;
+          dst[f0 / 2] |= static_cast<uint8_t>(code << (4 * (f0 % 2)));
+        }
+      }
+    e = L.tc_mem.alloc(&L.wq, hb.size());
+    if (e == cudaSuccess) e = cudaMemcpy(L.wq, hb.data(), hb.size(), cudaMemcpyHostToDevice);
+  }
+  if (e == cudaSuccess) e = L.tc_mem.alloc(&L.codes, static_cast<size_t>(L.N) * row_bytes);
+  if (e == cudaSuccess && f.k_splits > 1) e = L.tc_mem.alloc(&L.ws, static_cast<size_t>(L.N) * L.No);
+  if (e == cudaSuccess && f.k_splits > 1) e = cudaMemset(L.ws, 0, sizeof(float) * static_cast<size_t>(L.N) * L.No);
+  if (e == cudaSuccess && f.k_splits > 1)
+    e = L.tc_mem.alloc(&L.fc_count, static_cast<size_t>(f.m_tiles) * f.n_tiles);
+  if (e == cudaSuccess && f.k_splits > 1)
+    e = cudaMemset(L.fc_count, 0, sizeof(uint32_t) * static_cast<size_t>(f.m_tiles) * f.n_tiles);
+  if (e != cudaSuccess) return from_cuda(e);
+  bool ok = encode_2d(&L.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.codes, static_cast<uint64_t>(row_bytes),
+                      static_cast<uint64_t>(L.N), static_cast<uint64_t>(row_bytes), 128, 128);
+  ok = ok && encode_2d(&L.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(row_bytes),
+                       static_cast<uint64_t>(rows), static_cast<uint64_t>(row_bytes), 128, 256);
+  if (ok && f.k_splits > 1)
+    ok = encode_2d(&L.tmWs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.ws, static_cast<uint64_t>(L.No),
+                   static_cast<uint64_t>(L.N), static_cast<uint64_t>(L.No) * 4, 32, 128);
+  if (!ok) return BCONV_OK;  // the POPC path stays available
+  f.scale = L.scale;
+  f.bias = L.bias;
+  f.relu = L.relu;
+  f.err = L.err;
+  f.ws = L.ws;
+  f.count = L.fc_count;
+  L.tc.kind = 2;
+  L.tc.BN = 256;
+  L.tc.n_tiles = f.n_tiles;
+  L.tc.k_splits = f.k_splits;
+  L.tc.N = L.N;
+  L.tc.No = L.No;
+  L.fcb = true;
+  L.tc_ok = true;
+  return BCONV_OK;
+}
+
 bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   if (L.No % 4 != 0 || L.N == 0) return BCONV_OK;
   if (!tensor_map_encoder()) return BCONV_OK;
@@ -283,7 +386,16 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   // (kind 1).
   const int mode = g_cta_mode.load();
   const int codes = L.codes_override >= 0 ? L.codes_override : g_tc_codes.load();
-  t.kind = L.type == kBinaryWeights ? 1 : (codes == BCONV_CODES_INT8 || mode == BCONV_CTA_PAIR) ? 0 : 2;
+  // An XNOR / AND window sum adds up to (reduction length) terms of magnitude 1.  fp32 adds
+  // such integers exactly only below 2^24: beyond that the e2m1 path (fp32 accumulators) and the
+  // FC's split reduction (fp32 reduce-add) could round, so such layers keep int32 sums -- int8
+  // codes with s32 accumulators for a convolution, the POPC family (int32 split sums) for an FC.
+  const int64_t red_len = L.fc ? static_cast<int64_t>(L.H) * L.W * L.Ni : static_cast<int64_t>(taps) * L.Ni;
+  const bool fp32_exact = red_len <= (int64_t{1} << 24);
+  if (L.type != kBinaryWeights && !fp32_exact && L.fc) return BCONV_OK;
+  t.kind = L.type == kBinaryWeights                                                   ? 1
+           : (codes == BCONV_CODES_INT8 || mode == BCONV_CTA_PAIR || !fp32_exact) ? 0
+                                                                                   : 2;
   // channels per part, padded to whole 128-byte rows; bytes of activation operand per pixel
   // (kind 1: three bf16 parts) and of weights per output channel and tap (kind 1: one bf16
   // copy, which every part is multiplied with; kind 2: two codes per byte)
@@ -293,6 +405,8 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   t.kb_px = bpb / 128;
   t.px_bytes = bpp;
   t.part_bytes = t.kind == 1 ? 2 * L.cip : 0;
+  L.fcb = false;
+  if (L.fc && t.kind == 2) return setup_fc(L, packed);
   // The FC runs on SM pairs when its batch fills both CTAs of a pair (256 images per pair
   // tile, so the weight matrix streams from memory once, with half of every weight tile per
   // SM); otherwise a single SM keeps up to 256 images in one tile (two 128-row sub-tiles
@@ -379,6 +493,37 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   t.stages = pairs > 0 ? tc2_stages(t.kind, t.BN) : tc_stages(t.kind, t.BN, t.mt);
   if (t.stages < 2) return BCONV_OK;  // no room for a pipeline: the SIMT family stays
 
+  // Rows-staged contraction: e2m1 codes, stride 1, image rows that fit a tile (kernel
+  // tc_halo_kernel); its codes live in a zero-bordered grid
+  L.halo = false;
+  L.halo2 = false;
+  L.pad = PadMap{};
+  const int staging = g_staging.load();
+  if (t.kind == 2 && !L.fc && L.sy == 1 && L.sx == 1 && pairs == 0 && !L.halo_off &&
+      staging != BCONV_STAGING_PER_TAP) {
+    HaloArgs& h = L.hx;
+    h = HaloArgs{};
+    h.N = L.N; h.H = L.H; h.W = L.W; h.kh = L.kh; h.kw = L.kw;
+    h.Hp = L.H + L.kh - 1;
+    h.Wp = L.W + L.kw - 1;
+    h.kb_per_tap = t.kb_per_tap;
+    h.BN = t.BN; h.n_tiles = t.n_tiles; h.No = L.No;
+    // more than 128 output channels: SM pairs with 256-channel MMAs (each SM's MMAs then run
+    // at the tensor pipe's rate); else one SM per 128-slot tile
+    HaloArgs h2 = h;
+    if (mode != BCONV_CTA_SINGLE && tc_halo2_plan(h2, 0)) {
+      h = h2;
+      L.halo = true;
+      L.halo2 = true;
+    } else if (mode != BCONV_CTA_PAIR && tc_halo_plan(h, current_sm_count())) {
+      L.halo = true;
+    }
+    if (L.halo) {
+      L.pad = PadMap{L.H, L.W, h.Hp, h.Wp, L.kh / 2, L.kw / 2};
+      t.BN = h.BN;  // the plan may narrow (one SM) or widen (pairs) the tiles
+      t.n_tiles = h.n_tiles;
+    }
+  }
   // Weights [no_tc][taps][bpb bytes]: kind 0 int8 +-1 (XNOR) or 0/1 (AND); kind 1 bf16 +-1.
   // Every padding slot is 0.
   const int no_tc = t.n_tiles * t.BN;
@@ -404,7 +549,7 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
           memcpy(row + 2 * f, &v, 2);
         }
       }
-  if (pairs == 0 && !borrowed) {
+  if (pairs == 0 && !L.halo2 && !borrowed) {
     // the one-SM kernel copies each (N tile, k-block) stage of BN rows x 128 bytes as one
     // block: lay the blocks out contiguously with the 128-byte swizzle already applied
     const int kbt = static_cast<int>(kt / 128);
@@ -418,7 +563,7 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
         }
     hq.swap(tiles);
   }
-  const int64_t npix = static_cast<int64_t>(L.N) * L.H * L.W;
+  const int64_t npix = L.halo ? static_cast<int64_t>(L.N) * L.hx.Hp * L.hx.Wp : static_cast<int64_t>(L.N) * L.H * L.W;
   cudaError_t e = cudaSuccess;
   if (borrowed) {
     L.wq = src->wq;
@@ -427,12 +572,23 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
     if (e == cudaSuccess) e = cudaMemcpy(L.wq, hq.data(), hq.size(), cudaMemcpyHostToDevice);
   }
   if (e == cudaSuccess) e = L.tc_mem.alloc(&L.codes, static_cast<size_t>(npix) * bpp);
+  // the border of the padded grid is written once, here, and never again
+  if (e == cudaSuccess && L.halo) e = cudaMemset(L.codes, 0, static_cast<size_t>(npix) * bpp);
+  if (e == cudaSuccess && L.halo && L.use_beta()) e = L.tc_mem.alloc(&L.A_pad, static_cast<size_t>(npix));
+  if (e == cudaSuccess && L.halo && L.use_beta()) e = cudaMemset(L.A_pad, 0, sizeof(float) * static_cast<size_t>(npix));
   if (e == cudaSuccess && t.k_splits > 1) e = L.tc_mem.alloc(&L.ws, static_cast<size_t>(L.N) * L.No);
   if (e == cudaSuccess && t.k_splits > 1) e = cudaMemset(L.ws, 0, sizeof(float) * static_cast<size_t>(L.N) * L.No);
   if (e != cudaSuccess) return from_cuda(e);
 
   bool ok = true;
-  if (L.fc) {
+  if (L.halo) {
+    ok = encode_2d(&L.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.codes, static_cast<uint64_t>(bpp),
+                   static_cast<uint64_t>(npix), static_cast<uint64_t>(bpp), 128,
+                   static_cast<uint32_t>(L.hx.halo_rows));
+    if (L.halo2)  // each CTA of a pair reads its 128 rows of a 256-row weight tile
+      ok = ok && encode_2d(&L.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(kt),
+                           static_cast<uint64_t>(no_tc), static_cast<uint64_t>(kt), 128, 128);
+  } else if (L.fc) {
     const uint64_t K = static_cast<uint64_t>(L.H) * L.W * bpp;
     const uint64_t dims[4] = {K, 1, 1, static_cast<uint64_t>(L.N)};
     const uint64_t strides[3] = {K, K, K};
@@ -470,6 +626,11 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   } else {
     t.grid_ctas = tc_plan(t, current_sm_count());  // work list: tail tiles cut along N
     t.b_tiles = L.wq;
+    L.hx.b_tiles = L.wq;
+    L.hx.scale = L.scale;
+    L.hx.bias = L.bias;
+    L.hx.relu = L.relu;
+    L.hx.err = L.err;
   }
   if (ok && t.k_splits > 1) ok = encode_out_map(L, &L.tmWs, L.ws);
   if (!ok) return BCONV_OK;  // the POPC path stays available
@@ -646,8 +807,12 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
   const float* A = io.in_bits ? io.in_a : L.A;
   cudaError_t e;
   if (io.in_bits) {
-    e = (L.tc.kind == 2 ? launch_unpack_bits_f4 : launch_unpack_bits_i8)(
-        io.in_bits, static_cast<int64_t>(L.N) * L.H * L.W, L.Ni, L.cip, L.type, L.codes, s);
+    e = L.tc.kind == 2 ? launch_unpack_bits_f4(io.in_bits, static_cast<int64_t>(L.N) * L.H * L.W, L.Ni, L.cip,
+                                               L.type, L.codes, s, L.pad)
+                       : launch_unpack_bits_i8(io.in_bits, static_cast<int64_t>(L.N) * L.H * L.W, L.Ni, L.cip,
+                                               L.type, L.codes, s);
+    if (e == cudaSuccess && L.halo && beta)  // the caller's A into the padded grid the kernel reads
+      e = launch_pad_copy(io.in_a, static_cast<int64_t>(L.N) * L.H * L.W, L.pad, L.A_pad, s);
   } else if (L.tc.kind != 1) {
     PackI8Args p{};
     p.in = in;
@@ -657,9 +822,10 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
     p.in_scale = L.in_scale;
     p.in_bias = L.in_bias;
     p.codes = L.codes;
-    p.A = beta ? L.A : nullptr;
+    p.A = beta ? (L.halo ? L.A_pad : L.A) : nullptr;  // A follows the codes into the padded grid
     p.op = L.type;
     p.f4 = L.tc.kind == 2;
+    p.pad = L.pad;
     e = launch_pack_i8(p, s);
   } else {
     PackBf16x3Args p{};
@@ -674,6 +840,22 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
     e = launch_pack_bf16x3(p, s);
   }
   if (e != cudaSuccess) return from_cuda(e);
+  if (L.fcb) {  // the FC kernel forms beta and finishes split tiles in its own epilogue
+    FcArgs f = L.fx;
+    f.A = beta ? A : nullptr;
+    f.out = out;
+    if (out != L.tm_out_ptr) {
+      if (!encode_2d(&L.tmOut, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, out, static_cast<uint64_t>(L.No),
+                     static_cast<uint64_t>(L.N), static_cast<uint64_t>(L.No) * 4, 32, 128))
+        return BCONV_ERR_CUDA;
+      L.tm_out_ptr = out;
+    }
+    const bool timed = L.prof.take();
+    if (timed) cudaEventRecord(L.prof.start[L.prof.used], s);
+    e = launch_tc_fc(&L.tmA, &L.tmB, &L.tmWs, &L.tmOut, f, s);
+    if (timed) cudaEventRecord(L.prof.stop[L.prof.used++], s);
+    return from_cuda(e);
+  }
   // the convolution forms beta from A inside its epilogue, a split FC inside the finalize
   if (beta && L.fc && L.tc.k_splits == 1) {
     BetaArgs b{A, L.beta, L.N, L.H, L.W, L.Ho, L.Wo, L.kh, L.kw, L.sy, L.sx};
@@ -697,7 +879,7 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
     om = &L.tmOut;
   } else if (t.k_splits > 1) {
     // the workspace is zero: at allocation, then as each finalize reads it
-  } else {
+  } else if (!L.halo) {  // the rows-staged kernel stores without a tensor map
     if (out != L.tm_out_ptr) {
       if (!encode_out_map(L, &L.tmOut, out)) return BCONV_ERR_CUDA;
       L.tm_out_ptr = out;
@@ -706,7 +888,14 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
   }
   const bool timed = L.prof.take();
   if (timed) cudaEventRecord(L.prof.start[L.prof.used], s);
-  e = L.tc_pair ? launch_tc_conv2(&L.tmA, &L.tmB, &L.tmBp, om, t, s) : launch_tc_conv(&L.tmA, om, t, s);
+  if (L.halo) {
+    HaloArgs h = L.hx;
+    h.A = beta ? L.A_pad : nullptr;
+    h.out = out;
+    e = L.halo2 ? launch_tc_halo2(&L.tmA, &L.tmB, h, s) : launch_tc_halo(&L.tmA, h, s);
+  } else {
+    e = L.tc_pair ? launch_tc_conv2(&L.tmA, &L.tmB, &L.tmBp, om, t, s) : launch_tc_conv(&L.tmA, om, t, s);
+  }
   if (timed) cudaEventRecord(L.prof.stop[L.prof.used++], s);
   if (e != cudaSuccess) return from_cuda(e);
   if (t.k_splits > 1)
@@ -824,7 +1013,10 @@ bconv_status_t run_io(Layer& L, const Io& io, cudaStream_t s) {
     p.A = io.out_a;
     return from_cuda(launch_pack(p, s));
   }
-  return use_tc(L) ? run_forward_tc(L, io, s) : run_forward_simt(L, io, s);
+  // The tensor-core kernels write the output in 16-byte pieces (TMA boxes, float4 stores); an
+  // output that is not 16-byte aligned goes to the SIMT family, which can write it.
+  const bool aligned = (reinterpret_cast<uintptr_t>(io.out) & 15u) == 0;
+  return use_tc(L) && aligned ? run_forward_tc(L, io, s) : run_forward_simt(L, io, s);
 }
 
 bconv_status_t run_forward(Layer& L, const float* in, float* out, cudaStream_t s) {
@@ -846,6 +1038,11 @@ bconv_status_t replan_tc(Layer& L, int codes) {
   L.codes = nullptr;
   L.ws = nullptr;
   L.tm_out_ptr = nullptr;
+  L.halo = false;
+  L.halo2 = false;
+  L.A_pad = nullptr;
+  L.fcb = false;
+  L.fc_count = nullptr;
   L.codes_override = codes;
   return setup_tc(L, L.h_packed.data());
 }
@@ -882,7 +1079,12 @@ bconv_status_t set_output_terms(Layer& L, const float* next_scale, const float* 
   // 16, 56 x 56, 256 -> 256 as a chain's middle layer: 53.3 us per forward on e2m1 codes
   // (two 128-channel tiles), 37.1 us on int8.
   if (L.tc_ok && L.tc.kind == 2 && !L.fc && L.tc.n_tiles > 1 && L.codes_override < 0) {
+    L.halo_off = true;
     const bconv_status_t st = replan_tc(L, BCONV_CODES_INT8);
+    if (st != BCONV_OK) return st;
+  } else if (L.halo) {  // the rows-staged kernel writes fp32 only: the per-tap kernel emits the bits
+    L.halo_off = true;
+    const bconv_status_t st = replan_tc(L, L.codes_override);
     if (st != BCONV_OK) return st;
   }
   L.has_next = true;
@@ -1025,6 +1227,7 @@ bconv_status_t sync_status(Layer& L, cudaStream_t s) {
     if (L.a_count) cudaMemset(L.a_count, 0, sizeof(uint32_t) * L.tc.m_tiles);  // an aborted launch may leave counts
     if (L.tc.sk_flag) cudaMemset(L.tc.sk_flag, 0, sizeof(uint32_t) * (L.tc.grid_ctas / 2 - 1) * 2);  // and flags
     if (L.ws) cudaMemset(L.ws, 0, sizeof(float) * static_cast<size_t>(L.N) * L.No);  // and partial sums
+    if (L.fc_count) cudaMemset(L.fc_count, 0, sizeof(uint32_t) * static_cast<size_t>(L.fx.m_tiles) * L.fx.n_tiles);
     if (word & kErrTimeout) return BCONV_ERR_TIMEOUT;
     return BCONV_ERR_CUDA;  // kErrLayout: a kernel refused an unexpected shared-memory layout
   }
@@ -1044,6 +1247,7 @@ bconv_status_t set_algo(Layer& L, int algo) {
 }
 
 int launches_per_forward(const Layer& L) {
+  if (L.N > 0 && use_tc(L) && L.fcb) return 2;  // pack, the FC kernel (which finishes its own tiles)
   if (L.N > 0 && use_tc(L))  // pack, contraction; a split FC adds the finalize, an unsplit FC with beta its mean
     return 2 + (L.tc.k_splits > 1 ? 1 : ((L.fc && L.use_beta()) ? 1 : 0));
   int n = 1;  // contraction
@@ -1129,14 +1333,8 @@ bconv_status_t bconv_create(const bconv_desc_t* d, const uint32_t* packed_weight
   *out = nullptr;
   if (!d || !packed_weights) return BCONV_ERR_INVALID_ARG;
   if (!valid_type(type) || (flags & ~static_cast<uint32_t>(BCONV_FLAG_USE_BETA_SCALING))) return BCONV_ERR_INVALID_ARG;
-  if (d->neuron != BCONV_NEURON_NONE && d->neuron != BCONV_NEURON_RELU) return BCONV_ERR_INVALID_ARG;
-  if (d->batch < 0 || d->in_h <= 0 || d->in_w <= 0 || d->in_channels <= 0 || d->out_channels <= 0 ||
-      d->kernel_h <= 0 || d->kernel_w <= 0 || d->stride_y <= 0 || d->stride_x <= 0 || d->groups <= 0)
-    return BCONV_ERR_INVALID_ARG;
-  if (d->groups != 1) return BCONV_ERR_UNSUPPORTED;
-  if (d->kernel_h > d->in_h * 2 + 1 || d->kernel_w > d->in_w * 2 + 1 || d->kernel_h * d->kernel_w > 4096 ||
-      d->in_channels > (1 << 20) || d->out_channels > (1 << 20))
-    return BCONV_ERR_UNSUPPORTED;
+  const bconv_status_t shape = check_conv_shape(d);
+  if (shape != BCONV_OK) return shape;
   bconv_handle_s* h = new (std::nothrow) bconv_handle_s();
   if (!h) return BCONV_ERR_OOM;
   h->magic = kConvMagic;
@@ -1389,12 +1587,24 @@ bconv_status_t bconv_set_cta_mode(bconv_cta_mode_t mode) {
 
 int32_t bconv_cta_mode(bconv_handle_t h) {
   if (!checked(h, kConvMagic)) return -1;
-  return h->L.tc_ok ? (h->L.tc_pair ? BCONV_CTA_PAIR : BCONV_CTA_SINGLE) : 0;
+  return h->L.tc_ok ? ((h->L.tc_pair || h->L.halo2) ? BCONV_CTA_PAIR : BCONV_CTA_SINGLE) : 0;
 }
 
 int32_t bfc_cta_mode(bfc_handle_t h) {
   if (!checked(h, kFcMagic)) return -1;
   return h->L.tc_ok ? (h->L.tc_pair ? BCONV_CTA_PAIR : BCONV_CTA_SINGLE) : 0;
+}
+
+bconv_status_t bconv_set_staging(bconv_staging_t staging) {
+  if (staging < BCONV_STAGING_AUTO || staging > BCONV_STAGING_ROWS) return BCONV_ERR_INVALID_ARG;
+  g_staging.store(staging);
+  return BCONV_OK;
+}
+
+int32_t bconv_staging(bconv_handle_t h) {
+  if (!checked(h, kConvMagic)) return -1;
+  if (!h->L.tc_ok) return 0;
+  return h->L.halo ? BCONV_STAGING_ROWS : BCONV_STAGING_PER_TAP;
 }
 
 bconv_status_t bconv_set_tc_codes(bconv_tc_codes_t codes) {

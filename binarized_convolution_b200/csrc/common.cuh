@@ -6,7 +6,14 @@
 
 #include <utility>
 
+#include "bconv.h"
+
 namespace bconv {
+
+// Shape checks of a convolution descriptor shared by every entry point that takes one (neuron,
+// positive sizes, groups == 1, window and channel limits, int32 window sums); OK, INVALID_ARG
+// or UNSUPPORTED.
+bconv_status_t check_conv_shape(const bconv_desc_t* d);
 
 enum Op : int { kBinaryWeights = 0, kXnor = 1, kAnd = 2 };
 
@@ -24,6 +31,29 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Multiprocessor count of the current device (cached per device).
 int current_sm_count();
+
+// Per-CTA timeline of a kernel's phases, for diagnosis: compiled in only when the library is
+// built with -DBCONV_TIMELINE, where BCONV_STAMP(slot) writes %globaltimer into a device array
+// (64 slots per CTA, one array per source file) that the host reads through the function
+// BCONV_TIMELINE_READER(name) defines; otherwise both are empty.
+#ifdef BCONV_TIMELINE
+static __device__ unsigned long long g_bconv_timeline[1024 * 64];  // one array per source file
+#define BCONV_TIMELINE_READER(name)                                                       \
+  extern "C" int name(unsigned long long* host, int n) {                                 \
+    return static_cast<int>(cudaMemcpyFromSymbol(host, bconv::g_bconv_timeline, sizeof(unsigned long long) * n)); \
+  }
+#define BCONV_STAMP(slot)                                                                              \
+  do {                                                                                                 \
+    unsigned long long t_;                                                                             \
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                            \
+    if (blockIdx.x < 1024) g_bconv_timeline[blockIdx.x * 64 + (slot)] = t_;                            \
+  } while (0)
+#else
+#define BCONV_TIMELINE_READER(name)
+#define BCONV_STAMP(slot) \
+  do {                    \
+  } while (0)
+#endif
 
 // Programmatic dependent launch, used by the kernels of the tensor-core forward: a kernel
 // started with launch_overlapped may be scheduled while the previous kernel of the stream is
@@ -48,6 +78,20 @@ cudaError_t launch_overlapped(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
+
+// Where pixel p = (n, y, x) of an [N][h][w] image lands in a zero-bordered [N][hp][wp] grid
+// (at (n, y + pad_t, x + pad_l)); hp == 0 means no border (the pixel keeps its index).
+struct PadMap {
+  int h, w, hp, wp, pad_t, pad_l;
+  __host__ __device__ __forceinline__ int64_t operator()(int64_t p) const {
+    if (hp == 0) return p;
+    const int64_t hw = static_cast<int64_t>(h) * w;
+    const int64_t n = p / hw;
+    const int r = static_cast<int>(p - n * hw);
+    const int y = r / w, x = r - y * w;
+    return (n * hp + y + pad_t) * wp + x + pad_l;
+  }
+};
 
 // ------------------------------------------------------------------------------------
 // Input transform, sign and pack (one pass over the fp32 input).
@@ -74,7 +118,9 @@ cudaError_t launch_unpack_bits_i8(const uint32_t* bits, int64_t npix, int ni, in
 // ... or into e2m1 (fp4) codes [npix][cip / 2] bytes, two channels per byte (XNOR: 1 -> +1.0
 // = 0x2, 0 -> -1.0 = 0xA; AND: 1 -> 0x2, 0 -> 0; channels >= ni -> 0; cip a multiple of 32).
 cudaError_t launch_unpack_bits_f4(const uint32_t* bits, int64_t npix, int ni, int cip, int op, int8_t* codes,
-                                  cudaStream_t s);
+                                  cudaStream_t s, PadMap pad = PadMap{});
+// Copy an [N][h][w] float image into the same pixels of a zero-bordered grid.
+cudaError_t launch_pad_copy(const float* src, int64_t npix, PadMap pad, float* dst, cudaStream_t s);
 
 // ------------------------------------------------------------------------------------
 // Beta: box filter of A over the window (conv) or mean of A over the image (FC).

@@ -1,12 +1,11 @@
 // bconv_forward_noalloc: an XNOR / AND convolution forward that allocates no memory.
 //
 // Who needs it: code that must not call cudaMalloc at the moment it runs a layer -- for
-// example a caller that has handed all device memory to its own pool allocator, a real-time
-// loop where an allocation could block on a device-wide synchronisation, or code running
-// while a CUDA stream is being captured into a graph, where allocation calls are not
-// allowed.  Such callers cannot create a handle (bconv_create allocates the weights and the
-// workspace), so this entry point takes every operand as caller-owned device memory and keeps
-// its working buffers in one fixed array that lives in this library's device image.
+// example a caller that has handed all device memory to its own pool allocator, or a
+// real-time loop where an allocation could block on a device-wide synchronisation.  Such
+// callers cannot create a handle (bconv_create allocates the weights and the workspace), so
+// this entry point takes every operand as caller-owned device memory and keeps its working
+// buffers in one fixed array that lives in this library's device image.
 //
 // The scratch array is `g_noalloc_scratch` below (BCONV_NOALLOC_SCRATCH_BYTES).  It is
 // allocated by the CUDA runtime when the library's module is loaded on a device and is held
@@ -15,8 +14,10 @@
 // device address is looked up once per device with cudaGetSymbolAddress, with that device
 // current, on the first call made on that device.
 //
-// It reuses the library's own kernels (pack, beta, POPC contraction) and adds one small
-// kernel that lays the caller's packed weights out for the contraction.  Every call rewrites
+// It runs the SIMT kernel family -- the library's own pack, beta and POPC contraction (int32
+// window sums), not the tensor cores, whose weight layout is prepared on the host when a layer
+// is created -- and adds one small kernel that lays the caller's packed weights out for the
+// contraction.  Every call rewrites
 // all of the scratch it reads, so nothing carries over between calls; but all calls share the
 // one array, so calls whose GPU work overlaps (two streams, or two host threads) race.
 #include <mutex>
@@ -104,14 +105,9 @@ extern "C" bconv_status_t bconv_forward_noalloc(const bconv_desc_t* d, bconv_typ
   if (!d || !packed_weights) return BCONV_ERR_INVALID_ARG;
   if (type != BCONV_TYPE_XNOR && type != BCONV_TYPE_AND) return BCONV_ERR_INVALID_ARG;
   if (flags & ~static_cast<uint32_t>(BCONV_FLAG_USE_BETA_SCALING)) return BCONV_ERR_INVALID_ARG;
-  if (d->neuron != BCONV_NEURON_NONE && d->neuron != BCONV_NEURON_RELU) return BCONV_ERR_INVALID_ARG;
-  if (d->batch < 0 || d->in_h <= 0 || d->in_w <= 0 || d->in_channels <= 0 || d->out_channels <= 0 ||
-      d->kernel_h <= 0 || d->kernel_w <= 0 || d->stride_y <= 0 || d->stride_x <= 0 || d->groups <= 0)
-    return BCONV_ERR_INVALID_ARG;
-  if (d->groups != 1) return BCONV_ERR_UNSUPPORTED;
+  const bconv_status_t shape = check_conv_shape(d);  // the same shapes bconv_create accepts
+  if (shape != BCONV_OK) return shape;
   if (d->batch > 0 && (!in || !out)) return BCONV_ERR_INVALID_ARG;
-  if (d->kernel_h * d->kernel_w > 4096 || d->in_channels > (1 << 20) || d->out_channels > (1 << 20))
-    return BCONV_ERR_UNSUPPORTED;
 
   const int N = d->batch, H = d->in_h, W = d->in_w, Ni = d->in_channels, No = d->out_channels;
   const int kh = d->kernel_h, kw = d->kernel_w, sy = d->stride_y, sx = d->stride_x;

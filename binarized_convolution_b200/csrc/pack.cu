@@ -192,6 +192,7 @@ __global__ void __launch_bounds__(kPackThreads, 2) pack_i8_vec_kernel(PackI8Args
     for (int g = 0; g < kG; ++g) {
       const int64_t p = p0 + g;
       if (p >= a.npix) break;  // warp-uniform
+      const int64_t q = a.pad(p);  // the pixel's place in the code buffer
       float asum = 0.f;
 #pragma unroll
       for (int c = 0; c < kC; ++c) {
@@ -208,13 +209,13 @@ __global__ void __launch_bounds__(kPackThreads, 2) pack_i8_vec_kernel(PackI8Args
           word = kF4 ? nibbles4<kOp>(t) : codes4<kOp>(t);
         }
         if (kF4)  // e2m1 codes: cip / 2 bytes per pixel, 64 bytes per 128-channel chunk
-          *reinterpret_cast<uint16_t*>(codes + p * (a.cip / 2) + c * 64 + lane * 2) = static_cast<uint16_t>(word);
+          *reinterpret_cast<uint16_t*>(codes + q * (a.cip / 2) + c * 64 + lane * 2) = static_cast<uint16_t>(word);
         else
-          *reinterpret_cast<uint32_t*>(codes + p * a.cip + c * 128 + lane * 4) = word;
+          *reinterpret_cast<uint32_t*>(codes + q * a.cip + c * 128 + lane * 4) = word;
       }
       if (kA) {
         asum = warp_sum(asum);
-        if (lane == 0) a.A[p] = asum / static_cast<float>(ni);
+        if (lane == 0) a.A[q] = asum / static_cast<float>(ni);  // A follows the codes' grid
       }
     }
 #pragma unroll
@@ -238,7 +239,8 @@ __global__ void __launch_bounds__(kPackThreads) pack_i8_scalar_kernel(PackI8Args
   constexpr int kPer = kF4 ? 2 : 1;  // channels per lane and step
   for (int64_t p = warp; p < a.npix; p += nwarps) {
     const float* row = a.in + p * ni;
-    int8_t* crow = a.codes + p * (a.cip / kPer);
+    const int64_t q = a.pad(p);  // the pixel's place in the code buffer (and in A)
+    int8_t* crow = a.codes + q * (a.cip / kPer);
     float asum = 0.f;
     for (int f0 = 0; f0 < a.cip; f0 += 32 * kPer) {
       uint32_t byte = 0u;
@@ -258,7 +260,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_i8_scalar_kernel(PackI8Args
     }
     if (kA) {
       asum = warp_sum(asum);
-      if (lane == 0) a.A[p] = asum / static_cast<float>(ni);
+      if (lane == 0) a.A[q] = asum / static_cast<float>(ni);
     }
   }
 }
@@ -513,17 +515,18 @@ __device__ __forceinline__ uint32_t f4_codes_of_byte(uint32_t b, int nvalid) {
 template <int kOp>
 __global__ void __launch_bounds__(256) unpack_bits_f4_kernel(const uint32_t* __restrict__ bits, uint32_t total,
                                                               uint32_t groups, int nw_in, int ni,
-                                                              uint4* __restrict__ codes) {
+                                                              uint4* __restrict__ codes, PadMap pad) {
   wait_prior_grid();
   allow_next_grid();
   for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
     const uint32_t p = i / groups;
     const int g = static_cast<int>(i - p * groups);
+    const int64_t o = pad(p) * groups + g;  // this 16-byte group's place in the code buffer
     const int c0 = g * 32;
     uint32_t word = 0;
     if (c0 < ni) word = __ldg(bits + static_cast<size_t>(p) * nw_in + g);
     const int nv = ni - c0;
-    codes[i] = make_uint4(f4_codes_of_byte<kOp>(word, nv), f4_codes_of_byte<kOp>(word >> 8, nv - 8),
+    codes[o] = make_uint4(f4_codes_of_byte<kOp>(word, nv), f4_codes_of_byte<kOp>(word >> 8, nv - 8),
                           f4_codes_of_byte<kOp>(word >> 16, nv - 16), f4_codes_of_byte<kOp>(word >> 24, nv - 24));
   }
 }
@@ -544,6 +547,16 @@ __global__ void __launch_bounds__(256) repack_bits_kernel(const uint32_t* __rest
   }
 }
 
+// src [N][h][w] -> dst at the same pixels of a zero-bordered [N][hp][wp] grid.
+__global__ void __launch_bounds__(256) pad_copy_kernel(const float* __restrict__ src, int64_t npix, PadMap pad,
+                                                        float* __restrict__ dst) {
+  wait_prior_grid();
+  allow_next_grid();
+  for (int64_t p = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; p < npix;
+       p += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    dst[pad(p)] = __ldg(src + p);
+}
+
 unsigned grid_for(int64_t threads) {
   int64_t blocks = ceil_div(threads, 256);
   const int64_t cap = static_cast<int64_t>(current_sm_count()) * 8;
@@ -553,14 +566,14 @@ unsigned grid_for(int64_t threads) {
 }  // namespace
 
 cudaError_t launch_unpack_bits_f4(const uint32_t* bits, int64_t npix, int ni, int cip, int op, int8_t* codes,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, PadMap pad) {
   if (npix == 0) return cudaSuccess;
   const int64_t total = npix * (cip / 32);
   if (total >= (int64_t{1} << 31)) return cudaErrorInvalidValue;
   const uint32_t t = static_cast<uint32_t>(total), g = static_cast<uint32_t>(cip / 32);
   uint4* out = reinterpret_cast<uint4*>(codes);
   return launch_overlapped(op == kXnor ? unpack_bits_f4_kernel<kXnor> : unpack_bits_f4_kernel<kAnd>,
-                           dim3(grid_for(total)), dim3(256), 0, s, bits, t, g, words_for(ni), ni, out);
+                           dim3(grid_for(total)), dim3(256), 0, s, bits, t, g, words_for(ni), ni, out, pad);
 }
 
 cudaError_t launch_unpack_bits_i8(const uint32_t* bits, int64_t npix, int ni, int cip, int op, int8_t* codes,
@@ -572,6 +585,11 @@ cudaError_t launch_unpack_bits_i8(const uint32_t* bits, int64_t npix, int ni, in
   uint4* out = reinterpret_cast<uint4*>(codes);
   return launch_overlapped(op == kXnor ? unpack_bits_i8_kernel<kXnor> : unpack_bits_i8_kernel<kAnd>,
                            dim3(grid_for(total)), dim3(256), 0, s, bits, t, g, words_for(ni), ni, out);
+}
+
+cudaError_t launch_pad_copy(const float* src, int64_t npix, PadMap pad, float* dst, cudaStream_t s) {
+  if (npix == 0) return cudaSuccess;
+  return launch_overlapped(pad_copy_kernel, dim3(grid_for(npix)), dim3(256), 0, s, src, npix, pad, dst);
 }
 
 cudaError_t launch_repack_bits(const uint32_t* bits, int64_t npix, int ni, int nw_pad, uint32_t* out, cudaStream_t s) {

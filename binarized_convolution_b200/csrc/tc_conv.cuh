@@ -73,6 +73,73 @@ struct TcArgs {
   const int8_t* b_tiles;
 };
 
+// Convolution with the activation rows held in shared memory (stride 1, e2m1 codes, fp32 output):
+// codes (and A) in a zero-bordered [N][Hp][Wp] grid (Hp = H + kh - 1, Wp = W + kw - 1), outputs
+// enumerated over the same grid, a tile = 128 consecutive slots, one halo load per k-block
+// serving every tap.
+struct HaloArgs {
+  int N, H, W, Hp, Wp;
+  int kh, kw;
+  int kb_per_tap;      // 128-byte k-blocks per pixel
+  int BN, n_tiles, No;
+  // filled by tc_halo_plan
+  int m_tiles;         // ceil(N * Hp * Wp / 128)
+  int halo_len;        // rows a tile's MMAs read: 128 + (kh - 1) * Wp + kw - 1
+  int halo_rows;       // rows per halo box (<= 256)
+  int halo_boxes;      // boxes per halo
+  int halo_bytes;      // shared memory per halo stage (a 1024-byte multiple)
+  int resident;        // the weights of the CTA's N tile stay in shared memory
+  int wstages;         // weight ring stages otherwise
+  int grid_ctas;       // a multiple of n_tiles
+  uint32_t tmem_cols;
+  const float* scale;
+  const float* bias;
+  const float* A;      // [N][Hp][Wp] channel means in the zero-bordered grid, or nullptr
+  int relu;
+  uint32_t* err;
+  const int8_t* b_tiles;  // [n_tiles][kh * kw * kb_per_tap][BN][128] bytes, pre-swizzled
+  float* out;             // [N][H][W][No] fp32, 16-byte aligned
+};
+bool tc_halo_plan(HaloArgs& a, int sm_count);  // false: the shape does not fit this kernel
+int tc_halo_smem_bytes(const HaloArgs& a);
+// tmA: 2-D map over the padded codes [N*Hp*Wp][bytes per pixel], box 128 bytes x halo_rows,
+// 128-byte swizzle.
+cudaError_t launch_tc_halo(const CUtensorMap* tmA, const HaloArgs& a, cudaStream_t s);
+
+// Fully-connected layer on e2m1 codes: activations [N][K / 2] bytes, weights
+// [n_tiles * 256][K / 2] bytes (K = the flattened image's padded channels; a k-block = 256 codes
+// = 128 bytes); items of 128 images x 256 channels x a share of the k-blocks, one per CTA.
+struct FcArgs {
+  int N, No;
+  int hw;             // pixels per image (the window of beta)
+  int kb_total;       // k-blocks of the flattened image
+  // filled by tc_fc_plan
+  int m_tiles, n_tiles, k_splits, kb_per_split;
+  const float* scale;
+  const float* bias;
+  const float* A;     // [N][hw] channel means, or nullptr (no beta)
+  int relu;
+  uint32_t* err;
+  float* ws;          // [N][No] fp32 partial sums (split reductions), zero between launches
+  float* out;         // [N][No] output, 16-byte aligned
+  uint32_t* count;    // [m_tiles * n_tiles] finished items per tile, zero between launches
+};
+void tc_fc_plan(FcArgs& a, int sm_count);
+int tc_fc_smem_bytes();
+// tmA: 2-D map over the activation codes {K / 2 bytes, N}, box 128 x 128; tmB: 2-D map over the
+// weight codes {K / 2 bytes, n_tiles * 256}, box 128 x 256; tmWs / tmOut: 2-D maps {No, N} fp32
+// over the workspace and the output, box 32 x 128; all 128-byte swizzled.
+cudaError_t launch_tc_fc(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmWs,
+                         const CUtensorMap* tmOut, const FcArgs& a, cudaStream_t s);
+
+// The same on SM pairs (tc_halo2_kernel): M = 256 over two CTAs, N = 256 channels per pair,
+// each CTA holding half of the weight tile.  Weights row-major [n_tiles * 256][kh * kw *
+// kb_per_tap * 128] bytes, read through tmB (box 128 bytes x 128 rows, 128-byte swizzle).
+// max_pairs <= 0: the co-resident two-CTA clusters of the current device.
+bool tc_halo2_plan(HaloArgs& a, int max_pairs);
+int tc_halo2_max_pairs(const HaloArgs& a);
+cudaError_t launch_tc_halo2(const CUtensorMap* tmA, const CUtensorMap* tmB, const HaloArgs& a, cudaStream_t s);
+
 int tc_stages(int kind, int bn, int mt);  // stages that fit; < 2: the layout does not fit
 int tc_smem_bytes(const TcArgs& a);
 // One CTA per tile; weights from a.b_tiles.
@@ -109,6 +176,10 @@ struct PackI8Args {
   float* A;               // [npix] or nullptr
   int op;                 // kXnor or kAnd
   int f4;
+  // Destination grid: pixel (n, y, x) of the [N][h][w] input goes to code pixel
+  // (n, y + pad_t, x + pad_l) of an [N][hp][wp] buffer whose other pixels are left alone
+  // (hp == 0: the codes have the input's own [N][h][w] layout).
+  PadMap pad;
 };
 cudaError_t launch_pack_i8(const PackI8Args& a, cudaStream_t s);
 

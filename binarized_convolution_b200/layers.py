@@ -138,6 +138,9 @@ class BinaryConv2d(_Layer):
     def tc_codes(self) -> int:
         return nat.bconv_tc_codes(self.handle)
 
+    def staging(self) -> int:
+        return nat.bconv_staging(self.handle)
+
     def forward_into(self, x, out):
         import torch
 

@@ -242,6 +242,28 @@ bconv_status_t bconv_set_tc_codes(bconv_tc_codes_t codes);
 int32_t bconv_tc_codes(bconv_handle_t h);
 
 /*
+ * How the XNOR / AND tensor-core contraction of a stride-1 convolution on e2m1 codes brings the
+ * activations into shared memory, for layers created after the call (process-wide, like
+ * bconv_set_cta_mode).
+ *   PER_TAP  for every tap of the window, a box of the tile's pixels shifted by the tap offset
+ *            (each activation code is loaded once per tap).
+ *   ROWS     the codes sit in a zero-bordered copy of the image; a tile is 128 consecutive
+ *            positions of that grid, and one load of them plus the window's reach serves every
+ *            tap (the taps differ only in where their operand starts in shared memory); the
+ *            weights of a CTA's output channels stay in shared memory when they fit.  Needs
+ *            (kernel_h - 1) * (in_w + kernel_w - 1) + kernel_w - 1 <= 896 and an fp32 output;
+ *            a bit-packed output (bconv_set_output_terms) moves the layer to PER_TAP.
+ *   AUTO     ROWS where it applies, else PER_TAP.
+ * Returns INVALID_ARG for an unknown value.
+ */
+typedef enum { BCONV_STAGING_AUTO = 0, BCONV_STAGING_PER_TAP = 1, BCONV_STAGING_ROWS = 2 } bconv_staging_t;
+bconv_status_t bconv_set_staging(bconv_staging_t staging);
+
+/* The staging a layer's tensor-core contraction uses (BCONV_STAGING_PER_TAP or ROWS); 0 when the
+ * layer has no tensor-core path, -1 for a bad handle. */
+int32_t bconv_staging(bconv_handle_t h);
+
+/*
  * Wait for `stream`, then read and clear the handle's device error word.  Returns OK,
  * TIMEOUT (a kernel gave up a bounded wait), or CUDA (a pending CUDA error).
  */
@@ -357,10 +379,9 @@ bconv_status_t bconv_check_wait_timeout(double limit_ms);
 /* ------------------------------------------------------------------------------------
  * Forward without any allocation.  (The pages have no counterpart to this entry point; it
  * exists for callers of this library that cannot allocate device memory when they run a
- * layer: code whose device memory is all owned by its own pool, real-time loops where an
- * allocation may stall on a device-wide synchronisation, or work issued while a stream is
- * being captured into a CUDA graph, where allocation calls are not permitted.  Such callers
- * cannot use bconv_create, which allocates.)
+ * layer: code whose device memory is all owned by its own pool allocator, or real-time loops
+ * where an allocation may stall on a device-wide synchronisation.  Such callers cannot use
+ * bconv_create, which allocates the weights and the workspace.)
  * ------------------------------------------------------------------------------------ */
 
 /* Size of the one fixed scratch array this entry point works in (16 MiB).  Every device that
@@ -369,7 +390,11 @@ bconv_status_t bconv_check_wait_timeout(double limit_ms);
 
 /*
  * XNOR or AND convolution (the same result as bconv_create + bconv_forward with the same
- * arguments), computed with no cudaMalloc, cudaFree or other allocating call.
+ * arguments), computed with no cudaMalloc, cudaFree or other allocating call.  It runs the
+ * SIMT (POPC) kernel family -- a weight-layout kernel, pack, beta, then the XOR/AND + POPC
+ * contraction with int32 sums -- not the tensor cores, whose weight layout is prepared on
+ * the host at creation: on large layers it is several times slower than a created layer
+ * (batch 16, 56x56, 256 -> 256, 3x3: about 8x).
  *   desc            host; as for bconv_create (groups must be 1).
  *   type            BCONV_TYPE_XNOR or BCONV_TYPE_AND (binaryWeights -> INVALID_ARG).
  *   flags           BCONV_FLAG_* bits.

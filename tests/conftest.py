@@ -43,3 +43,4 @@ def _default_cta_mode():
     if _native._lib is not None:
         _native.bconv_set_cta_mode(_native.CTA_AUTO)
         _native.bconv_set_tc_codes(_native.CODES_AUTO)
+        _native.bconv_set_staging(_native.STAGING_AUTO)

@@ -43,9 +43,12 @@ def make_layer(w: synth.Workload, inp: synth.Inputs, *, sums: bool = False):
                         (w.stride_y, w.stride_x), wbits=inp.wbits, **kw)
 
 
-# Kernel families a parity case runs on: the library's choice (e2m1 codes for XNOR/AND), the
-# SIMT family, and the tensor cores with int8 codes forced onto one SM per tile or onto SM pairs.
-FAMILIES = ["auto", "alt", "single", "pair"]
+# Kernel families a parity case runs on: the library's choice (e2m1 codes for XNOR/AND; the
+# rows-staged kernel for stride-1 convolutions it fits, on SM pairs above 128 output channels),
+# the same codes with the per-tap staging forced, the rows-staged kernel forced onto one SM per
+# tile, the SIMT family, and the tensor cores with int8 codes forced onto one SM per tile or onto
+# SM pairs.
+FAMILIES = ["auto", "per_tap", "rows_single", "alt", "single", "pair"]
 
 
 def algo_for(w: synth.Workload, name: str):
@@ -57,8 +60,10 @@ def algo_for(w: synth.Workload, name: str):
     settings back to AUTO)."""
     import binarized_convolution_b200 as bc
 
-    bc.bconv_set_cta_mode({"single": bc.CTA_SINGLE, "pair": bc.CTA_PAIR}.get(name, bc.CTA_AUTO))
+    bc.bconv_set_cta_mode({"single": bc.CTA_SINGLE, "pair": bc.CTA_PAIR, "rows_single": bc.CTA_SINGLE}.get(
+        name, bc.CTA_AUTO))
     bc.bconv_set_tc_codes(bc.CODES_INT8 if name in ("single", "pair") else bc.CODES_AUTO)
+    bc.bconv_set_staging(bc.STAGING_PER_TAP if name == "per_tap" else bc.STAGING_AUTO)
     if name == "alt":
         return bc.ALGO_SIMT_F32 if w.op == synth.BINARY_WEIGHTS else bc.ALGO_POPC
     return bc.ALGO_AUTO

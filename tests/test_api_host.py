@@ -148,3 +148,22 @@ def test_create_without_a_device_reports_no_device():
 def test_python_layer_raises_on_bad_input():
     with pytest.raises((bc.BconvError, ValueError)):
         bc.BinaryConv2d(1, 4, 4, 8, 2, 3, 1, wbits=np.zeros((2, 3, 3, 8), np.uint8), groups=2)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(kernel_h=65536, kernel_w=65536, in_h=1 << 20, in_w=1 << 20),  # 2^32 taps: rejected before any product
+    dict(kernel_h=10, in_h=4),                                          # wider than 2 x the image + 1
+    dict(kernel_h=4097, in_h=4096),
+    dict(kernel_h=64, kernel_w=64, in_h=64, in_w=64, in_channels=1 << 20),  # 2^32-term sums overflow int32
+])
+def test_create_and_noalloc_reject_the_same_oversize_shapes(kw):
+    """bconv_create and bconv_forward_noalloc share one shape check (status 2 = UNSUPPORTED),
+    returned on the host before any weight is read or any device work is queued."""
+    lib = bc.load_library()
+    d = _desc(**kw)
+    dummy = (ctypes.c_uint32 * 4)()
+    h = ctypes.c_void_p()
+    assert lib.bconv_create(ctypes.byref(d), dummy, None, None, None, None, 1, 0, ctypes.byref(h)) == 2
+    assert h.value is None
+    assert lib.bconv_forward_noalloc(ctypes.byref(d), nat.TYPE_XNOR, 0, 16, None, None, None, None, 16, 16,
+                                     None) == 2

@@ -337,3 +337,93 @@ def test_e2m1_code_layouts(w, cuda_device):
     finally:
         layer.close()
     _check(w)
+
+
+@pytest.mark.parametrize("op", [synth.AND, synth.XNOR])
+def test_window_sums_past_2p24_stay_exact(op, cuda_device):
+    """A window sum of more than 2^24 unit terms (1 x 17 kernel over 2^20 channels, every input
+    bit 1, 99 % of the weight bits 1): fp32 accumulation would round such sums, so the library
+    keeps int32 sums even when e2m1 codes are asked for.  With scale 1 and no bias the fp32
+    output must be the exact integer sum rounded once to fp32, on every kernel family."""
+    import oracle
+    import torch
+
+    ni, no, width, k = 1 << 20, 4, 17, 17
+    rng = np.random.default_rng(77)
+    x = (np.abs(rng.standard_normal((1, 1, width, ni), dtype=np.float32)) + 0.25).astype(np.float32)
+    wbits = np.ones((no, 1, k, ni), np.uint8)
+    flat = wbits.reshape(-1)
+    flat[rng.integers(0, flat.size, flat.size // 100)] = 0
+    otype = {synth.AND: oracle.ORACLE_AND, synth.XNOR: oracle.ORACLE_XNOR}[op]
+    S, _, _ = oracle.conv(x, wbits, type=otype, scale_value=1.0)
+    assert np.abs(S).max() > 2 ** 24
+    if op == synth.AND:  # XNOR sums have the parity of the window size (even here); AND sums need not
+        assert np.any(S % 2 == 1)
+    want = S.astype(np.float32)
+    for name in ("auto", "alt", "single", "pair"):
+        algo = pu.algo_for(synth.small_case(op=op), name)
+        if name == "auto":
+            bc.bconv_set_tc_codes(bc.CODES_FP4)  # asked for e2m1: the sums must still stay int32
+        layer = bc.BinaryConv2d(1, 1, width, ni, no, (1, k), (1, 1), wbits=wbits, op=op, scale=None,
+                                scale_value=1.0)
+        try:
+            layer.set_algo(algo)
+            if layer.effective_algo() == bc.ALGO_TCGEN05:
+                assert layer.tc_codes() == bc.CODES_INT8
+            y = layer(torch.from_numpy(x).cuda())
+            layer.sync_status()
+            y = y.reshape(-1, no).cpu().numpy()
+        finally:
+            layer.close()
+        assert np.array_equal(y, want), f"{name}: {np.abs(y.astype(np.float64) - S).max()}"
+    bc.bconv_set_cta_mode(bc.CTA_AUTO)
+    bc.bconv_set_tc_codes(bc.CODES_AUTO)
+
+
+def test_staging_choice(cuda_device):
+    """The rows-staged kernel serves e2m1 stride-1 convolutions whose padded rows fit a tile; strided
+    layers, wide images, a forced per-tap setting and a bit-packed output use the per-tap kernel."""
+    def layer(h, w, stride=1, no=64):
+        c = synth.small_case(batch=2, h=h, w=w, ni=64, no=no, k=3, stride=stride, op=synth.XNOR, seed=7)
+        inp = synth.make_inputs(c)
+        return bc.BinaryConv2d(c.batch, c.in_h, c.in_w, c.in_channels, c.out_channels, 3, stride, wbits=inp.wbits)
+
+    with layer(12, 56) as l:
+        assert l.staging() == bc.STAGING_ROWS and l.tc_codes() == bc.CODES_FP4
+    with layer(12, 56, stride=2) as l:
+        assert l.staging() == bc.STAGING_PER_TAP
+    with layer(4, 500) as l:  # a window reaching 2 x 502 + 2 slots past the tile is too long
+        assert l.staging() == bc.STAGING_PER_TAP
+    with layer(4, 200) as l:  # wide rows are fine: tiles run across them
+        assert l.staging() == bc.STAGING_ROWS
+    with layer(12, 56) as l:
+        l.set_output_terms(None, None)
+        assert l.staging() == bc.STAGING_PER_TAP
+    bc.bconv_set_staging(bc.STAGING_PER_TAP)
+    with layer(12, 56) as l:
+        assert l.staging() == bc.STAGING_PER_TAP
+    bc.bconv_set_staging(bc.STAGING_AUTO)
+
+
+@pytest.mark.parametrize("kind", ["conv", "fc"])
+def test_output_not_16_byte_aligned(kind, cuda_device):
+    """An output buffer 4 bytes past a 16-byte boundary: the tensor-core kernels write 16-byte
+    pieces, so such a forward runs on the SIMT family and must still match the oracle."""
+    import torch
+
+    w = synth.small_case(batch=3, h=6, w=7, ni=40, no=36, k=3, kind=kind, op=synth.XNOR, use_beta=True, relu=True,
+                         in_terms=True, seed=61)
+    inp = synth.make_inputs(w)
+    S_ref, beta_ref, y_ref = pu.run_oracle(w, inp)
+    layer = pu.make_layer(w, inp)
+    try:
+        n_out = int(np.prod(layer.out_dims))
+        buf = torch.zeros(n_out + 4, dtype=torch.float32, device="cuda")
+        out = buf[1:1 + n_out].view(layer.out_dims)
+        assert out.data_ptr() % 16 == 4
+        layer.forward_into(torch.from_numpy(inp.x).cuda(), out)
+        layer.sync_status()
+        y = out.reshape(-1, w.out_channels).cpu().numpy()
+    finally:
+        layer.close()
+    pu.assert_outputs_close(w, inp, y, S_ref, beta_ref, y_ref)
