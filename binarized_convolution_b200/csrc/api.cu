@@ -144,10 +144,9 @@ struct Layer {
   HaloArgs hx{};
   PadMap pad{};
   float* A_pad = nullptr;  // A in the zero-bordered grid (rows-staged layers with beta)
-  // Fully-connected contraction with 256-channel items (tc_fc_kernel): its plan and counters
+  // Fully-connected contraction with 256-channel items (tc_fc_kernel): its plan
   bool fcb = false;
   FcArgs fx{};
-  uint32_t* fc_count = nullptr;
   CUtensorMap tmA{}, tmB{}, tmBp{}, tmWs{}, tmOut{};
   const float* tm_out_ptr = nullptr;
   // chained layers: the next layer's input terms (bit-packed output) and what emitting the
@@ -344,27 +343,16 @@ bconv_status_t setup_fc(Layer& L, const uint32_t* packed) {
     if (e == cudaSuccess) e = cudaMemcpy(L.wq, hb.data(), hb.size(), cudaMemcpyHostToDevice);
   }
   if (e == cudaSuccess) e = L.tc_mem.alloc(&L.codes, static_cast<size_t>(L.N) * row_bytes);
-  if (e == cudaSuccess && f.k_splits > 1) e = L.tc_mem.alloc(&L.ws, static_cast<size_t>(L.N) * L.No);
-  if (e == cudaSuccess && f.k_splits > 1) e = cudaMemset(L.ws, 0, sizeof(float) * static_cast<size_t>(L.N) * L.No);
-  if (e == cudaSuccess && f.k_splits > 1)
-    e = L.tc_mem.alloc(&L.fc_count, static_cast<size_t>(f.m_tiles) * f.n_tiles);
-  if (e == cudaSuccess && f.k_splits > 1)
-    e = cudaMemset(L.fc_count, 0, sizeof(uint32_t) * static_cast<size_t>(f.m_tiles) * f.n_tiles);
   if (e != cudaSuccess) return from_cuda(e);
   bool ok = encode_2d(&L.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.codes, static_cast<uint64_t>(row_bytes),
                       static_cast<uint64_t>(L.N), static_cast<uint64_t>(row_bytes), 128, 128);
   ok = ok && encode_2d(&L.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(row_bytes),
                        static_cast<uint64_t>(rows), static_cast<uint64_t>(row_bytes), 128, 256);
-  if (ok && f.k_splits > 1)
-    ok = encode_2d(&L.tmWs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L.ws, static_cast<uint64_t>(L.No),
-                   static_cast<uint64_t>(L.N), static_cast<uint64_t>(L.No) * 4, 32, 128);
   if (!ok) return BCONV_OK;  // the POPC path stays available
   f.scale = L.scale;
   f.bias = L.bias;
   f.relu = L.relu;
   f.err = L.err;
-  f.ws = L.ws;
-  f.count = L.fc_count;
   L.tc.kind = 2;
   L.tc.BN = 256;
   L.tc.n_tiles = f.n_tiles;
@@ -844,15 +832,9 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
     FcArgs f = L.fx;
     f.A = beta ? A : nullptr;
     f.out = out;
-    if (out != L.tm_out_ptr) {
-      if (!encode_2d(&L.tmOut, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, out, static_cast<uint64_t>(L.No),
-                     static_cast<uint64_t>(L.N), static_cast<uint64_t>(L.No) * 4, 32, 128))
-        return BCONV_ERR_CUDA;
-      L.tm_out_ptr = out;
-    }
     const bool timed = L.prof.take();
     if (timed) cudaEventRecord(L.prof.start[L.prof.used], s);
-    e = launch_tc_fc(&L.tmA, &L.tmB, &L.tmWs, &L.tmOut, f, s);
+    e = launch_tc_fc(&L.tmA, &L.tmB, f, s);
     if (timed) cudaEventRecord(L.prof.stop[L.prof.used++], s);
     return from_cuda(e);
   }
@@ -1042,7 +1024,6 @@ bconv_status_t replan_tc(Layer& L, int codes) {
   L.halo2 = false;
   L.A_pad = nullptr;
   L.fcb = false;
-  L.fc_count = nullptr;
   L.codes_override = codes;
   return setup_tc(L, L.h_packed.data());
 }
@@ -1078,7 +1059,9 @@ bconv_status_t set_output_terms(Layer& L, const float* next_scale, const float* 
   // formed within one work item instead of being added across items.  Measured on B200, batch
   // 16, 56 x 56, 256 -> 256 as a chain's middle layer: 53.3 us per forward on e2m1 codes
   // (two 128-channel tiles), 37.1 us on int8.
-  if (L.tc_ok && L.tc.kind == 2 && !L.fc && L.tc.n_tiles > 1 && L.codes_override < 0) {
+  // (The per-tap kernel's e2m1 tiles are at most 128 channels wide, whatever the rows-staged
+  // plan used.)
+  if (L.tc_ok && L.tc.kind == 2 && !L.fc && L.No > 128 && L.codes_override < 0) {
     L.halo_off = true;
     const bconv_status_t st = replan_tc(L, BCONV_CODES_INT8);
     if (st != BCONV_OK) return st;
@@ -1227,7 +1210,6 @@ bconv_status_t sync_status(Layer& L, cudaStream_t s) {
     if (L.a_count) cudaMemset(L.a_count, 0, sizeof(uint32_t) * L.tc.m_tiles);  // an aborted launch may leave counts
     if (L.tc.sk_flag) cudaMemset(L.tc.sk_flag, 0, sizeof(uint32_t) * (L.tc.grid_ctas / 2 - 1) * 2);  // and flags
     if (L.ws) cudaMemset(L.ws, 0, sizeof(float) * static_cast<size_t>(L.N) * L.No);  // and partial sums
-    if (L.fc_count) cudaMemset(L.fc_count, 0, sizeof(uint32_t) * static_cast<size_t>(L.fx.m_tiles) * L.fx.n_tiles);
     if (word & kErrTimeout) return BCONV_ERR_TIMEOUT;
     return BCONV_ERR_CUDA;  // kErrLayout: a kernel refused an unexpected shared-memory layout
   }

@@ -106,32 +106,6 @@ int tc_halo_smem_bytes(const HaloArgs& a);
 // 128-byte swizzle.
 cudaError_t launch_tc_halo(const CUtensorMap* tmA, const HaloArgs& a, cudaStream_t s);
 
-// Fully-connected layer on e2m1 codes: activations [N][K / 2] bytes, weights
-// [n_tiles * 256][K / 2] bytes (K = the flattened image's padded channels; a k-block = 256 codes
-// = 128 bytes); items of 128 images x 256 channels x a share of the k-blocks, one per CTA.
-struct FcArgs {
-  int N, No;
-  int hw;             // pixels per image (the window of beta)
-  int kb_total;       // k-blocks of the flattened image
-  // filled by tc_fc_plan
-  int m_tiles, n_tiles, k_splits, kb_per_split;
-  const float* scale;
-  const float* bias;
-  const float* A;     // [N][hw] channel means, or nullptr (no beta)
-  int relu;
-  uint32_t* err;
-  float* ws;          // [N][No] fp32 partial sums (split reductions), zero between launches
-  float* out;         // [N][No] output, 16-byte aligned
-  uint32_t* count;    // [m_tiles * n_tiles] finished items per tile, zero between launches
-};
-void tc_fc_plan(FcArgs& a, int sm_count);
-int tc_fc_smem_bytes();
-// tmA: 2-D map over the activation codes {K / 2 bytes, N}, box 128 x 128; tmB: 2-D map over the
-// weight codes {K / 2 bytes, n_tiles * 256}, box 128 x 256; tmWs / tmOut: 2-D maps {No, N} fp32
-// over the workspace and the output, box 32 x 128; all 128-byte swizzled.
-cudaError_t launch_tc_fc(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmWs,
-                         const CUtensorMap* tmOut, const FcArgs& a, cudaStream_t s);
-
 // The same on SM pairs (tc_halo2_kernel): M = 256 over two CTAs, N = 256 channels per pair,
 // each CTA holding half of the weight tile.  Weights row-major [n_tiles * 256][kh * kw *
 // kb_per_tap * 128] bytes, read through tmB (box 128 bytes x 128 rows, 128-byte swizzle).
@@ -139,6 +113,31 @@ cudaError_t launch_tc_fc(const CUtensorMap* tmA, const CUtensorMap* tmB, const C
 bool tc_halo2_plan(HaloArgs& a, int max_pairs);
 int tc_halo2_max_pairs(const HaloArgs& a);
 cudaError_t launch_tc_halo2(const CUtensorMap* tmA, const CUtensorMap* tmB, const HaloArgs& a, cudaStream_t s);
+
+// Fully-connected layer on e2m1 codes: activations [N][K / 2] bytes, weights
+// [n_tiles * 256][K / 2] bytes (K = the flattened image's padded channels; a k-block = 256 codes
+// = 128 bytes); items of 128 images x 256 channels x a share of the k-blocks, one per CTA, the
+// k_splits items of a tile forming one cluster that adds its partial sums through distributed
+// shared memory.
+struct FcArgs {
+  int N, No;
+  int hw;             // pixels per image (the window of beta)
+  int kb_total;       // k-blocks of the flattened image
+  // filled by tc_fc_plan
+  int m_tiles, n_tiles, k_splits, kb_per_split;  // k_splits: 1..8, a divisor of 128
+  const float* scale;
+  const float* bias;
+  const float* A;     // [N][hw] channel means, or nullptr (no beta)
+  int relu;
+  uint32_t* err;
+  float* out;         // [N][No] output, 16-byte aligned
+};
+void tc_fc_plan(FcArgs& a, int sm_count);
+int tc_fc_smem_bytes();
+// tmA: 2-D map over the activation codes {K / 2 bytes, N}, box 128 x 128; tmB: 2-D map over the
+// weight codes {K / 2 bytes, n_tiles * 256}, box 128 x 256; both 128-byte swizzled.
+cudaError_t launch_tc_fc(const CUtensorMap* tmA, const CUtensorMap* tmB, const FcArgs& a, cudaStream_t s);
+
 
 int tc_stages(int kind, int bn, int mt);  // stages that fit; < 2: the layout does not fit
 int tc_smem_bytes(const TcArgs& a);

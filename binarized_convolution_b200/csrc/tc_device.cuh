@@ -335,5 +335,50 @@ __device__ __forceinline__ bool named_all(bool v, uint32_t n) {
   return r != 0;
 }
 
+// XNOR-Net beta of the rows-staged kernels' output slots, for `count` tiles of 128 consecutive
+// slots (tile t starts at slot (first + t * step) * 128): beta = (sum of A over the kh x kw
+// window) / (kh * kw), A being the channel means in the zero-bordered [N][Hp][Wp] grid
+// (`total` slots), so the window of slot s is s + ty * wp + tx.  The `nthreads` threads of
+// named barrier 1 (index et) first stage the tiles' strips of A -- len = 128 + (kh - 1) * wp +
+// kw - 1 floats each, count * len <= the floats `strip` holds -- with eight independent loads
+// in flight per thread; then each thread forms the betas of its row (`writer` picks one thread
+// per row) into betas[t * 128 + row].  Barriers before (the strip's other users are done with
+// it), between, and after (the strip is free again and every beta is visible).
+__device__ __forceinline__ void tile_betas(const float* __restrict__ A, int total, int first, int step, int count,
+                                           int len, int kh, int kw, int wp, float* strip, float* betas, int row,
+                                           bool writer, int et, int nthreads) {
+  named_barrier(static_cast<uint32_t>(nthreads));
+  const int n = count * len;
+  for (int base = 0; base < n; base += 8 * nthreads) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int f = base + j * nthreads + et;
+      v[j] = 0.f;
+      if (f < n) {
+        const int t = f / len;
+        const int s = (first + t * step) * 128 + (f - t * len);
+        if (s < total) v[j] = __ldg(A + s);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int f = base + j * nthreads + et;
+      if (f < n) strip[f] = v[j];
+    }
+  }
+  named_barrier(static_cast<uint32_t>(nthreads));
+  if (writer) {
+    for (int t = 0; t < count; ++t) {
+      const float* w = strip + t * len + row;
+      float sum = 0.f;
+      for (int ty = 0; ty < kh; ++ty)
+        for (int tx = 0; tx < kw; ++tx) sum += w[ty * wp + tx];
+      betas[t * 128 + row] = sum / static_cast<float>(kh * kw);
+    }
+  }
+  named_barrier(static_cast<uint32_t>(nthreads));
+}
+
 }  // namespace tcdev
 }  // namespace bconv

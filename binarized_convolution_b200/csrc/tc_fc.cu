@@ -14,18 +14,19 @@
 // weight codes (both 128-byte swizzled) feed four M128 N256 K64 MMAs: the activations are read
 // once per 256 channels, the weights once per 128 images.
 //
-// The epilogue stages the item's whole 128 x 256 tile in the idle stage memory and moves it by
-// TMA.  A split item adds its exact partial sums into an fp32 workspace by TMA reduce-add
-// (integers below 2^24 add exactly in any order); the last item of a tile to finish (an atomic
-// count per tile, after proxy and memory fences) loads the tile's sums back, applies the
-// epilogue with the betas the epilogue warps formed during the main loop, stores the output,
-// zeroes the workspace and resets the count -- no separate finalize launch.  An unsplit item
-// stores y itself.
+// The k_splits items of a tile form one cluster.  After its MMAs each CTA writes its exact
+// partial sums (a 128 x 256 fp32 tile, 16-byte pieces XOR-swizzled within each row) into its
+// own shared memory; after a cluster barrier each CTA finishes 128 / k_splits rows: it reads the
+// rows of every CTA's partial tile through distributed shared memory, adds them in rank order
+// (integers below 2^24: exact in fp32 in any order), applies beta (formed by the epilogue warps
+// while the MMAs run), scale, bias and the neuron, and writes each output row with coalesced
+// stores.  A second cluster barrier keeps every CTA's shared memory alive until all have read it.
+// No workspace and no second launch.
 //
 // Roles (6 warps): warp 0 TMA producer (4-stage ring); warp 1 TMEM allocation and, from one
 // thread, the MMAs; warps 2-5 the epilogue.  Every mbarrier wait gives up after one second of
 // %globaltimer, sets the error word and makes all roles stop; TMEM is released on every exit
-// path.
+// path; the cluster barriers are reached on every path.
 #include <cuda.h>
 
 #include <algorithm>
@@ -55,15 +56,73 @@ struct __align__(16) FcBars {
   uint64_t done;
   uint32_t tmem_base;
   uint32_t abort_flag;
-  uint64_t fin_full;  // the finishing CTA's load of the tile's sums
-  uint32_t last;      // this CTA finishes its tile
   float2 sb[kBN];
   float beta[128];
 };
 
+// Offset, within a CTA's partial tile (128 rows x 1 KB), of float4 `k` (0..63) of row `r`: the
+// low three bits of the float4 index are XORed with the row's, so that 32 consecutive rows
+// writing the same float4 index hit different banks.
+__device__ __forceinline__ uint32_t part_off(int r, int k) {
+  return static_cast<uint32_t>(r * 1024 + (((k & ~7) | ((k & 7) ^ (r & 7))) * 16));
+}
+
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+
+// Rows [split * 128 / KS, (split + 1) * 128 / KS) of the tile from the KS partial tiles of the
+// cluster: warp q of the epilogue takes every fourth row, lane l channels 8 l .. 8 l + 7.  All
+// KS x 2 distributed-shared-memory loads of a row (two rows when KS <= 4) are issued before any
+// is used, so that a row costs one remote latency rather than KS of them.
+template <int KS>
+__device__ __forceinline__ void finish_rows(const FcArgs& a, const FcBars* B, const uint8_t* smem, int split, int m0,
+                                            int c0, int q, int lane) {
+  constexpr int kRowsPer = 128 / KS;
+  constexpr int kUnroll = KS <= 4 ? 2 : 1;  // rows in flight per warp
+  uint32_t base[KS];
+#pragma unroll
+  for (int p = 0; p < KS; ++p) base[p] = mapa(smem, static_cast<uint32_t>(p));
+  for (int r0 = split * kRowsPer + q; r0 < (split + 1) * kRowsPer; r0 += 4 * kUnroll) {
+    float4 u[kUnroll][KS][2];
+#pragma unroll
+    for (int h = 0; h < kUnroll; ++h)
+#pragma unroll
+      for (int p = 0; p < KS; ++p) {
+        const int r = r0 + 4 * h;
+        u[h][p][0] = ld_cluster_f4(base[p] + part_off(r, 2 * lane));
+        u[h][p][1] = ld_cluster_f4(base[p] + part_off(r, 2 * lane + 1));
+      }
+#pragma unroll
+    for (int h = 0; h < kUnroll; ++h) {
+      const int r = r0 + 4 * h;
+      const int nn = m0 + r;
+      if (nn >= a.N) continue;
+      float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int p = 0; p < KS; ++p) {  // rank order
+        y[0] += u[h][p][0].x; y[1] += u[h][p][0].y; y[2] += u[h][p][0].z; y[3] += u[h][p][0].w;
+        y[4] += u[h][p][1].x; y[5] += u[h][p][1].y; y[6] += u[h][p][1].z; y[7] += u[h][p][1].w;
+      }
+      const float bb = B->beta[r];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float2 p = B->sb[8 * lane + j];
+        const float v = a.A ? fmaf(y[j] * p.x, bb, p.y) : fmaf(y[j], p.x, p.y);
+        y[j] = a.relu ? fmaxf(v, 0.f) : v;
+      }
+      const int c = c0 + 8 * lane;
+      float* o = a.out + static_cast<int64_t>(nn) * a.No + c;
+      if (c < a.No) *reinterpret_cast<float4*>(o) = make_float4(y[0], y[1], y[2], y[3]);
+      if (c + 4 < a.No) *reinterpret_cast<float4*>(o + 4) = make_float4(y[4], y[5], y[6], y[7]);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-    tc_fc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ CUtensorMap tmWs, const __grid_constant__ CUtensorMap tmOut, const FcArgs a) {
+    tc_fc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const FcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0u) {
     if (threadIdx.x == 0) atomicOr(a.err, kErrLayout);
@@ -73,9 +132,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw;
   FcBars* B = reinterpret_cast<FcBars*>(smem + kStages * kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // item -> (split, N tile, M tile)
+  // item -> (split = the CTA's rank in its cluster, N tile, M tile)
   int t = blockIdx.x;
-  const int split = t % a.k_splits;
+  const int split = static_cast<int>(cluster_rank());
   t /= a.k_splits;
   const int ntile = t % a.n_tiles;
   const int mtile = t / a.n_tiles;
@@ -91,14 +150,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&B->tmem_full, 1);
     mbar_init(&B->done, 1);
-    mbar_init(&B->fin_full, 1);
     B->abort_flag = 0;
-    B->last = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tensor_map(&tmA);
     prefetch_tensor_map(&tmB);
-    prefetch_tensor_map(&tmOut);
-    if (a.k_splits > 1) prefetch_tensor_map(&tmWs);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&B->tmem_base)),
@@ -177,11 +232,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
-    // The whole 128 x 256 tile is staged in the (by then idle) stage memory as 8 chunks of
-    // 128 rows x 32 fp32 (16 KB each; 16-byte chunk k of row r at k ^ (r % 8)) and moved by TMA:
-    // reduce-add into the workspace (split) or store into the output (unsplit).  The finishing
-    // item of a split tile loads the tile's sums back by TMA, applies the epilogue in shared
-    // memory, stores the output and zeroes the workspace, again by TMA.
     const int et = threadIdx.x - 64;  // 0..127
     const int q = warp & 3;
     const int row = q * 32 + lane;    // TMEM lane = image m0 + row
@@ -197,108 +247,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       B->beta[et] = b;
     }
-    auto epilogue_row = [&](float (&y)[32], int ch, float beta) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float2 p = B->sb[ch * 32 + j];
-        const float r = a.A ? fmaf(y[j] * p.x, beta, p.y) : fmaf(y[j], p.x, p.y);
-        y[j] = a.relu ? fmaxf(r, 0.f) : r;
-      }
-    };
-    if (epi_all(mbar_wait(&B->tmem_full, 0, B, a.err, true, true))) {
+    bool ok = epi_all(mbar_wait(&B->tmem_full, 0, B, a.err, true, true));
+    if (ok) {
       tc_fence_after();
       if (et == 0) BCONV_STAMP(4);
-      const float beta = B->beta[row];
+      // this CTA's partial tile into its (now idle) stage memory; a split past the last k-block
+      // (k_splits * kb_per_split may exceed kb_total by up to a share) issued no MMA and adds 0
+      const bool no_kb = kb1 <= kb0;
       for (int ch = 0; ch < kBN / 32; ++ch) {
         uint32_t v[32];
-        tc_ld_32x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ch * 32), v);
-        float y[32];
+        if (no_kb) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(v[j]);
-        if (a.k_splits == 1) epilogue_row(y, ch, beta);
-        float4* orow = reinterpret_cast<float4*>(smem + ch * 16384 + row * 128);
+          for (int j = 0; j < 32; ++j) v[j] = 0u;
+        } else {
+          tc_ld_32x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ch * 32), v);
+        }
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          orow[k ^ (row & 7)] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
+          *reinterpret_cast<float4*>(smem + part_off(row, ch * 8 + k)) =
+              make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]), __uint_as_float(v[4 * k + 2]),
+                          __uint_as_float(v[4 * k + 3]));
       }
-      fence_proxy_async();
-      epi_barrier();
-      if (et == 0) {
-        for (int ch = 0; ch < kBN / 32; ++ch) {
-          if (c0 + ch * 32 >= a.No) break;
-          if (a.k_splits > 1)
-            tma_reduce_add_2d(&tmWs, smem + ch * 16384, c0 + ch * 32, m0);  // integers below 2^24: exact
-          else
-            tma_store_2d(&tmOut, smem + ch * 16384, c0 + ch * 32, m0);
-        }
-        bulk_commit();
-        bulk_wait_all();
-        BCONV_STAMP(5);
-        if (a.k_splits > 1) {
-          // this item's partial sums are in the workspace: count it in; the last item finishes the tile
-          asm volatile("fence.proxy.async.global;" ::: "memory");
-          __threadfence();
-          const uint32_t old = atomicAdd(a.count + mtile * a.n_tiles + ntile, 1u);
-          B->last = (old == static_cast<uint32_t>(a.k_splits - 1)) ? 1u : 0u;
-        }
-      }
-      epi_barrier();
-      if (a.k_splits > 1 && B->last) {
-        int nch = 0;
-        if (et == 0) {
-          __threadfence();
-          asm volatile("fence.proxy.async.global;" ::: "memory");
-          for (int ch = 0; ch < kBN / 32 && c0 + ch * 32 < a.No; ++ch) ++nch;
-          mbar_expect_tx(&B->fin_full, static_cast<uint32_t>(nch * 16384));
-          for (int ch = 0; ch < nch; ++ch)
-            tma_load_2d(smem + ch * 16384, &tmWs, &B->fin_full, c0 + ch * 32, m0);
-        }
-        if (epi_all(mbar_wait(&B->fin_full, 0, B, a.err, true, true))) {
-          for (int ch = 0; ch < kBN / 32; ++ch) {
-            float4* orow = reinterpret_cast<float4*>(smem + ch * 16384 + row * 128);
-            float y[32];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const float4 t4 = orow[k ^ (row & 7)];
-              y[4 * k] = t4.x;
-              y[4 * k + 1] = t4.y;
-              y[4 * k + 2] = t4.z;
-              y[4 * k + 3] = t4.w;
-            }
-            epilogue_row(y, ch, beta);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              orow[k ^ (row & 7)] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
-          }
-          fence_proxy_async();
-          epi_barrier();
-          if (et == 0) {
-            for (int ch = 0; ch < kBN / 32 && c0 + ch * 32 < a.No; ++ch)
-              tma_store_2d(&tmOut, smem + ch * 16384, c0 + ch * 32, m0);
-            bulk_commit();
-            bulk_wait_read_0();
-          }
-          epi_barrier();
-          // zero the workspace tile for the next forward: a zero chunk stored over every chunk
-          float4* z = reinterpret_cast<float4*>(smem);
-          for (int i = et; i < 16384 / 16; i += kEpiThreads) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-          fence_proxy_async();
-          epi_barrier();
-          if (et == 0) {
-            for (int ch = 0; ch < kBN / 32 && c0 + ch * 32 < a.No; ++ch)
-              tma_store_2d(&tmWs, smem, c0 + ch * 32, m0);
-            bulk_commit();
-            bulk_wait_all();
-            a.count[mtile * a.n_tiles + ntile] = 0u;
-            BCONV_STAMP(6);
-          }
-        }
-      }
+      if (et == 0) BCONV_STAMP(5);
     }
   }
 
+  // every CTA of the cluster reaches both barriers, whatever happened above
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // every partial tile of the cluster is written
+  if (warp >= 2 && !*reinterpret_cast<volatile uint32_t*>(&B->abort_flag)) {
+    switch (a.k_splits) {
+      case 1: finish_rows<1>(a, B, smem, split, m0, c0, warp & 3, lane); break;
+      case 2: finish_rows<2>(a, B, smem, split, m0, c0, warp & 3, lane); break;
+      case 4: finish_rows<4>(a, B, smem, split, m0, c0, warp & 3, lane); break;
+      default: finish_rows<8>(a, B, smem, split, m0, c0, warp & 3, lane); break;
+    }
+    if (warp == 2 && lane == 0) BCONV_STAMP(6);
+  }
+  cluster_sync();  // no CTA leaves while another may still read its partial tile
   allow_next_grid();
   if (warp == 1) {
     tc_fence_after();
@@ -310,27 +297,76 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 int tc_fc_smem_bytes() { return kStages * kStageBytes + static_cast<int>(sizeof(FcBars)); }
 
+namespace {
+// Clusters of `ks` CTAs of the FC kernel that can be resident at once (0 if unknown).
+int fc_max_clusters(int ks) {
+  const int smem = tc_fc_smem_bytes();
+  if (cudaFuncSetAttribute(tc_fc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ks));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(ks);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, tc_fc_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+}  // namespace
+
 void tc_fc_plan(FcArgs& a, int sm_count) {
   a.m_tiles = (a.N + 127) / 128;
   a.n_tiles = (a.No + kBN - 1) / kBN;
   const int tiles = a.m_tiles * a.n_tiles;
-  // the most splits that keep every item on its own SM, each with at least 4 k-blocks
+  // the most splits (a cluster of at most 8 CTAs per tile) that keep every item on its own SM
+  // in one wave of resident clusters, each with at least 4 k-blocks and an even share of the
+  // tile's 128 rows
   int ks = std::max(1, sm_count / std::max(tiles, 1));
-  ks = std::min(ks, std::max(1, a.kb_total / 4));
+  ks = std::min({ks, 8, std::max(1, a.kb_total / 4)});
+  while (ks > 1 && (128 % ks != 0 || fc_max_clusters(ks) < tiles)) --ks;
   a.kb_per_split = (a.kb_total + ks - 1) / ks;
-  a.k_splits = (a.kb_total + a.kb_per_split - 1) / a.kb_per_split;
+  a.k_splits = ks;
 }
 
-cudaError_t launch_tc_fc(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmWs,
-                         const CUtensorMap* tmOut, const FcArgs& a, cudaStream_t s) {
+cudaError_t launch_tc_fc(const CUtensorMap* tmA, const CUtensorMap* tmB, const FcArgs& a, cudaStream_t s) {
   const int items = a.m_tiles * a.n_tiles * a.k_splits;
   if (items == 0) return cudaSuccess;
-  if (!a.out || (reinterpret_cast<uintptr_t>(a.out) & 15u) != 0 || (a.k_splits > 1 && (!a.ws || !a.count)))
+  if (!a.out || (reinterpret_cast<uintptr_t>(a.out) & 15u) != 0 || a.k_splits < 1 || a.k_splits > 8 ||
+      128 % a.k_splits != 0)
     return cudaErrorInvalidValue;
   const int smem = tc_fc_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(tc_fc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess && a.k_splits > 1)
+    e = cudaFuncSetAttribute(tc_fc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
   if (e != cudaSuccess) return e;
-  return launch_overlapped(tc_fc_kernel, dim3(items), dim3(kThreads), smem, s, *tmA, *tmB, *tmWs, *tmOut, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(items));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;  // the k splits of a tile
+  attr[0].val.clusterDim.x = static_cast<unsigned>(a.k_splits);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may overlap the pack's tail
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  e = cudaLaunchKernelEx(&cfg, tc_fc_kernel, *tmA, *tmB, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 }  // namespace bconv

@@ -30,12 +30,13 @@
 //   warp 1      allocates TMEM (two BN-column fp32 accumulators + the unit scale factors)
 //               and, from one thread, issues kh * kw * kb_per_tap groups of four
 //               tcgen05.mma.kind::mxf4 (M = 128, N = BN, K = 64 each) per tile.
-//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time, beta from the tile's strip of A,
-//               scale / bias / neuron in fp32; each warp stages its 32 rows in its own 4 KB of
-//               shared memory (128-byte swizzle) and reads them back so that each store
-//               instruction writes 4 output rows x 128 contiguous bytes; junk rows are skipped.
-//               No TMA store and no barrier across warps: a chunk never waits for another
-//               chunk's store.
+//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time, scale / bias / neuron in fp32;
+//               each warp stages its 32 rows in its own 4 KB of shared memory (128-byte
+//               swizzle) and reads them back so that each store instruction writes 4 output
+//               rows x 128 contiguous bytes; junk rows are skipped.  No TMA store, and a chunk
+//               never waits for another warp's stores.  Beta is formed ahead for a batch of
+//               tiles at a time (the first batch while the first tile's MMAs run) from their
+//               strips of A, staged through the same buffers.
 // Every mbarrier wait gives up after one second of %globaltimer, sets the error word and
 // makes all roles stop; TMEM is released on every exit path.
 #include <cuda.h>
@@ -56,7 +57,9 @@ constexpr int kEpiThreads = 128;
 constexpr int kHaloStages = 2;
 constexpr int kMaxWStages = 8;
 constexpr int kWarpStageBytes = 32 * 128;           // one epilogue warp's 32 rows x 32 fp32
-constexpr int kAStrip = 1024;                        // floats of A a tile's beta reads, at most
+constexpr int kAStrip = 1024;                        // longest halo (and strip of A) a tile reads
+constexpr int kStripFloats = 4 * kWarpStageBytes / 4;  // strips of A staged in the epilogue's buffers
+constexpr int kMaxTiles = 6;                         // tiles whose betas are formed in one batch
 constexpr int kMinResidentBN = 128;                  // narrowest tile the plan narrows to
 
 struct __align__(8) HaloBars {
@@ -69,8 +72,8 @@ struct __align__(8) HaloBars {
   uint64_t done;
   uint32_t tmem_base;
   uint32_t abort_flag;
-  float2 sb[256];  // (scale, bias) of the CTA's output channels
-  float astrip[kAStrip];  // the tile's rows of A (with the window's margin), zero outside the image
+  float2 sb[128];                // (scale, bias) of the CTA's output channels (BN <= 128)
+  float betas[kMaxTiles * 128];  // beta of each row of the current batch of tiles
 };
 
 // 16 consecutive 32-bit TMEM columns of this warp's 32 lanes.
@@ -283,21 +286,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     const int et = threadIdx.x - 64;
+    // betas are formed for a batch of tiles at a time, the first batch while the first tile's
+    // MMAs run, through the (then idle) staging buffers
+    const int batch = min(kMaxTiles, kStripFloats / a.halo_len);
     int ti = 0;
     for (int m = slot0; m < a.m_tiles; m += slots, ++ti) {
       const int s0 = m * 128;
-      float beta = 1.f;
-      if (a.A) {
-        // beta = sum of A over the window / (kh*kw): A lies in the zero-bordered grid, so the
-        // tile's strip of it (one coalesced pass) holds every position its slots' windows cover
-        for (int i = et; i < a.halo_len; i += kEpiThreads)
-          B->astrip[i] = s0 + i < total_slots ? __ldg(a.A + s0 + i) : 0.f;
-        epi_barrier();
-        float sum = 0.f;
-        for (int ty = 0; ty < a.kh; ++ty)
-          for (int tx = 0; tx < a.kw; ++tx) sum += B->astrip[row + ty * a.Wp + tx];
-        beta = sum / static_cast<float>(a.kh * a.kw);
-      }
+      if (a.A && ti % batch == 0)
+        tile_betas(a.A, total_slots, m, slots, min(batch, (a.m_tiles - m + slots - 1) / slots), a.halo_len,
+                   a.kh, a.kw, a.Wp, reinterpret_cast<float*>(stage_out), B->betas, row, true, et, kEpiThreads);
+      const float beta = a.A ? B->betas[(ti % batch) * 128 + row] : 1.f;
       // the output rows this lane stores: rows 4i + lane / 8 of the warp's 32 (i = 0..7)
       int64_t dst[8];
 #pragma unroll
@@ -308,8 +306,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool ok = sl < total_slots && oy < a.H && ox < a.W;
         dst[i] = ok ? ((static_cast<int64_t>(n) * a.H + oy) * a.W + ox) * a.No : -1;
       }
-      // (a barrier across the epilogue warps: every row's beta is formed before the strip is
-      // overwritten for the next tile)
       if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err, true, true))) break;
       tc_fence_after();
       if (et == 0 && ti < 8) BCONV_STAMP(21 + 2 * ti);
@@ -384,7 +380,7 @@ bool tc_halo_plan(HaloArgs& a, int sm_count) {
   if (static_cast<int64_t>(a.N) * a.Hp * a.Wp + 1024 >= (int64_t{1} << 31)) return false;  // int32 slot indices
   // every row any tile's MMAs read: the 128 slots plus the window's reach
   a.halo_len = 128 + (a.kh - 1) * a.Wp + (a.kw - 1);
-  if (a.halo_len > kAStrip) return false;  // the tile's strip of A must fit
+  if (a.halo_len > kAStrip) return false;  // at least four tiles' strips of A fit the staging
   a.m_tiles = static_cast<int>((static_cast<int64_t>(a.N) * a.Hp * a.Wp + 127) / 128);
   a.halo_boxes = (a.halo_len + 255) / 256;
   a.halo_rows = round_up((a.halo_len + a.halo_boxes - 1) / a.halo_boxes, 8);

@@ -21,7 +21,10 @@
 // both CTAs; warps 2-9 of each CTA (two per TMEM lane quarter, 128 columns each) read the
 // accumulator into registers at once and hand it back -- there is room in TMEM for one 256-column
 // accumulator and the scale factors only -- then apply beta, scale, bias and the neuron and
-// store 16 channels at a time through 2 KB of shared memory per warp.  TMEM is allocated with
+// store 32 channels x 16 rows at a time through 2 KB of shared memory per warp, so that every
+// store instruction writes whole 128-byte lines (the SMs' write requests, not bytes, bound
+// this epilogue).  Beta is formed ahead for a batch of tiles from their strips of A, staged
+// through the same buffers while the first tile's MMAs run.  TMEM is allocated with
 // cta_group::2 in both CTAs; the pair synchronises (cluster barrier) after set-up and before
 // exit.  Every mbarrier wait gives up after one second of %globaltimer, sets the error word and
 // makes all roles stop; TMEM is released on every exit path.
@@ -45,9 +48,12 @@ constexpr int kMaxWStages = 10;
 constexpr int kBN = 256;                       // output channels per pair item
 constexpr int kHalfRows = kBN / 2;             // weight rows each CTA holds
 constexpr int kWBlock = kHalfRows * 128;       // one (tap, k-block) weight block of one CTA: 16 KB
-constexpr int kOutCols = 16;                   // output channels per epilogue chunk
-constexpr int kWarpStage = 32 * kOutCols * 4;  // one epilogue warp's 32 rows x 16 fp32
-constexpr int kAStrip = 1024;
+constexpr int kOutCols = 32;                   // output channels per epilogue chunk: 128-byte row pieces
+constexpr int kStageRows = 16;                 // rows staged at a time (half a warp's 32)
+constexpr int kWarpStage = kStageRows * kOutCols * 4;  // 2 KB per epilogue warp
+constexpr int kAStrip = 1024;                  // longest halo (and strip of A) a tile reads
+constexpr int kStripFloats = 8 * kWarpStage / 4;  // strips of A staged in the epilogue's buffers
+constexpr int kMaxTiles = 4;                   // tiles whose betas are formed in one batch
 constexpr uint32_t kTmemCols = 512;            // the accumulator (256) and 64 scale-factor columns
 
 struct __align__(16) PairHaloBars {
@@ -61,7 +67,7 @@ struct __align__(16) PairHaloBars {
   uint32_t tmem_base;
   uint32_t abort_flag;
   float2 sb[kBN];                // (scale, bias) of the pair's 256 output channels
-  float astrip[kAStrip];         // the tile's strip of A in the zero-bordered grid
+  float betas[kMaxTiles * 128];  // beta of each row of the current batch of this CTA's tiles
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -262,32 +268,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int et = threadIdx.x - 64;          // 0..255
     uint8_t* wst = stage_out + (warp - 2) * kWarpStage;
     const uint32_t empty_leader = mapa(&B->tmem_empty, 0);
+    // betas are formed for a batch of tiles at a time, the first batch while the first tile's
+    // MMAs run, through the (then idle) staging buffers
+    const int batch = min(kMaxTiles, kStripFloats / a.halo_len);
     int ti = 0;
     for (int pt = pslot0; pt < pair_tiles; pt += pslots, ++ti) {
       const int s0 = (2 * pt + static_cast<int>(rank)) * 128;
-      float beta = 1.f;
-      if (a.A) {
-        // beta = sum of A over the window / (kh*kw), from the tile's strip of the zero-bordered A
-        for (int i = et; i < a.halo_len; i += kEpiThreads)
-          B->astrip[i] = s0 + i < total_slots ? __ldg(a.A + s0 + i) : 0.f;
-        named_barrier(kEpiThreads);
-        float sum = 0.f;
-        for (int ty = 0; ty < a.kh; ++ty)
-          for (int tx = 0; tx < a.kw; ++tx) sum += B->astrip[row + ty * a.Wp + tx];
-        beta = sum / static_cast<float>(a.kh * a.kw);
-      }
-      // this lane's store rows: 8 i + lane / 4 of the warp's 32 (i = 0..3), 16 bytes each of 64
-      int64_t dst[4];
+      if (a.A && ti % batch == 0)
+        tile_betas(a.A, total_slots, 2 * pt + static_cast<int>(rank), 2 * pslots,
+                   min(batch, (pair_tiles - pt + pslots - 1) / pslots), a.halo_len, a.kh, a.kw, a.Wp,
+                   reinterpret_cast<float*>(stage_out), B->betas, row, half == 0, et, kEpiThreads);
+      const float beta = a.A ? B->betas[(ti % batch) * 128 + row] : 1.f;
+      // this lane's store rows: 4 i + lane / 8 of the warp's 32 (i = 0..7), 16 bytes each of 128;
+      // their output pixels (N * H * W < 2^31), or -1 for junk slots
+      int dst[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int sl = s0 + q * 32 + 8 * i + (lane >> 2);
+      for (int i = 0; i < 8; ++i) {
+        const int sl = s0 + q * 32 + 4 * i + (lane >> 3);
         const int n = sl / rows_per_img, rem = sl - n * rows_per_img;
         const int oy = rem / a.Wp, ox = rem - oy * a.Wp;
         const bool ok = sl < total_slots && oy < a.H && ox < a.W;
-        dst[i] = ok ? ((static_cast<int64_t>(n) * a.H + oy) * a.W + ox) * a.No : -1;
+        dst[i] = ok ? (n * a.H + oy) * a.W + ox : -1;
       }
-      // (a barrier across the epilogue warps: every row's beta is formed before the strip is
-      // overwritten for the next tile)
       if (!named_all(mbar_wait(&B->tmem_full, ti & 1, B, a.err, true, true), kEpiThreads)) break;
       tc_fence_after();
       if (et == 0 && ti < 8) BCONV_STAMP(21 + 2 * ti);
@@ -309,26 +311,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < kOutCols; ++j) {
           const float2 p = B->sb[half * 128 + ch * kOutCols + j];
-          const float s = __uint_as_float(v[ch * kOutCols + j]);
-          const float r = a.A ? fmaf(s * p.x, beta, p.y) : fmaf(s, p.x, p.y);
+          const float sv = __uint_as_float(v[ch * kOutCols + j]);
+          const float r = a.A ? fmaf(sv * p.x, beta, p.y) : fmaf(sv, p.x, p.y);
           y[j] = a.relu ? fmaxf(r, 0.f) : r;
         }
-        // 64-byte row per lane, 16-byte chunk k at k ^ ((row >> 1) & 3)
-        float4* orow = reinterpret_cast<float4*>(wst + lane * 64);
+        const int c = cbase + ch * kOutCols + 4 * (lane & 7);
+        // 16 rows at a time through the warp's 2 KB (16-byte piece k of row r at k ^ (r % 8)):
+        // each store instruction then writes 4 rows x 128 contiguous bytes
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          orow[k ^ ((lane >> 1) & 3)] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
-        __syncwarp();
-        const int c = cbase + ch * kOutCols + 4 * (lane & 3);
-        if (c < a.No) {  // No % 4 == 0: a float4 of channels is all real or all padding
+        for (int h = 0; h < 32 / kStageRows; ++h) {
+          if ((lane >> 4) == h) {
+            float4* orow = reinterpret_cast<float4*>(wst + (lane & 15) * 128);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = 8 * i + (lane >> 2);
-            const float4 val = reinterpret_cast<const float4*>(wst + r * 64)[(lane & 3) ^ ((r >> 1) & 3)];
-            if (dst[i] >= 0) *reinterpret_cast<float4*>(a.out + dst[i] + c) = val;
+            for (int k = 0; k < 8; ++k)
+              orow[k ^ (lane & 7)] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
           }
+          __syncwarp();
+          if (c < a.No) {  // No % 4 == 0: a float4 of channels is all real or all padding
+#pragma unroll
+            for (int i = 0; i < kStageRows / 4; ++i) {
+              const int r = 4 * i + (lane >> 3);
+              const float4 val = reinterpret_cast<const float4*>(wst + r * 128)[(lane & 7) ^ (r & 7)];
+              const int d = dst[h * (kStageRows / 4) + i];
+              if (d >= 0) *reinterpret_cast<float4*>(a.out + static_cast<int64_t>(d) * a.No + c) = val;
+            }
+          }
+          __syncwarp();  // the rows are read before the next ones overwrite them
         }
-        __syncwarp();
       }
       if (et == 0 && ti < 8) BCONV_STAMP(22 + 2 * ti);
     }

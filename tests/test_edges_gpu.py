@@ -264,17 +264,18 @@ def _spread(w, mode=None, codes=None):
 
 
 def test_spread_choice(cuda_device):
-    """AUTO: XNOR/AND on e2m1 codes, one SM per tile; with int8 codes one SM per tile where the
-    pair plan is not clearly shorter (equal waves), SM pairs where their balanced split evens
-    out a ragged last wave by more and for the FC with batch > 128; binaryWeights on bf16 parts
-    (its 24 against 27 stages on pairs is not enough for them); forced modes are kept where the
-    layer allows them."""
+    """AUTO: XNOR/AND on e2m1 codes -- stride-1 layers rows-staged, on SM pairs above 128 output
+    channels, else one SM per tile; with int8 codes one SM per tile where the pair plan is not
+    clearly shorter (equal waves), SM pairs where their balanced split evens out a ragged last
+    wave by more and for the FC with batch > 128; binaryWeights on bf16 parts (its 24 against 27
+    stages on pairs is not enough for them); forced modes are kept where the layer allows them."""
     S, P, I8, F4, BF = bc.CTA_SINGLE, bc.CTA_PAIR, bc.CODES_INT8, bc.CODES_FP4, bc.CODES_BF16X3
     c2 = synth.workload("xnor_beta_n16_56x56_c256_k256_3x3")
-    assert _spread(c2) == (S, F4)
+    assert _spread(c2) == (P, F4)  # rows-staged on SM pairs, 256-channel MMAs
+    assert _spread(c2, mode=S) == (S, F4)
     assert _spread(c2, codes=I8) == (S, I8)
-    assert _spread(c2, mode=P) == (P, I8)  # SM pairs take int8 codes
-    assert _spread(synth.workload("and_n32_28x28_c512_k512_3x3")) == (S, F4)
+    assert _spread(c2, mode=P) == (P, I8)  # forced pairs take the int8 per-tap pair kernel
+    assert _spread(synth.workload("and_n32_28x28_c512_k512_3x3")) == (P, F4)
     assert _spread(synth.workload("binw_n8_112x112_c128_k128_3x3_s2")) == (S, BF)
     assert _spread(synth.workload("fc_xnor_beta_n256_7x7x512_k4096"), codes=I8) == (P, I8)
     ragged = synth.small_case(batch=4, h=70, w=70, ni=32, no=32, k=3, op=synth.XNOR, seed=27)
