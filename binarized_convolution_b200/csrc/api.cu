@@ -319,7 +319,7 @@ bconv_status_t setup_fc(Layer& L, const uint32_t* packed) {
   f.No = L.No;
   f.hw = hw;
   f.kb_total = hw * (L.cip / 256);
-  tc_fc_plan(f, current_sm_count());
+  if (!tc_fc_plan(f, current_sm_count())) return BCONV_OK;  // (checked by the caller)
   const int64_t rows = static_cast<int64_t>(f.n_tiles) * 256;
   const int64_t row_bytes = static_cast<int64_t>(hw) * px_bytes;
   const Layer* src = L.weights_from;
@@ -384,6 +384,13 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   t.kind = L.type == kBinaryWeights                                                   ? 1
            : (codes == BCONV_CODES_INT8 || mode == BCONV_CTA_PAIR || !fp32_exact) ? 0
                                                                                    : 2;
+  if (L.fc && t.kind == 2) {  // the e2m1 FC kernel adds int16 partial sums: at most 127 k-blocks a split
+    FcArgs f{};
+    f.N = L.N;
+    f.No = L.No;
+    f.kb_total = L.H * L.W * (round_up(L.Ni, 256) / 256);
+    if (!tc_fc_plan(f, current_sm_count())) t.kind = 0;
+  }
   // channels per part, padded to whole 128-byte rows; bytes of activation operand per pixel
   // (kind 1: three bf16 parts) and of weights per output channel and tap (kind 1: one bf16
   // copy, which every part is multiplied with; kind 2: two codes per byte)

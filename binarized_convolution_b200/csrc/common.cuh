@@ -83,13 +83,35 @@ cudaError_t launch_overlapped(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 // (at (n, y + pad_t, x + pad_l)); hp == 0 means no border (the pixel keeps its index).
 struct PadMap {
   int h, w, hp, wp, pad_t, pad_l;
+  // (A zero-bordered grid is only planned when N * hp * wp < 2^31, so p fits 32 bits then.)
   __host__ __device__ __forceinline__ int64_t operator()(int64_t p) const {
     if (hp == 0) return p;
-    const int64_t hw = static_cast<int64_t>(h) * w;
-    const int64_t n = p / hw;
-    const int r = static_cast<int>(p - n * hw);
-    const int y = r / w, x = r - y * w;
-    return (n * hp + y + pad_t) * wp + x + pad_l;
+    const uint32_t pp = static_cast<uint32_t>(p), hw = static_cast<uint32_t>(h) * static_cast<uint32_t>(w);
+    const uint32_t n = pp / hw, r = pp - n * hw;
+    const uint32_t y = r / static_cast<uint32_t>(w), x = r - y * static_cast<uint32_t>(w);
+    return (static_cast<int64_t>(n) * hp + y + pad_t) * wp + x + pad_l;
+  }
+  // The place of pixel p + 1 from that of pixel p, whose column and row are x and y (updated).
+  __host__ __device__ __forceinline__ int64_t next(int64_t q, int& y, int& x) const {
+    if (hp == 0) return q + 1;
+    ++q;
+    if (++x == w) {
+      x = 0;
+      q += wp - w;
+      if (++y == h) {
+        y = 0;
+        q += static_cast<int64_t>(hp - h) * wp;
+      }
+    }
+    return q;
+  }
+  // Column and row of pixel p.
+  __host__ __device__ __forceinline__ void yx(int64_t p, int& y, int& x) const {
+    if (hp == 0) return;
+    const uint32_t pp = static_cast<uint32_t>(p), hw = static_cast<uint32_t>(h) * static_cast<uint32_t>(w);
+    const uint32_t r = pp % hw;
+    y = static_cast<int>(r / static_cast<uint32_t>(w));
+    x = static_cast<int>(r - static_cast<uint32_t>(y) * static_cast<uint32_t>(w));
   }
 };
 

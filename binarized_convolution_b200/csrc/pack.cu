@@ -188,11 +188,16 @@ __global__ void __launch_bounds__(kPackThreads, 2) pack_i8_vec_kernel(PackI8Args
   for (; p0 < a.npix; p0 += step) {
     float4 nxt[kG][kC];
     if (p0 + step < a.npix) load_group<kG, kC>(nxt, in, p0 + step, a.npix, ni, live, lane);
+    // the places of the step's pixels in the code buffer: one division for the first, then
+    // steps along the row (over the border at a row's or an image's end)
+    int py = 0, px = 0;
+    a.pad.yx(p0, py, px);
+    int64_t q = a.pad(p0);
 #pragma unroll
     for (int g = 0; g < kG; ++g) {
       const int64_t p = p0 + g;
       if (p >= a.npix) break;  // warp-uniform
-      const int64_t q = a.pad(p);  // the pixel's place in the code buffer
+      if (g > 0) q = a.pad.next(q, py, px);
       float asum = 0.f;
 #pragma unroll
       for (int c = 0; c < kC; ++c) {

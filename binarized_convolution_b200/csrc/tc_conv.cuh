@@ -124,7 +124,7 @@ struct FcArgs {
   int hw;             // pixels per image (the window of beta)
   int kb_total;       // k-blocks of the flattened image
   // filled by tc_fc_plan
-  int m_tiles, n_tiles, k_splits, kb_per_split;  // k_splits: 1..8, a divisor of 128
+  int m_tiles, n_tiles, k_splits, kb_per_split;  // k_splits: 1, 2, 4 or 8; kb_per_split <= 127
   const float* scale;
   const float* bias;
   const float* A;     // [N][hw] channel means, or nullptr (no beta)
@@ -132,7 +132,9 @@ struct FcArgs {
   uint32_t* err;
   float* out;         // [N][No] output, 16-byte aligned
 };
-void tc_fc_plan(FcArgs& a, int sm_count);
+// false: the shape does not fit this kernel (more than 127 k-blocks per split even with 8
+// splits, whose int16 partial sums would overflow, or no cluster fits the device)
+bool tc_fc_plan(FcArgs& a, int sm_count);
 int tc_fc_smem_bytes();
 // tmA: 2-D map over the activation codes {K / 2 bytes, N}, box 128 x 128; tmB: 2-D map over the
 // weight codes {K / 2 bytes, n_tiles * 256}, box 128 x 256; both 128-byte swizzled.

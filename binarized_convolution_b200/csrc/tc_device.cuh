@@ -59,21 +59,28 @@ __device__ __forceinline__ bool mbar_try_suspend(uint64_t* bar, uint32_t parity,
 // Wait for the phase with the given parity to complete; false after the time limit or, when
 // `follow_abort`, as soon as another role has given up (the caller then stops).  `idle`
 // waits (the epilogue's wait for an accumulator, the final drain) suspend between checks.
+// The polling loop is out of line: inlined into an MMA-issuing loop, even untaken, it slowed
+// the issue enough to starve the tensor pipe; the inlined part is one try_wait.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint32_t* abort_flag,
+                                                   uint32_t* err, bool follow_abort, bool idle, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (idle ? mbar_try_suspend(bar, parity, 20000u) : mbar_try(bar, parity)) return true;
+    if (follow_abort && *reinterpret_cast<volatile uint32_t*>(abort_flag)) return false;
+    if (globaltimer() - t0 > limit_ns) {
+      atomicOr(err, kErrTimeout);
+      atomicExch(abort_flag, 1u);
+      return false;
+    }
+  }
+}
+
 template <class Bars>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Bars* B, uint32_t* err,
                                           bool follow_abort = true, bool idle = false,
                                           uint64_t limit_ns = kTimeoutNs) {
   if (mbar_try(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-    if (idle ? mbar_try_suspend(bar, parity, 20000u) : mbar_try(bar, parity)) return true;
-    if (follow_abort && *reinterpret_cast<volatile uint32_t*>(&B->abort_flag)) return false;
-    if (globaltimer() - t0 > limit_ns) {
-      atomicOr(err, kErrTimeout);
-      atomicExch(&B->abort_flag, 1u);
-      return false;
-    }
-  }
+  return mbar_wait_slow(bar, parity, &B->abort_flag, err, follow_abort, idle, limit_ns);
 }
 
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
@@ -288,8 +295,11 @@ __device__ __forceinline__ uint32_t mapa(const void* p, uint32_t rank) {
   return r;
 }
 
+// (Release semantics at CTA scope, the default: what the arrival hands over -- TMEM columns
+// read with tcgen05.ld and waited for -- is ordered by the tcgen05 fences, not by this fence; a
+// cluster-scope release waited for this thread's earlier global stores, about a microsecond.)
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,

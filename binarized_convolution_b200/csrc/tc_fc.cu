@@ -14,14 +14,18 @@
 // weight codes (both 128-byte swizzled) feed four M128 N256 K64 MMAs: the activations are read
 // once per 256 channels, the weights once per 128 images.
 //
-// The k_splits items of a tile form one cluster.  After its MMAs each CTA writes its exact
-// partial sums (a 128 x 256 fp32 tile, 16-byte pieces XOR-swizzled within each row) into its
-// own shared memory; after a cluster barrier each CTA finishes 128 / k_splits rows: it reads the
-// rows of every CTA's partial tile through distributed shared memory, adds them in rank order
-// (integers below 2^24: exact in fp32 in any order), applies beta (formed by the epilogue warps
-// while the MMAs run), scale, bias and the neuron, and writes each output row with coalesced
-// stores.  A second cluster barrier keeps every CTA's shared memory alive until all have read it.
-// No workspace and no second launch.
+// The k_splits items of a tile form one cluster, and each CTA finishes 128 / k_splits rows of
+// the tile.  Once every CTA of the cluster has completed its MMAs (a cluster barrier), their
+// stage memory is idle and becomes receive buffers (k_splits slots x the owner's rows x 256
+// int16): each CTA reads its accumulator and sends every row's exact partial sums, as int16
+// (|partial| <= 256 x k-blocks per split <= 32512), to the row's owner -- st.async into the
+// peers, completing on the owner's mbarrier, and plain stores for its own rows.  The owner
+// adds the slots in rank order (int32, exact), applies beta (formed by the epilogue warps
+// while the MMAs run), scale, bias and the neuron and writes each output row with coalesced
+// stores.  (The barrier costs nothing on the critical path: an owner needs every split's
+// partial sums, so it waits for the slowest CTA of its cluster anyway.)  A second cluster
+// barrier keeps every CTA alive until the pushes into it are done.  No workspace, no second
+// launch.
 //
 // Roles (6 warps): warp 0 TMA producer (4-stage ring); warp 1 TMEM allocation and, from one
 // thread, the MMAs; warps 2-5 the epilogue.  Every mbarrier wait gives up after one second of
@@ -48,77 +52,45 @@ constexpr int kABytes = 128 * 128;     // 128 images x one k-block of codes
 constexpr int kBBytes = kBN * 128;     // 256 channels x one k-block of codes
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kTmemCols = 512;    // the accumulator (256) and 64 scale-factor columns
+constexpr int kRowBytes = kBN * 2;     // one row of int16 partial sums
+constexpr int kRecvBytes = 128 * kRowBytes;  // k_splits slots x (128 / k_splits) rows, in stage memory
+constexpr int kMaxKbPerSplit = 127;    // 256 codes per k-block: |partial| <= 32512 fits int16
 
 struct __align__(16) FcBars {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t tmem_full;
   uint64_t done;
+  uint64_t recv;  // this CTA's rows of every split's partial sums have arrived
   uint32_t tmem_base;
   uint32_t abort_flag;
   float2 sb[kBN];
   float beta[128];
 };
 
-// Offset, within a CTA's partial tile (128 rows x 1 KB), of float4 `k` (0..63) of row `r`: the
-// low three bits of the float4 index are XORed with the row's, so that 32 consecutive rows
-// writing the same float4 index hit different banks.
-__device__ __forceinline__ uint32_t part_off(int r, int k) {
-  return static_cast<uint32_t>(r * 1024 + (((k & ~7) | ((k & 7) ^ (r & 7))) * 16));
+static_assert(kRecvBytes <= kStages * kStageBytes, "the receive buffers live in the stage memory");
+static_assert(kStages * kStageBytes + sizeof(FcBars) <= 227 * 1024, "shared memory of one CTA");
+
+// Byte offset, in a receive buffer, of 16-byte piece k (0..31: columns 8 k .. 8 k + 7) of slot
+// row sr: the piece index is XORed with the row's low five bits, so that 32 consecutive rows
+// writing (or a row's 32 pieces read) hit distinct banks.
+__device__ __forceinline__ uint32_t recv_off(int sr, int k) {
+  return static_cast<uint32_t>(sr * kRowBytes + ((k ^ (sr & 31)) * 16));
 }
 
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
-  return v;
+// 16 bytes into another CTA's shared memory (cluster address), completing `bytes` on its mbarrier.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w,
+                                            uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   addr),
+               "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+               : "memory");
 }
 
-// Rows [split * 128 / KS, (split + 1) * 128 / KS) of the tile from the KS partial tiles of the
-// cluster: warp q of the epilogue takes every fourth row, lane l channels 8 l .. 8 l + 7.  All
-// KS x 2 distributed-shared-memory loads of a row (two rows when KS <= 4) are issued before any
-// is used, so that a row costs one remote latency rather than KS of them.
-template <int KS>
-__device__ __forceinline__ void finish_rows(const FcArgs& a, const FcBars* B, const uint8_t* smem, int split, int m0,
-                                            int c0, int q, int lane) {
-  constexpr int kRowsPer = 128 / KS;
-  constexpr int kUnroll = KS <= 4 ? 2 : 1;  // rows in flight per warp
-  uint32_t base[KS];
-#pragma unroll
-  for (int p = 0; p < KS; ++p) base[p] = mapa(smem, static_cast<uint32_t>(p));
-  for (int r0 = split * kRowsPer + q; r0 < (split + 1) * kRowsPer; r0 += 4 * kUnroll) {
-    float4 u[kUnroll][KS][2];
-#pragma unroll
-    for (int h = 0; h < kUnroll; ++h)
-#pragma unroll
-      for (int p = 0; p < KS; ++p) {
-        const int r = r0 + 4 * h;
-        u[h][p][0] = ld_cluster_f4(base[p] + part_off(r, 2 * lane));
-        u[h][p][1] = ld_cluster_f4(base[p] + part_off(r, 2 * lane + 1));
-      }
-#pragma unroll
-    for (int h = 0; h < kUnroll; ++h) {
-      const int r = r0 + 4 * h;
-      const int nn = m0 + r;
-      if (nn >= a.N) continue;
-      float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int p = 0; p < KS; ++p) {  // rank order
-        y[0] += u[h][p][0].x; y[1] += u[h][p][0].y; y[2] += u[h][p][0].z; y[3] += u[h][p][0].w;
-        y[4] += u[h][p][1].x; y[5] += u[h][p][1].y; y[6] += u[h][p][1].z; y[7] += u[h][p][1].w;
-      }
-      const float bb = B->beta[r];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float2 p = B->sb[8 * lane + j];
-        const float v = a.A ? fmaf(y[j] * p.x, bb, p.y) : fmaf(y[j], p.x, p.y);
-        y[j] = a.relu ? fmaxf(v, 0.f) : v;
-      }
-      const int c = c0 + 8 * lane;
-      float* o = a.out + static_cast<int64_t>(nn) * a.No + c;
-      if (c < a.No) *reinterpret_cast<float4*>(o) = make_float4(y[0], y[1], y[2], y[3]);
-      if (c + 4 < a.No) *reinterpret_cast<float4*>(o + 4) = make_float4(y[4], y[5], y[6], y[7]);
-    }
-  }
+// Two integer-valued fp32 sums (|v| < 2^15) as int16 halves of one word.
+__device__ __forceinline__ uint32_t pack_i16x2(uint32_t lo_f, uint32_t hi_f) {
+  const int lo = __float2int_rn(__uint_as_float(lo_f)), hi = __float2int_rn(__uint_as_float(hi_f));
+  return (static_cast<uint32_t>(lo) & 0xFFFFu) | (static_cast<uint32_t>(hi) << 16);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -128,8 +100,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) atomicOr(a.err, kErrLayout);
     return;
   }
-  // stage s: [A codes 16 KB][B codes 32 KB]; the epilogue reuses the first stage
+  // stage s: [A codes 16 KB][B codes 32 KB]; once the cluster's MMAs are done the first 64 KB
+  // receive the partial sums
   uint8_t* smem = smem_raw;
+  uint8_t* recv = smem;
   FcBars* B = reinterpret_cast<FcBars*>(smem + kStages * kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // item -> (split = the CTA's rank in its cluster, N tile, M tile)
@@ -150,8 +124,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&B->tmem_full, 1);
     mbar_init(&B->done, 1);
+    mbar_init(&B->recv, 1);
     B->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    // the one arrival, before any byte can land: the other splits' slots of this CTA's rows
+    mbar_expect_tx(&B->recv, static_cast<uint32_t>((a.k_splits - 1) * (128 / a.k_splits) * kRowBytes));
     prefetch_tensor_map(&tmA);
     prefetch_tensor_map(&tmB);
   }
@@ -233,8 +210,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
     const int et = threadIdx.x - 64;  // 0..127
-    const int q = warp & 3;
-    const int row = q * 32 + lane;    // TMEM lane = image m0 + row
     // betas of the tile's images, while the MMAs run: beta_n = mean of A over the image
     {
       float b = 1.f;
@@ -247,45 +222,89 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       B->beta[et] = b;
     }
-    bool ok = epi_all(mbar_wait(&B->tmem_full, 0, B, a.err, true, true));
-    if (ok) {
+    if (__all_sync(0xffffffffu, mbar_wait(&B->tmem_full, 0, B, a.err, true, true))) {
       tc_fence_after();
       if (et == 0) BCONV_STAMP(4);
-      // this CTA's partial tile into its (now idle) stage memory; a split past the last k-block
-      // (k_splits * kb_per_split may exceed kb_total by up to a share) issued no MMA and adds 0
-      const bool no_kb = kb1 <= kb0;
-      for (int ch = 0; ch < kBN / 32; ++ch) {
-        uint32_t v[32];
-        if (no_kb) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0u;
-        } else {
-          tc_ld_32x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ch * 32), v);
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          *reinterpret_cast<float4*>(smem + part_off(row, ch * 8 + k)) =
-              make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]), __uint_as_float(v[4 * k + 2]),
-                          __uint_as_float(v[4 * k + 3]));
-      }
-      if (et == 0) BCONV_STAMP(5);
     }
   }
 
   // every CTA of the cluster reaches both barriers, whatever happened above
   tc_fence_before();
   __syncthreads();
-  cluster_sync();  // every partial tile of the cluster is written
+  cluster_sync();  // every MMA of the cluster has completed: all stage memory is idle
   if (warp >= 2 && !*reinterpret_cast<volatile uint32_t*>(&B->abort_flag)) {
-    switch (a.k_splits) {
-      case 1: finish_rows<1>(a, B, smem, split, m0, c0, warp & 3, lane); break;
-      case 2: finish_rows<2>(a, B, smem, split, m0, c0, warp & 3, lane); break;
-      case 4: finish_rows<4>(a, B, smem, split, m0, c0, warp & 3, lane); break;
-      default: finish_rows<8>(a, B, smem, split, m0, c0, warp & 3, lane); break;
+    tc_fence_after();
+    const int et = threadIdx.x - 64;
+    const int q = warp & 3;
+    const int row = q * 32 + lane;  // TMEM lane = image m0 + row
+    const int rows_per = 128 / a.k_splits;
+    // this row's partial sums to its owner: slot row split * rows_per + (row % rows_per) of CTA
+    // row / rows_per; a split past the last k-block (k_splits * kb_per_split may exceed
+    // kb_total by up to a share) issued no MMA and sends zeros
+    const int owner = row / rows_per;
+    const int sr = split * rows_per + (row - owner * rows_per);
+    const bool local = owner == split;
+    const uint32_t dst = mapa(recv, static_cast<uint32_t>(owner));
+    const uint32_t bar = mapa(&B->recv, static_cast<uint32_t>(owner));
+    const bool no_kb = kb1 <= kb0;
+    for (int ch = 0; ch < kBN / 32; ++ch) {
+      uint32_t v[32];
+      if (no_kb) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0u;
+      } else {
+        tc_ld_32x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ch * 32), v);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {  // piece 4 ch + i: columns 32 ch + 8 i .. + 7
+        const uint32_t w0 = pack_i16x2(v[8 * i], v[8 * i + 1]), w1 = pack_i16x2(v[8 * i + 2], v[8 * i + 3]);
+        const uint32_t w2 = pack_i16x2(v[8 * i + 4], v[8 * i + 5]), w3 = pack_i16x2(v[8 * i + 6], v[8 * i + 7]);
+        if (local)
+          *reinterpret_cast<uint4*>(recv + recv_off(sr, 4 * ch + i)) = make_uint4(w0, w1, w2, w3);
+        else
+          st_async_v4(dst + recv_off(sr, 4 * ch + i), w0, w1, w2, w3, bar);
+      }
     }
-    if (warp == 2 && lane == 0) BCONV_STAMP(6);
+    if (et == 0) BCONV_STAMP(5);
+    // this CTA's rows: every split's partial sums, added in rank order
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&B->recv, 0, B, a.err, true, true));
+    epi_barrier();  // (the local slots, written by the other epilogue warps)
+    if (ok) {
+      for (int r = q; r < rows_per; r += 4) {
+        const int tr = split * rows_per + r;  // row of the tile
+        const int nn = m0 + tr;
+        if (nn >= a.N) break;
+        int acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (int p = 0; p < a.k_splits; ++p) {
+          const int psr = p * rows_per + r;
+          const uint4 w = *reinterpret_cast<const uint4*>(recv + recv_off(psr, lane));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            acc[2 * j] += static_cast<int>(static_cast<int16_t>(ww[j] & 0xFFFFu));
+            acc[2 * j + 1] += static_cast<int>(ww[j]) >> 16;
+          }
+        }
+        const float bb = B->beta[tr];
+        float y[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float2 p = B->sb[8 * lane + j];
+          const float sv = static_cast<float>(acc[j]);  // |S| < 2^24: exact
+          const float v = a.A ? fmaf(sv * p.x, bb, p.y) : fmaf(sv, p.x, p.y);
+          y[j] = a.relu ? fmaxf(v, 0.f) : v;
+        }
+        const int c = c0 + 8 * lane;
+        float* o = a.out + static_cast<int64_t>(nn) * a.No + c;
+        if (c < a.No) *reinterpret_cast<float4*>(o) = make_float4(y[0], y[1], y[2], y[3]);
+        if (c + 4 < a.No) *reinterpret_cast<float4*>(o + 4) = make_float4(y[4], y[5], y[6], y[7]);
+      }
+      if (et == 0) BCONV_STAMP(6);
+    }
   }
-  cluster_sync();  // no CTA leaves while another may still read its partial tile
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while a peer may still push into its receive buffer
   allow_next_grid();
   if (warp == 1) {
     tc_fence_after();
@@ -325,7 +344,7 @@ int fc_max_clusters(int ks) {
 }
 }  // namespace
 
-void tc_fc_plan(FcArgs& a, int sm_count) {
+bool tc_fc_plan(FcArgs& a, int sm_count) {
   a.m_tiles = (a.N + 127) / 128;
   a.n_tiles = (a.No + kBN - 1) / kBN;
   const int tiles = a.m_tiles * a.n_tiles;
@@ -335,15 +354,19 @@ void tc_fc_plan(FcArgs& a, int sm_count) {
   int ks = std::max(1, sm_count / std::max(tiles, 1));
   ks = std::min({ks, 8, std::max(1, a.kb_total / 4)});
   while (ks > 1 && (128 % ks != 0 || fc_max_clusters(ks) < tiles)) --ks;
+  // each split's partial sums travel as int16: at most kMaxKbPerSplit k-blocks per split
+  while ((a.kb_total + ks - 1) / ks > kMaxKbPerSplit && ks < 8) ks *= 2;
+  if ((a.kb_total + ks - 1) / ks > kMaxKbPerSplit || fc_max_clusters(ks) < 1) return false;
   a.kb_per_split = (a.kb_total + ks - 1) / ks;
   a.k_splits = ks;
+  return true;
 }
 
 cudaError_t launch_tc_fc(const CUtensorMap* tmA, const CUtensorMap* tmB, const FcArgs& a, cudaStream_t s) {
   const int items = a.m_tiles * a.n_tiles * a.k_splits;
   if (items == 0) return cudaSuccess;
   if (!a.out || (reinterpret_cast<uintptr_t>(a.out) & 15u) != 0 || a.k_splits < 1 || a.k_splits > 8 ||
-      128 % a.k_splits != 0)
+      128 % a.k_splits != 0 || a.kb_per_split > kMaxKbPerSplit)
     return cudaErrorInvalidValue;
   const int smem = tc_fc_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(tc_fc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

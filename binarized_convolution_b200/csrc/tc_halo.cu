@@ -62,7 +62,7 @@ constexpr int kStripFloats = 4 * kWarpStageBytes / 4;  // strips of A staged in 
 constexpr int kMaxTiles = 6;                         // tiles whose betas are formed in one batch
 constexpr int kMinResidentBN = 128;                  // narrowest tile the plan narrows to
 
-struct __align__(8) HaloBars {
+struct __align__(16) HaloBars {
   uint64_t hfull[kHaloStages];
   uint64_t hempty[kHaloStages];
   uint64_t wfull[kMaxWStages];
@@ -75,17 +75,6 @@ struct __align__(8) HaloBars {
   float2 sb[128];                // (scale, bias) of the CTA's output channels (BN <= 128)
   float betas[kMaxTiles * 128];  // beta of each row of the current batch of tiles
 };
-
-// 16 consecutive 32-bit TMEM columns of this warp's 32 lanes.
-__device__ __forceinline__ void tc_ld_32x16(uint32_t taddr, uint32_t (&v)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15}, [%16];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
-        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
     tc_halo_kernel(const __grid_constant__ CUtensorMap tmA, const HaloArgs a) {
@@ -212,6 +201,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // B operand by one weight block per tap
       const uint64_t row_step = 128 >> 4, wrap_step = static_cast<uint64_t>(a.Wp - a.kw + 1) * (128 >> 4);
       const uint64_t wb_step = static_cast<uint64_t>(a.kb_per_tap) * wblock >> 4;
+      // streamed weights: stage s's descriptor is the first one plus s blocks
+      const uint64_t wdesc0 = smem_desc_sw128(wsm), wstage_step = static_cast<uint64_t>(wblock) >> 4;
+      const uint32_t sfa = tmem_base + sf_col, sfb = tmem_base + sf_col + 16u;
+      const int kw = a.kw;
       for (int m = slot0; m < a.m_tiles && ok; m += slots, ++ti) {
         if (!mbar_wait(&B->tmem_empty[acc], acc_phase ^ 1u, B, a.err)) break;
         tc_fence_after();
@@ -223,37 +216,52 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           if (kb == 0 && ti < 8) BCONV_STAMP(3 + 2 * ti);
+          // The issuing loops are kept free of anything but the MMAs and their descriptors: the
+          // tensor pipe runs dry when the single issuing thread spends more than a few cycles
+          // between MMAs (a branch holding an mbarrier wait in this loop, even never taken,
+          // cost about half the pipe's rate).
           uint64_t da = smem_desc_sw128(halo + hs * a.halo_bytes);
-          uint64_t db = smem_desc_sw128(wsm + kb * wblock);
-          int tx = 0;
-          for (int tap = 0; tap < taps; ++tap) {
-            uint64_t dbt = db;
-            if (!a.resident) {
+          const uint32_t acc0 = kb > 0 ? 1u : 0u;
+          if (a.resident) {
+            uint64_t db = smem_desc_sw128(wsm + kb * wblock);
+            int tx = 0;
+            for (int tap = 0; tap < taps; ++tap) {
+              tc_mma_f4(d_tmem, da, db, idesc, tap > 0 ? 1u : acc0, sfa, sfb);
+              tc_mma_f4(d_tmem, da + 2u, db + 2u, idesc, 1u, sfa, sfb);
+              tc_mma_f4(d_tmem, da + 4u, db + 4u, idesc, 1u, sfa, sfb);
+              tc_mma_f4(d_tmem, da + 6u, db + 6u, idesc, 1u, sfa, sfb);
+              db += wb_step;
+              if (++tx == kw) {
+                tx = 0;
+                da += wrap_step;
+              } else {
+                da += row_step;
+              }
+            }
+          } else {
+            int tx = 0;
+            for (int tap = 0; tap < taps; ++tap) {
               if (!mbar_wait(&B->wfull[ws], wphase, B, a.err)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
-              dbt = smem_desc_sw128(wsm + ws * wblock);
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {  // four 32-byte (64-code) K steps across the 128-byte row
-              const uint32_t accum = (kb > 0 || tap > 0 || j > 0) ? 1u : 0u;
-              tc_mma_f4(d_tmem, da + 2u * j, dbt + 2u * j, idesc, accum, tmem_base + sf_col, tmem_base + sf_col + 16u);
-            }
-            if (!a.resident) {
+              const uint64_t db = wdesc0 + static_cast<uint64_t>(ws) * wstage_step;
+              tc_mma_f4(d_tmem, da, db, idesc, tap > 0 ? 1u : acc0, sfa, sfb);
+              tc_mma_f4(d_tmem, da + 2u, db + 2u, idesc, 1u, sfa, sfb);
+              tc_mma_f4(d_tmem, da + 4u, db + 4u, idesc, 1u, sfa, sfb);
+              tc_mma_f4(d_tmem, da + 6u, db + 6u, idesc, 1u, sfa, sfb);
               tc_commit(&B->wempty[ws]);
               if (++ws == a.wstages) {
                 ws = 0;
                 wphase ^= 1u;
               }
-            }
-            db += wb_step;
-            if (++tx == a.kw) {
-              tx = 0;
-              da += wrap_step;
-            } else {
-              da += row_step;
+              if (++tx == kw) {
+                tx = 0;
+                da += wrap_step;
+              } else {
+                da += row_step;
+              }
             }
           }
           if (!ok) break;
@@ -278,8 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
     // Each warp turns its 32 TMEM lanes (tile rows) into output rows 32 channels at a time:
-    // rows into its own 4 KB of shared memory (16-byte chunk k of row r at k ^ (r % 8)), then
-    // read back so that each store instruction writes 4 rows x 128 contiguous bytes.
+    // raw rows into its own 4 KB of shared memory (16-byte chunk k of row r at k ^ (r % 8)),
+    // then read back, with the terms applied, so that each store instruction writes 4 rows x
+    // 128 contiguous bytes.
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
     uint8_t* wst = stage_out + q * kWarpStageBytes;
@@ -289,15 +298,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // betas are formed for a batch of tiles at a time, the first batch while the first tile's
     // MMAs run, through the (then idle) staging buffers
     const int batch = min(kMaxTiles, kStripFloats / a.halo_len);
+    // Each warp moves on to the next tile as soon as its own stores are issued (no barrier
+    // across the epilogue warps but tile_betas' own); after an abort a warp keeps walking the
+    // tile list without waiting or storing, so that it still meets the others in tile_betas.
+    bool ok = true;
     int ti = 0;
     for (int m = slot0; m < a.m_tiles; m += slots, ++ti) {
       const int s0 = m * 128;
       if (a.A && ti % batch == 0)
         tile_betas(a.A, total_slots, m, slots, min(batch, (a.m_tiles - m + slots - 1) / slots), a.halo_len,
                    a.kh, a.kw, a.Wp, reinterpret_cast<float*>(stage_out), B->betas, row, true, et, kEpiThreads);
-      const float beta = a.A ? B->betas[(ti % batch) * 128 + row] : 1.f;
-      // the output rows this lane stores: rows 4i + lane / 8 of the warp's 32 (i = 0..7)
+      // the output rows this lane stores: rows 4i + lane / 8 of the warp's 32 (i = 0..7), and
+      // their betas
       int64_t dst[8];
+      float rb[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int sl = s0 + q * 32 + 4 * i + (lane >> 3);
@@ -305,8 +319,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int oy = rem / a.Wp, ox = rem - oy * a.Wp;
         const bool ok = sl < total_slots && oy < a.H && ox < a.W;
         dst[i] = ok ? ((static_cast<int64_t>(n) * a.H + oy) * a.W + ox) * a.No : -1;
+        rb[i] = a.A ? B->betas[(ti % batch) * 128 + q * 32 + 4 * i + (lane >> 3)] : 1.f;
       }
-      if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err, true, true))) break;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err, true, true));
+      if (!ok) {
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+        continue;
+      }
       tc_fence_after();
       if (et == 0 && ti < 8) BCONV_STAMP(21 + 2 * ti);
       const uint32_t tbase =
@@ -318,33 +338,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           if (lane == 0) mbar_arrive(&B->tmem_empty[acc]);
         }
-        const float4* sb4 = reinterpret_cast<const float4*>(&B->sb[ch * 32]);
-        float y[32];
+        // raw sums through the staging buffer; the terms are applied as they are read back,
+        // where a lane holds 4 channels of 8 rows (two float4 loads of (scale, bias) per chunk)
+        uint4* orow = reinterpret_cast<uint4*>(wst + lane * 128);
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float4 p = sb4[j / 2];  // (scale, bias) of channels j, j+1
-          const float s0 = __uint_as_float(v[j]), s1 = __uint_as_float(v[j + 1]);
-          float r0 = a.A ? fmaf(s0 * p.x, beta, p.y) : fmaf(s0, p.x, p.y);
-          float r1 = a.A ? fmaf(s1 * p.z, beta, p.w) : fmaf(s1, p.z, p.w);
-          if (a.relu) {
-            r0 = fmaxf(r0, 0.f);
-            r1 = fmaxf(r1, 0.f);
-          }
-          y[j] = r0;
-          y[j + 1] = r1;
-        }
-        float4* orow = reinterpret_cast<float4*>(wst + lane * 128);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          orow[k ^ (lane & 7)] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
+        for (int k = 0; k < 8; ++k) orow[k ^ (lane & 7)] = make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
         __syncwarp();
-        const int c = ntile * a.BN + ch * 32 + 4 * (lane & 7);
+        const int cl = ch * 32 + 4 * (lane & 7);  // this lane's first channel in the tile
+        const int c = ntile * a.BN + cl;
         if (c < a.No) {  // No % 4 == 0: a float4 of channels is all real or all padding
+          const float4 p01 = *reinterpret_cast<const float4*>(&B->sb[cl]);      // (s0, b0, s1, b1)
+          const float4 p23 = *reinterpret_cast<const float4*>(&B->sb[cl + 2]);  // (s2, b2, s3, b3)
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int r = 4 * i + (lane >> 3);
-            const float4 val = reinterpret_cast<const float4*>(wst + r * 128)[(lane & 7) ^ (r & 7)];
-            if (dst[i] >= 0) *reinterpret_cast<float4*>(a.out + dst[i] + c) = val;
+            const float4 sv = reinterpret_cast<const float4*>(wst + r * 128)[(lane & 7) ^ (r & 7)];
+            const float beta = rb[i];
+            float4 y;
+            y.x = a.A ? fmaf(sv.x * p01.x, beta, p01.y) : fmaf(sv.x, p01.x, p01.y);
+            y.y = a.A ? fmaf(sv.y * p01.z, beta, p01.w) : fmaf(sv.y, p01.z, p01.w);
+            y.z = a.A ? fmaf(sv.z * p23.x, beta, p23.y) : fmaf(sv.z, p23.x, p23.y);
+            y.w = a.A ? fmaf(sv.w * p23.z, beta, p23.w) : fmaf(sv.w, p23.z, p23.w);
+            if (a.relu) {
+              y.x = fmaxf(y.x, 0.f);
+              y.y = fmaxf(y.y, 0.f);
+              y.z = fmaxf(y.z, 0.f);
+              y.w = fmaxf(y.w, 0.f);
+            }
+            if (dst[i] >= 0) *reinterpret_cast<float4*>(a.out + dst[i] + c) = y;
           }
         }
         __syncwarp();  // the rows are read before the next chunk overwrites them

@@ -200,6 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // descriptor start-address units are 16 bytes: a tap moves the A operand by whole rows
       const uint64_t row_step = 128 >> 4, wrap_step = static_cast<uint64_t>(a.Wp - a.kw + 1) * (128 >> 4);
       const uint64_t wb_step = static_cast<uint64_t>(a.kb_per_tap) * kWBlock >> 4;
+      const uint64_t wdesc0 = smem_desc_sw128(wsm);  // streamed weights: stage s is s blocks on
+      const uint32_t sfa = tmem_base + sf_col, sfb = tmem_base + sf_col + 32u;
+      const int kw = a.kw;
       for (int pt = pslot0; pt < pair_tiles && ok; pt += pslots, ++ti) {
         // the single accumulator: wait until both CTAs' epilogues have read the previous tile
         if (!mbar_wait(&B->tmem_empty, (ti & 1) ^ 1u, B, a.err)) break;
@@ -211,38 +214,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           if (kb == 0 && ti < 8) BCONV_STAMP(3 + 2 * ti);
+          // The issuing loops hold nothing but the MMAs and their descriptors: the tensor pipes
+          // run dry when the single issuing thread spends more than a few cycles between MMAs.
           uint64_t da = smem_desc_sw128(halo + hs * a.halo_bytes);
-          uint64_t db = smem_desc_sw128(wsm + kb * kWBlock);
-          int tx = 0;
-          for (int tap = 0; tap < taps; ++tap) {
-            uint64_t dbt = db;
-            if (!a.resident) {
+          const uint32_t acc0 = kb > 0 ? 1u : 0u;
+          if (a.resident) {
+            uint64_t db = smem_desc_sw128(wsm + kb * kWBlock);
+            int tx = 0;
+            for (int tap = 0; tap < taps; ++tap) {
+              tc_mma_f4_pair(tmem_base, da, db, idesc, tap > 0 ? 1u : acc0, sfa, sfb);
+              tc_mma_f4_pair(tmem_base, da + 2u, db + 2u, idesc, 1u, sfa, sfb);
+              tc_mma_f4_pair(tmem_base, da + 4u, db + 4u, idesc, 1u, sfa, sfb);
+              tc_mma_f4_pair(tmem_base, da + 6u, db + 6u, idesc, 1u, sfa, sfb);
+              db += wb_step;
+              if (++tx == kw) {
+                tx = 0;
+                da += wrap_step;
+              } else {
+                da += row_step;
+              }
+            }
+          } else {
+            int tx = 0;
+            for (int tap = 0; tap < taps; ++tap) {
               if (!mbar_wait(&B->wfull[ws], wphase, B, a.err)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
-              dbt = smem_desc_sw128(wsm + ws * kWBlock);
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {  // four 32-byte (64-code) K steps across the 128-byte row
-              const uint32_t accum = (kb > 0 || tap > 0 || j > 0) ? 1u : 0u;
-              tc_mma_f4_pair(tmem_base, da + 2u * j, dbt + 2u * j, idesc, accum, tmem_base + sf_col,
-                             tmem_base + sf_col + 32u);
-            }
-            if (!a.resident) {
+              const uint64_t db = wdesc0 + static_cast<uint64_t>(ws) * (kWBlock >> 4);
+              tc_mma_f4_pair(tmem_base, da, db, idesc, tap > 0 ? 1u : acc0, sfa, sfb);
+              tc_mma_f4_pair(tmem_base, da + 2u, db + 2u, idesc, 1u, sfa, sfb);
+              tc_mma_f4_pair(tmem_base, da + 4u, db + 4u, idesc, 1u, sfa, sfb);
+              tc_mma_f4_pair(tmem_base, da + 6u, db + 6u, idesc, 1u, sfa, sfb);
               tc_commit_pair(&B->wempty[ws]);
               if (++ws == a.wstages) {
                 ws = 0;
                 wphase ^= 1u;
               }
-            }
-            db += wb_step;
-            if (++tx == a.kw) {
-              tx = 0;
-              da += wrap_step;
-            } else {
-              da += row_step;
+              if (++tx == kw) {
+                tx = 0;
+                da += wrap_step;
+              } else {
+                da += row_step;
+              }
             }
           }
           if (!ok) break;
@@ -271,6 +286,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // betas are formed for a batch of tiles at a time, the first batch while the first tile's
     // MMAs run, through the (then idle) staging buffers
     const int batch = min(kMaxTiles, kStripFloats / a.halo_len);
+    // Each warp moves on to the next tile as soon as its own stores are issued (no barrier
+    // across the epilogue warps but tile_betas' own); after an abort a warp keeps walking the
+    // tile list without waiting or storing, so that it still meets the others in tile_betas.
+    bool ok = true;
     int ti = 0;
     for (int pt = pslot0; pt < pair_tiles; pt += pslots, ++ti) {
       const int s0 = (2 * pt + static_cast<int>(rank)) * 128;
@@ -278,7 +297,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tile_betas(a.A, total_slots, 2 * pt + static_cast<int>(rank), 2 * pslots,
                    min(batch, (pair_tiles - pt + pslots - 1) / pslots), a.halo_len, a.kh, a.kw, a.Wp,
                    reinterpret_cast<float*>(stage_out), B->betas, row, half == 0, et, kEpiThreads);
-      const float beta = a.A ? B->betas[(ti % batch) * 128 + row] : 1.f;
       // this lane's store rows: 4 i + lane / 8 of the warp's 32 (i = 0..7), 16 bytes each of 128;
       // their output pixels (N * H * W < 2^31), or -1 for junk slots
       int dst[8];
@@ -290,7 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool ok = sl < total_slots && oy < a.H && ox < a.W;
         dst[i] = ok ? (n * a.H + oy) * a.W + ox : -1;
       }
-      if (!named_all(mbar_wait(&B->tmem_full, ti & 1, B, a.err, true, true), kEpiThreads)) break;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&B->tmem_full, ti & 1, B, a.err, true, true));
+      if (!ok) continue;
       tc_fence_after();
       if (et == 0 && ti < 8) BCONV_STAMP(21 + 2 * ti);
       // the whole 128-column half of this warp's lanes into registers, then the accumulator back
@@ -304,36 +323,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(empty_leader);
-      const int cbase = ntile * kBN + half * 128;
+      // Raw sums go through the staging buffer; the terms are applied as they are read back,
+      // where a lane holds 4 channels of 4 rows: its (scale, bias) pairs are two float4 loads
+      // per chunk.
+      const float* tb_beta = B->betas + (ti % batch) * 128 + q * 32 + (lane >> 3);
 #pragma unroll
       for (int ch = 0; ch < 128 / kOutCols; ++ch) {
-        float y[kOutCols];
-#pragma unroll
-        for (int j = 0; j < kOutCols; ++j) {
-          const float2 p = B->sb[half * 128 + ch * kOutCols + j];
-          const float sv = __uint_as_float(v[ch * kOutCols + j]);
-          const float r = a.A ? fmaf(sv * p.x, beta, p.y) : fmaf(sv, p.x, p.y);
-          y[j] = a.relu ? fmaxf(r, 0.f) : r;
-        }
-        const int c = cbase + ch * kOutCols + 4 * (lane & 7);
+        const int cl = half * 128 + ch * kOutCols + 4 * (lane & 7);  // this lane's first channel in the tile
+        const float4 p01 = *reinterpret_cast<const float4*>(&B->sb[cl]);      // (s0, b0, s1, b1)
+        const float4 p23 = *reinterpret_cast<const float4*>(&B->sb[cl + 2]);  // (s2, b2, s3, b3)
+        const int c = ntile * kBN + cl;
         // 16 rows at a time through the warp's 2 KB (16-byte piece k of row r at k ^ (r % 8)):
         // each store instruction then writes 4 rows x 128 contiguous bytes
 #pragma unroll
         for (int h = 0; h < 32 / kStageRows; ++h) {
           if ((lane >> 4) == h) {
-            float4* orow = reinterpret_cast<float4*>(wst + (lane & 15) * 128);
+            uint4* orow = reinterpret_cast<uint4*>(wst + (lane & 15) * 128);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-              orow[k ^ (lane & 7)] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
+              orow[k ^ (lane & 7)] = make_uint4(v[ch * kOutCols + 4 * k], v[ch * kOutCols + 4 * k + 1],
+                                                v[ch * kOutCols + 4 * k + 2], v[ch * kOutCols + 4 * k + 3]);
           }
           __syncwarp();
           if (c < a.No) {  // No % 4 == 0: a float4 of channels is all real or all padding
 #pragma unroll
             for (int i = 0; i < kStageRows / 4; ++i) {
               const int r = 4 * i + (lane >> 3);
-              const float4 val = reinterpret_cast<const float4*>(wst + r * 128)[(lane & 7) ^ (r & 7)];
+              const float4 sv = reinterpret_cast<const float4*>(wst + r * 128)[(lane & 7) ^ (r & 7)];
+              const float beta = a.A ? tb_beta[4 * (h * (kStageRows / 4) + i)] : 1.f;
+              float4 y;
+              y.x = a.A ? fmaf(sv.x * p01.x, beta, p01.y) : fmaf(sv.x, p01.x, p01.y);
+              y.y = a.A ? fmaf(sv.y * p01.z, beta, p01.w) : fmaf(sv.y, p01.z, p01.w);
+              y.z = a.A ? fmaf(sv.z * p23.x, beta, p23.y) : fmaf(sv.z, p23.x, p23.y);
+              y.w = a.A ? fmaf(sv.w * p23.z, beta, p23.w) : fmaf(sv.w, p23.z, p23.w);
+              if (a.relu) {
+                y.x = fmaxf(y.x, 0.f);
+                y.y = fmaxf(y.y, 0.f);
+                y.z = fmaxf(y.z, 0.f);
+                y.w = fmaxf(y.w, 0.f);
+              }
               const int d = dst[h * (kStageRows / 4) + i];
-              if (d >= 0) *reinterpret_cast<float4*>(a.out + static_cast<int64_t>(d) * a.No + c) = val;
+              if (d >= 0) *reinterpret_cast<float4*>(a.out + static_cast<int64_t>(d) * a.No + c) = y;
             }
           }
           __syncwarp();  // the rows are read before the next ones overwrite them

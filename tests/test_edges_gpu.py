@@ -187,6 +187,27 @@ def test_fc_split_reduction_repeated(cuda_device):
         sums.close()
 
 
+def test_fc_int16_partials_at_their_limit(cuda_device):
+    """The e2m1 FC sends each split's partial sums to the row's owner as int16, at most 127
+    k-blocks of 256 codes a split (|partial| <= 32512).  With every product +1 (positive
+    input, all weight bits set) the sums equal the code count: 508 k-blocks run on e2m1 codes
+    (4 splits of 127, or 8 of 64 where clusters of 8 fit), 1016 on e2m1 codes with 8 splits of
+    127 where those fit and on int8 codes otherwise, 1017 always on int8 codes."""
+    for kb, want in ((508, bc.CODES_FP4), (1016, None), (1017, bc.CODES_INT8)):
+        w = synth.small_case(batch=1, h=1, w=1, ni=kb * 256, no=32, kind="fc", op=synth.XNOR, p=1.0, seed=41)
+        base = synth.make_inputs(w)
+        inp = synth.Inputs(np.abs(base.x) + 0.01, base.wbits, base.scale, base.bias, None, None)
+        layer = pu.make_layer(w, inp, sums=True)
+        try:
+            assert layer.tc_codes() in ((want,) if want is not None else (bc.CODES_FP4, bc.CODES_INT8))
+        finally:
+            layer.close()
+        S_dev = pu.run_device(w, inp, sums=True)
+        S_sum, _, _ = pu.run_oracle(w, inp, sums=True)
+        assert np.all(S_sum == kb * 256)
+        pu.assert_sums_exact(S_dev, S_sum)
+
+
 def test_bounded_wait_gives_up_and_device_stays_usable(cuda_device):
     """The kernels' mbarrier waits are bounded: a wait on a barrier that nothing completes ends
     with a timeout status (not a hang), and the device keeps working afterwards."""
@@ -277,7 +298,9 @@ def test_spread_choice(cuda_device):
     assert _spread(c2, mode=P) == (P, I8)  # forced pairs take the int8 per-tap pair kernel
     assert _spread(synth.workload("and_n32_28x28_c512_k512_3x3")) == (P, F4)
     assert _spread(synth.workload("binw_n8_112x112_c128_k128_3x3_s2")) == (S, BF)
-    assert _spread(synth.workload("fc_xnor_beta_n256_7x7x512_k4096"), codes=I8) == (P, I8)
+    fc5 = synth.workload("fc_xnor_beta_n256_7x7x512_k4096")
+    assert _spread(fc5) == (S, F4)  # the e2m1 FC kernel (one SM per item, clusters per tile)
+    assert _spread(fc5, codes=I8) == (P, I8)
     ragged = synth.small_case(batch=4, h=70, w=70, ni=32, no=32, k=3, op=synth.XNOR, seed=27)
     assert _spread(ragged, codes=I8) == (P, I8)  # 162 tiles: 18 stages on single SMs, 10 on pairs
     assert _spread(ragged) == (S, F4)
