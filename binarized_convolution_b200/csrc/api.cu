@@ -821,6 +821,7 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
     p.op = L.type;
     p.f4 = L.tc.kind == 2;
     p.pad = L.pad;
+    p.err = L.err;
     e = launch_pack_i8(p, s);
   } else {
     PackBf16x3Args p{};

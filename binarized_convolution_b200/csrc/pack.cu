@@ -12,7 +12,10 @@
 // keeps a kilobyte in flight; the kernel is bound by the fp32 read.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "common.cuh"
+#include "tc_device.cuh"
 
 namespace bconv {
 namespace {
@@ -157,9 +160,37 @@ __device__ __forceinline__ void load_group(float4 (&v)[kG][kC], const float* __r
     }
 }
 
+// The sums over the warp of kG values per lane, for kG pixels at once (kG = 1, 2, 4 or 8):
+// halving exchanges first (offsets 16, 8, ... while a lane holds more than one value), then
+// the plain butterfly.  Each pixel's total is formed by the same pairing tree as a butterfly
+// over its own per-lane values, so it is bit-identical to one; lane l returns the total of
+// pixel l / (32 / kG).
+template <int kG>
+__device__ __forceinline__ float warp_sum_multi(float (&v)[kG], int lane) {
+  static_assert(kG == 1 || kG == 2 || kG == 4 || kG == 8, "pixels per step");
+  constexpr int kLog = kG == 1 ? 0 : kG == 2 ? 1 : kG == 4 ? 2 : 3;
+#pragma unroll
+  for (int lvl = 0; lvl < kLog; ++lvl) {
+    const int off = 16 >> lvl;
+    const int n = kG >> (lvl + 1);  // values a lane keeps after this level
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int j = 0; j < n; ++j) {
+      const float keep = upper ? v[j + n] : v[j];
+      const float send = upper ? v[j] : v[j + n];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  float t = v[0];
+#pragma unroll
+  for (int off = 16 >> kLog; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+  return t;
+}
+
 template <bool kTerms, bool kA, int kOp, int kC, bool kF4>
 __global__ void __launch_bounds__(kPackThreads, 2) pack_i8_vec_kernel(PackI8Args a) {
   constexpr int kG = 8 / kC;  // pixels per warp step
+  constexpr int kLanesPerPix = 32 / kG;  // lanes holding one pixel's A after warp_sum_multi
   wait_prior_grid();
   allow_next_grid();
   const int lane = threadIdx.x & 31;
@@ -168,6 +199,7 @@ __global__ void __launch_bounds__(kPackThreads, 2) pack_i8_vec_kernel(PackI8Args
   const int ni = a.ni;
   const float* __restrict__ in = a.in;
   int8_t* __restrict__ codes = a.codes;
+  const int64_t pbytes = kF4 ? a.cip / 2 : a.cip;  // code bytes per pixel
   float4 sc[kC], bi[kC];
   bool live[kC];
 #pragma unroll
@@ -181,24 +213,30 @@ __global__ void __launch_bounds__(kPackThreads, 2) pack_i8_vec_kernel(PackI8Args
       bi[c] = __ldg(reinterpret_cast<const float4*>(a.in_bias + f));
     }
   }
-  const int64_t step = nwarps * kG;
+  // Each warp packs one contiguous range of whole steps: a pixel's place in the code grid then
+  // follows from the previous pixel's (one division per warp, none per pixel), and each warp
+  // streams one stretch of the input.
+  const int64_t steps = (a.npix + kG - 1) / kG;
+  const int64_t per_warp = (steps + nwarps - 1) / nwarps;
+  int64_t p0 = warp * per_warp * kG;
+  const int64_t p_end = min(a.npix, p0 + per_warp * kG);
+  if (p0 >= p_end) return;
+  int py = 0, px = 0;
+  a.pad.yx(p0, py, px);
+  int64_t q = a.pad(p0);  // place of the next pixel to pack
   float4 v[kG][kC];
-  int64_t p0 = warp * kG;
-  if (p0 < a.npix) load_group<kG, kC>(v, in, p0, a.npix, ni, live, lane);
-  for (; p0 < a.npix; p0 += step) {
+  load_group<kG, kC>(v, in, p0, p_end, ni, live, lane);
+  for (; p0 < p_end; p0 += kG) {
     float4 nxt[kG][kC];
-    if (p0 + step < a.npix) load_group<kG, kC>(nxt, in, p0 + step, a.npix, ni, live, lane);
-    // the places of the step's pixels in the code buffer: one division for the first, then
-    // steps along the row (over the border at a row's or an image's end)
-    int py = 0, px = 0;
-    a.pad.yx(p0, py, px);
-    int64_t q = a.pad(p0);
+    if (p0 + kG < p_end) load_group<kG, kC>(nxt, in, p0 + kG, p_end, ni, live, lane);
+    float asum[kG];
+    int64_t qa = q;  // place of this lane's pixel for A (set below)
 #pragma unroll
     for (int g = 0; g < kG; ++g) {
-      const int64_t p = p0 + g;
-      if (p >= a.npix) break;  // warp-uniform
-      if (g > 0) q = a.pad.next(q, py, px);
-      float asum = 0.f;
+      asum[g] = 0.f;
+      if (p0 + g >= p_end) continue;  // warp-uniform
+      if (g == lane / kLanesPerPix) qa = q;
+      int8_t* crow = codes + q * pbytes;
 #pragma unroll
       for (int c = 0; c < kC; ++c) {
         uint32_t word = 0u;
@@ -210,18 +248,21 @@ __global__ void __launch_bounds__(kPackThreads, 2) pack_i8_vec_kernel(PackI8Args
             t.z = fmaf(t.z, sc[c].z, bi[c].z);
             t.w = fmaf(t.w, sc[c].w, bi[c].w);
           }
-          if (kA) asum += (fabsf(t.x) + fabsf(t.y)) + (fabsf(t.z) + fabsf(t.w));
+          if (kA) asum[g] += (fabsf(t.x) + fabsf(t.y)) + (fabsf(t.z) + fabsf(t.w));
           word = kF4 ? nibbles4<kOp>(t) : codes4<kOp>(t);
         }
         if (kF4)  // e2m1 codes: cip / 2 bytes per pixel, 64 bytes per 128-channel chunk
-          *reinterpret_cast<uint16_t*>(codes + q * (a.cip / 2) + c * 64 + lane * 2) = static_cast<uint16_t>(word);
+          *reinterpret_cast<uint16_t*>(crow + c * 64 + lane * 2) = static_cast<uint16_t>(word);
         else
-          *reinterpret_cast<uint32_t*>(codes + q * a.cip + c * 128 + lane * 4) = word;
+          *reinterpret_cast<uint32_t*>(crow + c * 128 + lane * 4) = word;
       }
-      if (kA) {
-        asum = warp_sum(asum);
-        if (lane == 0) a.A[q] = asum / static_cast<float>(ni);  // A follows the codes' grid
-      }
+      q = a.pad.next(q, py, px);
+    }
+    if (kA) {
+      // one reduction for the step's pixels; lanes g * kLanesPerPix hold pixel g's sum
+      const float total = warp_sum_multi<kG>(asum, lane);
+      const int g = lane / kLanesPerPix;
+      if ((lane % kLanesPerPix) == 0 && p0 + g < p_end) a.A[qa] = total / static_cast<float>(ni);
     }
 #pragma unroll
     for (int g = 0; g < kG; ++g)
@@ -270,6 +311,171 @@ __global__ void __launch_bounds__(kPackThreads) pack_i8_scalar_kernel(PackI8Args
   }
 }
 
+// ------------------------------------------------------------------------------------
+// e2m1 codes through a bulk-copy ring.  The register-fed kernels above keep a few kilobytes in
+// flight per warp and spend ~140 instructions per 256-channel pixel; this one has one thread
+// stream each CTA's contiguous stretch of pixels into shared memory (kStagedStages stages of
+// up to 8 KB: 128 KB in flight per SM) and eight warps convert it, each a whole stage of kSP
+// pixels at a time -- lane l takes channels 8 l .. 8 l + 7 of each 256-channel pass, whose
+// eight codes are one 32-bit store -- so that a pixel's place in the code grid follows from the
+// previous one's and one reduction forms the stage's kSP values of A.
+// ------------------------------------------------------------------------------------
+constexpr int kStagedStages = 16;
+constexpr int kStagedBytes = 8192;
+constexpr int kStagedWarps = 8;  // converting warps; one more warp feeds the ring
+
+struct __align__(8) StagedBars {
+  uint64_t full[kStagedStages];
+  uint64_t empty[kStagedStages];
+  uint32_t abort_flag;
+  uint32_t err_word;  // stands in for a missing error word
+};
+
+template <bool kTerms, bool kA, int kOp, int kSP>
+__global__ void __launch_bounds__((kStagedWarps + 1) * 32, 1) pack_f4_staged_kernel(PackI8Args a, int64_t per_cta) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  StagedBars* B = reinterpret_cast<StagedBars*>(sm + kStagedStages * kStagedBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ni = a.ni;
+  const int64_t p_begin = static_cast<int64_t>(blockIdx.x) * per_cta;
+  const int64_t p_end = min(a.npix, p_begin + per_cta);
+  const int64_t nst = p_begin < p_end ? (p_end - p_begin + kSP - 1) / kSP : 0;  // stages of this CTA
+  uint32_t* err = a.err ? a.err : &B->err_word;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStagedStages; ++i) {
+      tcdev::mbar_init(&B->full[i], 1);
+      tcdev::mbar_init(&B->empty[i], 1);
+    }
+    B->abort_flag = 0;
+    B->err_word = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  wait_prior_grid();  // the input and the code buffer belong to the previous kernels until here
+  allow_next_grid();
+  if (warp == kStagedWarps) {
+    if (lane == 0) {
+      int64_t issued = 0;
+      for (int64_t st = 0; st < nst; ++st) {
+        const int slot = static_cast<int>(st % kStagedStages);
+        const int64_t use = st / kStagedStages;
+        if (use > 0 && !tcdev::mbar_wait(&B->empty[slot], static_cast<uint32_t>((use - 1) & 1), B, err)) break;
+        const int64_t p = p_begin + st * kSP;
+        const int np = static_cast<int>(min(static_cast<int64_t>(kSP), p_end - p));
+        const uint32_t bytes = static_cast<uint32_t>(np) * static_cast<uint32_t>(ni) * 4u;
+        tcdev::mbar_expect_tx(&B->full[slot], bytes);
+        tcdev::bulk_load(sm + slot * kStagedBytes, a.in + p * ni, bytes, &B->full[slot]);
+        issued = st + 1;
+      }
+      // every copy has landed before the CTA may leave (after an abort too): the last phase
+      // of each slot used
+      for (int i = 0; i < kStagedStages && i < issued; ++i)
+        tcdev::mbar_wait(&B->full[i], static_cast<uint32_t>(((issued - 1 - i) / kStagedStages) & 1), B, err, false);
+    }
+  } else {
+  constexpr uint32_t kPos = 0x2u;
+  constexpr uint32_t kNeg = kOp == kXnor ? 0xAu : 0x0u;
+  const int npass = a.cip / 256;
+  const int64_t pbytes = a.cip / 2;
+  for (int64_t st = warp; st < nst; st += kStagedWarps) {
+    const int slot = static_cast<int>(st % kStagedStages);
+    const int64_t use = st / kStagedStages;
+    if (!__all_sync(0xffffffffu, tcdev::mbar_wait(&B->full[slot], static_cast<uint32_t>(use & 1), B, err))) break;
+    const int64_t p0 = p_begin + st * kSP;
+    const int np = static_cast<int>(min(static_cast<int64_t>(kSP), p_end - p0));
+    const float* stage = reinterpret_cast<const float*>(sm + slot * kStagedBytes);
+    // the stage's pixels' places in the code grid (one division per stage)
+    int64_t qs[kSP];
+    {
+      int py = 0, px = 0;
+      a.pad.yx(p0, py, px);
+      int64_t q = a.pad(p0);
+#pragma unroll
+      for (int g = 0; g < kSP; ++g) {
+        qs[g] = q;
+        if (g + 1 < kSP) q = a.pad.next(q, py, px);
+      }
+    }
+    float asum[kSP];
+#pragma unroll
+    for (int g = 0; g < kSP; ++g) asum[g] = 0.f;
+    for (int pass = 0; pass < npass; ++pass) {
+      const int f0 = pass * 256 + 8 * lane;  // this lane's first channel
+      const bool live0 = f0 < ni, live1 = f0 + 4 < ni;
+      float4 sc0 = make_float4(1.f, 1.f, 1.f, 1.f), sc1 = sc0;
+      float4 bi0 = make_float4(0.f, 0.f, 0.f, 0.f), bi1 = bi0;
+      if (kTerms) {
+        if (live0) {
+          sc0 = __ldg(reinterpret_cast<const float4*>(a.in_scale + f0));
+          bi0 = __ldg(reinterpret_cast<const float4*>(a.in_bias + f0));
+        }
+        if (live1) {
+          sc1 = __ldg(reinterpret_cast<const float4*>(a.in_scale + f0 + 4));
+          bi1 = __ldg(reinterpret_cast<const float4*>(a.in_bias + f0 + 4));
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < kSP; ++g) {
+        if (g >= np) break;  // warp-uniform
+        float t[8];
+        {
+          const float4 u0 = live0 ? *reinterpret_cast<const float4*>(stage + g * ni + f0) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 u1 = live1 ? *reinterpret_cast<const float4*>(stage + g * ni + f0 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          t[0] = u0.x; t[1] = u0.y; t[2] = u0.z; t[3] = u0.w;
+          t[4] = u1.x; t[5] = u1.y; t[6] = u1.z; t[7] = u1.w;
+        }
+        if (kTerms) {
+          t[0] = fmaf(t[0], sc0.x, bi0.x); t[1] = fmaf(t[1], sc0.y, bi0.y);
+          t[2] = fmaf(t[2], sc0.z, bi0.z); t[3] = fmaf(t[3], sc0.w, bi0.w);
+          t[4] = fmaf(t[4], sc1.x, bi1.x); t[5] = fmaf(t[5], sc1.y, bi1.y);
+          t[6] = fmaf(t[6], sc1.z, bi1.z); t[7] = fmaf(t[7], sc1.w, bi1.w);
+        }
+        uint32_t word = 0u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const bool ok = j < 4 ? live0 : live1;
+          if (kA && ok) asum[g] += fabsf(t[j]);
+          word |= (ok ? ((t[j] < 0.f) ? kNeg : kPos) : 0u) << (4 * j);
+        }
+        *reinterpret_cast<uint32_t*>(a.codes + qs[g] * pbytes + pass * 128 + lane * 4) = word;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) tcdev::mbar_arrive(&B->empty[slot]);  // the stage's input has been read
+    if (kA) {
+      // lanes g * (32 / kSP) hold pixel g's sum
+      const float total = warp_sum_multi<kSP>(asum, lane);
+      const int g = lane / (32 / kSP);
+      int64_t qa = qs[0];
+#pragma unroll
+      for (int j = 1; j < kSP; ++j)
+        if (g == j) qa = qs[j];
+      if ((lane % (32 / kSP)) == 0 && g < np) a.A[qa] = total / static_cast<float>(ni);
+    }
+  }
+  }
+  __syncthreads();
+}
+
+template <bool kTerms, bool kA, int kOp>
+cudaError_t launch_f4_staged(const PackI8Args& a, cudaStream_t s) {
+  const int sp_max = kStagedBytes / (4 * a.ni);  // >= 1 (checked by the caller)
+  const int sp = sp_max >= 8 ? 8 : sp_max >= 4 ? 4 : sp_max >= 2 ? 2 : 1;
+  const int sms = current_sm_count();
+  const int64_t stages = ceil_div(a.npix, sp);
+  const int64_t ctas = std::min<int64_t>(sms, stages);
+  const int64_t per_cta = ceil_div(stages, ctas) * sp;
+  const int grid = static_cast<int>(ceil_div(a.npix, per_cta));
+  const int smem = kStagedStages * kStagedBytes + static_cast<int>(sizeof(StagedBars));
+  auto kern = sp == 8   ? pack_f4_staged_kernel<kTerms, kA, kOp, 8>
+              : sp == 4 ? pack_f4_staged_kernel<kTerms, kA, kOp, 4>
+              : sp == 2 ? pack_f4_staged_kernel<kTerms, kA, kOp, 2>
+                        : pack_f4_staged_kernel<kTerms, kA, kOp, 1>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return launch_overlapped(kern, dim3(grid), dim3((kStagedWarps + 1) * 32), smem, s, a, per_cta);
+}
+
 template <bool kTerms, bool kA, int kOp, bool kF4>
 cudaError_t launch_i8_f(const PackI8Args& a, int chunks, dim3 grid, cudaStream_t s) {
   auto kern = chunks == 1   ? pack_i8_vec_kernel<kTerms, kA, kOp, 1, kF4>
@@ -298,6 +504,14 @@ cudaError_t launch_pack_i8(const PackI8Args& a, cudaStream_t s) {
   const int sms = current_sm_count();
   const bool vec = (a.ni % 4) == 0 && (reinterpret_cast<uintptr_t>(a.in) & 15) == 0 &&
                    (!a.in_scale || ((reinterpret_cast<uintptr_t>(a.in_scale) | reinterpret_cast<uintptr_t>(a.in_bias)) & 15) == 0);
+  // e2m1 codes with up to 2048 channels a pixel: the staged (bulk-copy-fed) kernel
+  if (vec && a.f4 && a.ni <= kStagedBytes / 4 && a.cip % 256 == 0) {
+    if (a.in_scale)
+      return a.A ? (a.op == kXnor ? launch_f4_staged<true, true, kXnor>(a, s) : launch_f4_staged<true, true, kAnd>(a, s))
+                 : (a.op == kXnor ? launch_f4_staged<true, false, kXnor>(a, s) : launch_f4_staged<true, false, kAnd>(a, s));
+    return a.A ? (a.op == kXnor ? launch_f4_staged<false, true, kXnor>(a, s) : launch_f4_staged<false, true, kAnd>(a, s))
+               : (a.op == kXnor ? launch_f4_staged<false, false, kXnor>(a, s) : launch_f4_staged<false, false, kAnd>(a, s));
+  }
   const int chunks = vec ? a.cip / 128 : 0;  // 1, 2, 4 -> vector kernel; anything else -> scalar
   int64_t blocks = ceil_div(a.npix, kPackThreads / 32);
   const int64_t cap = static_cast<int64_t>(sms) * (chunks ? 2 : 3);  // one wave

@@ -181,6 +181,7 @@ struct PackI8Args {
   // (n, y + pad_t, x + pad_l) of an [N][hp][wp] buffer whose other pixels are left alone
   // (hp == 0: the codes have the input's own [N][h][w] layout).
   PadMap pad;
+  uint32_t* err;          // error word for a wait that timed out (the staged e2m1 kernel), or nullptr
 };
 cudaError_t launch_pack_i8(const PackI8Args& a, cudaStream_t s);
 
