@@ -241,14 +241,30 @@ def measured_traffic(kernel: str, workload: str, sources) -> float | None:
     return rec.get("dram_bytes_per_launch")
 
 
+_TC_COMMON = ["binarized_convolution_b200/csrc/tc_device.cuh", "binarized_convolution_b200/csrc/tc_conv.cuh",
+              "binarized_convolution_b200/csrc/common.cuh"]
+# the sources each contraction kernel is built from (a change voids its recorded DRAM traffic)
 KERNEL_SOURCES = {
     "popc_gemm": ["binarized_convolution_b200/csrc/popc_gemm.cu", "binarized_convolution_b200/csrc/common.cuh"],
     "bw_conv": ["binarized_convolution_b200/csrc/bw_conv.cu", "binarized_convolution_b200/csrc/common.cuh"],
-    "tc_conv": ["binarized_convolution_b200/csrc/tc_conv.cu", "binarized_convolution_b200/csrc/tc_conv2.cu",
-                "binarized_convolution_b200/csrc/tc_conv.cuh", "binarized_convolution_b200/csrc/tc_device.cuh",
-                "binarized_convolution_b200/csrc/tc_bits.cuh"],
+    "tc_conv": ["binarized_convolution_b200/csrc/tc_conv.cu", "binarized_convolution_b200/csrc/tc_bits.cuh"] + _TC_COMMON,
+    "tc_conv2": ["binarized_convolution_b200/csrc/tc_conv2.cu", "binarized_convolution_b200/csrc/tc_bits.cuh"] + _TC_COMMON,
+    "tc_halo": ["binarized_convolution_b200/csrc/tc_halo.cu"] + _TC_COMMON,
+    "tc_halo2": ["binarized_convolution_b200/csrc/tc_halo2.cu"] + _TC_COMMON,
+    "tc_fc": ["binarized_convolution_b200/csrc/tc_fc.cu"] + _TC_COMMON,
 }
 ALGO_KERNEL = {1: "popc_gemm", 2: "bw_conv", 3: "tc_conv"}
+
+
+def tc_kernel_name(bc, layer, w: synth.Workload) -> str:
+    """The tensor-core kernel a layer's plan runs: the e2m1 FC kernel, the rows-staged
+    convolution (one SM or SM pairs) or the per-tap convolution (one SM or SM pairs)."""
+    pair = layer.cta_mode() == bc.CTA_PAIR
+    if w.kind == "fc":
+        return "tc_fc" if layer.tc_codes() == CODES_FP4 else ("tc_conv2" if pair else "tc_conv")
+    if layer.staging() == bc.STAGING_ROWS:
+        return "tc_halo2" if pair else "tc_halo"
+    return "tc_conv2" if pair else "tc_conv"
 
 
 def measured_peaks() -> dict:
@@ -523,13 +539,14 @@ def measure_workload(args, w: synth.Workload, device, bits_io: bool = False, cpu
     max_mhz = clock_info.get("sm_max_mhz") or 1965.0
     kname = ALGO_KERNEL[layer.effective_algo()]
     codes = layer.tc_codes() if kname == "tc_conv" else 0
+    kernel = tc_kernel_name(bc, layer, w) if kname == "tc_conv" else kname
     peak, bound, how = derived_peak(w, sms, max_mhz, kname, codes)
     achieved = ops_step / (kern_ms_max * 1e-3) / 1e12
     # the captured traffic is that of the library's own choice of spread and codes
-    traffic = (measured_traffic(kname, w.name, KERNEL_SOURCES[kname])
+    traffic = (measured_traffic(kernel, w.name, KERNEL_SOURCES[kernel])
                if args.cta == "auto" and args.codes == "auto" and not bits_io else None)
     roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
-            "traffic": traffic, "kernel": kname, "kernel_ms": kern_ms_max,
+            "traffic": traffic, "kernel": kernel, "kernel_ms": kern_ms_max,
             "kernel_launches_timed": kern_n, "timed_every": every,
             "peak_source": how if bound == "tensor" else f"derived: {how}"}
     if kname == "tc_conv":

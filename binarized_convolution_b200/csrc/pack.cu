@@ -15,6 +15,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "pack_stage.cuh"
 #include "tc_device.cuh"
 
 namespace bconv {
@@ -160,33 +161,6 @@ __device__ __forceinline__ void load_group(float4 (&v)[kG][kC], const float* __r
     }
 }
 
-// The sums over the warp of kG values per lane, for kG pixels at once (kG = 1, 2, 4 or 8):
-// halving exchanges first (offsets 16, 8, ... while a lane holds more than one value), then
-// the plain butterfly.  Each pixel's total is formed by the same pairing tree as a butterfly
-// over its own per-lane values, so it is bit-identical to one; lane l returns the total of
-// pixel l / (32 / kG).
-template <int kG>
-__device__ __forceinline__ float warp_sum_multi(float (&v)[kG], int lane) {
-  static_assert(kG == 1 || kG == 2 || kG == 4 || kG == 8, "pixels per step");
-  constexpr int kLog = kG == 1 ? 0 : kG == 2 ? 1 : kG == 4 ? 2 : 3;
-#pragma unroll
-  for (int lvl = 0; lvl < kLog; ++lvl) {
-    const int off = 16 >> lvl;
-    const int n = kG >> (lvl + 1);  // values a lane keeps after this level
-    const bool upper = (lane & off) != 0;
-#pragma unroll
-    for (int j = 0; j < n; ++j) {
-      const float keep = upper ? v[j + n] : v[j];
-      const float send = upper ? v[j] : v[j + n];
-      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-    }
-  }
-  float t = v[0];
-#pragma unroll
-  for (int off = 16 >> kLog; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-  return t;
-}
-
 template <bool kTerms, bool kA, int kOp, int kC, bool kF4>
 __global__ void __launch_bounds__(kPackThreads, 2) pack_i8_vec_kernel(PackI8Args a) {
   constexpr int kG = 8 / kC;  // pixels per warp step
@@ -260,7 +234,7 @@ __global__ void __launch_bounds__(kPackThreads, 2) pack_i8_vec_kernel(PackI8Args
     }
     if (kA) {
       // one reduction for the step's pixels; lanes g * kLanesPerPix hold pixel g's sum
-      const float total = warp_sum_multi<kG>(asum, lane);
+      const float total = packdev::warp_sum_multi<kG>(asum, lane);
       const int g = lane / kLanesPerPix;
       if ((lane % kLanesPerPix) == 0 && p0 + g < p_end) a.A[qa] = total / static_cast<float>(ni);
     }
@@ -320,7 +294,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_i8_scalar_kernel(PackI8Args
 // eight codes are one 32-bit store -- so that a pixel's place in the code grid follows from the
 // previous one's and one reduction forms the stage's kSP values of A.
 // ------------------------------------------------------------------------------------
-constexpr int kStagedStages = 16;
+constexpr int kStagedStages = 16;  // two per converting warp
 constexpr int kStagedBytes = 8192;
 constexpr int kStagedWarps = 8;  // converting warps; one more warp feeds the ring
 
@@ -350,9 +324,11 @@ __global__ void __launch_bounds__((kStagedWarps + 1) * 32, 1) pack_f4_staged_ker
     B->err_word = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (threadIdx.x == 0) BCONV_STAMP(0);
   __syncthreads();
   wait_prior_grid();  // the input and the code buffer belong to the previous kernels until here
   allow_next_grid();
+  if (threadIdx.x == 0) BCONV_STAMP(1);
   if (warp == kStagedWarps) {
     if (lane == 0) {
       int64_t issued = 0;
@@ -373,10 +349,6 @@ __global__ void __launch_bounds__((kStagedWarps + 1) * 32, 1) pack_f4_staged_ker
         tcdev::mbar_wait(&B->full[i], static_cast<uint32_t>(((issued - 1 - i) / kStagedStages) & 1), B, err, false);
     }
   } else {
-  constexpr uint32_t kPos = 0x2u;
-  constexpr uint32_t kNeg = kOp == kXnor ? 0xAu : 0x0u;
-  const int npass = a.cip / 256;
-  const int64_t pbytes = a.cip / 2;
   for (int64_t st = warp; st < nst; st += kStagedWarps) {
     const int slot = static_cast<int>(st % kStagedStages);
     const int64_t use = st / kStagedStages;
@@ -384,77 +356,13 @@ __global__ void __launch_bounds__((kStagedWarps + 1) * 32, 1) pack_f4_staged_ker
     const int64_t p0 = p_begin + st * kSP;
     const int np = static_cast<int>(min(static_cast<int64_t>(kSP), p_end - p0));
     const float* stage = reinterpret_cast<const float*>(sm + slot * kStagedBytes);
-    // the stage's pixels' places in the code grid (one division per stage)
-    int64_t qs[kSP];
-    {
-      int py = 0, px = 0;
-      a.pad.yx(p0, py, px);
-      int64_t q = a.pad(p0);
-#pragma unroll
-      for (int g = 0; g < kSP; ++g) {
-        qs[g] = q;
-        if (g + 1 < kSP) q = a.pad.next(q, py, px);
-      }
-    }
-    float asum[kSP];
-#pragma unroll
-    for (int g = 0; g < kSP; ++g) asum[g] = 0.f;
-    for (int pass = 0; pass < npass; ++pass) {
-      const int f0 = pass * 256 + 8 * lane;  // this lane's first channel
-      const bool live0 = f0 < ni, live1 = f0 + 4 < ni;
-      float4 sc0 = make_float4(1.f, 1.f, 1.f, 1.f), sc1 = sc0;
-      float4 bi0 = make_float4(0.f, 0.f, 0.f, 0.f), bi1 = bi0;
-      if (kTerms) {
-        if (live0) {
-          sc0 = __ldg(reinterpret_cast<const float4*>(a.in_scale + f0));
-          bi0 = __ldg(reinterpret_cast<const float4*>(a.in_bias + f0));
-        }
-        if (live1) {
-          sc1 = __ldg(reinterpret_cast<const float4*>(a.in_scale + f0 + 4));
-          bi1 = __ldg(reinterpret_cast<const float4*>(a.in_bias + f0 + 4));
-        }
-      }
-#pragma unroll
-      for (int g = 0; g < kSP; ++g) {
-        if (g >= np) break;  // warp-uniform
-        float t[8];
-        {
-          const float4 u0 = live0 ? *reinterpret_cast<const float4*>(stage + g * ni + f0) : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float4 u1 = live1 ? *reinterpret_cast<const float4*>(stage + g * ni + f0 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-          t[0] = u0.x; t[1] = u0.y; t[2] = u0.z; t[3] = u0.w;
-          t[4] = u1.x; t[5] = u1.y; t[6] = u1.z; t[7] = u1.w;
-        }
-        if (kTerms) {
-          t[0] = fmaf(t[0], sc0.x, bi0.x); t[1] = fmaf(t[1], sc0.y, bi0.y);
-          t[2] = fmaf(t[2], sc0.z, bi0.z); t[3] = fmaf(t[3], sc0.w, bi0.w);
-          t[4] = fmaf(t[4], sc1.x, bi1.x); t[5] = fmaf(t[5], sc1.y, bi1.y);
-          t[6] = fmaf(t[6], sc1.z, bi1.z); t[7] = fmaf(t[7], sc1.w, bi1.w);
-        }
-        uint32_t word = 0u;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const bool ok = j < 4 ? live0 : live1;
-          if (kA && ok) asum[g] += fabsf(t[j]);
-          word |= (ok ? ((t[j] < 0.f) ? kNeg : kPos) : 0u) << (4 * j);
-        }
-        *reinterpret_cast<uint32_t*>(a.codes + qs[g] * pbytes + pass * 128 + lane * 4) = word;
-      }
-    }
+    packdev::pack_stage_f4<kSP>(a, stage, p0, np, kTerms, kA, kOp == kXnor ? 0xAu : 0x0u, lane);
     __syncwarp();
     if (lane == 0) tcdev::mbar_arrive(&B->empty[slot]);  // the stage's input has been read
-    if (kA) {
-      // lanes g * (32 / kSP) hold pixel g's sum
-      const float total = warp_sum_multi<kSP>(asum, lane);
-      const int g = lane / (32 / kSP);
-      int64_t qa = qs[0];
-#pragma unroll
-      for (int j = 1; j < kSP; ++j)
-        if (g == j) qa = qs[j];
-      if ((lane % (32 / kSP)) == 0 && g < np) a.A[qa] = total / static_cast<float>(ni);
-    }
   }
   }
   __syncthreads();
+  if (threadIdx.x == 0) BCONV_STAMP(2);
 }
 
 template <bool kTerms, bool kA, int kOp>
@@ -821,3 +729,5 @@ cudaError_t launch_repack_bits(const uint32_t* bits, int64_t npix, int ni, int n
 }
 
 }  // namespace bconv
+
+BCONV_TIMELINE_READER(bconv_timeline_pack)
