@@ -26,7 +26,7 @@ NEURON_NONE, NEURON_RELU = 0, 1
 ALGO_AUTO, ALGO_POPC, ALGO_SIMT_F32, ALGO_TCGEN05 = 0, 1, 2, 3
 CTA_AUTO, CTA_SINGLE, CTA_PAIR = 0, 1, 2
 CODES_AUTO, CODES_INT8, CODES_FP4, CODES_BF16X3 = 0, 1, 2, 3
-STAGING_AUTO, STAGING_PER_TAP, STAGING_ROWS = 0, 1, 2
+STAGING_AUTO, STAGING_PER_TAP, STAGING_ROWS, STAGING_INPUT = 0, 1, 2, 3
 
 _STATUS = {0: "BCONV_OK", 1: "BCONV_ERR_INVALID_ARG", 2: "BCONV_ERR_UNSUPPORTED", 3: "BCONV_ERR_CUDA",
            4: "BCONV_ERR_OOM", 5: "BCONV_ERR_TIMEOUT", 6: "BCONV_ERR_NO_DEVICE"}
@@ -294,7 +294,7 @@ def bconv_tc_codes(h) -> int:
 
 
 def bconv_set_staging(staging: int):
-    """Activation staging of the e2m1 stride-1 contraction for layers created from now on (STAGING_*)."""
+    """Activation staging of the tensor-core contraction for layers created from now on (STAGING_*)."""
     _check(load_library().bconv_set_staging(int(staging)), "bconv_set_staging")
 
 

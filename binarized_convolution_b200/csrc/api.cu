@@ -144,6 +144,11 @@ struct Layer {
   HaloArgs hx{};
   PadMap pad{};
   float* A_pad = nullptr;  // A in the zero-bordered grid (rows-staged layers with beta)
+  bool f32_off = false;  // binaryWeights: a bit-packed output asks for the parts path (not tc.f32)
+  // tc.f32: tensor maps over the last few input buffers, reused by pointer
+  CUtensorMap tmX[4];
+  const float* tmX_ptr[4] = {nullptr, nullptr, nullptr, nullptr};
+  int tmX_next = 0;
   // Fully-connected contraction with 256-channel items (tc_fc_kernel): its plan
   bool fcb = false;
   FcArgs fx{};
@@ -277,6 +282,28 @@ bool encode_out_map(Layer& L, CUtensorMap* m, const float* out) {
   const uint32_t box[4] = {32, static_cast<uint32_t>(L.tc.Cw), static_cast<uint32_t>(L.tc.R),
                            static_cast<uint32_t>(L.tc.Bn)};
   return encode_4d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, out, d, strides, box);
+}
+
+// Map over `in` ([N][H][W][Ni] fp32) for binaryWeights from fp32 input (tc.f32): boxes of 32
+// channels (128-byte rows, 128-byte swizzle) x Cw x R x Bn pixels stepping by the strides, as
+// the one-SM kernel loads them per tap.  Maps of the last four input buffers are kept;
+// nullptr if `in` cannot be mapped (not 16-byte aligned).
+const CUtensorMap* input_map(Layer& L, const float* in) {
+  for (int i = 0; i < 4; ++i)
+    if (L.tmX_ptr[i] == in) return &L.tmX[i];
+  if ((reinterpret_cast<uintptr_t>(in) & 15u) != 0) return nullptr;
+  const int i = L.tmX_next;
+  const uint64_t dims[4] = {static_cast<uint64_t>(L.Ni), static_cast<uint64_t>(L.W), static_cast<uint64_t>(L.H),
+                            static_cast<uint64_t>(L.N)};
+  const uint64_t row = static_cast<uint64_t>(L.Ni) * sizeof(float);
+  const uint64_t strides[3] = {row, row * L.W, row * L.W * L.H};
+  const uint32_t box[4] = {32, static_cast<uint32_t>(L.tc.sx * L.tc.Cw), static_cast<uint32_t>(L.tc.sy * L.tc.R),
+                           static_cast<uint32_t>(L.tc.Bn)};
+  const uint32_t estr[4] = {1, static_cast<uint32_t>(L.tc.sx), static_cast<uint32_t>(L.tc.sy), 1};
+  if (!encode_4d(&L.tmX[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, in, dims, strides, box, estr)) return nullptr;
+  L.tmX_ptr[i] = in;
+  L.tmX_next = (i + 1) % 4;
+  return &L.tmX[i];
 }
 
 // The tensor-core path: XNOR/AND as int8 codes (kind 0) and binaryWeights as three exact
@@ -475,17 +502,26 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
   // 112 x 112, 128 -> 128, stride 2, binaryWeights (27 stages on single SMs with the tail cut
   // in halves, 24 on pairs with the balanced split) 46.9 us against 53.7 us.
   const double pair_factor = t.kind == 1 ? 0.80 : 0.95;
+  // binaryWeights without beta: the contraction reads the fp32 input itself and splits it in
+  // shared memory (no 3-part buffer: the parts cost 1.5x the input to write and again to read)
+  t.f32 = (t.kind == 1 && !L.fc && !L.use_beta() && !L.f32_off && L.Ni % 4 == 0 && mode != BCONV_CTA_PAIR &&
+           g_staging.load() != BCONV_STAGING_PER_TAP && tc_f32_stages(t.BN) > 0)
+              ? 1
+              : 0;
+  t.in_scale = L.in_scale;
+  t.in_bias = L.in_bias;
+  t.Ni = L.Ni;
   int pairs = 0;
   if (L.fc) {
     pairs = fc_pair ? tc2_max_pairs(t.kind, t.BN) : 0;
-  } else if (mode != BCONV_CTA_SINGLE && t.kind != 2) {
+  } else if (mode != BCONV_CTA_SINGLE && t.kind != 2 && !t.f32) {
     pairs = tc2_max_pairs(t.kind, t.BN);
     if (pairs > 0 && mode == BCONV_CTA_AUTO &&
         !(plan_stages_pair(t, pairs) < pair_factor * plan_stages_single(t, current_sm_count())))
       pairs = 0;
   }
 
-  t.stages = pairs > 0 ? tc2_stages(t.kind, t.BN) : tc_stages(t.kind, t.BN, t.mt);
+  t.stages = pairs > 0 ? tc2_stages(t.kind, t.BN) : t.f32 ? tc_f32_stages(t.BN) : tc_stages(t.kind, t.BN, t.mt);
   if (t.stages < 2) return BCONV_OK;  // no room for a pipeline: the SIMT family stays
 
   // Rows-staged contraction: e2m1 codes, stride 1, image rows that fit a tile (kernel
@@ -566,7 +602,7 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
     e = L.tc_mem.alloc(&L.wq, hq.size());
     if (e == cudaSuccess) e = cudaMemcpy(L.wq, hq.data(), hq.size(), cudaMemcpyHostToDevice);
   }
-  if (e == cudaSuccess) e = L.tc_mem.alloc(&L.codes, static_cast<size_t>(npix) * bpp);
+  if (e == cudaSuccess && !t.f32) e = L.tc_mem.alloc(&L.codes, static_cast<size_t>(npix) * bpp);
   // the border of the padded grid is written once, here, and never again
   if (e == cudaSuccess && L.halo) e = cudaMemset(L.codes, 0, static_cast<size_t>(npix) * bpp);
   if (e == cudaSuccess && L.halo && L.use_beta()) e = L.tc_mem.alloc(&L.A_pad, static_cast<size_t>(npix));
@@ -589,6 +625,8 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
     const uint64_t strides[3] = {K, K, K};
     const uint32_t box[4] = {128, 1, 1, 128};
     ok = encode_4d(&L.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.codes, dims, strides, box);
+  } else if (t.f32) {
+    // the activation map is over each forward's input (input_map)
   } else {
     // box: 128 bytes of channels x (stride x Cw) columns x (stride x R) rows x Bn images,
     // stepping by the stride, so the copy lands Cw x R x Bn pixels = 128 rows
@@ -800,7 +838,7 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
   float* out = io.out;
   const bool beta = L.use_beta();
   const float* A = io.in_bits ? io.in_a : L.A;
-  cudaError_t e;
+  cudaError_t e = cudaSuccess;
   if (io.in_bits) {
     e = L.tc.kind == 2 ? launch_unpack_bits_f4(io.in_bits, static_cast<int64_t>(L.N) * L.H * L.W, L.Ni, L.cip,
                                                L.type, L.codes, s, L.pad)
@@ -823,6 +861,8 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
     p.pad = L.pad;
     p.err = L.err;
     e = launch_pack_i8(p, s);
+  } else if (L.tc.f32) {
+    e = cudaSuccess;  // binaryWeights from fp32 input: the contraction reads `in` itself (no pack, no A)
   } else {
     PackBf16x3Args p{};
     p.in = in;
@@ -883,6 +923,9 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
     h.A = beta ? L.A_pad : nullptr;
     h.out = out;
     e = L.halo2 ? launch_tc_halo2(&L.tmA, &L.tmB, h, s) : launch_tc_halo(&L.tmA, h, s);
+  } else if (t.f32) {
+    const CUtensorMap* xm = input_map(L, in);
+    e = xm ? launch_tc_conv(xm, om, t, s) : cudaErrorInvalidValue;
   } else {
     e = L.tc_pair ? launch_tc_conv2(&L.tmA, &L.tmB, &L.tmBp, om, t, s) : launch_tc_conv(&L.tmA, om, t, s);
   }
@@ -982,6 +1025,12 @@ bconv_status_t run_forward_simt(Layer& L, const Io& io, cudaStream_t s) {
 }
 
 // One forward with the given input and output forms.
+// The fp32-input binaryWeights contraction maps the input for the TMA: it needs it 16-byte
+// aligned (a forward with another input runs on the SIMT family).
+bool tc_input_ok(const Layer& L, const float* in) {
+  return use_tc(L) && (!L.tc.f32 || (reinterpret_cast<uintptr_t>(in) & 15u) == 0);
+}
+
 bconv_status_t run_io(Layer& L, const Io& io, cudaStream_t s) {
   if (L.N == 0) return BCONV_OK;
   if (io.out_bits && !tc_emits_bits(L)) {
@@ -990,7 +1039,7 @@ bconv_status_t run_io(Layer& L, const Io& io, cudaStream_t s) {
     fp.out = L.y_scratch;
     fp.out_bits = nullptr;
     fp.out_a = nullptr;
-    bconv_status_t st = use_tc(L) ? run_forward_tc(L, fp, s) : run_forward_simt(L, fp, s);
+    bconv_status_t st = tc_input_ok(L, io.in) ? run_forward_tc(L, fp, s) : run_forward_simt(L, fp, s);
     if (st != BCONV_OK) return st;
     PackArgs p{};
     p.in = L.y_scratch;
@@ -1006,7 +1055,7 @@ bconv_status_t run_io(Layer& L, const Io& io, cudaStream_t s) {
   // The tensor-core kernels write the output in 16-byte pieces (TMA boxes, float4 stores); an
   // output that is not 16-byte aligned goes to the SIMT family, which can write it.
   const bool aligned = (reinterpret_cast<uintptr_t>(io.out) & 15u) == 0;
-  return use_tc(L) && aligned ? run_forward_tc(L, io, s) : run_forward_simt(L, io, s);
+  return tc_input_ok(L, io.in) && aligned ? run_forward_tc(L, io, s) : run_forward_simt(L, io, s);
 }
 
 bconv_status_t run_forward(Layer& L, const float* in, float* out, cudaStream_t s) {
@@ -1032,6 +1081,8 @@ bconv_status_t replan_tc(Layer& L, int codes) {
   L.halo2 = false;
   L.A_pad = nullptr;
   L.fcb = false;
+  for (int i = 0; i < 4; ++i) L.tmX_ptr[i] = nullptr;  // their boxes follow the old tile shape
+  L.tmX_next = 0;
   L.codes_override = codes;
   return setup_tc(L, L.h_packed.data());
 }
@@ -1075,6 +1126,10 @@ bconv_status_t set_output_terms(Layer& L, const float* next_scale, const float* 
     if (st != BCONV_OK) return st;
   } else if (L.halo) {  // the rows-staged kernel writes fp32 only: the per-tap kernel emits the bits
     L.halo_off = true;
+    const bconv_status_t st = replan_tc(L, L.codes_override);
+    if (st != BCONV_OK) return st;
+  } else if (L.tc_ok && L.tc.f32) {  // so does the fp32-input kernel: the parts path emits them
+    L.f32_off = true;
     const bconv_status_t st = replan_tc(L, L.codes_override);
     if (st != BCONV_OK) return st;
   }
@@ -1586,7 +1641,7 @@ int32_t bfc_cta_mode(bfc_handle_t h) {
 }
 
 bconv_status_t bconv_set_staging(bconv_staging_t staging) {
-  if (staging < BCONV_STAGING_AUTO || staging > BCONV_STAGING_ROWS) return BCONV_ERR_INVALID_ARG;
+  if (staging < BCONV_STAGING_AUTO || staging > BCONV_STAGING_INPUT) return BCONV_ERR_INVALID_ARG;
   g_staging.store(staging);
   return BCONV_OK;
 }
@@ -1594,7 +1649,7 @@ bconv_status_t bconv_set_staging(bconv_staging_t staging) {
 int32_t bconv_staging(bconv_handle_t h) {
   if (!checked(h, kConvMagic)) return -1;
   if (!h->L.tc_ok) return 0;
-  return h->L.halo ? BCONV_STAGING_ROWS : BCONV_STAGING_PER_TAP;
+  return h->L.halo ? BCONV_STAGING_ROWS : h->L.tc.f32 ? BCONV_STAGING_INPUT : BCONV_STAGING_PER_TAP;
 }
 
 bconv_status_t bconv_set_tc_codes(bconv_tc_codes_t codes) {

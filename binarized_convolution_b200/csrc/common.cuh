@@ -55,6 +55,23 @@ static __device__ unsigned long long g_bconv_timeline[1024 * 64];  // one array 
   } while (0)
 #endif
 
+// x~ as three bf16 parts whose sum is x~ exactly, for the binaryWeights contraction (which
+// multiplies each part by the same +-1 weights on the bf16 tensor cores): hi = x~ with the low
+// 16 bits of its fp32 encoding cleared (its leading 8 significant bits), r = x~ - hi (exact: a
+// subset of x~'s bits), mid = r cut the same way, lo = r - mid (exact, and with at most 8
+// significant bits left, itself a bf16 with zero low bits).  Every part is a normal bf16 (or 0)
+// for |x~| >= 2^-103.  Two values at a time as bf16x2 words (x0 in the low half); bit
+// operations and exact subtractions only, no conversion instructions.
+__device__ __forceinline__ void split3_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& mid, uint32_t& lo) {
+  const uint32_t u0 = __float_as_uint(x0), u1 = __float_as_uint(x1);
+  hi = __byte_perm(u0, u1, 0x7632);  // the high halves of both
+  const float r0 = x0 - __uint_as_float(u0 & 0xffff0000u), r1 = x1 - __uint_as_float(u1 & 0xffff0000u);
+  const uint32_t v0 = __float_as_uint(r0), v1 = __float_as_uint(r1);
+  mid = __byte_perm(v0, v1, 0x7632);
+  const float q0 = r0 - __uint_as_float(v0 & 0xffff0000u), q1 = r1 - __uint_as_float(v1 & 0xffff0000u);
+  lo = __byte_perm(__float_as_uint(q0), __float_as_uint(q1), 0x7632);
+}
+
 // Programmatic dependent launch, used by the kernels of the tensor-core forward: a kernel
 // started with launch_overlapped may be scheduled while the previous kernel of the stream is
 // finishing.  It calls wait_prior_grid() before it touches global memory (the previous kernel

@@ -10,7 +10,6 @@
 // one coalesced 128-byte line and __ballot_sync assembles the word in channel order
 // (LSB = lowest channel).  Eight words are loaded before any is used so that each warp
 // keeps a kilobyte in flight; the kernel is bound by the fp32 read.
-#include <cuda_bf16.h>
 
 #include <algorithm>
 
@@ -437,16 +436,8 @@ cudaError_t launch_pack_i8(const PackI8Args& a, cudaStream_t s) {
 // ------------------------------------------------------------------------------------
 namespace {
 
-__device__ __forceinline__ uint32_t split3_pair(float x0, float x1, uint32_t (&w)[3]) {
-  const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-  const float r0 = x0 - __bfloat162float(h0), r1 = x1 - __bfloat162float(h1);  // exact
-  const __nv_bfloat16 m0 = __float2bfloat16_rn(r0), m1 = __float2bfloat16_rn(r1);
-  const float q0 = r0 - __bfloat162float(m0), q1 = r1 - __bfloat162float(m1);  // exact
-  const __nv_bfloat16 l0 = __float2bfloat16_rn(q0), l1 = __float2bfloat16_rn(q1);
-  w[0] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-  w[1] = static_cast<uint32_t>(__bfloat16_as_ushort(m0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(m1)) << 16);
-  w[2] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
-  return 0;
+__device__ __forceinline__ void split3_pair(float x0, float x1, uint32_t (&w)[3]) {
+  split3_bf16x2(x0, x1, w[0], w[1], w[2]);
 }
 
 template <bool kTerms, bool kA>

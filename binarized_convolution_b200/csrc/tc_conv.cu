@@ -32,6 +32,10 @@
 //               With a split reduction (the FC layer), the partial sums are instead added
 //               into an fp32 workspace by TMA reduce-add (integers below 2^24 add exactly) and
 //               a small kernel applies the epilogue.
+//   binaryWeights straight from the fp32 input (TcArgs::f32): warp 0 loads each k-block's fp32
+//   input as two boxes of 32 channels into the stage's first two part tiles, and the weight
+//   block; eight more warps (6-13) read the boxes, form x~ and its three bf16 parts and
+//   write them over the boxes (each warp rewrites exactly the rows it read); 3 stages fit.
 // Every mbarrier wait gives up after one second of %globaltimer, sets the error word and
 // makes all roles stop; TMEM is released on every exit path.
 #include <cuda.h>
@@ -52,10 +56,15 @@ constexpr int kABytes = 128 * 128;  // 128 rows x 128 bytes
 constexpr int kThreadsTc = 192;
 constexpr int kEpiThreads = 128;
 constexpr int kStageOutBytes = 128 * 128;  // 128 rows x 32 fp32
+// binaryWeights from fp32 input: eight converting warps turn three stages' fp32 boxes into parts
+constexpr int kConvWarps = 8;
+constexpr int kThreadsF32 = kThreadsTc + 32 * kConvWarps;
+constexpr int kF32PartStages = 3;
 
 struct __align__(8) Barriers {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
+  uint64_t xfull[kMaxStages];  // fp32 input: the stage's fp32 boxes have landed
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t done;
@@ -96,10 +105,11 @@ __device__ __forceinline__ TileCoord tile_coord(const TcArgs& a, int w) {
   return c;
 }
 
-template <bool kSplit, int kKind, bool kBits>
-__global__ void __launch_bounds__(kThreadsTc, 1)
+template <bool kSplit, int kKind, bool kBits, bool kF32 = false>
+__global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
     tc_conv_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmOut,
                    const TcArgs a) {
+  static_assert(!kF32 || (kKind == 1 && !kSplit && !kBits), "fp32 input: binaryWeights, fp32 output");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The swizzled tiles need a 1024-byte aligned base, which the dynamic shared window has
   // when the kernel declares no static shared memory; anything else is refused before any
@@ -124,9 +134,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const uint32_t tmem_cols = a.tmem_cols;
 
   if (threadIdx.x == 0) {
+    BCONV_STAMP(0);
     for (int s = 0; s < stages; ++s) {
-      mbar_init(&B->full[s], 1);
+      // fp32 input: the weights' copy and the eight converting warps complete a stage
+      mbar_init(&B->full[s], kF32 ? 1 + kConvWarps : 1);
       mbar_init(&B->empty[s], 1);
+      mbar_init(&B->xfull[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&B->tmem_full[b], 1);
@@ -160,6 +173,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (!kBits) prefetch_tensor_map(&tmOut);  // a bit-packed output never uses (or encodes) it
   }
   wait_prior_grid();  // the codes, A and the output buffer are the previous kernels' business until here
+  if (threadIdx.x == 0) BCONV_STAMP(1);
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -172,6 +186,31 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         const int kb0 = tc.split * kb_per_split;
         const int kb1 = min(kb0 + kb_per_split, kb_total);
         for (int kb = kb0; kb < kb1; ++kb) {
+          if constexpr (kF32) {
+            // the fp32 input of the k-block as two boxes of 32 channels (128-byte rows, 128-byte
+            // swizzle) over the stage's hi and mid tiles, for the converting warps; the weights
+            if (!mbar_wait(&B->empty[stage], phase ^ 1u, B, a.err)) {
+              ok = false;
+              break;
+            }
+            if (t == static_cast<int>(blockIdx.x) && kb - kb0 < 8) BCONV_STAMP(56 + kb - kb0);
+            uint8_t* sa = smem + stage * stage_bytes;
+            mbar_expect_tx(&B->xfull[stage], static_cast<uint32_t>(2 * kABytes));
+            const int tap = kb / a.kb_per_tap, cb = kb - tap * a.kb_per_tap;
+            const int ky = tap / a.kw, kx = tap - ky * a.kw;
+            for (int h = 0; h < 2; ++h)
+              tma_load_4d(sa + h * kABytes, &tmA, &B->xfull[stage], cb * 64 + h * 32, tc.ox0 * a.sx + kx - a.kw / 2,
+                          tc.oy0 * a.sy + ky - a.kh / 2, tc.n0);
+            mbar_expect_tx(&B->full[stage], static_cast<uint32_t>(tc.bn * 128));
+            bulk_load(smem + stage * stage_bytes + a_bytes,
+                      a.b_tiles + ((static_cast<int64_t>(tc.ntile) * kb_total + kb) * a.BN + tc.noff) * 128,
+                      static_cast<uint32_t>(tc.bn * 128), &B->full[stage]);
+            if (++stage == stages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
           if (!mbar_wait(&B->empty[stage], phase ^ 1u, B, a.err)) {
             ok = false;
             break;
@@ -221,18 +260,21 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             ok = false;
             break;
           }
+          if (t == static_cast<int>(blockIdx.x) && kb - kb0 < 18) BCONV_STAMP(12 + kb - kb0);
           tc_fence_after();
           uint8_t* sa = smem + stage * stage_bytes;
           const uint64_t db = smem_desc_sw128(sa + a_bytes);
           if constexpr (kKind == 1) {
-            // the three parts of x~ against the same weight block, into one accumulator
-            for (int part = 0; part < 3; ++part) {
-              const uint64_t da = smem_desc_sw128(sa + part * kABytes);
+            // the three parts of x~ against the same weight block, into one accumulator (fully
+            // unrolled: the issuing thread must do nothing between MMAs but step descriptors)
+            const uint64_t da0 = smem_desc_sw128(sa);
+            const uint32_t acc0 = kb > kb0 ? 1u : 0u;
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {  // four 32-byte K steps across the 128-byte row
-                const uint32_t accum = (kb > kb0 || part > 0 || j > 0) ? 1u : 0u;
-                tc_mma_bf16(d_tmem, da + 2u * j, db + 2u * j, idesc, accum);
-              }
+            for (int part = 0; part < 3; ++part) {
+              const uint64_t da = da0 + static_cast<uint64_t>(part) * (kABytes >> 4);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)  // four 32-byte K steps across the 128-byte row
+                tc_mma_bf16(d_tmem, da + 2u * j, db + 2u * j, idesc, (part > 0 || j > 0) ? 1u : acc0);
             }
           } else if constexpr (kKind == 2) {
             const uint64_t da = smem_desc_sw128(sa);
@@ -259,6 +301,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
         if (!ok) break;
         tc_commit(&B->tmem_full[acc]);
+        {
+          const int ti = (t - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x);
+          if (ti < 4) BCONV_STAMP(2 + ti);
+        }
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
@@ -266,6 +312,93 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       // abort, so that TMEM is never released under a running MMA)
       tc_commit(&B->done);
       mbar_wait(&B->done, 0, B, a.err, false, true);
+    }
+  } else if (kF32 && warp >= 6) {
+    // ---------------- converting warps (fp32 input) ----------------
+    // Warp 6 + w takes tile rows (pixels) 16 w .. 16 w + 15: lane l row 16 w + l % 16 and the
+    // k-block's channels 32 (l / 16) .. + 31, i.e. row r of fp32 box l / 16, which lies in the
+    // hi (box 0) or mid (box 1) tile of the stage.  A lane reads its 32 values, forms x~ =
+    // fma(x, in_scale, in_bias) (0 for a tap outside the image or a channel >= Ni) and the three
+    // bf16 parts, and once the whole warp has its values writes them into the part tiles in the
+    // 128-byte-swizzled layout the MMAs read (8-channel piece m of row r at m ^ (r % 8)).  The
+    // bytes a warp overwrites in the hi and mid tiles are exactly the rows it read from the
+    // two boxes, so no other warp's reads are in the way.
+    const int cw_ = warp - 6;
+    const int r = cw_ * 16 + (lane & 15), half = lane >> 4;
+    const int rc = a.R * a.Cw;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      const TileCoord tc = tile_coord(a, t);
+      const int n = tc.n0 + r / rc, oy = tc.oy0 + (r / a.Cw) % a.R, ox = tc.ox0 + r % a.Cw;
+      const bool row_ok = n < a.N && oy < a.Ho && ox < a.Wo;
+      const int kb0 = tc.split * kb_per_split;
+      const int kb1 = min(kb0 + kb_per_split, kb_total);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&B->xfull[stage], phase, B, a.err))) {
+          ok = false;
+          break;
+        }
+        if (warp == 6 && lane == 0 && t == static_cast<int>(blockIdx.x) && kb - kb0 < 8) BCONV_STAMP(30 + kb - kb0);
+        uint8_t* sa = smem + stage * stage_bytes;
+        float4 u[8];  // 16-byte chunk j of the row holds channels 4 j .. 4 j + 3 of this half
+        {
+          const uint8_t* fb = sa + half * kABytes + r * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) u[j] = *reinterpret_cast<const float4*>(fb + ((j ^ (r & 7)) * 16));
+        }
+        const int tap = kb / a.kb_per_tap, cb = kb - tap * a.kb_per_tap;
+        const int ky = tap / a.kw, kx = tap - ky * a.kw;
+        const int iy = oy * a.sy + ky - a.kh / 2, ix = ox * a.sx + kx - a.kw / 2;
+        const bool in_img = row_ok && iy >= 0 && iy < a.H && ix >= 0 && ix < a.W;
+        uint32_t hi[4][4], mid[4][4], lo[4][4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // channels 8 q .. 8 q + 7 of this half
+          const int c = cb * 64 + half * 32 + 8 * q;
+          float v[8] = {u[2 * q].x, u[2 * q].y, u[2 * q].z, u[2 * q].w,
+                        u[2 * q + 1].x, u[2 * q + 1].y, u[2 * q + 1].z, u[2 * q + 1].w};
+          const bool live0 = in_img && c < a.Ni, live1 = in_img && c + 4 < a.Ni;
+          if (a.in_scale) {
+            if (live0) {
+              const float4 s4 = __ldg(reinterpret_cast<const float4*>(a.in_scale + c));
+              const float4 b4 = __ldg(reinterpret_cast<const float4*>(a.in_bias + c));
+              v[0] = fmaf(v[0], s4.x, b4.x); v[1] = fmaf(v[1], s4.y, b4.y);
+              v[2] = fmaf(v[2], s4.z, b4.z); v[3] = fmaf(v[3], s4.w, b4.w);
+            }
+            if (live1) {
+              const float4 s4 = __ldg(reinterpret_cast<const float4*>(a.in_scale + c + 4));
+              const float4 b4 = __ldg(reinterpret_cast<const float4*>(a.in_bias + c + 4));
+              v[4] = fmaf(v[4], s4.x, b4.x); v[5] = fmaf(v[5], s4.y, b4.y);
+              v[6] = fmaf(v[6], s4.z, b4.z); v[7] = fmaf(v[7], s4.w, b4.w);
+            }
+          }
+          // out-of-image taps and channels >= Ni read zeros from the box, but the terms would
+          // turn them into in_bias, and a row past the output reads some other pixel
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (!(j < 4 ? live0 : live1)) v[j] = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) split3_bf16x2(v[2 * j], v[2 * j + 1], hi[q][j], mid[q][j], lo[q][j]);
+        }
+        __syncwarp();  // every lane has read its values before any lane overwrites the boxes
+        uint8_t* db = sa + r * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int pos = ((half * 4 + q) ^ (r & 7)) * 16;
+          *reinterpret_cast<uint4*>(db + pos) = make_uint4(hi[q][0], hi[q][1], hi[q][2], hi[q][3]);
+          *reinterpret_cast<uint4*>(db + kABytes + pos) = make_uint4(mid[q][0], mid[q][1], mid[q][2], mid[q][3]);
+          *reinterpret_cast<uint4*>(db + 2 * kABytes + pos) = make_uint4(lo[q][0], lo[q][1], lo[q][2], lo[q][3]);
+        }
+        fence_proxy_async();  // the parts (generic stores) before the MMAs read them (async proxy)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B->full[stage]);
+        if (warp == 6 && lane == 0 && t == static_cast<int>(blockIdx.x) && kb - kb0 < 8) BCONV_STAMP(38 + kb - kb0);
+        if (++stage == stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
     }
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
@@ -320,6 +453,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
       }
       if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err, true, true))) break;
+      const int eti = (t - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x);
+      if (et == 0 && eti < 4) BCONV_STAMP(52 + eti);
       tc_fence_after();
       float bits_asum = 0.f;
       Words8 bits_w{};
@@ -392,6 +527,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         bits_finish_item(a, bits_pix, bits_valid, bits_asum, tc.mtile, tc.mtile, tc.ntile,
                          tc.ntile * a.pieces + tc.noff / tc.bn, bits_flag, et);
       }
+      if (et == 0 && eti < 4) BCONV_STAMP(48 + eti);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -467,6 +603,8 @@ __global__ void __launch_bounds__(kFinThreads) tc_finalize_kernel(float4* __rest
 
 }  // namespace
 
+BCONV_TIMELINE_READER(bconv_timeline_tc)
+
 constexpr int kSmemMax = 227 * 1024;  // dynamic shared memory one CTA may opt in to
 
 int tc_stages(int kind, int bn, int mt) {
@@ -479,6 +617,12 @@ int tc_stages(int kind, int bn, int mt) {
 int tc_smem_bytes(const TcArgs& a) {
   return a.stages * ((a.kind == 1 ? 3 : a.mt) * kABytes + a.BN * 128) + 2 * kStageOutBytes +
          static_cast<int>(sizeof(Barriers));
+}
+
+int tc_f32_stages(int bn) {
+  const int stage = 3 * kABytes + bn * 128;
+  const int fixed = 2 * kStageOutBytes + static_cast<int>(sizeof(Barriers));
+  return bn <= 128 && fixed + kF32PartStages * stage <= kSmemMax ? kF32PartStages : 0;
 }
 
 int tc_plan(TcArgs& a, int sm_count) {
@@ -504,6 +648,9 @@ cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmOut, con
   if (a.stages < 2 || a.stages > (a.kind == 0 ? kStages : kMaxStages) || (a.kind != 0 && a.mt != 1) ||
       (a.kind == 0 && a.stages != kStages) || (a.kind == 2 && 2 * a.BN + 32 > static_cast<int>(a.tmem_cols)))
     return cudaErrorInvalidValue;
+  if (a.f32 && (a.kind != 1 || a.k_splits != 1 || a.out_bits || a.stages != kF32PartStages || a.BN > 128 ||
+                a.Ni % 4 != 0 || (a.in_scale && !a.in_bias)))
+    return cudaErrorInvalidValue;
   const int smem = tc_smem_bytes(a);
   const int tiles = a.m_tiles * a.n_tiles * a.k_splits;
   if (tiles == 0) return cudaSuccess;
@@ -517,9 +664,10 @@ cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmOut, con
                                     tc_conv_kernel<false, 2, true>, a.kind)
                              : pick(tc_conv_kernel<false, 0, false>, tc_conv_kernel<false, 1, false>,
                                     tc_conv_kernel<false, 2, false>, a.kind);
+  if (a.f32) kern = tc_conv_kernel<false, 1, false, true>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  return launch_overlapped(kern, dim3(grid), dim3(kThreadsTc), smem, s, *tmA, *tmOut, a);
+  return launch_overlapped(kern, dim3(grid), dim3(a.f32 ? kThreadsF32 : kThreadsTc), smem, s, *tmA, *tmOut, a);
 }
 
 cudaError_t launch_tc_finalize(float* ws, float* out, const float* scale, const float* bias, const float* A, int hw,

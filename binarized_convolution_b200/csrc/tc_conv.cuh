@@ -66,6 +66,16 @@ struct TcArgs {
   int sk;
   uint32_t* sk_part;        // [pairs - 1][2][BN / 32][32][128] accumulator words
   uint32_t* sk_flag;        // [pairs - 1][2], zero between launches
+  // binaryWeights straight from the fp32 input (f32 != 0; one SM per tile, BN <= 128, no beta):
+  // tmA is then a map over the input x [N][H][W][Ni] fp32 (boxes of 32 channels x Cw x R x Bn
+  // pixels with the convolution's strides as element strides, 128-byte swizzle), and
+  // converting warps form x~ = fma(x, in_scale, in_bias) -- zero for out-of-image taps and
+  // channels >= Ni -- and its exact three bf16 parts in shared memory, so no parts buffer is
+  // written or read.
+  int f32;
+  const float* in_scale;  // [Ni] or nullptr
+  const float* in_bias;
+  int Ni;
   // Weights for the one-SM kernel: [n_tiles][kh * kw * kb_per_tap][BN][128] bytes, one
   // contiguous block per (N tile, k-block) already in the shared-memory order of the 128-byte
   // swizzle (16-byte chunk c of row r stored at chunk c ^ (r % 8)), so that each stage is one
@@ -142,6 +152,7 @@ cudaError_t launch_tc_fc(const CUtensorMap* tmA, const CUtensorMap* tmB, const F
 
 
 int tc_stages(int kind, int bn, int mt);  // stages that fit; < 2: the layout does not fit
+int tc_f32_stages(int bn);                // binaryWeights from fp32 input: part stages, 0 if it does not fit
 int tc_smem_bytes(const TcArgs& a);
 // One CTA per tile; weights from a.b_tiles.
 cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmOut, const TcArgs& a, cudaStream_t s);
@@ -186,8 +197,9 @@ struct PackI8Args {
 cudaError_t launch_pack_i8(const PackI8Args& a, cudaStream_t s);
 
 // binaryWeights operand for the tensor cores: x~ split exactly into three bf16 parts,
-// x~ = hi + mid + lo (hi = bf16(x~), mid = bf16(x~ - hi), lo = bf16(x~ - hi - mid); each
-// difference is exact in fp32), stored per pixel as [part][cip] bf16; channels in [ni, cip) are 0.
+// x~ = hi + mid + lo (each the leading 8 significant bits of what the previous parts leave;
+// every difference is exact in fp32), stored per pixel as [part][cip] bf16; channels in
+// [ni, cip) are 0.
 struct PackBf16x3Args {
   const float* in;        // [npix][ni]
   int64_t npix;

@@ -242,25 +242,37 @@ bconv_status_t bconv_set_tc_codes(bconv_tc_codes_t codes);
 int32_t bconv_tc_codes(bconv_handle_t h);
 
 /*
- * How the XNOR / AND tensor-core contraction of a stride-1 convolution on e2m1 codes brings the
- * activations into shared memory, for layers created after the call (process-wide, like
- * bconv_set_cta_mode).
+ * How the tensor-core contraction brings the activations into shared memory, for layers
+ * created after the call (process-wide, like bconv_set_cta_mode).
  *   PER_TAP  for every tap of the window, a box of the tile's pixels shifted by the tap offset
- *            (each activation code is loaded once per tap).
+ *            (each activation code is loaded once per tap); binaryWeights: of the three bf16
+ *            parts of x~ that a pack kernel wrote to memory before the contraction.
  *   ROWS     the codes sit in a zero-bordered copy of the image; a tile is 128 consecutive
  *            positions of that grid, and one load of them plus the window's reach serves every
  *            tap (the taps differ only in where their operand starts in shared memory); the
  *            weights of a CTA's output channels stay in shared memory when they fit.  Needs
  *            (kernel_h - 1) * (in_w + kernel_w - 1) + kernel_w - 1 <= 896 and an fp32 output;
  *            a bit-packed output (bconv_set_output_terms) moves the layer to PER_TAP.
- *   AUTO     ROWS where it applies, else PER_TAP.
+ *   INPUT    binaryWeights convolutions: per tap, a box of the fp32 input itself; converting
+ *            warps of the contraction form x~ = in_scale * x + in_bias and its three bf16 parts
+ *            in shared memory, so no parts buffer is written or read (no pack kernel runs).
+ *            Needs no beta,
+ *            in_c % 4 == 0, a 16-byte aligned input and an fp32 output; a bit-packed output
+ *            moves the layer to PER_TAP, and so does a forward whose input is not 16-byte
+ *            aligned (for that call only: it runs on the SIMT family).
+ *   AUTO     ROWS or INPUT where they apply, else PER_TAP.
  * Returns INVALID_ARG for an unknown value.
  */
-typedef enum { BCONV_STAGING_AUTO = 0, BCONV_STAGING_PER_TAP = 1, BCONV_STAGING_ROWS = 2 } bconv_staging_t;
+typedef enum {
+  BCONV_STAGING_AUTO = 0,
+  BCONV_STAGING_PER_TAP = 1,
+  BCONV_STAGING_ROWS = 2,
+  BCONV_STAGING_INPUT = 3
+} bconv_staging_t;
 bconv_status_t bconv_set_staging(bconv_staging_t staging);
 
-/* The staging a layer's tensor-core contraction uses (BCONV_STAGING_PER_TAP or ROWS); 0 when the
- * layer has no tensor-core path, -1 for a bad handle. */
+/* The staging a layer's tensor-core contraction uses (BCONV_STAGING_PER_TAP, ROWS or INPUT); 0
+ * when the layer has no tensor-core path, -1 for a bad handle. */
 int32_t bconv_staging(bconv_handle_t h);
 
 /*
