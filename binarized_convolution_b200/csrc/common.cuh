@@ -61,14 +61,24 @@ static __device__ unsigned long long g_bconv_timeline[1024 * 64];  // one array 
 // subset of x~'s bits), mid = r cut the same way, lo = r - mid (exact, and with at most 8
 // significant bits left, itself a bf16 with zero low bits).  Every part is a normal bf16 (or 0)
 // for |x~| >= 2^-103.  Two values at a time as bf16x2 words (x0 in the low half); bit
-// operations and exact subtractions only, no conversion instructions.
+// operations and exact subtractions (both values in one packed f32x2 subtraction, round to
+// nearest, no flush to zero) only, no conversion instructions.
+__device__ __forceinline__ void sub_f32x2(float a0, float a1, float b0, float b1, float& d0, float& d1) {
+  asm("{\n .reg .b64 a, b, d;\n mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %5};\n sub.rn.f32x2 d, a, b;\n"
+      " mov.b64 {%0, %1}, d;\n}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 __device__ __forceinline__ void split3_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& mid, uint32_t& lo) {
   const uint32_t u0 = __float_as_uint(x0), u1 = __float_as_uint(x1);
   hi = __byte_perm(u0, u1, 0x7632);  // the high halves of both
-  const float r0 = x0 - __uint_as_float(u0 & 0xffff0000u), r1 = x1 - __uint_as_float(u1 & 0xffff0000u);
+  float r0, r1;
+  sub_f32x2(x0, x1, __uint_as_float(u0 & 0xffff0000u), __uint_as_float(u1 & 0xffff0000u), r0, r1);
   const uint32_t v0 = __float_as_uint(r0), v1 = __float_as_uint(r1);
   mid = __byte_perm(v0, v1, 0x7632);
-  const float q0 = r0 - __uint_as_float(v0 & 0xffff0000u), q1 = r1 - __uint_as_float(v1 & 0xffff0000u);
+  float q0, q1;
+  sub_f32x2(r0, r1, __uint_as_float(v0 & 0xffff0000u), __uint_as_float(v1 & 0xffff0000u), q0, q1);
   lo = __byte_perm(__float_as_uint(q0), __float_as_uint(q1), 0x7632);
 }
 

@@ -373,11 +373,14 @@ __global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
               v[6] = fmaf(v[6], s4.z, b4.z); v[7] = fmaf(v[7], s4.w, b4.w);
             }
           }
-          // out-of-image taps and channels >= Ni read zeros from the box, but the terms would
-          // turn them into in_bias, and a row past the output reads some other pixel
+          // out-of-image taps and channels >= Ni read zeros from the box (a row past the output
+          // reads some other pixel, whose sums are never stored), but the terms would turn
+          // them into in_bias
+          if (a.in_scale) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (!(j < 4 ? live0 : live1)) v[j] = 0.f;
+            for (int j = 0; j < 8; ++j)
+              if (!(j < 4 ? live0 : live1)) v[j] = 0.f;
+          }
 #pragma unroll
           for (int j = 0; j < 4; ++j) split3_bf16x2(v[2 * j], v[2 * j + 1], hi[q][j], mid[q][j], lo[q][j]);
         }
