@@ -658,6 +658,21 @@ bconv_status_t setup_tc(Layer& L, const uint32_t* packed) {
                          static_cast<uint32_t>(t.BN / t.pieces / 2));
   } else {
     t.grid_ctas = tc_plan(t, current_sm_count());  // work list: tail tiles cut along N
+    if (t.f32 && t.m_tiles * t.n_tiles > t.grid_ctas) {
+      // binaryWeights from fp32 input: the converting warps' work does not shrink with a tail
+      // piece's channels, so the CTAs take equal contiguous shares of all tiles' k-blocks
+      // instead (a tile cut between two CTAs finished by the first, with the second's raw
+      // sums).  Batch 8, 112 x 112, 128 -> 128, stride 2: 36 k-blocks converted on the busiest
+      // SM with tail pieces, 24 with equal shares.
+      t.sk = 1;
+      t.pieces = 1;
+      t.full_tiles = t.m_tiles * t.n_tiles;
+      const int cuts = t.grid_ctas - 1;
+      cudaError_t e2 = L.tc_mem.alloc(&t.sk_part, static_cast<size_t>(cuts) * t.BN * 128);
+      if (e2 == cudaSuccess) e2 = L.tc_mem.alloc(&t.sk_flag, static_cast<size_t>(cuts));
+      if (e2 == cudaSuccess) e2 = cudaMemset(t.sk_flag, 0, sizeof(uint32_t) * cuts);
+      if (e2 != cudaSuccess) return from_cuda(e2);
+    }
     t.b_tiles = L.wq;
     L.hx.b_tiles = L.wq;
     L.hx.scale = L.scale;
@@ -1271,7 +1286,8 @@ bconv_status_t sync_status(Layer& L, cudaStream_t s) {
   if (word) {
     cudaMemset(L.err, 0, sizeof(uint32_t));
     if (L.a_count) cudaMemset(L.a_count, 0, sizeof(uint32_t) * L.tc.m_tiles);  // an aborted launch may leave counts
-    if (L.tc.sk_flag) cudaMemset(L.tc.sk_flag, 0, sizeof(uint32_t) * (L.tc.grid_ctas / 2 - 1) * 2);  // and flags
+    if (L.tc.sk_flag)  // and flags (pairs: two per cut between pairs; one SM: one per cut between CTAs)
+      cudaMemset(L.tc.sk_flag, 0, sizeof(uint32_t) * (L.tc_pair ? (L.tc.grid_ctas / 2 - 1) * 2 : L.tc.grid_ctas - 1));
     if (L.ws) cudaMemset(L.ws, 0, sizeof(float) * static_cast<size_t>(L.N) * L.No);  // and partial sums
     if (word & kErrTimeout) return BCONV_ERR_TIMEOUT;
     return BCONV_ERR_CUDA;  // kErrLayout: a kernel refused an unexpected shared-memory layout

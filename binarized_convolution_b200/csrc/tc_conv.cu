@@ -105,6 +105,50 @@ __device__ __forceinline__ TileCoord tile_coord(const TcArgs& a, int w) {
   return c;
 }
 
+// A CTA's work list: (tile, k-block range) items.  Without a.sk, tiles blockIdx.x, + gridDim.x,
+// ... with their split's k-blocks.  With a.sk (the fp32-input kernel when the tiles outnumber
+// the CTAs), a contiguous, equal share of all tiles' k-blocks in tile order: a tile cut between
+// CTA c and c + 1 has its first k-blocks as c's last item and the rest as c + 1's first item;
+// c + 1 leaves its raw sums in sk_part[c] and raises sk_flag[c], c adds them and finishes the
+// tile.  (Each share is at least a tile's k-blocks long, so no tile is cut twice.)
+struct ConvWork {
+  int64_t u, uend;
+  int t, ti;
+  __device__ ConvWork(const TcArgs& a, int total_tiles, int kb_total) : ti(0) {
+    const int64_t U = static_cast<int64_t>(total_tiles) * kb_total;
+    u = a.sk ? U * blockIdx.x / gridDim.x : 0;
+    uend = a.sk ? U * (blockIdx.x + 1) / gridDim.x : 0;
+    t = blockIdx.x;
+  }
+  __device__ bool next(const TcArgs& a, int total_tiles, int kb_total, int kb_per_split, int& tile, int& k0, int& k1) {
+    if (!a.sk) {
+      if (t >= total_tiles) return false;
+      tile = t;
+      k0 = tile_coord(a, t).split * kb_per_split;
+      k1 = min(k0 + kb_per_split, kb_total);
+      t += gridDim.x;
+    } else {
+      if (u >= uend) return false;
+      tile = static_cast<int>(u / kb_total);
+      k0 = static_cast<int>(u - static_cast<int64_t>(tile) * kb_total);
+      k1 = static_cast<int>(min(static_cast<int64_t>(kb_total), k0 + (uend - u)));
+      u += k1 - k0;
+    }
+    ++ti;
+    return true;
+  }
+};
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 template <bool kSplit, int kKind, bool kBits, bool kF32 = false>
 __global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
     tc_conv_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmOut,
@@ -181,10 +225,10 @@ __global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      ConvWork wk(a, total_tiles, kb_total);
+      int t, kb0, kb1;
+      while (ok && wk.next(a, total_tiles, kb_total, kb_per_split, t, kb0, kb1)) {
         const TileCoord tc = tile_coord(a, t);
-        const int kb0 = tc.split * kb_per_split;
-        const int kb1 = min(kb0 + kb_per_split, kb_total);
         for (int kb = kb0; kb < kb1; ++kb) {
           if constexpr (kF32) {
             // the fp32 input of the k-block as two boxes of 32 channels (128-byte rows, 128-byte
@@ -193,7 +237,7 @@ __global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
               ok = false;
               break;
             }
-            if (t == static_cast<int>(blockIdx.x) && kb - kb0 < 8) BCONV_STAMP(56 + kb - kb0);
+            if (wk.ti == 1 && kb - kb0 < 8) BCONV_STAMP(56 + kb - kb0);
             uint8_t* sa = smem + stage * stage_bytes;
             mbar_expect_tx(&B->xfull[stage], static_cast<uint32_t>(2 * kABytes));
             const int tap = kb / a.kb_per_tap, cb = kb - tap * a.kb_per_tap;
@@ -247,11 +291,11 @@ __global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      ConvWork wk(a, total_tiles, kb_total);
+      int t, kb0, kb1;
+      while (ok && wk.next(a, total_tiles, kb_total, kb_per_split, t, kb0, kb1)) {
         const TileCoord tc = tile_coord(a, t);
         const uint32_t idesc = idesc_for(kKind, 128, tc.bn);
-        const int kb0 = tc.split * kb_per_split;
-        const int kb1 = min(kb0 + kb_per_split, kb_total);
         if (!mbar_wait(&B->tmem_empty[acc], acc_phase ^ 1u, B, a.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.mt * a.BN);
@@ -260,7 +304,7 @@ __global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
             ok = false;
             break;
           }
-          if (t == static_cast<int>(blockIdx.x) && kb - kb0 < 18) BCONV_STAMP(12 + kb - kb0);
+          if (wk.ti == 1 && kb - kb0 < 18) BCONV_STAMP(12 + kb - kb0);
           tc_fence_after();
           uint8_t* sa = smem + stage * stage_bytes;
           const uint64_t db = smem_desc_sw128(sa + a_bytes);
@@ -301,10 +345,7 @@ __global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
         }
         if (!ok) break;
         tc_commit(&B->tmem_full[acc]);
-        {
-          const int ti = (t - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x);
-          if (ti < 4) BCONV_STAMP(2 + ti);
-        }
+        if (wk.ti <= 4) BCONV_STAMP(1 + wk.ti);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
@@ -329,18 +370,18 @@ __global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+    ConvWork wk(a, total_tiles, kb_total);
+    int t, kb0, kb1;
+    while (ok && wk.next(a, total_tiles, kb_total, kb_per_split, t, kb0, kb1)) {
       const TileCoord tc = tile_coord(a, t);
       const int n = tc.n0 + r / rc, oy = tc.oy0 + (r / a.Cw) % a.R, ox = tc.ox0 + r % a.Cw;
       const bool row_ok = n < a.N && oy < a.Ho && ox < a.Wo;
-      const int kb0 = tc.split * kb_per_split;
-      const int kb1 = min(kb0 + kb_per_split, kb_total);
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!__all_sync(0xffffffffu, mbar_wait(&B->xfull[stage], phase, B, a.err))) {
           ok = false;
           break;
         }
-        if (warp == 6 && lane == 0 && t == static_cast<int>(blockIdx.x) && kb - kb0 < 8) BCONV_STAMP(30 + kb - kb0);
+        if (warp == 6 && lane == 0 && wk.ti == 1 && kb - kb0 < 8) BCONV_STAMP(30 + kb - kb0);
         uint8_t* sa = smem + stage * stage_bytes;
         float4 u[8];  // 16-byte chunk j of the row holds channels 4 j .. 4 j + 3 of this half
         {
@@ -396,7 +437,7 @@ __global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
         fence_proxy_async();  // the parts (generic stores) before the MMAs read them (async proxy)
         __syncwarp();
         if (lane == 0) mbar_arrive(&B->full[stage]);
-        if (warp == 6 && lane == 0 && t == static_cast<int>(blockIdx.x) && kb - kb0 < 8) BCONV_STAMP(38 + kb - kb0);
+        if (warp == 6 && lane == 0 && wk.ti == 1 && kb - kb0 < 8) BCONV_STAMP(38 + kb - kb0);
         if (++stage == stages) {
           stage = 0;
           phase ^= 1u;
@@ -417,8 +458,34 @@ __global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
     constexpr bool bits_out = kBits && !kSplit;
     float2* next_t = reinterpret_cast<float2*>(stage_out);
     uint32_t* bits_flag = reinterpret_cast<uint32_t*>(stage_out + kStageOutBytes);
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+    ConvWork wk(a, total_tiles, kb_total);
+    int t, ek0, ek1;
+    while (wk.next(a, total_tiles, kb_total, kb_per_split, t, ek0, ek1)) {
       const TileCoord tc = tile_coord(a, t);
+      if (kF32 && a.sk && ek0 > 0) {
+        // the later k-blocks of a tile that CTA blockIdx.x - 1 finishes: leave the raw sums
+        if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err, true, true))) break;
+        tc_fence_after();
+        uint32_t* part = a.sk_part + static_cast<size_t>(blockIdx.x - 1) * a.BN * 128;
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
+        for (int ch = 0; ch < tc.bn / 32; ++ch) {
+          uint32_t v[32];
+          tc_ld_32x32(tb + static_cast<uint32_t>(ch * 32), v);
+          if (ch == tc.bn / 32 - 1) {
+            tc_fence_before();
+            if (lane == 0) mbar_arrive(&B->tmem_empty[acc]);
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) part[(ch * 32 + j) * 128 + row] = v[j];  // lanes write 128-byte rows
+        }
+        __threadfence();
+        epi_barrier();
+        if (et == 0) st_release_u32(a.sk_flag + blockIdx.x - 1, 1u);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+        continue;
+      }
+      const bool sk_owner = kF32 && a.sk && ek1 < kb_total;  // CTA blockIdx.x + 1 has the rest
       if (!kSplit && tc.ntile != loaded_ntile) {  // this tile's (scale, bias) into shared memory
         epi_barrier();
         for (int j = et; j < a.BN; j += kEpiThreads) {
@@ -455,8 +522,27 @@ __global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
           beta_h[h] = __ldg(a.beta + (static_cast<int64_t>(n) * a.Ho + oy) * a.Wo + ox);
         }
       }
+      const uint32_t* part = nullptr;
+      if (sk_owner) {  // wait (bounded) for the raw sums of this tile's later k-blocks
+        bool ready = true;
+        if (et == 0) {
+          const uint32_t* flag = a.sk_flag + blockIdx.x;
+          const uint64_t t0 = globaltimer();
+          while (ld_acquire_u32(flag) == 0u) {
+            if (*reinterpret_cast<volatile uint32_t*>(&B->abort_flag) || globaltimer() - t0 > kTimeoutNs) {
+              atomicOr(a.err, kErrTimeout);
+              atomicExch(&B->abort_flag, 1u);
+              ready = false;
+              break;
+            }
+          }
+        }
+        if (!epi_all(ready)) break;
+        __threadfence();
+        part = a.sk_part + static_cast<size_t>(blockIdx.x) * a.BN * 128;
+      }
       if (!epi_all(mbar_wait(&B->tmem_full[acc], acc_phase, B, a.err, true, true))) break;
-      const int eti = (t - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x);
+      const int eti = wk.ti - 1;
       if (et == 0 && eti < 4) BCONV_STAMP(52 + eti);
       tc_fence_after();
       float bits_asum = 0.f;
@@ -474,6 +560,11 @@ __global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
           if (h == a.mt - 1 && ch == tc.bn / 32 - 1) {  // accumulator fully read: hand it back
             tc_fence_before();
             if (lane == 0) mbar_arrive(&B->tmem_empty[acc]);
+          }
+          if (kF32 && part) {  // + the later k-blocks' sums, in this fixed order
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(__ldcg(part + (ch * 32 + j) * 128 + row)));
           }
           const int buf = chunk_count & 1;
           ++chunk_count;
@@ -529,6 +620,10 @@ __global__ void __launch_bounds__(kF32 ? kThreadsF32 : kThreadsTc, 1)
         if (bits_valid) words_store(a.out_bits + bits_pix * a.nwo + w0, bits_w, min(tc.bn / 32, a.nwo - w0));
         bits_finish_item(a, bits_pix, bits_valid, bits_asum, tc.mtile, tc.mtile, tc.ntile,
                          tc.ntile * a.pieces + tc.noff / tc.bn, bits_flag, et);
+      }
+      if (sk_owner) {  // every thread has read the partial sums: the slot is free for the next launch
+        epi_barrier();
+        if (et == 0) a.sk_flag[blockIdx.x] = 0u;
       }
       if (et == 0 && eti < 4) BCONV_STAMP(48 + eti);
       acc ^= 1;
@@ -654,11 +749,17 @@ cudaError_t launch_tc_conv(const CUtensorMap* tmA, const CUtensorMap* tmOut, con
   if (a.f32 && (a.kind != 1 || a.k_splits != 1 || a.out_bits || a.stages != kF32PartStages || a.BN > 128 ||
                 a.Ni % 4 != 0 || (a.in_scale && !a.in_bias)))
     return cudaErrorInvalidValue;
+  // the balanced work list: the fp32-input kernel only, whole tiles (no pieces), a grid of
+  // grid_ctas CTAs, all resident at once (one per SM), each with at least a tile's k-blocks
+  if (a.sk && (!a.f32 || !a.sk_part || !a.sk_flag || a.pieces != 1 || a.grid_ctas < 1 ||
+               a.grid_ctas > current_sm_count() || a.m_tiles * a.n_tiles < a.grid_ctas))
+    return cudaErrorInvalidValue;
   const int smem = tc_smem_bytes(a);
   const int tiles = a.m_tiles * a.n_tiles * a.k_splits;
   if (tiles == 0) return cudaSuccess;
   int grid = current_sm_count();
   if (grid > tiles) grid = tiles;
+  if (a.sk) grid = a.grid_ctas;  // the shares and the exchange slots were cut for this grid
   if ((a.out_bits && a.k_splits > 1) || !a.b_tiles) return cudaErrorInvalidValue;
   auto pick = [](auto k0, auto k1, auto k2, int kind) { return kind == 2 ? k2 : kind == 1 ? k1 : k0; };
   auto kern = a.k_splits > 1 ? pick(tc_conv_kernel<true, 0, false>, tc_conv_kernel<true, 1, false>,

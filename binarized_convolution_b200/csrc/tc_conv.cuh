@@ -63,9 +63,11 @@ struct TcArgs {
   // p and p+1 is finished by p (which computes its first k-blocks, last in its share); p+1
   // computes the rest first and leaves its raw partial sums in sk_part[p][rank] with
   // sk_flag[p][rank] = 1, which p adds (int32 exactly, fp32 in a fixed order) and resets.
+  // The one-SM fp32-input kernel does the same per CTA (sk_part[c], sk_flag[c] for the tile cut
+  // between CTAs c and c + 1) when the tiles outnumber the CTAs.
   int sk;
-  uint32_t* sk_part;        // [pairs - 1][2][BN / 32][32][128] accumulator words
-  uint32_t* sk_flag;        // [pairs - 1][2], zero between launches
+  uint32_t* sk_part;        // pairs: [pairs - 1][2][BN / 32][32][128]; one SM: [CTAs - 1][BN / 32][32][128] words
+  uint32_t* sk_flag;        // pairs: [pairs - 1][2]; one SM: [CTAs - 1]; zero between launches
   // binaryWeights straight from the fp32 input (f32 != 0; one SM per tile, BN <= 128, no beta):
   // tmA is then a map over the input x [N][H][W][Ni] fp32 (boxes of 32 channels x Cw x R x Bn
   // pixels with the convolution's strides as element strides, 128-byte swizzle), and

@@ -29,6 +29,18 @@ CASES = [
                      in_terms=True, seed=705),
     synth.small_case(batch=2, h=30, w=30, ni=68, no=128, k=3, op=synth.BINARY_WEIGHTS, use_beta=False, relu=True,
                      in_terms=False, seed=706),
+    # edges: the fewest channels, a wide reduction (32 k-blocks a tap), even and non-square
+    # windows, different strides per axis, a 1 x 1 image, a few output channels, and a batch
+    # whose last tile holds one image
+    synth.small_case(batch=3, h=7, w=9, ni=4, no=16, k=3, op=synth.BINARY_WEIGHTS, in_terms=True, seed=707),
+    synth.small_case(batch=1, h=6, w=7, ni=2048, no=64, k=3, op=synth.BINARY_WEIGHTS, in_terms=True, relu=True,
+                     seed=708),
+    synth.small_case(batch=2, h=13, w=12, ni=96, no=48, k=2, op=synth.BINARY_WEIGHTS, in_terms=True, seed=709),
+    synth.small_case(batch=2, h=11, w=14, ni=40, no=24, k=3, kw=1, stride=1, stride_x=2, op=synth.BINARY_WEIGHTS,
+                     in_terms=True, seed=710),
+    synth.small_case(batch=5, h=1, w=1, ni=64, no=8, k=3, op=synth.BINARY_WEIGHTS, in_terms=True, seed=711),
+    synth.small_case(batch=9, h=8, w=8, ni=64, no=128, k=5, stride=2, op=synth.BINARY_WEIGHTS, relu=True,
+                     in_terms=False, seed=712),
 ]
 
 
@@ -138,3 +150,33 @@ def test_input_buffers_rotate(cuda_device):
         inp = synth.Inputs(refs[j], base.wbits, base.scale, base.bias, base.in_scale, base.in_bias)
         S_ref, beta_ref, y_ref = pu.run_oracle(w, inp)
         pu.assert_outputs_close(w, inp, y, S_ref, beta_ref, y_ref)
+
+
+# more tiles than SMs: the CTAs take equal contiguous shares of all tiles' k-blocks, and a tile
+# cut between two CTAs is finished by the first with the second's fp32 partial sums -- another
+# order of the same fp32 additions, so these are held to the oracle's tolerance only
+SHARE_CASES = [
+    synth.small_case(batch=8, h=64, w=64, ni=64, no=64, k=3, op=synth.BINARY_WEIGHTS, relu=True, in_terms=True,
+                     seed=720),
+    synth.small_case(batch=8, h=56, w=56, ni=200, no=40, k=3, op=synth.BINARY_WEIGHTS, in_terms=False, seed=721),
+]
+
+
+@pytest.mark.parametrize("w", SHARE_CASES, ids=lambda w: w.name)
+def test_input_staging_equal_shares(w, cuda_device):
+    """Every output against the oracle, over three forwards of one layer (the exchange flags must
+    be back at zero after each launch)."""
+    import torch
+
+    inp = synth.make_inputs(w)
+    S_ref, beta_ref, y_ref = pu.run_oracle(w, inp)
+    layer = pu.make_layer(w, inp)
+    try:
+        assert layer.staging() == bc.STAGING_INPUT
+        x = torch.from_numpy(inp.x).cuda()
+        for _ in range(3):
+            y = layer(x)
+            layer.sync_status()
+            pu.assert_outputs_close(w, inp, y.reshape(-1, w.out_channels).cpu().numpy(), S_ref, beta_ref, y_ref)
+    finally:
+        layer.close()
