@@ -1308,6 +1308,7 @@ bconv_status_t set_algo(Layer& L, int algo) {
 }
 
 int launches_per_forward(const Layer& L) {
+  if (L.N > 0 && use_tc(L) && L.tc.f32) return 1;  // binaryWeights from fp32 input: the contraction alone
   if (L.N > 0 && use_tc(L) && L.fcb) return 2;  // pack, the FC kernel (which finishes its own tiles)
   if (L.N > 0 && use_tc(L))  // pack, contraction; a split FC adds the finalize, an unsplit FC with beta its mean
     return 2 + (L.tc.k_splits > 1 ? 1 : ((L.fc && L.use_beta()) ? 1 : 0));

@@ -83,8 +83,10 @@ def test_input_staging_choice(cuda_device):
 
     with layer() as l:
         assert l.staging() == bc.STAGING_INPUT and l.tc_codes() == bc.CODES_BF16X3
+        assert l.launches_per_forward() == 1  # no pack kernel
     with layer(use_beta=True) as l:
         assert l.staging() == bc.STAGING_PER_TAP
+        assert l.launches_per_forward() == 2
     with layer(ni=30) as l:
         assert l.staging() == bc.STAGING_PER_TAP
     with layer() as l:
