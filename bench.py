@@ -554,6 +554,10 @@ def measure_workload(args, w: synth.Workload, device, bits_io: bool = False, cpu
             layer.cta_mode(), "?")
         roof["codes"] = {CODES_INT8: "int8", CODES_FP4: "e2m1 (fp4), kind::mxf4",
                          CODES_BF16X3: "bf16 x3"}.get(codes, "?")
+        if w.kind != "fc":
+            roof["staging"] = {bc.STAGING_PER_TAP: "per tap", bc.STAGING_ROWS: "rows-staged",
+                               bc.STAGING_INPUT: "fp32 input split in shared memory (no pack kernel)"}.get(
+                layer.staging(), "?")
     sm_mhz = clock_info.get("sm_mhz")
     if sm_mhz and bound == "alu":
         p_obs, _, _ = derived_peak(w, sms, sm_mhz, kname, codes)

@@ -36,6 +36,9 @@
 //   input as two boxes of 32 channels into the stage's first two part tiles, and the weight
 //   block; eight more warps (6-13) read the boxes, form x~ and its three bf16 parts and
 //   write them over the boxes (each warp rewrites exactly the rows it read); 3 stages fit.
+//   When its tiles outnumber the CTAs, the CTAs take equal contiguous shares of all tiles'
+//   k-blocks (ConvWork), and a tile cut between two CTAs is finished by the one holding its
+//   first k-blocks, with the other's fp32 partial sums.
 // Every mbarrier wait gives up after one second of %globaltimer, sets the error word and
 // makes all roles stop; TMEM is released on every exit path.
 #include <cuda.h>
