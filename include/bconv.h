@@ -256,10 +256,9 @@ int32_t bconv_tc_codes(bconv_handle_t h);
  *   INPUT    binaryWeights convolutions: per tap, a box of the fp32 input itself; converting
  *            warps of the contraction form x~ = in_scale * x + in_bias and its three bf16 parts
  *            in shared memory, so no parts buffer is written or read (no pack kernel runs).
- *            Needs no beta,
- *            in_c % 4 == 0, a 16-byte aligned input and an fp32 output; a bit-packed output
- *            moves the layer to PER_TAP, and so does a forward whose input is not 16-byte
- *            aligned (for that call only: it runs on the SIMT family).
+ *            Needs no beta, in_c % 4 == 0, at most 128 output channels and an fp32 output; a
+ *            bit-packed output (bconv_set_output_terms) moves the layer to PER_TAP.  A forward
+ *            whose input is not 16-byte aligned runs on the SIMT family (that call only).
  *   AUTO     ROWS or INPUT where they apply, else PER_TAP.
  * Returns INVALID_ARG for an unknown value.
  */
