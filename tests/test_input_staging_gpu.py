@@ -74,10 +74,10 @@ def test_input_staging_parity(w, cuda_device):
 
 
 def test_input_staging_choice(cuda_device):
-    """INPUT where it applies; beta, in_c % 4 != 0, a forced per-tap setting and a bit-packed
-    output keep the parts buffer."""
-    def layer(ni=64, use_beta=False, **kw):
-        c = synth.small_case(batch=2, h=12, w=12, ni=ni, no=64, k=3, op=synth.BINARY_WEIGHTS, use_beta=use_beta,
+    """INPUT where it applies; beta, in_c % 4 != 0, more than 128 output channels, a forced
+    per-tap setting and a bit-packed output keep the parts buffer."""
+    def layer(ni=64, use_beta=False, no=64, **kw):
+        c = synth.small_case(batch=2, h=12, w=12, ni=ni, no=no, k=3, op=synth.BINARY_WEIGHTS, use_beta=use_beta,
                              seed=9, **kw)
         return pu.make_layer(c, synth.make_inputs(c))
 
@@ -88,6 +88,8 @@ def test_input_staging_choice(cuda_device):
         assert l.staging() == bc.STAGING_PER_TAP
         assert l.launches_per_forward() == 2
     with layer(ni=30) as l:
+        assert l.staging() == bc.STAGING_PER_TAP
+    with layer(no=160) as l:  # more than 128 output channels
         assert l.staging() == bc.STAGING_PER_TAP
     with layer() as l:
         l.set_output_terms(None, None)
