@@ -184,3 +184,18 @@ def test_input_staging_equal_shares(w, cuda_device):
             pu.assert_outputs_close(w, inp, y.reshape(-1, w.out_channels).cpu().numpy(), S_ref, beta_ref, y_ref)
     finally:
         layer.close()
+
+
+def test_input_staging_host_buffers(cuda_device):
+    """The host-buffer entry point (copies in, forward, copies out) on the fp32-input kernel: the
+    same output as the device forward, bit for bit."""
+    w = CASES[2]
+    inp = synth.make_inputs(w)
+    y_dev = pu.run_device(w, inp)
+    layer = pu.make_layer(w, inp)
+    try:
+        assert layer.staging() == bc.STAGING_INPUT
+        y_host = layer.forward_host(inp.x)
+    finally:
+        layer.close()
+    np.testing.assert_array_equal(y_host.reshape(y_dev.shape), y_dev)
