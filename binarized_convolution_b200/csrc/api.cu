@@ -366,16 +366,28 @@ bconv_status_t setup_fc(Layer& L, const uint32_t* packed) {
           dst[f0 / 2] |= static_cast<uint8_t>(code << (4 * (f0 % 2)));
         }
       }
+    // as contiguous (N tile, k-block) blocks of 256 rows x 128 bytes, each with the 128-byte
+    // swizzle applied (16-byte chunk c of row r at c ^ (r % 8)): one bulk copy per stage
+    {
+      std::vector<uint8_t> blocks(hb.size());
+      for (int nt = 0; nt < f.n_tiles; ++nt)
+        for (int kb = 0; kb < f.kb_total; ++kb)
+          for (int r = 0; r < 256; ++r) {
+            const uint8_t* src_row = hb.data() + static_cast<size_t>(nt * 256 + r) * row_bytes + static_cast<int64_t>(kb) * 128;
+            uint8_t* dst = blocks.data() + ((static_cast<size_t>(nt) * f.kb_total + kb) * 256 + r) * 128;
+            for (int c = 0; c < 8; ++c) memcpy(dst + 16 * (c ^ (r & 7)), src_row + 16 * c, 16);
+          }
+      hb.swap(blocks);
+    }
     e = L.tc_mem.alloc(&L.wq, hb.size());
     if (e == cudaSuccess) e = cudaMemcpy(L.wq, hb.data(), hb.size(), cudaMemcpyHostToDevice);
   }
   if (e == cudaSuccess) e = L.tc_mem.alloc(&L.codes, static_cast<size_t>(L.N) * row_bytes);
   if (e != cudaSuccess) return from_cuda(e);
-  bool ok = encode_2d(&L.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.codes, static_cast<uint64_t>(row_bytes),
-                      static_cast<uint64_t>(L.N), static_cast<uint64_t>(row_bytes), 128, 128);
-  ok = ok && encode_2d(&L.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.wq, static_cast<uint64_t>(row_bytes),
-                       static_cast<uint64_t>(rows), static_cast<uint64_t>(row_bytes), 128, 256);
+  const bool ok = encode_2d(&L.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.codes, static_cast<uint64_t>(row_bytes),
+                            static_cast<uint64_t>(L.N), static_cast<uint64_t>(row_bytes), 128, 128);
   if (!ok) return BCONV_OK;  // the POPC path stays available
+  f.b_blocks = reinterpret_cast<const uint8_t*>(L.wq);
   f.scale = L.scale;
   f.bias = L.bias;
   f.relu = L.relu;
@@ -897,7 +909,7 @@ bconv_status_t run_forward_tc(Layer& L, const Io& io, cudaStream_t s) {
     f.out = out;
     const bool timed = L.prof.take();
     if (timed) cudaEventRecord(L.prof.start[L.prof.used], s);
-    e = launch_tc_fc(&L.tmA, &L.tmB, f, s);
+    e = launch_tc_fc(&L.tmA, f, s);
     if (timed) cudaEventRecord(L.prof.stop[L.prof.used++], s);
     return from_cuda(e);
   }

@@ -143,14 +143,18 @@ struct FcArgs {
   int relu;
   uint32_t* err;
   float* out;         // [N][No] output, 16-byte aligned
+  // weight codes as contiguous blocks [n_tiles][kb_total][256 rows][128 bytes], each already in
+  // the shared-memory order of the 128-byte swizzle (16-byte chunk c of row r at c ^ (r % 8)):
+  // one 32 KB bulk copy per stage
+  const uint8_t* b_blocks;
 };
 // false: the shape does not fit this kernel (more than 127 k-blocks per split even with 8
 // splits, whose int16 partial sums would overflow, or no cluster fits the device)
 bool tc_fc_plan(FcArgs& a, int sm_count);
 int tc_fc_smem_bytes();
-// tmA: 2-D map over the activation codes {K / 2 bytes, N}, box 128 x 128; tmB: 2-D map over the
-// weight codes {K / 2 bytes, n_tiles * 256}, box 128 x 256; both 128-byte swizzled.
-cudaError_t launch_tc_fc(const CUtensorMap* tmA, const CUtensorMap* tmB, const FcArgs& a, cudaStream_t s);
+// tmA: 2-D map over the activation codes {K / 2 bytes, N}, box 128 x 128, 128-byte swizzled;
+// the weights come from a.b_blocks.
+cudaError_t launch_tc_fc(const CUtensorMap* tmA, const FcArgs& a, cudaStream_t s);
 
 
 int tc_stages(int kind, int bn, int mt);  // stages that fit; < 2: the layout does not fit

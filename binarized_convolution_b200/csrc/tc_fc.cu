@@ -10,9 +10,12 @@
 //
 // Work: an item is 128 images x 256 output channels x a share of the k-blocks (the reduction is
 // split so that the items fill the SMs once); one item per CTA, one 256-column fp32 accumulator
-// in TMEM.  Per k-block a 128 x 128-byte box of activation codes and a 256 x 128-byte box of
-// weight codes (both 128-byte swizzled) feed four M128 N256 K64 MMAs: the activations are read
-// once per 256 channels, the weights once per 128 images.
+// in TMEM.  Per k-block a 128 x 128-byte box of activation codes (TMA, 128-byte swizzled) and a
+// 256 x 128-byte block of weight codes (one 32 KB bulk copy of a block the layer laid out
+// contiguously, already swizzled: contiguous reads stream from HBM faster than 256 rows of 128
+// bytes) feed four M128 N256 K64 MMAs: the activations are read once per 256 channels, the
+// weights once per 128 images.  The first stages' weights are requested before the wait for
+// the previous kernel: they do not depend on it.
 //
 // The k_splits items of a tile form one cluster, and each CTA finishes 128 / k_splits rows of
 // the tile.  Once every CTA of the cluster has completed its MMAs (a cluster barrier), their
@@ -94,7 +97,7 @@ __device__ __forceinline__ uint32_t pack_i16x2(uint32_t lo_f, uint32_t hi_f) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    tc_fc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const FcArgs a) {
+    tc_fc_kernel(const __grid_constant__ CUtensorMap tmA, const FcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0u) {
     if (threadIdx.x == 0) atomicOr(a.err, kErrLayout);
@@ -130,7 +133,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the one arrival, before any byte can land: the other splits' slots of this CTA's rows
     mbar_expect_tx(&B->recv, static_cast<uint32_t>((a.k_splits - 1) * (128 / a.k_splits) * kRowBytes));
     prefetch_tensor_map(&tmA);
-    prefetch_tensor_map(&tmB);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&B->tmem_base)),
@@ -156,6 +158,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const uint8_t* wblocks = a.b_blocks + static_cast<int64_t>(ntile) * a.kb_total * kBBytes;
+  const int pre = min(kStages, max(kb1 - kb0, 0));  // stages whose weights are requested early
+  if (threadIdx.x == 0) {  // (the producer thread) the weights do not depend on the previous kernel
+    for (int i = 0; i < pre; ++i) {
+      uint8_t* st = smem + i * kStageBytes;
+      mbar_expect_tx(&B->full[i], static_cast<uint32_t>(kABytes + kBBytes));
+      bulk_load(st + kABytes, wblocks + static_cast<int64_t>(kb0 + i) * kBBytes, kBBytes, &B->full[i]);
+    }
+  }
   wait_prior_grid();  // the codes and A come from the previous kernel
   if (threadIdx.x == 0) BCONV_STAMP(1);
 
@@ -167,9 +178,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&B->empty[stage], phase ^ 1u, B, a.err)) break;
         uint8_t* st = smem + stage * kStageBytes;
-        mbar_expect_tx(&B->full[stage], static_cast<uint32_t>(kABytes + kBBytes));
+        if (kb - kb0 >= pre) {  // (the first stages' weights are on their way)
+          mbar_expect_tx(&B->full[stage], static_cast<uint32_t>(kABytes + kBBytes));
+          bulk_load(st + kABytes, wblocks + static_cast<int64_t>(kb) * kBBytes, kBBytes, &B->full[stage]);
+        }
         tma_load_2d(st, &tmA, &B->full[stage], kb * 128, m0);
-        tma_load_2d(st + kABytes, &tmB, &B->full[stage], kb * 128, c0);
         if (++stage == kStages) {
           stage = 0;
           phase ^= 1u;
@@ -362,10 +375,11 @@ bool tc_fc_plan(FcArgs& a, int sm_count) {
   return true;
 }
 
-cudaError_t launch_tc_fc(const CUtensorMap* tmA, const CUtensorMap* tmB, const FcArgs& a, cudaStream_t s) {
+cudaError_t launch_tc_fc(const CUtensorMap* tmA, const FcArgs& a, cudaStream_t s) {
   const int items = a.m_tiles * a.n_tiles * a.k_splits;
   if (items == 0) return cudaSuccess;
-  if (!a.out || (reinterpret_cast<uintptr_t>(a.out) & 15u) != 0 || a.k_splits < 1 || a.k_splits > 8 ||
+  if (!a.out || (reinterpret_cast<uintptr_t>(a.out) & 15u) != 0 || !a.b_blocks ||
+      (reinterpret_cast<uintptr_t>(a.b_blocks) & 15u) != 0 || a.k_splits < 1 || a.k_splits > 8 ||
       128 % a.k_splits != 0 || a.kb_per_split > kMaxKbPerSplit)
     return cudaErrorInvalidValue;
   const int smem = tc_fc_smem_bytes();
@@ -387,7 +401,7 @@ cudaError_t launch_tc_fc(const CUtensorMap* tmA, const CUtensorMap* tmB, const F
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, tc_fc_kernel, *tmA, *tmB, a);
+  e = cudaLaunchKernelEx(&cfg, tc_fc_kernel, *tmA, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
