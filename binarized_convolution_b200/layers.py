@@ -139,6 +139,9 @@ class BinaryConv2d(_Layer):
         return nat.bconv_tc_codes(self.handle)
 
     def staging(self) -> int:
+        """How the tensor-core contraction brings in its activations: STAGING_PER_TAP, STAGING_ROWS
+        (XNOR/AND, stride 1) or STAGING_INPUT (binaryWeights from the fp32 input, no pack
+        kernel); 0 without a tensor-core path."""
         return nat.bconv_staging(self.handle)
 
     def forward_into(self, x, out):
