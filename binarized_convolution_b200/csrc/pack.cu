@@ -293,9 +293,13 @@ __global__ void __launch_bounds__(kPackThreads) pack_i8_scalar_kernel(PackI8Args
 // eight codes are one 32-bit store -- so that a pixel's place in the code grid follows from the
 // previous one's and one reduction forms the stage's kSP values of A.
 // ------------------------------------------------------------------------------------
-constexpr int kStagedStages = 16;  // two per converting warp
+constexpr int kStagedStages = 16;  // two per converting warp (one CTA per SM)
 constexpr int kStagedBytes = 8192;
 constexpr int kStagedWarps = 8;  // converting warps; one more warp feeds the ring
+// A stretch of few stages per SM (a small input) runs as two CTAs per SM with half the ring
+// each: more copies start at once, and the ramp to full streaming is what such a pack costs.
+constexpr int kStagedStagesHalf = 8;
+constexpr int kFewStagesPerSm = 32;
 
 struct __align__(8) StagedBars {
   uint64_t full[kStagedStages];
@@ -304,8 +308,9 @@ struct __align__(8) StagedBars {
   uint32_t err_word;  // stands in for a missing error word
 };
 
-template <bool kTerms, bool kA, int kOp, int kSP>
-__global__ void __launch_bounds__((kStagedWarps + 1) * 32, 1) pack_f4_staged_kernel(PackI8Args a, int64_t per_cta) {
+template <bool kTerms, bool kA, int kOp, int kSP, int kStagedStages>
+__global__ void __launch_bounds__((kStagedWarps + 1) * 32, 16 / kStagedStages)
+    pack_f4_staged_kernel(PackI8Args a, int64_t per_cta) {
   extern __shared__ __align__(128) uint8_t sm[];
   StagedBars* B = reinterpret_cast<StagedBars*>(sm + kStagedStages * kStagedBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -364,23 +369,31 @@ __global__ void __launch_bounds__((kStagedWarps + 1) * 32, 1) pack_f4_staged_ker
   if (threadIdx.x == 0) BCONV_STAMP(2);
 }
 
+template <bool kTerms, bool kA, int kOp, int kStages>
+cudaError_t launch_f4_staged_n(const PackI8Args& a, int sp, int ctas_per_sm, cudaStream_t s) {
+  const int sms = current_sm_count();
+  const int64_t stages = ceil_div(a.npix, sp);
+  const int64_t ctas = std::min<int64_t>(static_cast<int64_t>(sms) * ctas_per_sm, stages);
+  const int64_t per_cta = ceil_div(stages, ctas) * sp;
+  const int grid = static_cast<int>(ceil_div(a.npix, per_cta));
+  const int smem = kStages * kStagedBytes + static_cast<int>(sizeof(StagedBars));
+  auto kern = sp == 8   ? pack_f4_staged_kernel<kTerms, kA, kOp, 8, kStages>
+              : sp == 4 ? pack_f4_staged_kernel<kTerms, kA, kOp, 4, kStages>
+              : sp == 2 ? pack_f4_staged_kernel<kTerms, kA, kOp, 2, kStages>
+                        : pack_f4_staged_kernel<kTerms, kA, kOp, 1, kStages>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return launch_overlapped(kern, dim3(grid), dim3((kStagedWarps + 1) * 32), smem, s, a, per_cta);
+}
+
 template <bool kTerms, bool kA, int kOp>
 cudaError_t launch_f4_staged(const PackI8Args& a, cudaStream_t s) {
   const int sp_max = kStagedBytes / (4 * a.ni);  // >= 1 (checked by the caller)
   const int sp = sp_max >= 8 ? 8 : sp_max >= 4 ? 4 : sp_max >= 2 ? 2 : 1;
-  const int sms = current_sm_count();
   const int64_t stages = ceil_div(a.npix, sp);
-  const int64_t ctas = std::min<int64_t>(sms, stages);
-  const int64_t per_cta = ceil_div(stages, ctas) * sp;
-  const int grid = static_cast<int>(ceil_div(a.npix, per_cta));
-  const int smem = kStagedStages * kStagedBytes + static_cast<int>(sizeof(StagedBars));
-  auto kern = sp == 8   ? pack_f4_staged_kernel<kTerms, kA, kOp, 8>
-              : sp == 4 ? pack_f4_staged_kernel<kTerms, kA, kOp, 4>
-              : sp == 2 ? pack_f4_staged_kernel<kTerms, kA, kOp, 2>
-                        : pack_f4_staged_kernel<kTerms, kA, kOp, 1>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  return launch_overlapped(kern, dim3(grid), dim3((kStagedWarps + 1) * 32), smem, s, a, per_cta);
+  if (stages < static_cast<int64_t>(current_sm_count()) * kFewStagesPerSm)
+    return launch_f4_staged_n<kTerms, kA, kOp, kStagedStagesHalf>(a, sp, 2, s);
+  return launch_f4_staged_n<kTerms, kA, kOp, kStagedStages>(a, sp, 1, s);
 }
 
 template <bool kTerms, bool kA, int kOp, bool kF4>
